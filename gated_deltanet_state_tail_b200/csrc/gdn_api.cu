@@ -1,0 +1,354 @@
+// gdn_api.cu -- host side of the Tail-Replay C ABI: argument validation, the
+// varlen plan (windows, work units, longest-first order) and kernel dispatch.
+//
+// The replay window follows "Tail-Replay: Escaping the Curse of Linear
+// Attention in Prefix Caching for Hybrid LLMs", section "Mecanismos
+// Principais", item "Reconstrucao de Estado Independente": only the most
+// recent R tokens of the matched prefix are replayed, from a zero state.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "gdn_internal.h"
+#include "gdn_tail_replay.h"
+
+using gdn::CallArgs;
+using gdn::Unit;
+using gdn::Window;
+using gdn::WorkspaceHeader;
+
+struct gdn_plan {
+    int kind;
+    int batch, num_heads, dk, dv, dtype, kernel;
+    int device;
+    std::vector<Window> windows;
+    std::vector<Unit> units;
+    long long total_tokens;
+    void* dev_block;          // windows then units
+    Window* d_windows;
+    Unit* d_units;
+};
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+gdn_status check_desc(const gdn_varlen_desc* d) {
+    if (!d || !d->seq_offsets_host) return GDN_ERR_INVALID_ARG;
+    if (d->batch < 1 || d->num_heads < 1) return GDN_ERR_INVALID_ARG;
+    if (d->dtype != GDN_F32 && d->dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
+    if ((d->d_k != 64 && d->d_k != 128) || (d->d_v != 64 && d->d_v != 128)) return GDN_ERR_UNSUPPORTED;
+    if (d->kernel < GDN_KERNEL_AUTO || d->kernel > GDN_KERNEL_CHUNKED_TC) return GDN_ERR_INVALID_ARG;
+    const int32_t* off = d->seq_offsets_host;
+    if (off[0] < 0) return GDN_ERR_INVALID_ARG;
+    for (int b = 0; b < d->batch; ++b)
+        if (off[b + 1] < off[b]) return GDN_ERR_INVALID_ARG;
+    // element offsets are 64-bit on the device; rows * H * d must fit comfortably
+    const long long rows = off[d->batch];
+    if (rows * d->num_heads > (1ll << 40)) return GDN_ERR_INVALID_ARG;
+    return GDN_OK;
+}
+
+int resolve_kernel(const gdn_varlen_desc* d) {
+    if (d->kernel != GDN_KERNEL_AUTO) return d->kernel;
+    return gdn::chunk_tc_supported(d->dtype, d->d_k, d->d_v) ? GDN_KERNEL_CHUNKED_TC
+                                                              : GDN_KERNEL_RECURRENT;
+}
+
+gdn_status finish_plan(gdn_plan* p, gdn_plan_t* out) {
+    // Work units: every (sequence, head); longest window first so the long
+    // units start early and the short ones fill the tail of the grid.
+    p->units.reserve((size_t)p->batch * p->num_heads);
+    for (int b = 0; b < p->batch; ++b)
+        for (int h = 0; h < p->num_heads; ++h) p->units.push_back(Unit{b, h});
+    std::stable_sort(p->units.begin(), p->units.end(), [p](const Unit& x, const Unit& y) {
+        return p->windows[x.seq].len > p->windows[y.seq].len;
+    });
+    p->total_tokens = 0;
+    for (const Window& w : p->windows) p->total_tokens += w.len;
+
+    if (cudaGetDevice(&p->device) != cudaSuccess) return GDN_ERR_CUDA;
+    const size_t wbytes = sizeof(Window) * p->windows.size();
+    const size_t ubytes = sizeof(Unit) * p->units.size();
+    if (cudaMalloc(&p->dev_block, wbytes + ubytes) != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_ALLOC;
+    }
+    p->d_windows = static_cast<Window*>(p->dev_block);
+    p->d_units = reinterpret_cast<Unit*>(static_cast<char*>(p->dev_block) + wbytes);
+    if (cudaMemcpy(p->d_windows, p->windows.data(), wbytes, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(p->d_units, p->units.data(), ubytes, cudaMemcpyHostToDevice) != cudaSuccess) {
+        cudaFree(p->dev_block);
+        p->dev_block = nullptr;
+        return GDN_ERR_CUDA;
+    }
+    *out = p;
+    return GDN_OK;
+}
+
+gdn_status check_replay_arrays(int batch, const int32_t* off, const int32_t* match_len,
+                               const int32_t* R) {
+    if (batch < 1 || !off || !match_len || !R) return GDN_ERR_INVALID_ARG;
+    if (off[0] < 0) return GDN_ERR_INVALID_ARG;
+    for (int b = 0; b < batch; ++b) {
+        const long long cached = (long long)off[b + 1] - off[b];
+        if (cached < 0) return GDN_ERR_INVALID_ARG;
+        if (match_len[b] < 0 || match_len[b] > cached) return GDN_ERR_INVALID_ARG;
+        if (R[b] < 0) return GDN_ERR_INVALID_ARG;
+    }
+    return GDN_OK;
+}
+
+gdn_plan* new_plan(const gdn_varlen_desc* d, int kind) {
+    gdn_plan* p = new (std::nothrow) gdn_plan();
+    if (!p) return nullptr;
+    p->kind = kind;
+    p->batch = d->batch;
+    p->num_heads = d->num_heads;
+    p->dk = d->d_k;
+    p->dv = d->d_v;
+    p->dtype = d->dtype;
+    p->kernel = resolve_kernel(d);
+    p->dev_block = nullptr;
+    return p;
+}
+
+gdn_status check_call_common(gdn_plan_t plan, void* workspace) {
+    if (!plan || !workspace) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(workspace)) return GDN_ERR_INVALID_ARG;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
+    if (dev != plan->device) return GDN_ERR_INVALID_ARG;
+    return GDN_OK;
+}
+
+gdn_status launch(gdn_plan_t plan, CallArgs& a, cudaStream_t stream) {
+    if (cudaMemsetAsync(a.ws, 0, sizeof(WorkspaceHeader), stream) != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_CUDA;
+    }
+    cudaError_t e = plan->kernel == GDN_KERNEL_CHUNKED_TC ? gdn::launch_chunk_tc(a, stream)
+                                                          : gdn::launch_recurrent(a, stream);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_CUDA;
+    }
+    return GDN_OK;
+}
+
+void fill_common(gdn_plan_t plan, CallArgs& a, void* workspace) {
+    a.kind = plan->kind;
+    a.dtype = plan->dtype;
+    a.num_heads = plan->num_heads;
+    a.dk = plan->dk;
+    a.dv = plan->dv;
+    a.batch = plan->batch;
+    a.units = (long long)plan->units.size();
+    a.windows = plan->d_windows;
+    a.unit_list = plan->d_units;
+    a.ws = static_cast<WorkspaceHeader*>(workspace);
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_plan_create_replay(const gdn_varlen_desc* cache, const int32_t* match_len_host,
+                                  const int32_t* R_host, gdn_plan_t* out) {
+    if (!out) return GDN_ERR_INVALID_ARG;
+    *out = nullptr;
+    gdn_status s = check_desc(cache);
+    if (s != GDN_OK) return s;
+    if (!match_len_host || !R_host) return GDN_ERR_INVALID_ARG;
+    const int32_t* off = cache->seq_offsets_host;
+    s = check_replay_arrays(cache->batch, off, match_len_host, R_host);
+    if (s != GDN_OK) return s;
+    if (resolve_kernel(cache) == GDN_KERNEL_CHUNKED_TC &&
+        !gdn::chunk_tc_supported(cache->dtype, cache->d_k, cache->d_v))
+        return GDN_ERR_UNSUPPORTED;
+    gdn_plan* p = new_plan(cache, gdn::kReplay);
+    if (!p) return GDN_ERR_ALLOC;
+    p->windows.resize(cache->batch);
+    std::vector<int64_t> row0(cache->batch);
+    std::vector<int32_t> len(cache->batch);
+    gdn_replay_windows(cache->batch, off, match_len_host, R_host, row0.data(), len.data());
+    for (int b = 0; b < cache->batch; ++b) {
+        const int L = match_len_host[b];
+        Window& w = p->windows[b];
+        std::memset(&w, 0, sizeof w);
+        w.row0 = row0[b];   // R > L clamps to L; R = 0 is the Zero-Only state
+        w.len = len[b];
+        w.expect_off = off[b];
+        w.expect_end = off[b + 1];
+        w.expect_match = L;
+        w.expect_budget = R_host[b];
+    }
+    s = finish_plan(p, out);
+    if (s != GDN_OK) delete p;
+    return s;
+}
+
+gdn_status gdn_plan_create_prefill(const gdn_varlen_desc* seqs, gdn_plan_t* out) {
+    if (!out) return GDN_ERR_INVALID_ARG;
+    *out = nullptr;
+    gdn_status s = check_desc(seqs);
+    if (s != GDN_OK) return s;
+    if (resolve_kernel(seqs) == GDN_KERNEL_CHUNKED_TC &&
+        !gdn::chunk_tc_supported(seqs->dtype, seqs->d_k, seqs->d_v))
+        return GDN_ERR_UNSUPPORTED;
+    gdn_plan* p = new_plan(seqs, gdn::kPrefill);
+    if (!p) return GDN_ERR_ALLOC;
+    const int32_t* off = seqs->seq_offsets_host;
+    p->windows.resize(seqs->batch);
+    for (int b = 0; b < seqs->batch; ++b) {
+        Window& w = p->windows[b];
+        std::memset(&w, 0, sizeof w);
+        w.row0 = off[b];
+        w.len = off[b + 1] - off[b];
+        w.expect_off = off[b];
+        w.expect_end = off[b + 1];
+    }
+    s = finish_plan(p, out);
+    if (s != GDN_OK) delete p;
+    return s;
+}
+
+gdn_status gdn_replay_windows(int32_t batch, const int32_t* seq_offsets_host,
+                              const int32_t* match_len_host, const int32_t* R_host,
+                              int64_t* row0_out, int32_t* len_out) {
+    if (!row0_out || !len_out) return GDN_ERR_INVALID_ARG;
+    gdn_status s = check_replay_arrays(batch, seq_offsets_host, match_len_host, R_host);
+    if (s != GDN_OK) return s;
+    for (int b = 0; b < batch; ++b) {
+        const int L = match_len_host[b];
+        const int reff = std::min(R_host[b], L);
+        row0_out[b] = (int64_t)seq_offsets_host[b] + L - reff;
+        len_out[b] = reff;
+    }
+    return GDN_OK;
+}
+
+void gdn_plan_destroy(gdn_plan_t plan) {
+    if (!plan) return;
+    if (plan->dev_block) cudaFree(plan->dev_block);
+    delete plan;
+}
+
+gdn_status gdn_plan_window(gdn_plan_t plan, int32_t b, int64_t* row0, int32_t* len) {
+    if (!plan || !row0 || !len || b < 0 || b >= plan->batch) return GDN_ERR_INVALID_ARG;
+    *row0 = plan->windows[b].row0;
+    *len = plan->windows[b].len;
+    return GDN_OK;
+}
+
+gdn_status gdn_plan_info(gdn_plan_t plan, int64_t* units, int64_t* total_tokens, int32_t* kernel) {
+    if (!plan) return GDN_ERR_INVALID_ARG;
+    if (units) *units = (int64_t)plan->units.size();
+    if (total_tokens) *total_tokens = plan->total_tokens;
+    if (kernel) *kernel = plan->kernel;
+    return GDN_OK;
+}
+
+size_t gdn_workspace_bytes(gdn_plan_t plan) {
+    (void)plan;
+    return sizeof(WorkspaceHeader);
+}
+
+gdn_status gdn_tail_replay_state(gdn_plan_t plan, const void* q, const void* k, const void* v,
+                                 const float* alpha, const float* beta,
+                                 const int32_t* seq_offsets, const int32_t* match_len,
+                                 const int32_t* R, float* state_out, void* workspace,
+                                 void* stream) {
+    gdn_status s = check_call_common(plan, workspace);
+    if (s != GDN_OK) return s;
+    if (plan->kind != gdn::kReplay) return GDN_ERR_INVALID_ARG;
+    if (!state_out || !aligned16(state_out)) return GDN_ERR_INVALID_ARG;
+    if (plan->total_tokens > 0) {
+        if (!k || !v || !alpha || !beta) return GDN_ERR_INVALID_ARG;
+        if (!aligned16(k) || !aligned16(v) || !aligned16(alpha) || !aligned16(beta))
+            return GDN_ERR_INVALID_ARG;
+    }
+    CallArgs a;
+    std::memset(&a, 0, sizeof a);
+    fill_common(plan, a, workspace);
+    a.chk_offsets = seq_offsets;
+    a.chk_match = match_len;
+    a.chk_budget = R;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.alpha = alpha;
+    a.beta = beta;
+    a.state_in = nullptr;
+    a.o_out = nullptr;
+    a.state_out = state_out;
+    return launch(plan, a, static_cast<cudaStream_t>(stream));
+}
+
+gdn_status gdn_chunk_prefill(gdn_plan_t plan, const void* q, const void* k, const void* v,
+                             const float* alpha, const float* beta, const int32_t* cu_seqlens,
+                             const float* state_in, void* o_out, float* state_out,
+                             void* workspace, void* stream) {
+    gdn_status s = check_call_common(plan, workspace);
+    if (s != GDN_OK) return s;
+    if (plan->kind != gdn::kPrefill) return GDN_ERR_INVALID_ARG;
+    if (plan->total_tokens > 0) {
+        if (!q || !k || !v || !alpha || !beta || !o_out) return GDN_ERR_INVALID_ARG;
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(alpha) ||
+            !aligned16(beta) || !aligned16(o_out))
+            return GDN_ERR_INVALID_ARG;
+    }
+    if ((state_in && !aligned16(state_in)) || (state_out && !aligned16(state_out)))
+        return GDN_ERR_INVALID_ARG;
+    CallArgs a;
+    std::memset(&a, 0, sizeof a);
+    fill_common(plan, a, workspace);
+    a.chk_offsets = cu_seqlens;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.alpha = alpha;
+    a.beta = beta;
+    a.state_in = state_in;
+    a.o_out = o_out;
+    a.state_out = state_out;
+    return launch(plan, a, static_cast<cudaStream_t>(stream));
+}
+
+gdn_status gdn_workspace_status(const void* workspace, void* stream) {
+    if (!workspace) return GDN_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_CUDA;
+    }
+    unsigned int status = 0;
+    if (cudaMemcpy(&status, workspace, sizeof status, cudaMemcpyDeviceToHost) != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_CUDA;
+    }
+    if (status & gdn::kStatusTimeout) return GDN_ERR_TIMEOUT;
+    if (status & gdn::kStatusMismatch) return GDN_ERR_MISMATCH;
+    return GDN_OK;
+}
+
+const char* gdn_status_string(gdn_status s) {
+    switch (s) {
+        case GDN_OK: return "ok";
+        case GDN_ERR_INVALID_ARG: return "invalid argument";
+        case GDN_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case GDN_ERR_CUDA: return "CUDA error";
+        case GDN_ERR_TIMEOUT: return "device wait timed out";
+        case GDN_ERR_ALLOC: return "allocation failed";
+        case GDN_ERR_MISMATCH: return "device descriptor arrays disagree with the plan";
+    }
+    return "unknown status";
+}
+
+int32_t gdn_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,89 @@
+// gdn_internal.h -- structures shared by the host API and the kernels of the
+// Tail-Replay library.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdn {
+
+// Work window of one sequence, as validated on the host by the plan.
+//   replay : rows [row0, row0 + len) are the tail of the matched prefix
+//   prefill: rows [row0, row0 + len) are the whole sequence
+// The expect_* fields are the descriptor values the window was derived from;
+// kernels compare them with the device copies a caller passes.
+struct Window {
+    long long row0;
+    int len;
+    int expect_off;       // seq_offsets[b]
+    int expect_end;       // seq_offsets[b + 1]
+    int expect_match;     // replay: match_len[b]; prefill: unused
+    int expect_budget;    // replay: R[b]; prefill: unused
+    int pad;
+};
+static_assert(sizeof(Window) == 32, "Window is 32 bytes");
+
+// One (sequence, head) work unit.  Plans order units longest first.
+struct Unit {
+    int seq;
+    int head;
+};
+
+// Per-call device scratch at the start of the caller's workspace.
+struct WorkspaceHeader {
+    unsigned int status;        // bit set of kStatus*
+    unsigned int next_unit;     // dynamic scheduler counter
+    unsigned int timeout_where; // first wait that gave up (kernel-defined code)
+    unsigned int pad[61];
+};
+static_assert(sizeof(WorkspaceHeader) == 256, "header is 256 bytes");
+
+constexpr unsigned int kStatusMismatch = 1u;
+constexpr unsigned int kStatusTimeout = 2u;
+
+enum PlanKind { kReplay = 0, kPrefill = 1 };
+
+// Everything a kernel needs for one call.
+struct CallArgs {
+    int kind;               // PlanKind
+    int dtype;              // 0 = fp32, 1 = bf16 (q, k, v, o)
+    int num_heads;
+    int dk, dv;
+    int batch;
+    long long units;
+    const Window* windows;  // [batch], plan-owned device memory
+    const Unit* unit_list;  // [units], longest first
+    // optional device descriptor arrays to check against the plan
+    const int* chk_offsets; // [batch + 1] or null
+    const int* chk_match;   // [batch] or null (replay)
+    const int* chk_budget;  // [batch] or null (replay)
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* alpha;
+    const float* beta;
+    const float* state_in;  // null = zero state
+    void* o_out;            // null for replay
+    float* state_out;       // may be null for prefill
+    WorkspaceHeader* ws;
+};
+
+// Device-side check of one unit's window against the caller's descriptor
+// arrays.  Returns true if the unit may run.
+__device__ __forceinline__ bool window_agrees(const CallArgs& a, int b) {
+    const Window& w = a.windows[b];
+    if (a.chk_offsets) {
+        if (a.chk_offsets[b] != w.expect_off || a.chk_offsets[b + 1] != w.expect_end) return false;
+    }
+    if (a.kind == kReplay) {
+        if (a.chk_match && a.chk_match[b] != w.expect_match) return false;
+        if (a.chk_budget && a.chk_budget[b] != w.expect_budget) return false;
+    }
+    return true;
+}
+
+cudaError_t launch_recurrent(const CallArgs& a, cudaStream_t stream);
+cudaError_t launch_chunk_tc(const CallArgs& a, cudaStream_t stream);
+bool chunk_tc_supported(int dtype, int dk, int dv);
+
+}  // namespace gdn

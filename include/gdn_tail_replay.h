@@ -1,0 +1,199 @@
+/*
+ * gdn_tail_replay.h -- C ABI of the Tail-Replay state rebuild and chunked
+ * suffix prefill for Gated DeltaNet layers on B200 (sm_100a).
+ *
+ * The method ("Tail-Replay: Escaping the Curse of Linear Attention in Prefix
+ * Caching for Hybrid LLMs", gist.science summary, section "Mecanismos
+ * Principais", item "Reconstrucao de Estado Independente"): on a prefix-cache
+ * hit the recurrent state of each linear-attention (Gated DeltaNet) layer is
+ * rebuilt by taking only the most recent R tokens of the matched prefix,
+ * starting from a zero state, and replaying the layer's recurrence over that
+ * tail.  The same page's "Resultados" section times the first token after
+ * the hit, i.e. the prefill of the request's new suffix that continues from
+ * the rebuilt state.
+ *
+ * The recurrence (Gated DeltaNet's gated delta rule), per head, with a
+ * d_k x d_v state S whose rows are indexed by the key dimension:
+ *     S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t
+ * alpha_t is the gate value in [0, 1] (not its log); no query scaling.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  Layout.  q, k: [rows, H, d_k]; v, o: [rows, H, d_v]; token-major packed
+ *    rows, contiguous (row stride H*d elements).  alpha, beta: [rows, H]
+ *    fp32 always (bf16 would round 0.999 to 1).  States: [batch, H, d_k,
+ *    d_v] fp32, row-major, key dimension first.
+ *  dtype.  q, k, v and o share one element type: GDN_F32 or GDN_BF16.
+ *  Ownership.  The caller owns every buffer.  The library allocates device
+ *    memory only inside gdn_plan_create_* (a small schedule table) and frees
+ *    it in gdn_plan_destroy.  No call on the hot path allocates.
+ *  Streams.  `stream` is a cudaStream_t passed as void* (NULL = legacy
+ *    default stream).  Every hot-path call is asynchronous on that stream.
+ *  Errors.  Arguments are validated on the host before anything is
+ *    launched; a rejected call launches nothing and returns a status.  Device
+ *    code never traps: problems it detects (a descriptor array that disagrees
+ *    with the plan, a wait that ran out) set bits in the workspace status
+ *    word, which gdn_workspace_status() reads after the stream.
+ *  Pointers.  Device buffers must be 16-byte aligned.
+ *  Determinism.  Reruns on the same inputs give bit-identical results.
+ *  Threads.  A plan is immutable after creation and may be used from
+ *    several host threads; concurrent calls need separate workspaces.
+ */
+#ifndef GDN_TAIL_REPLAY_H
+#define GDN_TAIL_REPLAY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gdn_status {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,  /* null pointer, bad size, bad offsets, misaligned buffer */
+    GDN_ERR_UNSUPPORTED = 2,  /* head dims or dtype this build has no kernel for */
+    GDN_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+    GDN_ERR_TIMEOUT = 4,      /* a device-side wait gave up (reported via the workspace) */
+    GDN_ERR_ALLOC = 5,        /* plan creation could not allocate */
+    GDN_ERR_MISMATCH = 6      /* device descriptor arrays disagree with the plan */
+} gdn_status;
+
+typedef enum gdn_dtype { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
+
+/* Kernel selection.  AUTO picks the tensor-core chunked kernel for bf16 with
+ * d_k = d_v = 128 and the exact fp32 CUDA-core recurrent kernel otherwise. */
+typedef enum gdn_kernel {
+    GDN_KERNEL_AUTO = 0,
+    GDN_KERNEL_RECURRENT = 1,   /* token-recurrent, fp32 CUDA cores, any supported shape */
+    GDN_KERNEL_CHUNKED_TC = 2   /* chunked WY/UT form on tcgen05 tensor cores (bf16, d = 128) */
+} gdn_kernel;
+
+/* Varlen batch descriptor.  Sequence b occupies rows [seq_offsets[b],
+ * seq_offsets[b+1]) of the packed buffers.  Layer stacks are folded in by
+ * treating (layer, request) pairs as sequences of one packed batch. */
+typedef struct gdn_varlen_desc {
+    int32_t batch;                    /* number of sequences, >= 1 */
+    int32_t num_heads;                /* H, >= 1 */
+    int32_t d_k;                      /* key head dim: 64 or 128 */
+    int32_t d_v;                      /* value head dim: 64 or 128 */
+    int32_t dtype;                    /* gdn_dtype of q, k, v, o */
+    int32_t kernel;                   /* gdn_kernel; 0 = AUTO */
+    const int32_t* seq_offsets_host;  /* [batch + 1] host copy; non-decreasing, [0] >= 0 */
+} gdn_varlen_desc;
+
+typedef struct gdn_plan* gdn_plan_t;
+
+/*
+ * Build the schedule of a tail replay ("Mecanismos Principais", item
+ * "Reconstrucao de Estado Independente": the last k tokens of the matched
+ * prefix, replayed from a zero state).
+ *   cache          descriptor of the packed prefix cache; the cached entry of
+ *                  sequence b may be longer than its match.
+ *   match_len_host [batch] matched prefix length L_b, 0 <= L_b <= cached length.
+ *   R_host         [batch] replay budget R_b >= 0; R_b > L_b is clamped to L_b,
+ *                  R_b = 0 (or L_b = 0) yields the zero state ("Zero-Only").
+ * Sequence b's window is rows [off_b + L_b - min(R_b, L_b), off_b + L_b).
+ * The plan copies what it needs; the host arrays may be freed afterwards.
+ * Returns GDN_OK, INVALID_ARG, UNSUPPORTED, ALLOC or CUDA.
+ */
+GDN_API gdn_status gdn_plan_create_replay(const gdn_varlen_desc* cache, const int32_t* match_len_host,
+                                  const int32_t* R_host, gdn_plan_t* out);
+
+/*
+ * Build the schedule of a chunked prefill over whole sequences (the suffix
+ * prefill that follows the rebuild, "Resultados" section: time to first
+ * token; with a zero initial state over prefix ++ suffix it is the full
+ * prefill the pages compare against).  Sequence b is rows [off_b, off_b+1).
+ */
+GDN_API gdn_status gdn_plan_create_prefill(const gdn_varlen_desc* seqs, gdn_plan_t* out);
+
+/* The replay windows a replay plan would use, computed on the host with no
+ * device work: row0_out[b] = seq_offsets[b] + L_b - min(R_b, L_b) and
+ * len_out[b] = min(R_b, L_b).  Same validation as gdn_plan_create_replay
+ * (INVALID_ARG for a match longer than its cached entry, R_b < 0, offsets
+ * that decrease, or null pointers); nothing is written on error. */
+GDN_API gdn_status gdn_replay_windows(int32_t batch, const int32_t* seq_offsets_host,
+                                      const int32_t* match_len_host, const int32_t* R_host,
+                                      int64_t* row0_out, int32_t* len_out);
+
+/* Free a plan (NULL is ignored).  Synchronises with nothing; do not destroy a
+ * plan while a call that uses it may still be running. */
+GDN_API void gdn_plan_destroy(gdn_plan_t plan);
+
+/* First row and length of sequence b's work window (replay: the tail window;
+ * prefill: the whole sequence).  For tests and schedulers. */
+GDN_API gdn_status gdn_plan_window(gdn_plan_t plan, int32_t b, int64_t* row0, int32_t* len);
+
+/* Number of (sequence, head) work units and the kernel the plan will run. */
+GDN_API gdn_status gdn_plan_info(gdn_plan_t plan, int64_t* units, int64_t* total_tokens,
+                         int32_t* kernel);
+
+/* Bytes of device workspace a call on this plan needs (>= 256, multiple of
+ * 256).  The caller allocates it (16-byte aligned) and passes it to each
+ * call; calls running concurrently need separate workspaces. */
+GDN_API size_t gdn_workspace_bytes(gdn_plan_t plan);
+
+/*
+ * Tail replay: rebuild the state at the end of each matched prefix.
+ *   q            unused by the state-only replay; may be NULL.
+ *   k, v         packed cache rows, dtype of the plan.
+ *   alpha, beta  [rows, H] fp32 gates of the cached rows.
+ *   seq_offsets, match_len, R
+ *                device copies of the arrays given to the plan ([batch+1],
+ *                [batch], [batch] int32), or NULL.  When given, each work
+ *                unit checks its window against them; a disagreement skips
+ *                the unit and sets GDN_ERR_MISMATCH in the workspace.
+ *                Addressing always uses the plan's validated copy.
+ *   state_out    [batch, H, d_k, d_v] fp32, written in full.
+ *   workspace    gdn_workspace_bytes(plan) bytes of device memory.
+ *   stream       cudaStream_t.
+ * Host-side return: GDN_OK or an argument/launch error.  Device-side
+ * problems are read with gdn_workspace_status().
+ */
+GDN_API gdn_status gdn_tail_replay_state(gdn_plan_t plan, const void* q, const void* k, const void* v,
+                                 const float* alpha, const float* beta,
+                                 const int32_t* seq_offsets, const int32_t* match_len,
+                                 const int32_t* R, float* state_out, void* workspace,
+                                 void* stream);
+
+/*
+ * Chunked prefill over each sequence of a prefill plan, continuing from
+ * state_in, emitting o_t = S_t^T q_t for every row and the final state.
+ *   q, k, v      packed rows, dtype of the plan.
+ *   alpha, beta  [rows, H] fp32.
+ *   cu_seqlens   device copy of the plan's offsets ([batch+1] int32) or NULL;
+ *                checked like the replay's descriptor arrays.
+ *   state_in     [batch, H, d_k, d_v] fp32, or NULL for the zero state.
+ *   o_out        [rows, H, d_v] in the plan's dtype; rows of the sequences
+ *                are written, other rows are left untouched.
+ *   state_out    [batch, H, d_k, d_v] fp32, or NULL.  May alias state_in.
+ */
+GDN_API gdn_status gdn_chunk_prefill(gdn_plan_t plan, const void* q, const void* k, const void* v,
+                             const float* alpha, const float* beta, const int32_t* cu_seqlens,
+                             const float* state_in, void* o_out, float* state_out,
+                             void* workspace, void* stream);
+
+/* Synchronise `stream`, then return the status the device recorded in
+ * `workspace` during the last call (GDN_OK, GDN_ERR_TIMEOUT or
+ * GDN_ERR_MISMATCH), or GDN_ERR_CUDA if the stream itself failed. */
+GDN_API gdn_status gdn_workspace_status(const void* workspace, void* stream);
+
+/* Static description of a status code. */
+GDN_API const char* gdn_status_string(gdn_status s);
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+GDN_API int32_t gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_TAIL_REPLAY_H */

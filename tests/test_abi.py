@@ -1,0 +1,123 @@
+"""C-ABI tests that need no GPU: the library loads, exports every symbol the
+headers declare, and the host-side validation and window arithmetic behave."""
+import ctypes
+import glob
+import os
+import re
+
+import numpy as np
+import pytest
+
+import gated_deltanet_state_tail_b200 as gdn
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        for m in re.finditer(r"GDN_API\s+[\w\s\*]+?\b(gdn_\w+)\s*\(", text):
+            names.add(m.group(1))
+    return names
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_symbols()
+    assert len(names) >= 12
+    lib = gdn.library()
+    for n in sorted(names):
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+    assert set(gdn.EXPORTED) <= names
+
+
+def test_version_and_status_strings():
+    assert gdn.gdn_version() >= 100
+    for s in range(7):
+        assert gdn.gdn_status_string(s)
+    assert gdn.gdn_status_string(0) == "ok"
+    assert "unknown" in gdn.gdn_status_string(99)
+
+
+def _desc(batch=1, H=2, dk=128, dv=128, dtype=gdn.GDN_BF16, kernel=0, offsets=None):
+    off = np.asarray(offsets if offsets is not None else [0, 100], np.int32)
+    d = gdn.gdn_varlen_desc()
+    d.batch, d.num_heads, d.d_k, d.d_v, d.dtype, d.kernel = batch, H, dk, dv, dtype, kernel
+    d.seq_offsets_host = off.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    return d, off
+
+
+def _create_replay(d, ml, R):
+    lib = gdn.library()
+    ml = np.asarray(ml, np.int32)
+    R = np.asarray(R, np.int32)
+    h = ctypes.c_void_p()
+    return lib.gdn_plan_create_replay(ctypes.byref(d), ml.ctypes.data, R.ctypes.data, ctypes.byref(h))
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dk=96), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dv=32), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dtype=7), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(batch=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(H=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(kernel=9), gdn.GDN_ERR_INVALID_ARG),
+    (dict(offsets=[-1, 100]), gdn.GDN_ERR_INVALID_ARG),
+])
+def test_descriptor_rejected_before_any_device_work(kw, status):
+    d, off = _desc(**kw)
+    assert _create_replay(d, [50], [10]) == status
+
+
+def test_replay_arrays_rejected():
+    d, off = _desc(batch=2, offsets=[0, 100, 90])          # decreasing offsets
+    assert _create_replay(d, [50, 10], [10, 1]) == gdn.GDN_ERR_INVALID_ARG
+    d, off = _desc(batch=2, offsets=[0, 100, 150])
+    assert _create_replay(d, [101, 10], [10, 1]) == gdn.GDN_ERR_INVALID_ARG   # match > cached
+    assert _create_replay(d, [50, 10], [10, -1]) == gdn.GDN_ERR_INVALID_ARG   # negative budget
+    assert _create_replay(d, [-5, 10], [10, 1]) == gdn.GDN_ERR_INVALID_ARG    # negative match
+    lib = gdn.library()
+    h = ctypes.c_void_p()
+    assert lib.gdn_plan_create_replay(None, None, None, ctypes.byref(h)) == gdn.GDN_ERR_INVALID_ARG
+    assert lib.gdn_plan_create_replay(ctypes.byref(d), None, None, ctypes.byref(h)) == gdn.GDN_ERR_INVALID_ARG
+    assert lib.gdn_plan_create_replay(ctypes.byref(d), None, None, None) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_chunked_kernel_needs_bf16_d128():
+    d, off = _desc(dtype=gdn.GDN_F32, kernel=gdn.GDN_KERNEL_CHUNKED_TC)
+    assert _create_replay(d, [50], [10]) == gdn.GDN_ERR_UNSUPPORTED
+    d, off = _desc(dk=64, dv=64, kernel=gdn.GDN_KERNEL_CHUNKED_TC)
+    assert _create_replay(d, [50], [10]) == gdn.GDN_ERR_UNSUPPORTED
+
+
+def test_null_plan_calls_rejected():
+    lib = gdn.library()
+    assert lib.gdn_tail_replay_state(None, *([None] * 11)) == gdn.GDN_ERR_INVALID_ARG
+    assert lib.gdn_chunk_prefill(None, *([None] * 11)) == gdn.GDN_ERR_INVALID_ARG
+    assert lib.gdn_plan_window(None, 0, None, None) == gdn.GDN_ERR_INVALID_ARG
+    assert lib.gdn_workspace_status(None, None) == gdn.GDN_ERR_INVALID_ARG
+    lib.gdn_plan_destroy(None)
+
+
+def test_replay_windows_match_oracle_bit_exact():
+    r = np.random.default_rng(0)
+    for trial in range(50):
+        B = int(r.integers(1, 40))
+        cached = r.integers(0, 5000, B)
+        off = np.concatenate([[int(r.integers(0, 100))], cached]).cumsum().astype(np.int32)
+        ml = (cached * r.random(B)).astype(np.int32)
+        ml[r.random(B) < 0.1] = 0
+        R = r.integers(0, 6000, B).astype(np.int32)
+        R[r.random(B) < 0.1] = 0
+        row0, ln = gdn.gdn_replay_windows(off, ml, R)
+        for b in range(B):
+            assert oracle.replay_window(off, ml, R, b) == (row0[b], ln[b])
+
+
+def test_replay_windows_edge_cases():
+    off = [0, 256, 256, 300]
+    row0, ln = gdn.gdn_replay_windows(off, [256, 0, 44], [32, 5, 100])
+    assert list(row0) == [224, 256, 256] and list(ln) == [32, 0, 44]
+    with pytest.raises(gdn.GdnError):
+        gdn.gdn_replay_windows(off, [257, 0, 0], [1, 1, 1])
