@@ -28,6 +28,7 @@ struct gdn_plan {
     std::vector<Window> windows;
     std::vector<Unit> units;
     long long total_tokens;
+    long long rows_total;     // seq_offsets[batch]
     void* dev_block;          // windows then units
     Window* d_windows;
     Unit* d_units;
@@ -69,7 +70,11 @@ gdn_status finish_plan(gdn_plan* p, gdn_plan_t* out) {
         return p->windows[x.seq].len > p->windows[y.seq].len;
     });
     p->total_tokens = 0;
-    for (const Window& w : p->windows) p->total_tokens += w.len;
+    p->rows_total = 0;
+    for (const Window& w : p->windows) {
+        p->total_tokens += w.len;
+        p->rows_total = std::max(p->rows_total, (long long)w.expect_end);
+    }
 
     if (cudaGetDevice(&p->device) != cudaSuccess) return GDN_ERR_CUDA;
     const size_t wbytes = sizeof(Window) * p->windows.size();
@@ -148,6 +153,7 @@ void fill_common(gdn_plan_t plan, CallArgs& a, void* workspace) {
     a.dv = plan->dv;
     a.batch = plan->batch;
     a.units = (long long)plan->units.size();
+    a.rows_total = plan->rows_total;
     a.windows = plan->d_windows;
     a.unit_list = plan->d_units;
     a.ws = static_cast<WorkspaceHeader*>(workspace);

@@ -51,6 +51,7 @@ struct CallArgs {
     int dk, dv;
     int batch;
     long long units;
+    long long rows_total;   // rows of the packed buffers the plan addresses (max offset)
     const Window* windows;  // [batch], plan-owned device memory
     const Unit* unit_list;  // [units], longest first
     // optional device descriptor arrays to check against the plan
