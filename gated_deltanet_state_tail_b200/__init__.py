@@ -29,7 +29,7 @@ EXPORTED = (
     "gdn_plan_create_replay", "gdn_plan_create_prefill", "gdn_plan_destroy", "gdn_replay_windows",
     "gdn_plan_window",
     "gdn_plan_info", "gdn_workspace_bytes", "gdn_tail_replay_state", "gdn_chunk_prefill",
-    "gdn_workspace_status", "gdn_status_string", "gdn_version",
+    "gdn_workspace_status", "gdn_status_string", "gdn_version", "gdn_tail_replay_state_noalloc",
 )
 
 
@@ -72,6 +72,7 @@ def _load():
         "gdn_workspace_status": (I32, [P, P]),
         "gdn_status_string": (ctypes.c_char_p, [I32]),
         "gdn_version": (I32, []),
+        "gdn_tail_replay_state_noalloc": (I32, [pd, P, P, P, P, P, P, P, P, ctypes.POINTER(ctypes.c_uint32)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -218,6 +219,23 @@ def gdn_chunk_prefill(handle, q, k, v, alpha, beta, cu_seqlens, state_in, o_out,
                                   _ptr(cu_seqlens), _ptr(state_in), _ptr(o_out), _ptr(state_out),
                                   _ptr(workspace), _stream_handle(stream)),
            "gdn_chunk_prefill")
+
+
+def gdn_tail_replay_state_noalloc(H, dk, dv, dtype, seq_offsets, match_len, R, k, v, alpha, beta,
+                                  state_out, kernel=GDN_KERNEL_AUTO, stream=None, wait_status=True):
+    """Replay without any device allocation (schedule in the library's fixed
+    device array).  Returns the device status word when wait_status is set."""
+    off, ml, rr = _i32(seq_offsets), _i32(match_len), _i32(R)
+    if len(off) != len(ml) + 1 or len(rr) != len(ml):
+        raise ValueError("seq_offsets must have batch + 1 entries, match_len and R batch entries")
+    d = _make_desc(len(ml), H, dk, dv, dtype, kernel, off)
+    st = ctypes.c_uint32(0xFFFFFFFF)
+    _check(_lib.gdn_tail_replay_state_noalloc(ctypes.byref(d), ml.ctypes.data, rr.ctypes.data,
+                                              _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+                                              _ptr(state_out), _stream_handle(stream),
+                                              ctypes.byref(st) if wait_status else None),
+           "gdn_tail_replay_state_noalloc")
+    return st.value if wait_status else None
 
 
 def gdn_workspace_status(workspace, stream=None) -> int:

@@ -181,6 +181,42 @@ GDN_API gdn_status gdn_chunk_prefill(gdn_plan_t plan, const void* q, const void*
                              const float* state_in, void* o_out, float* state_out,
                              void* workspace, void* stream);
 
+/*
+ * Tail replay that allocates nothing (the pages describe no counterpart; this
+ * is a deployment variant of gdn_tail_replay_state).
+ *
+ * For callers that cannot call cudaMalloc -- code running inside a memory
+ * pool that owns the whole device heap, or a runtime that only hands out its
+ * own input and output buffers -- and so can neither create a plan (its
+ * schedule table is device memory) nor provide a workspace.  The schedule
+ * and the status word live in one fixed 64 KB __device__ array inside the
+ * library, which every GPU that loads the library holds until the process
+ * exits.  The call validates like gdn_plan_create_replay, builds the
+ * schedule in a host stack buffer, copies it into that array on `stream`,
+ * clears the status word and launches the same kernel a plan would.  No
+ * cudaMalloc, cudaFree or other allocating routine is called.
+ *   cache, match_len_host, R_host   as for gdn_plan_create_replay.
+ *   k, v, alpha, beta, state_out    as for gdn_tail_replay_state.
+ *   stream                          cudaStream_t.
+ *   status_out                      NULL, or a host word that receives the
+ *                                   device status (0 = ok, else the bit set
+ *                                   gdn_workspace_status decodes); the call
+ *                                   then waits for `stream`.
+ * Limit: 256 + 32 * batch + 8 * batch * num_heads bytes (plus 16 * batch of
+ * host temporaries) must fit in 64 KB; larger batches return
+ * GDN_ERR_UNSUPPORTED before anything is launched.
+ * The first call on a device resolves the array's device address; make that
+ * first call before any stream capture.  Every call on a device shares the
+ * array, which keeps the last call's contents, so calls whose work overlaps
+ * on the GPU (different streams, or several host threads) race.
+ */
+GDN_API gdn_status gdn_tail_replay_state_noalloc(const gdn_varlen_desc* cache,
+                                                 const int32_t* match_len_host,
+                                                 const int32_t* R_host, const void* k,
+                                                 const void* v, const float* alpha,
+                                                 const float* beta, float* state_out,
+                                                 void* stream, uint32_t* status_out);
+
 /* Synchronise `stream`, then return the status the device recorded in
  * `workspace` during the last call (GDN_OK, GDN_ERR_TIMEOUT or
  * GDN_ERR_MISMATCH), or GDN_ERR_CUDA if the stream itself failed. */
