@@ -81,54 +81,65 @@ def sum_over_ranks(x, world):
 # --------------------------------------------------------------------------
 # clocks sampled during the timed region
 # --------------------------------------------------------------------------
-CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+# NVML clock-event reason bits (nvmlClocksEventReason*)
+_REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
 
 class ClockSampler:
-    def __init__(self, device_index):
+    """Samples the SM clock and the clock-event reasons through NVML every few
+    milliseconds while the timed region runs (a background thread)."""
+
+    def __init__(self, device_index, period_s=0.005):
         self.dev = device_index
-        self.proc = None
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self._stop = None
+
+    def _handle(self, pynvml):
+        try:
+            props = torch.cuda.get_device_properties(self.dev)
+            uuid = str(props.uuid)
+            return pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.dev)
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={CLOCK_FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            import pynvml
+            pynvml.nvmlInit()
+            h = self._handle(pynvml)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
         except Exception:
-            self.proc = None
+            return self
+        self._stop = threading.Event()
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                    reasons = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append((float(mhz), int(reasons)))
+                except Exception:
+                    pass
+                self._stop.wait(self.period)
+
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except Exception:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+        if self._stop is not None:
+            self._stop.set()
+            self._thread.join(timeout=2)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in getattr(self, "lines", []):
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for name, val in zip(names, f[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        sm = [m for m, _ in self.samples]
+        reasons = sorted({name for _, r in self.samples for name, bit in _REASON_BITS.items() if r & bit})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(sm), "source": "NVML, 5 ms period"}
 
 
 # --------------------------------------------------------------------------
@@ -184,10 +195,15 @@ class StackData:
     """Per-layer buffers of prefix ++ suffix rows, laid out launch-major:
     buffer slot s = j * GROUPS + g holds GDN layer 3g + j (seed = layer id)."""
 
-    def __init__(self, wl, device):
+    def __init__(self, wl, device, compact=False):
+        # compact: keep only the replay window and the suffix of each layer
+        # (rows [L - R, L + N)); the replay reads exactly the same work, but
+        # the full-prefill comparator needs the whole prefix.
         self.wl = wl
         self.layers = wl.layers
         L, N = wl.match_len[0], wl.suffix_len[0]
+        if compact:
+            L = wl.R[0]
         self.L, self.N, self.R = L, N, wl.R[0]
         self.seq = L + N
         rows = self.layers * self.seq
@@ -302,7 +318,7 @@ def bench_ours(args, rank, world, local):
     wl = inputs.stack_workload(args.layers)
     kernel = {"auto": gdn.GDN_KERNEL_AUTO, "recurrent": gdn.GDN_KERNEL_RECURRENT,
               "chunked": gdn.GDN_KERNEL_CHUNKED_TC}[args.kernel]
-    data = StackData(wl, "cuda")
+    data = StackData(wl, "cuda", compact=args.no_comparator)
     rp, pp, state, o, st_out, n_launch = build_stack_runner(data, kernel)
     kernel_used = rp[0].info["kernel"]
     kname = {1: "recurrent", 2: "chunked_tc"}[kernel_used]
@@ -368,7 +384,8 @@ def bench_ours(args, rank, world, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": wl.dtype, "data": "synthetic (seeded q/k/v/alpha/beta; no datasets or weights)",
         "config": {"workload": wl.name, "layers": wl.layers, "heads": wl.H, "d_k": wl.dk,
-                   "d_v": wl.dv, "matched_prefix": data.L, "replay": data.R, "suffix": data.N,
+                   "d_v": wl.dv, "matched_prefix": wl.match_len[0], "replay": data.R, "suffix": data.N,
+                   "resident_prefix_rows": data.L,
                    "launches_per_phase": n_launch, "layers_per_launch": data.per_launch,
                    "kernel": kname, "l2": "inputs larger than L2 and a 256 MB flush between steps",
                    "parallelism": f"replicas x{world}"},

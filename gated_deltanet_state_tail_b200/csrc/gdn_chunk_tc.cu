@@ -15,157 +15,99 @@
 //   U    = U' - W S0
 //   S_C  = gamma_C S0 + K^T diag(gamma_C / gamma) U
 //   O    = diag(gamma) Q S0 + (tril(Q K^T) * exp(G_i - G_j)) U
-// Every contraction is a tcgen05.mma with M = 128 (the key or value
-// dimension, or the 64 chunk rows of K stacked on 64 rows of Q/V), operands in
-// 128-byte-swizzled shared memory (TMA-loaded tiles or tiles the epilogues
-// write), accumulators in TMEM.  T is built on CUDA cores in fp32.
+// Every chunk contraction is a tcgen05.mma with M = 128 (the key or value
+// dimension, or the 64 chunk rows of K stacked on 64 rows of Q/V) and
+// accumulators in TMEM.  The state lives in TMEM transposed (lane = value
+// row) as S / sigma with a running scalar sigma, so the state-dependent
+// product U' - W S reads it straight from TMEM as a tf32 operand and the
+// decay costs no pass over the state (sigma is folded back only when it gets
+// small).  T is built from 16 x 16 diagonal inverses on CUDA cores and
+// warp-level tf32 tensor-core products for the blocks below the diagonal.
 //
-// Work: one CTA per (sequence, head) unit, 4 warps, chunks in order.  Thread
-// t owns TMEM lane t in every epilogue.  Replay: 96 KB shared memory and 256
-// TMEM columns, so two CTAs share an SM and overlap each other's serial
-// chain.  Prefill adds the output path (152 KB, 512 columns).
+// Work: one CTA per (sequence, head) unit, 4 warps, chunks in order; the
+// next chunk's tiles stream in by TMA while the current chunk is computed.
+// Thread t owns TMEM lane t in every epilogue.  Replay: 96 KB of shared
+// memory and 256 TMEM columns, so two CTAs share an SM and overlap each
+// other's serial chain.  Prefill adds the output path (184 KB, 512 columns).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
-#include "gdn_internal.h"
-#include "gdn_sm100.h"
+#include "gdn_chunk_common.h"
 
 namespace gdn {
 namespace {
 
 using namespace sm100;
+using namespace chunk;
 
-constexpr int C = 64;        // chunk length
-constexpr int D = 128;       // d_k = d_v
 constexpr int NT = 128;      // threads per CTA
-constexpr uint64_t kWaitNs = 1000000000ull;   // 1 s per wait
-constexpr float kLog2Floor = -115.0f;         // log2 of a zero gate, clamped (2^-115 ~ 2.4e-35)
 
 // ---- shared memory map (byte offsets from a 1 KB aligned base) ----
-// TILE: [K0 | X0 | K1 | X1], 8 KB boxes of 64 rows x 64 columns.  X = V
-//       (replay) or Q (prefill).  Block kb holds columns [64 kb, 64 kb + 64).
-// VT  : prefill only, [V0 | V1].
-// SB  : bf16 S as an MN-major operand (two 16 KB dv-blocks of 128 k-rows);
-//       during the chunk prep it holds A (fp32 64 x 64) and scratch.
-// UT  : bf16 diag(gamma_C / gamma) U, [dv][j]; during prep T diag(beta) and
-//       T diag(beta gamma) in bf16.
-// WT  : bf16 -W^T, [dk][j]; during prep T in fp32.
-// UB  : prefill, bf16 U^T unscaled, [dv][j].
-// MB  : prefill, bf16 masked decayed Q K^T, [i][j].
-// GQ  : prefill, bf16 diag(gamma) Q, [i][dk] as two 8 KB blocks.
-constexpr uint32_t OFF_TILE = 0;
-constexpr uint32_t OFF_SB = 32768;
-constexpr uint32_t OFF_UT = OFF_SB + 32768;
-constexpr uint32_t OFF_WT = OFF_UT + 16384;
-constexpr uint32_t SMEM_REPLAY = OFF_WT + 16384;        // 96 KB
-constexpr uint32_t OFF_VT = SMEM_REPLAY;
-constexpr uint32_t OFF_UB = OFF_VT + 16384;
-constexpr uint32_t OFF_MB = OFF_UB + 16384;
-constexpr uint32_t OFF_GQ = OFF_MB + 8192;
-constexpr uint32_t SMEM_PREFILL = OFF_GQ + 16384;       // 152 KB
-// fp32 scratch inside SB during the prep
-constexpr uint32_t OFF_A = OFF_SB;                      // 64 x 64 fp32
-constexpr uint32_t OFF_P = OFF_SB + 16384;              // up to 3 x 256 fp32
-constexpr uint32_t OFF_T = OFF_WT;                      // 64 x 64 fp32
-constexpr uint32_t OFF_TB = OFF_UT;                     // bf16 T diag(beta)
-constexpr uint32_t OFF_TBG = OFF_UT + 8192;             // bf16 T diag(beta gamma)
+// Two tile slots (chunk c in slot c % 2, the next chunk prefetched by TMA):
+//   replay : [K0 | V0 | K1 | V1]            (32 KB)
+//   prefill: [K0 | Q0 | K1 | Q1 | V0 | V1]  (48 KB)
+// 8 KB boxes of 64 rows x 64 columns; block kb holds columns [64 kb, 64 kb + 64).
+// PREP (32 KB) is reused within a chunk, in this order:
+//   A -> T in place (fp32 64 x LDT) and the product scratch,
+//   T diag(beta), T diag(beta gamma) (bf16 [j][j'], 8 KB each),
+//   BU = -sigma W (fp32, K-major [j][dk], four 8 KB key blocks),
+//   UT = diag(gamma_C / gamma) U / sigma (bf16 [dv][j], 16 KB).
+// Prefill adds UB (bf16 U^T [dv][j]), MB (bf16 masked decayed Q K^T [i][j])
+// and BQ (fp32 sigma diag(gamma) Q, K-major [i][dk], four 8 KB blocks).
+template <bool REPLAY>
+struct Layout {
+    static constexpr uint32_t TILE = REPLAY ? 32768u : 49152u;
+    static constexpr uint32_t OFF_TILE = 0;
+    static constexpr uint32_t OFF_PREP = 2 * TILE;
+    static constexpr uint32_t OFF_AT = OFF_PREP;
+    static constexpr uint32_t OFF_X = OFF_PREP + 17408;
+    static constexpr uint32_t OFF_TB = OFF_PREP;
+    static constexpr uint32_t OFF_TBG = OFF_PREP + 8192;
+    static constexpr uint32_t OFF_BU = OFF_PREP;
+    static constexpr uint32_t OFF_UT = OFF_PREP;
+    static constexpr uint32_t OFF_UB = OFF_PREP + 32768;
+    static constexpr uint32_t OFF_MB = OFF_UB + 16384;
+    static constexpr uint32_t OFF_BQ = OFF_MB + 8192;
+    static constexpr uint32_t BYTES = REPLAY ? OFF_PREP + 32768 : OFF_BQ + 32768;
+    // offsets inside a tile slot
+    static constexpr uint32_t K0 = 0, K1 = 16384;
+    static constexpr uint32_t X0 = 8192;                  // V (replay) or Q (prefill) block 0
+    static constexpr uint32_t V0 = REPLAY ? 8192u : 32768u;
+    static constexpr uint32_t V_LBO = REPLAY ? 16384u : 8192u;
+};
+static_assert(Layout<true>::OFF_X + 3 * 16 * 24 * 4 <= Layout<true>::OFF_PREP + 32768, "prep scratch fits");
 
 // TMEM columns
-constexpr uint32_t TM_S = 0;      // 128 columns: fp32 S, lane = key row
+constexpr uint32_t TM_S = 0;      // 128 columns: fp32 S^T / sigma, lane = value row, column = key
 constexpr uint32_t TM_U = 128;    // 64 columns: U'^T then U^T, lane = value row
-constexpr uint32_t TM_P = 192;    // 64 columns: [K;X] K^T, then W^T
-constexpr uint32_t TM_O = 256;    // 64 columns (prefill): O^T
+constexpr uint32_t TM_P = 192;    // 64 columns: K K^T ([K;Q] K^T for prefill), then W^T (lane = key)
+constexpr uint32_t TM_O = 256;    // 64 columns (prefill): O^T, lane = value row
 
 struct TcParams {
     CallArgs a;
-    long long rows_total;
 };
-
-__device__ __forceinline__ void st_shared_v4(uint8_t* base, uint32_t off, uint4 v) {
-    *reinterpret_cast<uint4*>(base + off) = v;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-    __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&p);
-}
-
-// Write 64 fp32 values (one row, columns 0..63) as bf16 into a 128-byte
-// swizzled row `row` of the tile at `tile`.
-__device__ __forceinline__ void write_row64_bf16(uint8_t* tile, int row, const float* v) {
-#pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
-        uint4 q;
-        q.x = pack_bf16(v[ch * 8 + 0], v[ch * 8 + 1]);
-        q.y = pack_bf16(v[ch * 8 + 2], v[ch * 8 + 3]);
-        q.z = pack_bf16(v[ch * 8 + 4], v[ch * 8 + 5]);
-        q.w = pack_bf16(v[ch * 8 + 6], v[ch * 8 + 7]);
-        st_shared_v4(tile, (uint32_t)(row * 128 + ((ch ^ (row & 7)) << 4)), q);
-    }
-}
-
-__device__ __forceinline__ float bf16_at(const uint8_t* tile, int row, int col) {
-    const __nv_bfloat16 x = *reinterpret_cast<const __nv_bfloat16*>(tile + sw128_offset(row, col));
-    return __bfloat162float(x);
-}
 
 // Block-wide agreement after a bounded wait: every thread leaves together.
 __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, const CallArgs& a, uint32_t where) {
     bool ok = mbar_wait_bounded(bar, parity, kWaitNs);
     ok = __syncthreads_and(ok) != 0;
-    if (!ok && threadIdx.x == 0) {
-        atomicOr(&a.ws->status, kStatusTimeout);
-        atomicCAS(&a.ws->timeout_where, 0u, where);
-    }
+    if (!ok && threadIdx.x == 0) report_timeout(a, where);
     return ok;
 }
 
-// T = (I + A)^-1 for the strictly lower triangular 64 x 64 A (fp32, row
-// stride 64), by 16 x 16 diagonal blocks (forward substitution) and the
-// block recurrence T_ba = -T_bb sum_{a <= m < b} A_bm T_ma.  Writes T (fp32,
-// lower triangle, zeros above) to Ts.
-__device__ void invert_unit_lower(const float* As, float* Ts, float* Ps) {
-    const int tid = threadIdx.x;
-    // zero T
-    for (int e = tid; e < C * C; e += NT) Ts[e] = 0.0f;
-    __syncthreads();
-    if (tid < 64) {
-        const int bb = tid >> 4, cc = tid & 15, o = bb * 16;
-        float x[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float acc = (i == cc) ? 1.0f : 0.0f;
-#pragma unroll
-            for (int j = 0; j < i; ++j) acc = fmaf(-As[(o + i) * C + o + j], x[j], acc);
-            x[i] = (i < cc) ? 0.0f : acc;
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) Ts[(o + i) * C + o + cc] = x[i];
-    }
-    __syncthreads();
-    for (int b = 1; b < 4; ++b) {
-        // P_ba = sum_{m=a}^{b-1} A_bm T_ma for a < b: b * 256 elements
-        for (int e = tid; e < b * 256; e += NT) {
-            const int a = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-            float acc = 0.0f;
-            for (int m = a; m < b; ++m) {
-#pragma unroll
-                for (int l = 0; l < 16; ++l)
-                    acc = fmaf(As[(16 * b + r) * C + 16 * m + l], Ts[(16 * m + l) * C + 16 * a + cc], acc);
-            }
-            Ps[e] = acc;
-        }
-        __syncthreads();
-        for (int e = tid; e < b * 256; e += NT) {
-            const int a = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-            float acc = 0.0f;
-#pragma unroll
-            for (int l = 0; l < 16; ++l)
-                acc = fmaf(Ts[(16 * b + r) * C + 16 * b + l], Ps[(a << 8) + (l << 4) + cc], acc);
-            Ts[(16 * b + r) * C + 16 * a + cc] = -acc;
-        }
-        __syncthreads();
+template <bool REPLAY>
+__device__ __forceinline__ void issue_tiles(uint8_t* tile, uint64_t* bar, const CUtensorMap* mk, const CUtensorMap* mv,
+                                            const CUtensorMap* mq, int h, int r0) {
+    using L = Layout<REPLAY>;
+    mbar_arrive_expect_tx(bar, L::TILE);
+    tma_load_3d(tile + L::K0, mk, bar, 0, h, r0);
+    tma_load_3d(tile + L::K1, mk, bar, 64, h, r0);
+    tma_load_3d(tile + L::V0, mv, bar, 0, h, r0);
+    tma_load_3d(tile + L::V0 + L::V_LBO, mv, bar, 64, h, r0);
+    if (!REPLAY) {
+        tma_load_3d(tile + L::X0, mq, bar, 0, h, r0);
+        tma_load_3d(tile + L::X0 + 16384, mq, bar, 64, h, r0);
     }
 }
 
@@ -173,11 +115,16 @@ template <bool REPLAY>
 __global__ void __launch_bounds__(NT, 1)
 chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_q) {
+    using L = Layout<REPLAY>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t bar_tma, bar_mma;
+    __shared__ uint64_t bar_tile[2], bar_mma;
     __shared__ uint32_t tmem_slot;
-    __shared__ float s_beta[C], s_g2[C], s_gam[C];
+    __shared__ alignas(16) float s_beta[C];
+    __shared__ alignas(16) float s_g2[C];
+    __shared__ alignas(16) float s_gam[C];
+    __shared__ alignas(16) float s_binv[C];
+    __shared__ alignas(16) float s_e[C];
     __shared__ float s_scan;
 
     const CallArgs& a = p.a;
@@ -191,9 +138,11 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         return;
     }
     const Window w = a.windows[b];
+    const int nchunks = (w.len + C - 1) / C;
 
     if (tid == 0) {
-        mbar_init(&bar_tma, 1);
+        mbar_init(&bar_tile[0], 1);
+        mbar_init(&bar_tile[1], 1);
         mbar_init(&bar_mma, 1);
         mbar_fence_init();
         tma_prefetch_desc(&map_k);
@@ -209,28 +158,24 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     tc_fence_after();
     const uint32_t tbase = tmem_slot;
     const uint32_t tlane = tbase + ((uint32_t)(warp * 32) << 16);   // this thread's lane, column 0
+    if (tid == 0 && nchunks > 0)
+        issue_tiles<REPLAY>(sm + L::OFF_TILE, &bar_tile[0], &map_k, &map_v, &map_q, h, (int)w.row0);
 
-    uint8_t* tile = sm + OFF_TILE;
-    uint8_t* vtile = REPLAY ? sm + OFF_TILE + 8192 : sm + OFF_VT;
-    const uint32_t v_lbo = REPLAY ? 16384u : 8192u;
-    const uint32_t s_tile = smem_u32(tile), s_vtile = smem_u32(vtile);
-    const uint32_t s_sb = smem_u32(sm + OFF_SB), s_ut = smem_u32(sm + OFF_UT), s_wt = smem_u32(sm + OFF_WT);
-    const uint32_t s_tb = smem_u32(sm + OFF_TB), s_tbg = smem_u32(sm + OFF_TBG);
-    const uint32_t s_ub = smem_u32(sm + OFF_UB), s_mb = smem_u32(sm + OFF_MB), s_gq = smem_u32(sm + OFF_GQ);
+    float* AT = reinterpret_cast<float*>(sm + L::OFF_AT);
+    float* Xs = reinterpret_cast<float*>(sm + L::OFF_X);
+    const uint32_t s_bu = smem_u32(sm + L::OFF_BU), s_ut = smem_u32(sm + L::OFF_UT);
+    const uint32_t s_tb = smem_u32(sm + L::OFF_TB), s_tbg = smem_u32(sm + L::OFF_TBG);
+    const uint32_t s_ub = smem_u32(sm + L::OFF_UB), s_mb = smem_u32(sm + L::OFF_MB), s_bq = smem_u32(sm + L::OFF_BQ);
 
-    // ---- initial state into TMEM (thread t = key row t) ----
+    // ---- initial state: TMEM lane dv = tid holds column dv of S (a row of S^T) ----
     const size_t state_base = ((size_t)b * H + h) * D * D;
     {
         float v[32];
 #pragma unroll
         for (int cb = 0; cb < 4; ++cb) {
             if (!REPLAY && a.state_in) {
-                const float4* src = reinterpret_cast<const float4*>(a.state_in + state_base + (size_t)tid * D + cb * 32);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    float4 x = src[i];
-                    v[4 * i] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z; v[4 * i + 3] = x.w;
-                }
+                for (int i = 0; i < 32; ++i) v[i] = a.state_in[state_base + (size_t)(cb * 32 + i) * D + tid];
             } else {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = 0.0f;
@@ -239,43 +184,44 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         }
         tmem_wait_st();
     }
+    float sigma = 1.0f;   // S = sigma * (TMEM state)
 
-    const uint32_t id_kk = idesc_bf16(128, 64, false, false);    // [K;X] K^T
+    const uint32_t id_kk = REPLAY ? idesc_bf16(64, 64, false, false)    // K K^T; row r in lane 32 (r/16) + r%16
+                                  : idesc_bf16(128, 64, false, false);  // [K;Q] K^T
     const uint32_t id_w = idesc_bf16(128, 64, true, false);      // K^T (T..)^T, V^T (T..)^T
-    const uint32_t id_u = idesc_bf16(128, 64, true, true);       // S^T (-W^T)
-    const uint32_t id_o1 = idesc_bf16(128, 64, true, false);     // S^T (gamma Q)^T
-    const uint32_t id_s = idesc_bf16(128, 128, true, false);     // K^T U~
+    const uint32_t id_u = idesc_tf32(128, 64, false, false);     // S^T (-sigma W^T), A in TMEM
+    const uint32_t id_s = idesc_bf16(128, 128, false, true);     // U~^T K
     const uint32_t id_o2 = idesc_bf16(128, 64, false, false);    // U^T M^T
 
-    uint32_t ph_tma = 0, ph_mma = 0;
+    uint32_t ph_mma = 0;
     bool ok = true;
-    const int nchunks = (w.len + C - 1) / C;
-    const uint32_t tile_bytes = REPLAY ? 4u * 8192u : 6u * 8192u;
+    // gates of the next chunk are fetched one chunk ahead (thread tid < 64 holds token tid)
+    float al_nxt = 1.0f, be_nxt = 0.0f;
+    if (tid < C && tid < w.len) {
+        al_nxt = a.alpha[(w.row0 + tid) * H + h];
+        be_nxt = a.beta[(w.row0 + tid) * H + h];
+    }
+    // prefill: outputs of the previous chunk are written once its products are known complete
+    long long o_r0 = 0;
+    int o_nc = 0;
 
     for (int c = 0; c < nchunks && ok; ++c) {
+        const int slot = c & 1;
         const long long r0 = w.row0 + (long long)c * C;
         const int nc = min(C, w.len - c * C);
+        uint8_t* tile = sm + L::OFF_TILE + slot * L::TILE;
+        const uint32_t s_tile = smem_u32(tile);
 
-        // ---- load the chunk's tiles (TMA) and gates ----
-        if (tid == 0) {
-            mbar_arrive_expect_tx(&bar_tma, tile_bytes);
-            tma_load_3d(tile, &map_k, &bar_tma, 0, h, (int)r0);
-            tma_load_3d(tile + 16384, &map_k, &bar_tma, 64, h, (int)r0);
-            tma_load_3d(vtile, &map_v, &bar_tma, 0, h, (int)r0);
-            tma_load_3d(vtile + v_lbo, &map_v, &bar_tma, 64, h, (int)r0);
-            if (!REPLAY) {
-                tma_load_3d(tile + 8192, &map_q, &bar_tma, 0, h, (int)r0);
-                tma_load_3d(tile + 24576, &map_q, &bar_tma, 64, h, (int)r0);
-            }
-        }
+        // ---- gates: cumulative log2 decay and the per-chunk factors ----
         if (tid < C) {
-            float al = 1.0f, be = 0.0f;
-            if (tid < nc) {
-                al = a.alpha[(r0 + tid) * H + h];
-                be = a.beta[(r0 + tid) * H + h];
+            const float al = al_nxt, be = be_nxt;
+            al_nxt = 1.0f;
+            be_nxt = 0.0f;
+            if ((c + 1) * C + tid < w.len) {
+                al_nxt = a.alpha[(r0 + C + tid) * H + h];
+                be_nxt = a.beta[(r0 + C + tid) * H + h];
             }
             float lg = al > 0.0f ? fmaxf(__log2f(al), kLog2Floor) : kLog2Floor;
-            // inclusive scan over the 64 tokens (two warps)
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 float y = __shfl_up_sync(0xffffffffu, lg, off);
@@ -283,28 +229,33 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             }
             if (tid == 31) s_scan = lg;
             s_beta[tid] = be;
-            s_g2[tid] = lg;   // warp 1 adds warp 0's total below
+            s_g2[tid] = lg;
         }
         __syncthreads();
         if (tid >= 32 && tid < C) s_g2[tid] += s_scan;
         __syncthreads();
-        if (tid < C) s_gam[tid] = exp2f(s_g2[tid]);
-        ok = wait_all(&bar_tma, ph_tma, a, 1);
-        ph_tma ^= 1;
+        const float g2C = s_g2[C - 1];
+        const bool fast = g2C >= kFastGateFloor;   // every partial product of gates is >= 2^-100
+        if (tid < C) {
+            const float gj = s_g2[tid];
+            s_gam[tid] = exp2f(gj);
+            s_binv[tid] = fast ? exp2f(-gj) : 0.0f;
+            s_e[tid] = exp2f(g2C - gj);
+        }
+        ok = wait_all(&bar_tile[slot], (c >> 1) & 1, a, 1);
         if (!ok) break;
         if (nc < C) {   // padded tokens are identity transitions: zero their rows
             const int nrows = C - nc;
-            const int ntiles = REPLAY ? 4 : 6;
-            for (int e = tid; e < ntiles * nrows * 8; e += NT) {
+            const int nbox = REPLAY ? 4 : 6;
+            for (int e = tid; e < nbox * nrows * 8; e += NT) {
                 const int t = e / (nrows * 8), rr = nc + (e / 8) % nrows, ch = e % 8;
-                uint8_t* base = (t < 4) ? tile + t * 8192 : vtile + (t - 4) * 8192;
-                st_shared_v4(base, (uint32_t)(rr * 128 + ch * 16), make_uint4(0, 0, 0, 0));
+                st_shared_v4(tile + t * 8192, (uint32_t)(rr * 128 + ch * 16), make_uint4(0, 0, 0, 0));
             }
             fence_proxy_async_smem();
         }
         __syncthreads();
 
-        // ---- MMA 1: [K; X] K^T -> TM_P (rows 0..63: K K^T, rows 64..127: Q K^T) ----
+        // ---- MMA 1: K K^T (replay, M = 64) or [K; Q] K^T (prefill) -> TM_P ----
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
@@ -315,69 +266,74 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             }
             mma_commit(&bar_mma);
         }
-        ok = wait_all(&bar_mma, ph_mma, a, 2);
+        ok = wait_all(&bar_mma, ph_mma, a, 2);   // also: every product of the previous chunk is done
         ph_mma ^= 1;
         if (!ok) break;
         tc_fence_after();
+        // the other tile slot is free: prefetch the next chunk
+        if (tid == 0 && c + 1 < nchunks)
+            issue_tiles<REPLAY>(sm + L::OFF_TILE + (slot ^ 1) * L::TILE, &bar_tile[slot ^ 1], &map_k, &map_v,
+                                &map_q, h, (int)(r0 + C));
 
-        // ---- epilogue 1: A (rows 0..63) and M (rows 64..127, prefill) ----
-        {
-            float* As = reinterpret_cast<float*>(sm + OFF_A);
-            const bool krow = tid < C;
-            if (krow || !REPLAY) {
-                const int i = krow ? tid : tid - C;
-                const float gi = s_g2[i];
-                const float bi = s_beta[i];
-                float v[64];
-                tmem_ld32(tlane + TM_P, v);
-                tmem_ld32(tlane + TM_P + 32, v + 32);
-                tmem_wait_ld();
-                if (krow) {
+        if (!REPLAY && c > 0) {
+            // ---- outputs of chunk c - 1: o[r0 + i, h, tid] ----
+            float v[64];
+            tmem_ld32(tlane + TM_O, v);
+            tmem_ld32(tlane + TM_O + 32, v + 32);
+            tmem_wait_ld();
+            __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o_out);
 #pragma unroll
-                    for (int j = 0; j < C; ++j)
-                        As[i * C + j] = (j < i) ? bi * exp2f(gi - s_g2[j]) * v[j] : 0.0f;
+            for (int i = 0; i < C; ++i)
+                if (i < o_nc) o[((o_r0 + i) * H + h) * (long long)D + tid] = __float2bfloat16_rn(v[i]);
+        }
+
+        // ---- epilogue 1: A = strict_tril(beta_i (gamma_i / gamma_j) K K^T) (fp32, in AT);
+        //      prefill: M = tril((gamma_i / gamma_j) Q K^T) (bf16, MB) ----
+        {
+            float v[64];
+            tmem_ld32(tlane + TM_P, v);
+            tmem_ld32(tlane + TM_P + 32, v + 32);
+            tmem_wait_ld();
+            const bool active = REPLAY ? (lane < 16) : true;
+            const bool krow = REPLAY ? true : (tid < C);
+            const int i = REPLAY ? warp * 16 + lane : (krow ? tid : tid - C);
+            if (active) {
+                const float gi = s_g2[i];
+                const float bi = krow ? s_beta[i] : 1.0f;
+                if (fast) {
+                    const float rowf = bi * s_gam[i];
+                    const float4* binv = reinterpret_cast<const float4*>(s_binv);
+#pragma unroll
+                    for (int q = 0; q < C / 4; ++q) {
+                        const float4 bv = binv[q];
+                        v[4 * q] *= rowf * bv.x;
+                        v[4 * q + 1] *= rowf * bv.y;
+                        v[4 * q + 2] *= rowf * bv.z;
+                        v[4 * q + 3] *= rowf * bv.w;
+                    }
                 } else {
 #pragma unroll
-                    for (int j = 0; j < C; ++j) v[j] = (j <= i) ? exp2f(gi - s_g2[j]) * v[j] : 0.0f;
-                    write_row64_bf16(sm + OFF_MB, i, v);
+                    for (int j = 0; j < C; ++j) v[j] *= bi * exp2f(gi - s_g2[j]);
+                }
+                if (krow) {
+#pragma unroll
+                    for (int j = 0; j < C; ++j) v[j] = (j < i) ? v[j] : 0.0f;
+#pragma unroll
+                    for (int j = 0; j < C; j += 4)
+                        *reinterpret_cast<float4*>(AT + i * LDT + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < C; ++j) v[j] = (j <= i) ? v[j] : 0.0f;
+                    write_row64_bf16(sm + L::OFF_MB, i, v);
                 }
             }
         }
         tc_fence_before();
         __syncthreads();
 
-        // ---- T = (I + A)^-1 and its two scaled bf16 copies ----
-        {
-            const float* As = reinterpret_cast<const float*>(sm + OFF_A);
-            float* Ts = reinterpret_cast<float*>(sm + OFF_T);
-            float* Ps = reinterpret_cast<float*>(sm + OFF_P);
-            invert_unit_lower(As, Ts, Ps);
-            const int j = tid >> 1, half = tid & 1;
-            float vb[32], vbg[32];
-#pragma unroll
-            for (int q = 0; q < 32; ++q) {
-                const int jp = half * 32 + q;
-                const float t = Ts[j * C + jp] * s_beta[jp];
-                vb[q] = t;
-                vbg[q] = t * s_gam[jp];
-            }
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                const int chunk = half * 4 + ch;
-                uint4 x, y;
-                x.x = pack_bf16(vb[ch * 8 + 0], vb[ch * 8 + 1]);
-                x.y = pack_bf16(vb[ch * 8 + 2], vb[ch * 8 + 3]);
-                x.z = pack_bf16(vb[ch * 8 + 4], vb[ch * 8 + 5]);
-                x.w = pack_bf16(vb[ch * 8 + 6], vb[ch * 8 + 7]);
-                y.x = pack_bf16(vbg[ch * 8 + 0], vbg[ch * 8 + 1]);
-                y.y = pack_bf16(vbg[ch * 8 + 2], vbg[ch * 8 + 3]);
-                y.z = pack_bf16(vbg[ch * 8 + 4], vbg[ch * 8 + 5]);
-                y.w = pack_bf16(vbg[ch * 8 + 6], vbg[ch * 8 + 7]);
-                const uint32_t off = (uint32_t)(j * 128 + ((chunk ^ (j & 7)) << 4));
-                st_shared_v4(sm + OFF_TB, off, x);
-                st_shared_v4(sm + OFF_TBG, off, y);
-            }
-        }
+        // ---- T = (I + A)^-1 in place, then T diag(beta) and T diag(beta gamma) in bf16 ----
+        invert_unit_lower_inplace(AT, Xs, tid, 0);
+        write_scaled_t(AT, s_beta, s_gam, sm + L::OFF_TB, sm + L::OFF_TBG, tid, 0);
         fence_proxy_async_smem();
         __syncthreads();
 
@@ -385,15 +341,13 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                mma_bf16_ss(tbase + TM_P, smem_desc_sw128(s_tile + kk * 2048, 16384, 1024),
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ss(tbase + TM_P, smem_desc_sw128(s_tile + L::K0 + kk * 2048, 16384, 1024),
                             smem_desc_sw128(s_tbg + kk * 32, 16, 1024), id_w, kk > 0);
-            }
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                mma_bf16_ss(tbase + TM_U, smem_desc_sw128(s_vtile + kk * 2048, v_lbo, 1024),
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ss(tbase + TM_U, smem_desc_sw128(s_tile + L::V0 + kk * 2048, L::V_LBO, 1024),
                             smem_desc_sw128(s_tb + kk * 32, 16, 1024), id_w, kk > 0);
-            }
             mma_commit(&bar_mma);
         }
         ok = wait_all(&bar_mma, ph_mma, a, 3);
@@ -401,70 +355,57 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         if (!ok) break;
         tc_fence_after();
 
-        // ---- epilogue 2: -W^T (bf16, row = key index) and diag(gamma) Q ----
+        // ---- epilogue 2: BU[j][dk] = -sigma W[j][dk] (fp32, K-major);
+        //      prefill: BQ[i][dk] = sigma gamma_i Q[i][dk] ----
         {
             float v[64];
             tmem_ld32(tlane + TM_P, v);
             tmem_ld32(tlane + TM_P + 32, v + 32);
             tmem_wait_ld();
+            uint8_t* bu = sm + L::OFF_BU + (tid >> 5) * 8192;   // key block of this thread
+            const int kc = tid & 31;
+            const float ns = -sigma;
 #pragma unroll
-            for (int j = 0; j < C; ++j) v[j] = -v[j];
-            write_row64_bf16(sm + OFF_WT, tid, v);
+            for (int j = 0; j < C; ++j) *reinterpret_cast<float*>(bu + sw128_offset_f32(j, kc)) = ns * v[j];
             if (!REPLAY) {
-                const int i = tid >> 1, half = tid & 1;   // row i, key block `half`
-                const uint8_t* qb = tile + half * 16384 + 8192;
-                const float gi = s_gam[i];
+                const int i = tid >> 1, half = tid & 1;   // row i, keys [64 half, 64 half + 64)
+                const uint8_t* qb = tile + L::X0 + half * 16384;
+                const float sg = sigma * s_gam[i];
 #pragma unroll
-                for (int col = 0; col < 64; ++col) v[col] = gi * bf16_at(qb, i, col);
-                write_row64_bf16(sm + OFF_GQ + half * 8192, i, v);
-            }
-        }
-        // ---- S epilogue: bf16 S_{c-1} for the operands, then S <- gamma_C S in TMEM ----
-        {
-            const float gC = s_gam[C - 1];
-            uint8_t* sb = sm + OFF_SB;
+                for (int ch = 0; ch < 8; ++ch) {       // 8 bf16 per 16-byte chunk of the Q row
+                    const uint4 raw = *reinterpret_cast<const uint4*>(qb + i * 128 + ((ch ^ (i & 7)) << 4));
+                    const uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
+                    float f[8];
 #pragma unroll
-            for (int cb = 0; cb < 4; ++cb) {
-                float v[32];
-                tmem_ld32(tlane + TM_S + cb * 32, v);
-                tmem_wait_ld();
-                // columns [32 cb, 32 cb + 32) of key row tid -> dv block (cb / 2)
-                uint8_t* blk = sb + (cb >> 1) * 16384;
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    const int chunk = (cb & 1) * 4 + ch;
-                    uint4 x;
-                    x.x = pack_bf16(v[ch * 8 + 0], v[ch * 8 + 1]);
-                    x.y = pack_bf16(v[ch * 8 + 2], v[ch * 8 + 3]);
-                    x.z = pack_bf16(v[ch * 8 + 4], v[ch * 8 + 5]);
-                    x.w = pack_bf16(v[ch * 8 + 6], v[ch * 8 + 7]);
-                    st_shared_v4(blk, (uint32_t)(tid * 128 + ((chunk ^ (tid & 7)) << 4)), x);
+                    for (int e = 0; e < 4; ++e) {
+                        f[2 * e] = sg * __uint_as_float(wds[e] << 16);
+                        f[2 * e + 1] = sg * __uint_as_float(wds[e] & 0xffff0000u);
+                    }
+                    const int col = half * 64 + ch * 8;                // key index of f[0]
+                    uint8_t* blk = sm + L::OFF_BQ + (col >> 5) * 8192;
+                    const int cc = col & 31;
+                    *reinterpret_cast<float4*>(blk + sw128_offset_f32(i, cc)) = make_float4(f[0], f[1], f[2], f[3]);
+                    *reinterpret_cast<float4*>(blk + sw128_offset_f32(i, cc + 4)) = make_float4(f[4], f[5], f[6], f[7]);
                 }
-#pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] *= gC;
-                tmem_st32(tlane + TM_S + cb * 32, v);
             }
-            tmem_wait_st();
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
 
-        // ---- MMA U: U^T += S^T (-W^T);  prefill: O^T = S^T (gamma Q)^T ----
+        // ---- MMA U: U^T += (S^T / sigma)(-sigma W^T), A from TMEM (tf32);
+        //      prefill: O^T = (S^T / sigma)(sigma gamma Q)^T ----
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                mma_bf16_ss(tbase + TM_U, smem_desc_sw128(s_sb + kk * 2048, 16384, 1024),
-                            smem_desc_sw128(s_wt + kk * 2048, 16384, 1024), id_u, 1u);
-            }
+            for (int kk = 0; kk < 16; ++kk)
+                mma_tf32_ts(tbase + TM_U, tbase + TM_S + kk * 8,
+                            smem_desc_sw128(s_bu + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_u, 1u);
             if (!REPLAY) {
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    mma_bf16_ss(tbase + TM_O, smem_desc_sw128(s_sb + kk * 2048, 16384, 1024),
-                                smem_desc_sw128(s_gq + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_o1,
-                                kk > 0);
-                }
+                for (int kk = 0; kk < 16; ++kk)
+                    mma_tf32_ts(tbase + TM_O, tbase + TM_S + kk * 8,
+                                smem_desc_sw128(s_bq + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_u, kk > 0);
             }
             mma_commit(&bar_mma);
         }
@@ -473,70 +414,88 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         if (!ok) break;
         tc_fence_after();
 
-        // ---- epilogue U: diag(gamma_C / gamma) U (and U itself for the outputs) ----
+        // ---- epilogue U: U~ = diag(gamma_C / gamma) U / sigma_new (and U for the outputs) ----
         {
             float v[64];
             tmem_ld32(tlane + TM_U, v);
             tmem_ld32(tlane + TM_U + 32, v + 32);
             tmem_wait_ld();
-            if (!REPLAY) write_row64_bf16(sm + OFF_UB, tid, v);
-            const float g2C = s_g2[C - 1];
+            if (!REPLAY) write_row64_bf16(sm + L::OFF_UB, tid, v);
+            float snew = sigma * s_gam[C - 1];
+            if (snew < kRenormBelow) {     // uniform: fold the scale into the TMEM state
 #pragma unroll
-            for (int j = 0; j < C; ++j) v[j] *= exp2f(g2C - s_g2[j]);
-            write_row64_bf16(sm + OFF_UT, tid, v);
+                for (int cb = 0; cb < 4; ++cb) {
+                    float sv[32];
+                    tmem_ld32(tlane + TM_S + cb * 32, sv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) sv[q] *= snew;
+                    tmem_st32(tlane + TM_S + cb * 32, sv);
+                }
+                tmem_wait_st();
+                snew = 1.0f;
+            }
+            sigma = snew;
+            const float inv = 1.0f / snew;
+            const float4* ev = reinterpret_cast<const float4*>(s_e);
+#pragma unroll
+            for (int q = 0; q < C / 4; ++q) {
+                const float4 e4 = ev[q];
+                v[4 * q] *= e4.x * inv;
+                v[4 * q + 1] *= e4.y * inv;
+                v[4 * q + 2] *= e4.z * inv;
+                v[4 * q + 3] *= e4.w * inv;
+            }
+            write_row64_bf16(sm + L::OFF_UT, tid, v);
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
 
-        // ---- MMA S: S += K^T U~ ;  prefill: O^T += U^T M^T ----
+        // ---- MMA S: S^T / sigma += U~^T K ;  prefill: O^T += U^T M^T.
+        //      Not waited for here: the next chunk's first commit covers it. ----
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                mma_bf16_ss(tbase + TM_S, smem_desc_sw128(s_tile + kk * 2048, 16384, 1024),
-                            smem_desc_sw128(s_ut + kk * 32, 16, 1024), id_s, 1u);
-            }
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ss(tbase + TM_S, smem_desc_sw128(s_ut + kk * 32, 16, 1024),
+                            smem_desc_sw128(s_tile + L::K0 + kk * 2048, 16384, 1024), id_s, 1u);
             if (!REPLAY) {
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
+                for (int kk = 0; kk < 4; ++kk)
                     mma_bf16_ss(tbase + TM_O, smem_desc_sw128(s_ub + kk * 32, 16, 1024),
                                 smem_desc_sw128(s_mb + kk * 32, 16, 1024), id_o2, 1u);
-                }
             }
-            mma_commit(&bar_mma);
         }
-        ok = wait_all(&bar_mma, ph_mma, a, 5);
-        ph_mma ^= 1;
-        if (!ok) break;
-        tc_fence_after();
-
-        // ---- epilogue O: o[r0 + i, h, tid] for the chunk's real rows ----
-        if (!REPLAY) {
-            float v[64];
-            tmem_ld32(tlane + TM_O, v);
-            tmem_ld32(tlane + TM_O + 32, v + 32);
-            tmem_wait_ld();
-            __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o_out);
-#pragma unroll
-            for (int i = 0; i < C; ++i)
-                if (i < nc) o[((r0 + i) * H + h) * (long long)D + tid] = __float2bfloat16_rn(v[i]);
-        }
-        tc_fence_before();
-        __syncthreads();
+        o_r0 = r0;
+        o_nc = nc;
     }
 
-    // ---- final state (thread t = key row t) ----
-    if (ok && a.state_out) {
+    // ---- drain: wait for the last products ----
+    if (ok) {
+        if (tid == 0) mma_commit(&bar_mma);
+        ok = wait_all(&bar_mma, ph_mma, a, 5);
         tc_fence_after();
+    }
+    if (ok && !REPLAY && nchunks > 0) {
+        float v[64];
+        tmem_ld32(tlane + TM_O, v);
+        tmem_ld32(tlane + TM_O + 32, v + 32);
+        tmem_wait_ld();
+        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o_out);
+#pragma unroll
+        for (int i = 0; i < C; ++i)
+            if (i < o_nc) o[((o_r0 + i) * H + h) * (long long)D + tid] = __float2bfloat16_rn(v[i]);
+    }
+    // ---- final state: S[dk][dv] = sigma * TMEM[lane dv][dk] ----
+    if (ok && a.state_out) {
 #pragma unroll
         for (int cb = 0; cb < 4; ++cb) {
             float v[32];
             tmem_ld32(tlane + TM_S + cb * 32, v);
             tmem_wait_ld();
-            float4* dst = reinterpret_cast<float4*>(a.state_out + state_base + (size_t)tid * D + cb * 32);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            for (int i = 0; i < 32; ++i) a.state_out[state_base + (size_t)(cb * 32 + i) * D + tid] = sigma * v[i];
         }
     }
     tc_fence_before();
@@ -547,7 +506,6 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     }
 }
 
-// ---- tensor maps ----
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
@@ -567,8 +525,10 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
+}  // namespace
+
 // [rows][H][128] bf16, box = 64 columns x 1 head x 64 rows, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, int H, long long rows) {
+bool make_tile_map(CUtensorMap* m, const void* base, int H, long long rows) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     if (rows < 1) rows = 1;
@@ -581,8 +541,6 @@ bool make_map(CUtensorMap* m, const void* base, int H, long long rows) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
-
 bool chunk_tc_supported(int dtype, int dk, int dv) { return dtype == 1 && dk == 128 && dv == 128; }
 
 cudaError_t launch_chunk_tc(const CallArgs& a, cudaStream_t stream) {
@@ -590,16 +548,15 @@ cudaError_t launch_chunk_tc(const CallArgs& a, cudaStream_t stream) {
     if (!chunk_tc_supported(a.dtype, a.dk, a.dv)) return cudaErrorInvalidValue;
     TcParams p;
     p.a = a;
-    p.rows_total = a.rows_total;
-    CUtensorMap mk, mv, mq;
-    if (!a.k || !a.v) return cudaErrorInvalidValue;
-    if (!make_map(&mk, a.k, a.num_heads, a.rows_total) || !make_map(&mv, a.v, a.num_heads, a.rows_total))
-        return cudaErrorInvalidValue;
     const bool replay = a.kind == kReplay;
-    if (!make_map(&mq, replay ? a.k : a.q, a.num_heads, a.rows_total)) return cudaErrorInvalidValue;
-    const uint32_t smem = (replay ? SMEM_REPLAY : SMEM_PREFILL) + 1024;
+    CUtensorMap mk, mv, mq;
+    if (!a.k || !a.v || (!replay && !a.q)) return cudaErrorInvalidValue;
+    if (!make_tile_map(&mk, a.k, a.num_heads, a.rows_total) || !make_tile_map(&mv, a.v, a.num_heads, a.rows_total) ||
+        !make_tile_map(&mq, replay ? a.k : a.q, a.num_heads, a.rows_total))
+        return cudaErrorInvalidValue;
     static bool attr_set[2] = {false, false};
     if (replay) {
+        const uint32_t smem = Layout<true>::BYTES + 1024;
         if (!attr_set[0]) {
             cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
             if (e != cudaSuccess) return e;
@@ -607,6 +564,7 @@ cudaError_t launch_chunk_tc(const CallArgs& a, cudaStream_t stream) {
         }
         chunk_tc_kernel<true><<<(unsigned)a.units, NT, smem, stream>>>(p, mk, mv, mq);
     } else {
+        const uint32_t smem = Layout<false>::BYTES + 1024;
         if (!attr_set[1]) {
             cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
             if (e != cudaSuccess) return e;
