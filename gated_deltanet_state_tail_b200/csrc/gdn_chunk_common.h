@@ -51,105 +51,109 @@ __device__ __forceinline__ void report_timeout(const CallArgs& a, uint32_t where
     atomicCAS(&a.ws->timeout_where, 0u, where);
 }
 
+// acc[nt] += A (16 x 8 ksteps) * B (8 ksteps x 16), nt = two 8-column halves
+// of the 16-wide result; A and B row-major fp32 in shared memory (strides
+// lda, ldb), read as tf32 (the tensor core uses the top 19 bits).
+__device__ __forceinline__ void mma16x16_tf32(float acc[2][4], const float* A, int lda, const float* B, int ldb,
+                                              int ksteps, int g, int t) {
+    for (int ks = 0; ks < ksteps; ++ks) {
+        uint32_t af[4], bf[2][2];
+        af[0] = __float_as_uint(A[g * lda + 8 * ks + t]);
+        af[1] = __float_as_uint(A[(g + 8) * lda + 8 * ks + t]);
+        af[2] = __float_as_uint(A[g * lda + 8 * ks + t + 4]);
+        af[3] = __float_as_uint(A[(g + 8) * lda + 8 * ks + t + 4]);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            bf[nt][0] = __float_as_uint(B[(8 * ks + t) * ldb + 8 * nt + g]);
+            bf[nt][1] = __float_as_uint(B[(8 * ks + t + 4) * ldb + 8 * nt + g]);
+        }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) mma_sync_tf32(acc[nt], af, bf[nt]);
+    }
+}
+
+// Store a 16 x 16 fragment pair (times `scale`) row-major at D (stride ldd).
+__device__ __forceinline__ void store16x16(float* D, int ldd, const float acc[2][4], float scale, int g, int t) {
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        D[g * ldd + 8 * nt + 2 * t] = scale * acc[nt][0];
+        D[g * ldd + 8 * nt + 2 * t + 1] = scale * acc[nt][1];
+        D[(g + 8) * ldd + 8 * nt + 2 * t] = scale * acc[nt][2];
+        D[(g + 8) * ldd + 8 * nt + 2 * t + 1] = scale * acc[nt][3];
+    }
+}
+
 // In place: on entry AT (fp32, 64 x LDT) holds the strictly lower triangular
 // A (entries on and above the diagonal are ignored); on exit it holds
 // T = (I + A)^-1 on and below the diagonal 16 x 16 blocks (the upper
 // triangles of the diagonal blocks are written as zeros; the blocks above
-// them are left untouched and must be read as zero).
+// them are left untouched and must be read as zero).  Xs is scratch of
+// 4 x 16 x 24 floats.
 //
-// The 16 x 16 diagonal blocks are inverted by forward substitution on CUDA
-// cores, one lane per column, right-looking (once x_j is final it is pushed
-// into the rows below, so the serial dependency is one FMA per row).  The
-// blocks below the diagonal follow from T_ba = -T_bb sum_{a <= m < b} A_bm
-// T_ma, one block row b at a time, as warp-level tf32 tensor-core products
-// (warp a computes block (b, a); the tensor core reads the top 19 bits of
-// the fp32 values).  ltid is the thread's index among the 128 threads that
-// run it; bar_id names the barrier those threads share.
+// Diagonal blocks: forward substitution on CUDA cores, warp w solves block w
+// with one lane per column (row i of the block is prefetched while row i - 1
+// finishes).  Then recursive doubling with warp-level tf32 tensor-core
+// products: 32 x 32 blocks T_10 = -D_1 A_10 D_0 and T_32 = -D_3 A_32 D_2,
+// then the lower-left 32 x 32 block -T_22 (A_21 T_11) (warp (r, c) computes
+// 16 x 16 block (r, c)).  ltid is the thread's index among the 128 threads
+// that run it; bar_id names the barrier those threads share.
 __device__ __forceinline__ void invert_unit_lower_inplace(float* AT, float* Xs, int ltid, uint32_t bar_id) {
     const int warp = ltid >> 5, lane = ltid & 31;
     {
         // every lane computes; lanes 16..31 repeat lanes 0..15 and do not store
         const int o = warp * 16, cc = lane & 15;
-        float acc[16];
+        float x[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i] = (i == cc) ? 1.0f : 0.0f;
+        for (int i = 0; i < 16; ++i) {
+            float s0 = (i == cc) ? 1.0f : 0.0f, s1 = 0.0f;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const float xj = acc[j];
-#pragma unroll
-            for (int i = j + 1; i < 16; ++i) acc[i] = fmaf(-AT[(o + i) * LDT + o + j], xj, acc[i]);
+            for (int j = 0; j < i; ++j) {
+                const float aij = AT[(o + i) * LDT + o + j];
+                if (j & 1) s1 = fmaf(-aij, x[j], s1);
+                else s0 = fmaf(-aij, x[j], s0);
+            }
+            x[i] = s0 + s1;
         }
         __syncwarp();
         if (lane < 16) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) AT[(o + i) * LDT + o + cc] = acc[i];
+            for (int i = 0; i < 16; ++i) AT[(o + i) * LDT + o + cc] = x[i];
         }
     }
     named_sync(bar_id, 128);
     const int g = lane >> 2, t = lane & 3;
-    for (int b = 1; b < 4; ++b) {
-        float* X = Xs + warp * (16 * 24);
-        if (warp < b) {
-            const int a = warp;
-            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            for (int m = a; m < b; ++m) {
-                uint32_t af[2][4], bf[2][2][2];
-#pragma unroll
-                for (int ks = 0; ks < 2; ++ks) {
-                    const int k0 = 16 * m + 8 * ks;
-                    af[ks][0] = __float_as_uint(AT[(16 * b + g) * LDT + k0 + t]);
-                    af[ks][1] = __float_as_uint(AT[(16 * b + g + 8) * LDT + k0 + t]);
-                    af[ks][2] = __float_as_uint(AT[(16 * b + g) * LDT + k0 + t + 4]);
-                    af[ks][3] = __float_as_uint(AT[(16 * b + g + 8) * LDT + k0 + t + 4]);
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
-                        bf[ks][nt][0] = __float_as_uint(AT[(k0 + t) * LDT + 16 * a + 8 * nt + g]);
-                        bf[ks][nt][1] = __float_as_uint(AT[(k0 + t + 4) * LDT + 16 * a + 8 * nt + g]);
-                    }
-                }
-#pragma unroll
-                for (int ks = 0; ks < 2; ++ks)
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) mma_sync_tf32(acc[nt], af[ks], bf[ks][nt]);
-            }
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                X[g * 24 + 8 * nt + 2 * t] = acc[nt][0];
-                X[g * 24 + 8 * nt + 2 * t + 1] = acc[nt][1];
-                X[(g + 8) * 24 + 8 * nt + 2 * t] = acc[nt][2];
-                X[(g + 8) * 24 + 8 * nt + 2 * t + 1] = acc[nt][3];
-            }
-        }
-        named_sync(bar_id, 128);   // every read of A_b* is done before T_b* overwrites it
-        if (warp < b) {
-            const int a = warp;
-            uint32_t af[2][4], bf[2][2][2];
-#pragma unroll
-            for (int ks = 0; ks < 2; ++ks) {
-                const int k0 = 8 * ks;
-                af[ks][0] = __float_as_uint(AT[(16 * b + g) * LDT + 16 * b + k0 + t]);
-                af[ks][1] = __float_as_uint(AT[(16 * b + g + 8) * LDT + 16 * b + k0 + t]);
-                af[ks][2] = __float_as_uint(AT[(16 * b + g) * LDT + 16 * b + k0 + t + 4]);
-                af[ks][3] = __float_as_uint(AT[(16 * b + g + 8) * LDT + 16 * b + k0 + t + 4]);
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
-                    bf[ks][nt][0] = __float_as_uint(X[(k0 + t) * 24 + 8 * nt + g]);
-                    bf[ks][nt][1] = __float_as_uint(X[(k0 + t + 4) * 24 + 8 * nt + g]);
-                }
-            }
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                float r[4] = {0.f, 0.f, 0.f, 0.f};
-                mma_sync_tf32(r, af[0], bf[0][nt]);
-                mma_sync_tf32(r, af[1], bf[1][nt]);
-                AT[(16 * b + g) * LDT + 16 * a + 8 * nt + 2 * t] = -r[0];
-                AT[(16 * b + g) * LDT + 16 * a + 8 * nt + 2 * t + 1] = -r[1];
-                AT[(16 * b + g + 8) * LDT + 16 * a + 8 * nt + 2 * t] = -r[2];
-                AT[(16 * b + g + 8) * LDT + 16 * a + 8 * nt + 2 * t + 1] = -r[3];
-            }
-        }
-        named_sync(bar_id, 128);
+    float* X = Xs + warp * (16 * 24);
+    // 32 x 32 merges: warp 0 -> block (1, 0), warp 1 -> block (3, 2)
+    if (warp < 2) {
+        const int bo = warp ? 48 : 16, ao = warp ? 32 : 0;   // row block b, column block a
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        mma16x16_tf32(acc, AT + bo * LDT + ao, LDT, AT + ao * LDT + ao, LDT, 2, g, t);     // A_ba D_a
+        store16x16(X, 24, acc, 1.0f, g, t);
+        __syncwarp();
+        float r[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        mma16x16_tf32(r, AT + bo * LDT + bo, LDT, X, 24, 2, g, t);                       // D_b (A_ba D_a)
+        store16x16(AT + bo * LDT + ao, LDT, r, -1.0f, g, t);
     }
+    named_sync(bar_id, 128);
+    // 64 x 64 merge: warp w -> block (r, c) = (2 + w / 2, w % 2) of X = A_21 T_11, then T_21 = -T_22 X
+    {
+        const int r = 2 + (warp >> 1), c = warp & 1;
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        for (int m = c; m < 2; ++m)
+            mma16x16_tf32(acc, AT + 16 * r * LDT + 16 * m, LDT, AT + 16 * m * LDT + 16 * c, LDT, 2, g, t);
+        store16x16(X, 24, acc, 1.0f, g, t);
+        named_sync(bar_id, 128);    // X blocks visible; every read of A_21 done
+        float rr[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        const float* X2c = Xs + c * (16 * 24);                   // X block (2, c), from warp c
+        if (r == 2) {
+            mma16x16_tf32(rr, AT + 32 * LDT + 32, LDT, X2c, 24, 2, g, t);               // D_2 X_2c
+        } else {
+            mma16x16_tf32(rr, AT + 48 * LDT + 32, LDT, X2c, 24, 2, g, t);               // T_32 X_2c
+            mma16x16_tf32(rr, AT + 48 * LDT + 48, LDT, X, 24, 2, g, t);                 // D_3 X_3c
+        }
+        store16x16(AT + 16 * r * LDT + 16 * c, LDT, rr, -1.0f, g, t);
+    }
+    named_sync(bar_id, 128);
 }
 
 // From the inverse T (in place in AT, see above) write the bf16 operands

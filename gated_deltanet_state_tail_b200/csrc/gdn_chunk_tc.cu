@@ -76,7 +76,7 @@ struct Layout {
     static constexpr uint32_t V0 = REPLAY ? 8192u : 32768u;
     static constexpr uint32_t V_LBO = REPLAY ? 16384u : 8192u;
 };
-static_assert(Layout<true>::OFF_X + 3 * 16 * 24 * 4 <= Layout<true>::OFF_PREP + 32768, "prep scratch fits");
+static_assert(Layout<true>::OFF_X + 4 * 16 * 24 * 4 <= Layout<true>::OFF_PREP + 32768, "prep scratch fits");
 
 // TMEM columns
 constexpr uint32_t TM_S = 0;      // 128 columns: fp32 S^T / sigma, lane = value row, column = key
@@ -87,6 +87,44 @@ constexpr uint32_t TM_O = 256;    // 64 columns (prefill): O^T, lane = value row
 struct TcParams {
     CallArgs a;
 };
+
+// Per-chunk gate factors: beta, G = cumulative log2 decay, gamma = 2^G,
+// binv = 2^-G (when the chunk's total decay is >= 2^-100), e = 2^(G_C - G).
+struct Gates {
+    alignas(16) float beta[C];
+    alignas(16) float g2[C];
+    alignas(16) float gam[C];
+    alignas(16) float binv[C];
+    alignas(16) float e[C];
+    float scan;
+};
+
+// Build the gate factors of one chunk from the fp32 gates of token `tid`
+// (threads 0..63; identity transitions past the window).  Every thread of the
+// CTA must call it: it contains two barriers.
+__device__ __forceinline__ void build_gates(Gates& G, float al, float be, int tid, int lane) {
+    if (tid < C) {
+        float lg = al > 0.0f ? fmaxf(__log2f(al), kLog2Floor) : kLog2Floor;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            float y = __shfl_up_sync(0xffffffffu, lg, off);
+            if (lane >= off) lg += y;
+        }
+        if (tid == 31) G.scan = lg;
+        G.beta[tid] = be;
+        G.g2[tid] = lg;
+    }
+    __syncthreads();
+    if (tid >= 32 && tid < C) G.g2[tid] += G.scan;
+    __syncthreads();
+    if (tid < C) {
+        const float g2C = G.g2[C - 1];
+        const float gj = G.g2[tid];
+        G.gam[tid] = exp2f(gj);
+        G.binv[tid] = g2C >= kFastGateFloor ? exp2f(-gj) : 0.0f;
+        G.e[tid] = exp2f(g2C - gj);
+    }
+}
 
 // Block-wide agreement after a bounded wait: every thread leaves together.
 __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, const CallArgs& a, uint32_t where) {
@@ -118,14 +156,9 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     using L = Layout<REPLAY>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t bar_tile[2], bar_mma;
+    __shared__ uint64_t bar_tile[2], bar_mma, bar_mma2;
     __shared__ uint32_t tmem_slot;
-    __shared__ alignas(16) float s_beta[C];
-    __shared__ alignas(16) float s_g2[C];
-    __shared__ alignas(16) float s_gam[C];
-    __shared__ alignas(16) float s_binv[C];
-    __shared__ alignas(16) float s_e[C];
-    __shared__ float s_scan;
+    __shared__ Gates s_gates[2];    // chunk c uses s_gates[c & 1]; chunk c + 1's are built during chunk c
 
     const CallArgs& a = p.a;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -144,6 +177,7 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         mbar_init(&bar_tile[0], 1);
         mbar_init(&bar_tile[1], 1);
         mbar_init(&bar_mma, 1);
+        mbar_init(&bar_mma2, 2);
         mbar_fence_init();
         tma_prefetch_desc(&map_k);
         tma_prefetch_desc(&map_v);
@@ -193,14 +227,54 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     const uint32_t id_s = idesc_bf16(128, 128, false, true);     // U~^T K
     const uint32_t id_o2 = idesc_bf16(128, 64, false, false);    // U^T M^T
 
-    uint32_t ph_mma = 0;
+    uint32_t ph_mma = 0, ph_mma2 = 0;
     bool ok = true;
-    // gates of the next chunk are fetched one chunk ahead (thread tid < 64 holds token tid)
-    float al_nxt = 1.0f, be_nxt = 0.0f;
-    if (tid < C && tid < w.len) {
-        al_nxt = a.alpha[(w.row0 + tid) * H + h];
-        be_nxt = a.beta[(w.row0 + tid) * H + h];
-    }
+    // gates: registers hold the next chunk's alpha, beta (thread tid < 64 = token tid)
+    auto load_gates = [&](int cc, float& al, float& be) {
+        al = 1.0f;
+        be = 0.0f;
+        if (tid < C && cc * C + tid < w.len) {
+            al = a.alpha[(w.row0 + (long long)cc * C + tid) * H + h];
+            be = a.beta[(w.row0 + (long long)cc * C + tid) * H + h];
+        }
+    };
+    float al_nxt, be_nxt;
+    load_gates(0, al_nxt, be_nxt);
+    build_gates(s_gates[0], al_nxt, be_nxt, tid, lane);
+    load_gates(1, al_nxt, be_nxt);
+
+    // K K^T of chunk cc into TM_P, issued as soon as its tiles are in (thread 0).
+    auto start_chunk = [&](int cc) -> bool {
+        const int slot = cc & 1;
+        uint8_t* tile = sm + L::OFF_TILE + slot * L::TILE;
+        bool good = wait_all(&bar_tile[slot], (cc >> 1) & 1, a, 1);
+        if (!good) return false;
+        const int ncc = min(C, w.len - cc * C);
+        if (ncc < C) {   // padded tokens are identity transitions: zero their rows
+            const int nrows = C - ncc;
+            const int nbox = REPLAY ? 4 : 6;
+            for (int e = tid; e < nbox * nrows * 8; e += NT) {
+                const int t = e / (nrows * 8), rr = ncc + (e / 8) % nrows, ch = e % 8;
+                st_shared_v4(tile + t * 8192, (uint32_t)(rr * 128 + ch * 16), make_uint4(0, 0, 0, 0));
+            }
+            fence_proxy_async_smem();
+        }
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t st = smem_u32(tile);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                mma_bf16_ss(tbase + TM_P, smem_desc_sw128(st + off, 16, 1024),
+                            smem_desc_sw128(st + off, 16, 1024), id_kk, kk > 0);
+            }
+            mma_commit(&bar_mma);
+        }
+        return true;
+    };
+    if (nchunks > 0) ok = start_chunk(0);
+
     // prefill: outputs of the previous chunk are written once its products are known complete
     long long o_r0 = 0;
     int o_nc = 0;
@@ -211,61 +285,10 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         const int nc = min(C, w.len - c * C);
         uint8_t* tile = sm + L::OFF_TILE + slot * L::TILE;
         const uint32_t s_tile = smem_u32(tile);
+        Gates& G = s_gates[c & 1];
+        const bool fast = G.g2[C - 1] >= kFastGateFloor;   // every partial product of gates is >= 2^-100
 
-        // ---- gates: cumulative log2 decay and the per-chunk factors ----
-        if (tid < C) {
-            const float al = al_nxt, be = be_nxt;
-            al_nxt = 1.0f;
-            be_nxt = 0.0f;
-            if ((c + 1) * C + tid < w.len) {
-                al_nxt = a.alpha[(r0 + C + tid) * H + h];
-                be_nxt = a.beta[(r0 + C + tid) * H + h];
-            }
-            float lg = al > 0.0f ? fmaxf(__log2f(al), kLog2Floor) : kLog2Floor;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                float y = __shfl_up_sync(0xffffffffu, lg, off);
-                if (lane >= off) lg += y;
-            }
-            if (tid == 31) s_scan = lg;
-            s_beta[tid] = be;
-            s_g2[tid] = lg;
-        }
-        __syncthreads();
-        if (tid >= 32 && tid < C) s_g2[tid] += s_scan;
-        __syncthreads();
-        const float g2C = s_g2[C - 1];
-        const bool fast = g2C >= kFastGateFloor;   // every partial product of gates is >= 2^-100
-        if (tid < C) {
-            const float gj = s_g2[tid];
-            s_gam[tid] = exp2f(gj);
-            s_binv[tid] = fast ? exp2f(-gj) : 0.0f;
-            s_e[tid] = exp2f(g2C - gj);
-        }
-        ok = wait_all(&bar_tile[slot], (c >> 1) & 1, a, 1);
-        if (!ok) break;
-        if (nc < C) {   // padded tokens are identity transitions: zero their rows
-            const int nrows = C - nc;
-            const int nbox = REPLAY ? 4 : 6;
-            for (int e = tid; e < nbox * nrows * 8; e += NT) {
-                const int t = e / (nrows * 8), rr = nc + (e / 8) % nrows, ch = e % 8;
-                st_shared_v4(tile + t * 8192, (uint32_t)(rr * 128 + ch * 16), make_uint4(0, 0, 0, 0));
-            }
-            fence_proxy_async_smem();
-        }
-        __syncthreads();
-
-        // ---- MMA 1: K K^T (replay, M = 64) or [K; Q] K^T (prefill) -> TM_P ----
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                mma_bf16_ss(tbase + TM_P, smem_desc_sw128(s_tile + off, 16, 1024),
-                            smem_desc_sw128(s_tile + off, 16, 1024), id_kk, kk > 0);
-            }
-            mma_commit(&bar_mma);
-        }
+        // ---- K K^T of this chunk (issued at the end of the previous one) ----
         ok = wait_all(&bar_mma, ph_mma, a, 2);   // also: every product of the previous chunk is done
         ph_mma ^= 1;
         if (!ok) break;
@@ -298,11 +321,11 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             const bool krow = REPLAY ? true : (tid < C);
             const int i = REPLAY ? warp * 16 + lane : (krow ? tid : tid - C);
             if (active) {
-                const float gi = s_g2[i];
-                const float bi = krow ? s_beta[i] : 1.0f;
+                const float gi = G.g2[i];
+                const float bi = krow ? G.beta[i] : 1.0f;
                 if (fast) {
-                    const float rowf = bi * s_gam[i];
-                    const float4* binv = reinterpret_cast<const float4*>(s_binv);
+                    const float rowf = bi * G.gam[i];
+                    const float4* binv = reinterpret_cast<const float4*>(G.binv);
 #pragma unroll
                     for (int q = 0; q < C / 4; ++q) {
                         const float4 bv = binv[q];
@@ -313,7 +336,7 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                     }
                 } else {
 #pragma unroll
-                    for (int j = 0; j < C; ++j) v[j] *= bi * exp2f(gi - s_g2[j]);
+                    for (int j = 0; j < C; ++j) v[j] *= bi * exp2f(gi - G.g2[j]);
                 }
                 if (krow) {
 #pragma unroll
@@ -333,25 +356,29 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
 
         // ---- T = (I + A)^-1 in place, then T diag(beta) and T diag(beta gamma) in bf16 ----
         invert_unit_lower_inplace(AT, Xs, tid, 0);
-        write_scaled_t(AT, s_beta, s_gam, sm + L::OFF_TB, sm + L::OFF_TBG, tid, 0);
+        write_scaled_t(AT, G.beta, G.gam, sm + L::OFF_TB, sm + L::OFF_TBG, tid, 0);
         fence_proxy_async_smem();
         __syncthreads();
 
-        // ---- MMA 2 / 3: W^T = K^T (T diag(beta gamma))^T -> TM_P, U'^T = V^T (T diag(beta))^T -> TM_U ----
+        // ---- MMA 2 / 3 (two issuing threads): W^T = K^T (T diag(beta gamma))^T -> TM_P,
+        //      U'^T = V^T (T diag(beta))^T -> TM_U ----
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 mma_bf16_ss(tbase + TM_P, smem_desc_sw128(s_tile + L::K0 + kk * 2048, 16384, 1024),
                             smem_desc_sw128(s_tbg + kk * 32, 16, 1024), id_w, kk > 0);
+            mma_commit(&bar_mma2);
+        } else if (tid == 32) {
+            tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 mma_bf16_ss(tbase + TM_U, smem_desc_sw128(s_tile + L::V0 + kk * 2048, L::V_LBO, 1024),
                             smem_desc_sw128(s_tb + kk * 32, 16, 1024), id_w, kk > 0);
-            mma_commit(&bar_mma);
+            mma_commit(&bar_mma2);
         }
-        ok = wait_all(&bar_mma, ph_mma, a, 3);
-        ph_mma ^= 1;
+        ok = wait_all(&bar_mma2, ph_mma2, a, 3);
+        ph_mma2 ^= 1;
         if (!ok) break;
         tc_fence_after();
 
@@ -370,7 +397,7 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             if (!REPLAY) {
                 const int i = tid >> 1, half = tid & 1;   // row i, keys [64 half, 64 half + 64)
                 const uint8_t* qb = tile + L::X0 + half * 16384;
-                const float sg = sigma * s_gam[i];
+                const float sg = sigma * G.gam[i];
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {       // 8 bf16 per 16-byte chunk of the Q row
                     const uint4 raw = *reinterpret_cast<const uint4*>(qb + i * 128 + ((ch ^ (i & 7)) << 4));
@@ -409,6 +436,11 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             }
             mma_commit(&bar_mma);
         }
+        // in its shadow: the next chunk's gate factors, and the gates after it
+        if (c + 1 < nchunks) {
+            build_gates(s_gates[(c + 1) & 1], al_nxt, be_nxt, tid, lane);
+            load_gates(c + 2, al_nxt, be_nxt);
+        }
         ok = wait_all(&bar_mma, ph_mma, a, 4);
         ph_mma ^= 1;
         if (!ok) break;
@@ -421,7 +453,7 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             tmem_ld32(tlane + TM_U + 32, v + 32);
             tmem_wait_ld();
             if (!REPLAY) write_row64_bf16(sm + L::OFF_UB, tid, v);
-            float snew = sigma * s_gam[C - 1];
+            float snew = sigma * G.gam[C - 1];
             if (snew < kRenormBelow) {     // uniform: fold the scale into the TMEM state
 #pragma unroll
                 for (int cb = 0; cb < 4; ++cb) {
@@ -437,7 +469,7 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             }
             sigma = snew;
             const float inv = 1.0f / snew;
-            const float4* ev = reinterpret_cast<const float4*>(s_e);
+            const float4* ev = reinterpret_cast<const float4*>(G.e);
 #pragma unroll
             for (int q = 0; q < C / 4; ++q) {
                 const float4 e4 = ev[q];
@@ -469,6 +501,11 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         }
         o_r0 = r0;
         o_nc = nc;
+        // ---- next chunk's K K^T goes in behind the state update ----
+        if (c + 1 < nchunks) {
+            ok = start_chunk(c + 1);
+            if (!ok) break;
+        }
     }
 
     // ---- drain: wait for the last products ----
