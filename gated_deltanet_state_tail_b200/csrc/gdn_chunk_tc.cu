@@ -44,15 +44,18 @@ using namespace chunk;
 constexpr int NT = 128;      // threads per CTA
 
 // ---- shared memory map (byte offsets from a 1 KB aligned base) ----
-// Two tile slots (chunk c in slot c % 2, the next chunk prefetched by TMA):
-//   replay : [K0 | V0 | K1 | V1]            (32 KB)
-//   prefill: [K0 | Q0 | K1 | Q1 | V0 | V1]  (48 KB)
-// 8 KB boxes of 64 rows x 64 columns; block kb holds columns [64 kb, 64 kb + 64).
+// Two tile slots (chunk c in slot c % 2, the next chunk prefetched by TMA),
+// made of 8 KB boxes of 64 rows x 64 columns:
+//   replay : [K0 | K1 | V0 | V1]            (32 KB)
+//   prefill: [K0 | Q0 | K1 | Q1 | V0 | V1]  (48 KB; K block stride 16 KB so
+//            that [K; Q] is one 128-row operand)
+// Once W and U' of a chunk are done, its V boxes take the U tile
+// diag(gamma_C / gamma) U / sigma (bf16 [dv][j], 16 KB) that the state update
+// of the same chunk reads.
 // PREP (32 KB) is reused within a chunk, in this order:
 //   A -> T in place (fp32 64 x LDT) and the product scratch,
 //   T diag(beta), T diag(beta gamma) (bf16 [j][j'], 8 KB each),
-//   BU = -sigma W (fp32, K-major [j][dk], four 8 KB key blocks),
-//   UT = diag(gamma_C / gamma) U / sigma (bf16 [dv][j], 16 KB).
+//   BU = -sigma W (fp32, K-major [j][dk], four 8 KB key blocks).
 // Prefill adds UB (bf16 U^T [dv][j]), MB (bf16 masked decayed Q K^T [i][j])
 // and BQ (fp32 sigma diag(gamma) Q, K-major [i][dk], four 8 KB blocks).
 template <bool REPLAY>
@@ -65,16 +68,16 @@ struct Layout {
     static constexpr uint32_t OFF_TB = OFF_PREP;
     static constexpr uint32_t OFF_TBG = OFF_PREP + 8192;
     static constexpr uint32_t OFF_BU = OFF_PREP;
-    static constexpr uint32_t OFF_UT = OFF_PREP;
     static constexpr uint32_t OFF_UB = OFF_PREP + 32768;
     static constexpr uint32_t OFF_MB = OFF_UB + 16384;
     static constexpr uint32_t OFF_BQ = OFF_MB + 8192;
     static constexpr uint32_t BYTES = REPLAY ? OFF_PREP + 32768 : OFF_BQ + 32768;
     // offsets inside a tile slot
-    static constexpr uint32_t K0 = 0, K1 = 16384;
-    static constexpr uint32_t X0 = 8192;                  // V (replay) or Q (prefill) block 0
-    static constexpr uint32_t V0 = REPLAY ? 8192u : 32768u;
-    static constexpr uint32_t V_LBO = REPLAY ? 16384u : 8192u;
+    static constexpr uint32_t K_BLK = REPLAY ? 8192u : 16384u;   // stride of the two K blocks
+    static constexpr uint32_t Q0 = 8192;                          // prefill only
+    static constexpr uint32_t V0 = REPLAY ? 16384u : 32768u;
+    static constexpr uint32_t V_LBO = 8192;
+    static constexpr uint32_t UT = V0;
 };
 static_assert(Layout<true>::OFF_X + 4 * 16 * 24 * 4 <= Layout<true>::OFF_PREP + 32768, "prep scratch fits");
 
@@ -99,11 +102,13 @@ struct Gates {
     float scan;
 };
 
+constexpr uint32_t BAR_GATES = 3;   // named barrier of warps 0-1
+
 // Build the gate factors of one chunk from the fp32 gates of token `tid`
-// (threads 0..63; identity transitions past the window).  Every thread of the
-// CTA must call it: it contains two barriers.
+// (identity transitions past the window).  Called by threads 0..63 only
+// (warps 0 and 1, which share a named barrier).
 __device__ __forceinline__ void build_gates(Gates& G, float al, float be, int tid, int lane) {
-    if (tid < C) {
+    {
         float lg = al > 0.0f ? fmaxf(__log2f(al), kLog2Floor) : kLog2Floor;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -114,10 +119,10 @@ __device__ __forceinline__ void build_gates(Gates& G, float al, float be, int ti
         G.beta[tid] = be;
         G.g2[tid] = lg;
     }
-    __syncthreads();
-    if (tid >= 32 && tid < C) G.g2[tid] += G.scan;
-    __syncthreads();
-    if (tid < C) {
+    named_sync(BAR_GATES, 64);
+    if (tid >= 32) G.g2[tid] += G.scan;
+    named_sync(BAR_GATES, 64);
+    {
         const float g2C = G.g2[C - 1];
         const float gj = G.g2[tid];
         G.gam[tid] = exp2f(gj);
@@ -139,13 +144,13 @@ __device__ __forceinline__ void issue_tiles(uint8_t* tile, uint64_t* bar, const 
                                             const CUtensorMap* mq, int h, int r0) {
     using L = Layout<REPLAY>;
     mbar_arrive_expect_tx(bar, L::TILE);
-    tma_load_3d(tile + L::K0, mk, bar, 0, h, r0);
-    tma_load_3d(tile + L::K1, mk, bar, 64, h, r0);
+    tma_load_3d(tile, mk, bar, 0, h, r0);
+    tma_load_3d(tile + L::K_BLK, mk, bar, 64, h, r0);
     tma_load_3d(tile + L::V0, mv, bar, 0, h, r0);
     tma_load_3d(tile + L::V0 + L::V_LBO, mv, bar, 64, h, r0);
     if (!REPLAY) {
-        tma_load_3d(tile + L::X0, mq, bar, 0, h, r0);
-        tma_load_3d(tile + L::X0 + 16384, mq, bar, 64, h, r0);
+        tma_load_3d(tile + L::Q0, mq, bar, 0, h, r0);
+        tma_load_3d(tile + L::Q0 + 16384, mq, bar, 64, h, r0);
     }
 }
 
@@ -156,7 +161,9 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     using L = Layout<REPLAY>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t bar_tile[2], bar_mma, bar_mma2;
+    // bar_w: W and U' (two issuers); bar_u: the state product and the next
+    // chunk's K K^T (two issuers); bar_s: the state update (one issuer)
+    __shared__ uint64_t bar_tile[2], bar_w, bar_u, bar_s;
     __shared__ uint32_t tmem_slot;
     __shared__ Gates s_gates[2];    // chunk c uses s_gates[c & 1]; chunk c + 1's are built during chunk c
 
@@ -176,8 +183,9 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     if (tid == 0) {
         mbar_init(&bar_tile[0], 1);
         mbar_init(&bar_tile[1], 1);
-        mbar_init(&bar_mma, 1);
-        mbar_init(&bar_mma2, 2);
+        mbar_init(&bar_w, 2);
+        mbar_init(&bar_u, 2);
+        mbar_init(&bar_s, 1);
         mbar_fence_init();
         tma_prefetch_desc(&map_k);
         tma_prefetch_desc(&map_v);
@@ -197,7 +205,7 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
 
     float* AT = reinterpret_cast<float*>(sm + L::OFF_AT);
     float* Xs = reinterpret_cast<float*>(sm + L::OFF_X);
-    const uint32_t s_bu = smem_u32(sm + L::OFF_BU), s_ut = smem_u32(sm + L::OFF_UT);
+    const uint32_t s_bu = smem_u32(sm + L::OFF_BU);
     const uint32_t s_tb = smem_u32(sm + L::OFF_TB), s_tbg = smem_u32(sm + L::OFF_TBG);
     const uint32_t s_ub = smem_u32(sm + L::OFF_UB), s_mb = smem_u32(sm + L::OFF_MB), s_bq = smem_u32(sm + L::OFF_BQ);
 
@@ -227,7 +235,7 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     const uint32_t id_s = idesc_bf16(128, 128, false, true);     // U~^T K
     const uint32_t id_o2 = idesc_bf16(128, 64, false, false);    // U^T M^T
 
-    uint32_t ph_mma = 0, ph_mma2 = 0;
+    uint32_t ph_w = 0, ph_u = 0, ph_s = 0;
     bool ok = true;
     // gates: registers hold the next chunk's alpha, beta (thread tid < 64 = token tid)
     auto load_gates = [&](int cc, float& al, float& be) {
@@ -238,17 +246,11 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             be = a.beta[(w.row0 + (long long)cc * C + tid) * H + h];
         }
     };
-    float al_nxt, be_nxt;
-    load_gates(0, al_nxt, be_nxt);
-    build_gates(s_gates[0], al_nxt, be_nxt, tid, lane);
-    load_gates(1, al_nxt, be_nxt);
-
-    // K K^T of chunk cc into TM_P, issued as soon as its tiles are in (thread 0).
-    auto start_chunk = [&](int cc) -> bool {
+    // Wait for chunk cc's tiles and zero the rows past the window.
+    auto tiles_ready = [&](int cc) -> bool {
         const int slot = cc & 1;
         uint8_t* tile = sm + L::OFF_TILE + slot * L::TILE;
-        bool good = wait_all(&bar_tile[slot], (cc >> 1) & 1, a, 1);
-        if (!good) return false;
+        if (!wait_all(&bar_tile[slot], (cc >> 1) & 1, a, 1)) return false;
         const int ncc = min(C, w.len - cc * C);
         if (ncc < C) {   // padded tokens are identity transitions: zero their rows
             const int nrows = C - ncc;
@@ -260,22 +262,46 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             fence_proxy_async_smem();
         }
         __syncthreads();
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t st = smem_u32(tile);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                mma_bf16_ss(tbase + TM_P, smem_desc_sw128(st + off, 16, 1024),
-                            smem_desc_sw128(st + off, 16, 1024), id_kk, kk > 0);
-            }
-            mma_commit(&bar_mma);
-        }
         return true;
     };
-    if (nchunks > 0) ok = start_chunk(0);
+    // K K^T (or [K; Q] K^T) of chunk cc into TM_P.
+    auto issue_kk = [&](int cc) {
+        const uint32_t st = smem_u32(sm + L::OFF_TILE + (cc & 1) * L::TILE);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * L::K_BLK + (kk & 3) * 32;
+            mma_bf16_ss(tbase + TM_P, smem_desc_sw128(st + off, 16, 1024), smem_desc_sw128(st + off, 16, 1024),
+                        id_kk, kk > 0);
+        }
+    };
+    auto write_outputs = [&](long long orow, int onc) {   // prefill: O of a finished chunk
+        float v[64];
+        tmem_ld32(tlane + TM_O, v);
+        tmem_ld32(tlane + TM_O + 32, v + 32);
+        tmem_wait_ld();
+        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o_out);
+#pragma unroll
+        for (int i = 0; i < C; ++i)
+            if (i < onc) o[((orow + i) * H + h) * (long long)D + tid] = __float2bfloat16_rn(v[i]);
+    };
 
-    // prefill: outputs of the previous chunk are written once its products are known complete
+    // ---- prologue: gates and K K^T of chunk 0 ----
+    float al_nxt, be_nxt;
+    load_gates(0, al_nxt, be_nxt);
+    if (tid < C) build_gates(s_gates[0], al_nxt, be_nxt, tid, lane);
+    load_gates(1, al_nxt, be_nxt);
+    if (nchunks > 0) {
+        ok = tiles_ready(0);
+        if (ok && tid == 96) {
+            tc_fence_after();
+            issue_kk(0);
+        }
+        if (ok && (tid == 64 || tid == 96)) mma_commit(&bar_u);
+        if (ok) {
+            ok = wait_all(&bar_u, ph_u, a, 2);
+            ph_u ^= 1;
+        }
+    }
     long long o_r0 = 0;
     int o_nc = 0;
 
@@ -287,27 +313,15 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         const uint32_t s_tile = smem_u32(tile);
         Gates& G = s_gates[c & 1];
         const bool fast = G.g2[C - 1] >= kFastGateFloor;   // every partial product of gates is >= 2^-100
-
-        // ---- K K^T of this chunk (issued at the end of the previous one) ----
-        ok = wait_all(&bar_mma, ph_mma, a, 2);   // also: every product of the previous chunk is done
-        ph_mma ^= 1;
-        if (!ok) break;
         tc_fence_after();
-        // the other tile slot is free: prefetch the next chunk
-        if (tid == 0 && c + 1 < nchunks)
-            issue_tiles<REPLAY>(sm + L::OFF_TILE + (slot ^ 1) * L::TILE, &bar_tile[slot ^ 1], &map_k, &map_v,
-                                &map_q, h, (int)(r0 + C));
 
         if (!REPLAY && c > 0) {
-            // ---- outputs of chunk c - 1: o[r0 + i, h, tid] ----
-            float v[64];
-            tmem_ld32(tlane + TM_O, v);
-            tmem_ld32(tlane + TM_O + 32, v + 32);
-            tmem_wait_ld();
-            __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o_out);
-#pragma unroll
-            for (int i = 0; i < C; ++i)
-                if (i < o_nc) o[((o_r0 + i) * H + h) * (long long)D + tid] = __float2bfloat16_rn(v[i]);
+            // the previous chunk's state update and outputs are complete before MB is rewritten
+            ok = wait_all(&bar_s, ph_s, a, 6);
+            ph_s ^= 1;
+            if (!ok) break;
+            tc_fence_after();
+            write_outputs(o_r0, o_nc);
         }
 
         // ---- epilogue 1: A = strict_tril(beta_i (gamma_i / gamma_j) K K^T) (fp32, in AT);
@@ -360,25 +374,41 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         fence_proxy_async_smem();
         __syncthreads();
 
-        // ---- MMA 2 / 3 (two issuing threads): W^T = K^T (T diag(beta gamma))^T -> TM_P,
-        //      U'^T = V^T (T diag(beta))^T -> TM_U ----
+        // ---- W^T = K^T (T diag(beta gamma))^T -> TM_P and U'^T = V^T (T diag(beta))^T -> TM_U ----
+        const uint32_t ph_s_prev = ph_s;   // replay: parity of the previous chunk's state update
+        if (REPLAY && c > 0) ph_s ^= 1;
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tbase + TM_P, smem_desc_sw128(s_tile + L::K0 + kk * 2048, 16384, 1024),
+                mma_bf16_ss(tbase + TM_P, smem_desc_sw128(s_tile + kk * 2048, L::K_BLK, 1024),
                             smem_desc_sw128(s_tbg + kk * 32, 16, 1024), id_w, kk > 0);
-            mma_commit(&bar_mma2);
+            mma_commit(&bar_w);
+            // prefetch the next chunk into the other slot once the previous chunk's state
+            // update (its last reader) is done; a timeout here leaves the tiles unloaded
+            // and the wait for them reports it
+            if (REPLAY && c > 0) {
+                if (mbar_wait_bounded(&bar_s, ph_s_prev, kWaitNs)) {
+                    if (c + 1 < nchunks)
+                        issue_tiles<REPLAY>(sm + L::OFF_TILE + (slot ^ 1) * L::TILE, &bar_tile[slot ^ 1], &map_k,
+                                            &map_v, &map_q, h, (int)(r0 + C));
+                } else {
+                    report_timeout(a, 6);
+                }
+            } else if (c + 1 < nchunks) {
+                issue_tiles<REPLAY>(sm + L::OFF_TILE + (slot ^ 1) * L::TILE, &bar_tile[slot ^ 1], &map_k, &map_v,
+                                    &map_q, h, (int)(r0 + C));
+            }
         } else if (tid == 32) {
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 mma_bf16_ss(tbase + TM_U, smem_desc_sw128(s_tile + L::V0 + kk * 2048, L::V_LBO, 1024),
                             smem_desc_sw128(s_tb + kk * 32, 16, 1024), id_w, kk > 0);
-            mma_commit(&bar_mma2);
+            mma_commit(&bar_w);
         }
-        ok = wait_all(&bar_mma2, ph_mma2, a, 3);
-        ph_mma2 ^= 1;
+        ok = wait_all(&bar_w, ph_w, a, 3);
+        ph_w ^= 1;
         if (!ok) break;
         tc_fence_after();
 
@@ -396,7 +426,7 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             for (int j = 0; j < C; ++j) *reinterpret_cast<float*>(bu + sw128_offset_f32(j, kc)) = ns * v[j];
             if (!REPLAY) {
                 const int i = tid >> 1, half = tid & 1;   // row i, keys [64 half, 64 half + 64)
-                const uint8_t* qb = tile + L::X0 + half * 16384;
+                const uint8_t* qb = tile + L::Q0 + half * 16384;
                 const float sg = sigma * G.gam[i];
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {       // 8 bf16 per 16-byte chunk of the Q row
@@ -418,11 +448,17 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();
+        // the next chunk's tiles (prefetched since epilogue 1) must be in before its K K^T
+        if (c + 1 < nchunks) {
+            ok = tiles_ready(c + 1);
+            if (!ok) break;
+        } else {
+            __syncthreads();
+        }
 
-        // ---- MMA U: U^T += (S^T / sigma)(-sigma W^T), A from TMEM (tf32);
-        //      prefill: O^T = (S^T / sigma)(sigma gamma Q)^T ----
-        if (tid == 0) {
+        // ---- the state product (tid 64) and the next chunk's K K^T (tid 96) go in together;
+        //      warps 0-1 build the next chunk's gate factors meanwhile ----
+        if (tid == 64) {
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 16; ++kk)
@@ -434,19 +470,22 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                     mma_tf32_ts(tbase + TM_O, tbase + TM_S + kk * 8,
                                 smem_desc_sw128(s_bq + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_u, kk > 0);
             }
-            mma_commit(&bar_mma);
-        }
-        // in its shadow: the next chunk's gate factors, and the gates after it
-        if (c + 1 < nchunks) {
+            mma_commit(&bar_u);
+        } else if (tid == 96) {
+            tc_fence_after();
+            if (c + 1 < nchunks) issue_kk(c + 1);
+            mma_commit(&bar_u);
+        } else if (tid < C && c + 1 < nchunks) {
             build_gates(s_gates[(c + 1) & 1], al_nxt, be_nxt, tid, lane);
-            load_gates(c + 2, al_nxt, be_nxt);
         }
-        ok = wait_all(&bar_mma, ph_mma, a, 4);
-        ph_mma ^= 1;
+        if (c + 1 < nchunks) load_gates(c + 2, al_nxt, be_nxt);
+        ok = wait_all(&bar_u, ph_u, a, 4);
+        ph_u ^= 1;
         if (!ok) break;
         tc_fence_after();
 
-        // ---- epilogue U: U~ = diag(gamma_C / gamma) U / sigma_new (and U for the outputs) ----
+        // ---- epilogue U: U~ = diag(gamma_C / gamma) U / sigma_new into this chunk's V boxes
+        //      (and U itself for the outputs) ----
         {
             float v[64];
             tmem_ld32(tlane + TM_U, v);
@@ -478,51 +517,36 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 v[4 * q + 2] *= e4.z * inv;
                 v[4 * q + 3] *= e4.w * inv;
             }
-            write_row64_bf16(sm + L::OFF_UT, tid, v);
+            write_row64_bf16(tile + L::UT, tid, v);
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
 
-        // ---- MMA S: S^T / sigma += U~^T K ;  prefill: O^T += U^T M^T.
-        //      Not waited for here: the next chunk's first commit covers it. ----
+        // ---- S^T / sigma += U~^T K ;  prefill: O^T += U^T M^T ----
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tbase + TM_S, smem_desc_sw128(s_ut + kk * 32, 16, 1024),
-                            smem_desc_sw128(s_tile + L::K0 + kk * 2048, 16384, 1024), id_s, 1u);
+                mma_bf16_ss(tbase + TM_S, smem_desc_sw128(s_tile + L::UT + kk * 32, 16, 1024),
+                            smem_desc_sw128(s_tile + kk * 2048, L::K_BLK, 1024), id_s, 1u);
             if (!REPLAY) {
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_bf16_ss(tbase + TM_O, smem_desc_sw128(s_ub + kk * 32, 16, 1024),
                                 smem_desc_sw128(s_mb + kk * 32, 16, 1024), id_o2, 1u);
             }
+            mma_commit(&bar_s);
         }
         o_r0 = r0;
         o_nc = nc;
-        // ---- next chunk's K K^T goes in behind the state update ----
-        if (c + 1 < nchunks) {
-            ok = start_chunk(c + 1);
-            if (!ok) break;
-        }
     }
 
-    // ---- drain: wait for the last products ----
-    if (ok) {
-        if (tid == 0) mma_commit(&bar_mma);
-        ok = wait_all(&bar_mma, ph_mma, a, 5);
+    // ---- drain: the last state update (and outputs) ----
+    if (ok && nchunks > 0) {
+        ok = wait_all(&bar_s, ph_s, a, 5);
         tc_fence_after();
-    }
-    if (ok && !REPLAY && nchunks > 0) {
-        float v[64];
-        tmem_ld32(tlane + TM_O, v);
-        tmem_ld32(tlane + TM_O + 32, v + 32);
-        tmem_wait_ld();
-        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o_out);
-#pragma unroll
-        for (int i = 0; i < C; ++i)
-            if (i < o_nc) o[((o_r0 + i) * H + h) * (long long)D + tid] = __float2bfloat16_rn(v[i]);
+        if (ok && !REPLAY) write_outputs(o_r0, o_nc);
     }
     // ---- final state: S[dk][dv] = sigma * TMEM[lane dv][dk] ----
     if (ok && a.state_out) {
