@@ -313,8 +313,6 @@ def oracle_replay_sample(wl, seconds_hint=15.0):
 # --------------------------------------------------------------------------
 def bench_ours(args, rank, world, local):
     import gated_deltanet_state_tail_b200 as gdn
-    if args.workload != "stack":
-        raise SystemExit("only --workload stack is a bench line; other workloads are parity cases")
     wl = inputs.stack_workload(args.layers)
     kernel = {"auto": gdn.GDN_KERNEL_AUTO, "recurrent": gdn.GDN_KERNEL_RECURRENT,
               "chunked": gdn.GDN_KERNEL_CHUNKED_TC}[args.kernel]
@@ -522,6 +520,88 @@ def e2e_host_buffers(data, kernel, args, world):
 
 
 # --------------------------------------------------------------------------
+# auxiliary workloads (not the headline line): budget sweep and varlen batch
+# --------------------------------------------------------------------------
+def _time_ms(fn, iters=5, flush=None):
+    fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(iters):
+        if flush is not None:
+            flush.fill_(1.0)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts)
+
+
+def bench_sweep(args):
+    """Replay budget R/L in {1, 2, 5, 10, 25, 100}% at L = 8K, 16K, 32K (one layer, 32 heads,
+    alpha ~ U[0.97, 0.9999]): replay latency, full-prefill latency, and the relative
+    Frobenius distance of the replayed state to the state of the whole prefix."""
+    import gated_deltanet_state_tail_b200 as gdn
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    lines = []
+    for L in (8192, 16384, 32768):
+        wl = [w for w in inputs.sweep_workloads() if w.match_len[0] == L]
+        H = wl[0].H
+        t = inputs.draw_tensors(L, H, 128, 128, "bf16", 0.97, 0.9999, 0, device="cuda")
+        full_state = torch.empty((1, H, 128, 128), device="cuda")
+        pf = gdn.PrefillPlan(H, 128, 128, "bf16", [0, L])
+        o = torch.empty((L, H, 128), dtype=torch.bfloat16, device="cuda")
+        full_ms = _time_ms(lambda: pf.run(t["q"], t["k"], t["v"], t["alpha"], t["beta"], o,
+                                          state_out=full_state), flush=flush)
+        pf.check()
+        for w in wl:
+            R = w.R[0]
+            plan = gdn.ReplayPlan(H, 128, 128, "bf16", [0, L], [L], [R])
+            st = torch.empty_like(full_state)
+            rep_ms = _time_ms(lambda: plan.run(t["k"], t["v"], t["alpha"], t["beta"], st), flush=flush)
+            plan.check()
+            e = ((st - full_state).flatten(2).norm(dim=2) / full_state.flatten(2).norm(dim=2))[0]
+            lines.append({"metric": "replay-budget sweep", "workload": w.name, "L": L, "pct": w.extra["pct"],
+                          "R": R, "replay_ms": rep_ms, "full_prefill_ms": full_ms,
+                          "replay_speedup_vs_full_prefill": full_ms / rep_ms,
+                          "replayed_tokens_per_s": R / (rep_ms / 1e3),
+                          "state_rel_frob": {"mean": float(e.mean()), "max": float(e.max())},
+                          "alpha": "U[0.97, 0.9999]", "heads": H, "dtype": "bf16", "data": "synthetic"})
+            plan.close()
+        pf.close()
+    return lines
+
+
+def bench_varlen(args):
+    """64 ragged requests (16 heads): replay of every tail, then every suffix."""
+    import gated_deltanet_state_tail_b200 as gdn
+    wl = inputs.varlen_workload(64, seed=0)
+    off, cu = wl.seq_offsets(), wl.suffix_cu()
+    H = wl.H
+    cache = inputs.draw_tensors(int(off[-1]), H, 128, 128, "bf16", wl.alpha_lo, wl.alpha_hi, 100,
+                                device="cuda", with_q=False)
+    suf = inputs.draw_tensors(int(cu[-1]), H, 128, 128, "bf16", wl.alpha_lo, wl.alpha_hi, 101, device="cuda")
+    rp = gdn.ReplayPlan(H, 128, 128, "bf16", off, wl.match_len, wl.R)
+    pp = gdn.PrefillPlan(H, 128, 128, "bf16", cu)
+    st = torch.empty((wl.batch, H, 128, 128), device="cuda")
+    st2 = torch.empty_like(st)
+    o = torch.empty((int(cu[-1]), H, 128), dtype=torch.bfloat16, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    rep_ms = _time_ms(lambda: rp.run(cache["k"], cache["v"], cache["alpha"], cache["beta"], st), 10, flush)
+    suf_ms = _time_ms(lambda: pp.run(suf["q"], suf["k"], suf["v"], suf["alpha"], suf["beta"], o,
+                                     state_in=st, state_out=st2), 10, flush)
+    rp.check()
+    pp.check()
+    return [{"metric": "varlen replay + suffix", "workload": wl.name, "requests": wl.batch, "heads": H,
+             "replayed_tokens": int(sum(min(r, l) for r, l in zip(wl.R, wl.match_len))),
+             "suffix_tokens": int(sum(wl.suffix_len)), "replay_ms": rep_ms, "suffix_prefill_ms": suf_ms,
+             "replayed_tokens_per_s": sum(min(r, l) for r, l in zip(wl.R, wl.match_len)) / (rep_ms / 1e3),
+             "match_len": wl.match_len, "R": wl.R, "suffix_len": wl.suffix_len, "dtype": "bf16",
+             "data": "synthetic"}]
+
+
+# --------------------------------------------------------------------------
 # reference arm: the fp64 CPU oracle as it stands
 # --------------------------------------------------------------------------
 def bench_reference(args, rank, world):
@@ -560,7 +640,8 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="stack")
+    ap.add_argument("--workload", default="stack", choices=["stack", "sweep", "varlen"],
+                    help="stack = the bench line; sweep / varlen print auxiliary lines")
     ap.add_argument("--layers", type=int, default=24,
                     help="GDN layers in the stack (a multiple of 3; 24 is the bench line, "
                          "fewer only for profiling captures)")
@@ -581,6 +662,13 @@ def main():
         return
 
     rank, world, local = dist_init(args.gpus)
+    if args.workload in ("sweep", "varlen"):
+        if rank == 0:
+            for line in (bench_sweep(args) if args.workload == "sweep" else bench_varlen(args)):
+                print(json.dumps(line), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
     try:
         res = bench_ours(args, rank, world, local)
         if rank == 0:
