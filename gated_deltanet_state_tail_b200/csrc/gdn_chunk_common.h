@@ -32,17 +32,18 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&p);
 }
 
-// Write 64 fp32 values (one row, columns 0..63) as bf16 into a 128-byte
-// swizzled row `row` of the tile at `tile`.
-__device__ __forceinline__ void write_row64_bf16(uint8_t* tile, int row, const float* v) {
+// Write 32 fp32 values as bf16 into the 16-byte chunks c0 .. c0 + 3
+// (columns 8 c0 .. 8 c0 + 31) of the 128-byte swizzled row `row` of the tile
+// at `tile`.
+__device__ __forceinline__ void write_row32_bf16(uint8_t* tile, int row, int c0, const float* v) {
 #pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
+    for (int ch = 0; ch < 4; ++ch) {
         uint4 q;
         q.x = pack_bf16(v[ch * 8 + 0], v[ch * 8 + 1]);
         q.y = pack_bf16(v[ch * 8 + 2], v[ch * 8 + 3]);
         q.z = pack_bf16(v[ch * 8 + 4], v[ch * 8 + 5]);
         q.w = pack_bf16(v[ch * 8 + 6], v[ch * 8 + 7]);
-        st_shared_v4(tile, (uint32_t)(row * 128 + ((ch ^ (row & 7)) << 4)), q);
+        st_shared_v4(tile, (uint32_t)(row * 128 + (((c0 + ch) ^ (row & 7)) << 4)), q);
     }
 }
 
@@ -91,26 +92,35 @@ __device__ __forceinline__ void store16x16(float* D, int ldd, const float acc[2]
 // 4 x 16 x 24 floats.
 //
 // Diagonal blocks: forward substitution on CUDA cores, warp w solves block w
-// with one lane per column (row i of the block is prefetched while row i - 1
-// finishes).  Then recursive doubling with warp-level tf32 tensor-core
-// products: 32 x 32 blocks T_10 = -D_1 A_10 D_0 and T_32 = -D_3 A_32 D_2,
-// then the lower-left 32 x 32 block -T_22 (A_21 T_11) (warp (r, c) computes
-// 16 x 16 block (r, c)).  ltid is the thread's index among the 128 threads
-// that run it; bar_id names the barrier those threads share.
+// with one lane per column.  Then recursive doubling with
+// warp-level tf32 tensor-core products: 32 x 32 blocks T_10 = -D_1 A_10 D_0
+// and T_32 = -D_3 A_32 D_2 (warps 0-1, while warps 2-3 form the parts of
+// X = A_21 T_11 that need only diagonal blocks), then the lower-left 32 x 32
+// block -T_22 X (warp (r, c) computes 16 x 16 block (r, c)).  ltid is the
+// thread's index among the 128 threads that run it; bar_id names the barrier
+// those threads share.
 __device__ __forceinline__ void invert_unit_lower_inplace(float* AT, float* Xs, int ltid, uint32_t bar_id) {
     const int warp = ltid >> 5, lane = ltid & 31;
     {
-        // every lane computes; lanes 16..31 repeat lanes 0..15 and do not store
+        // every lane computes; lanes 16..31 repeat lanes 0..15 and do not store.
+        // Row i of the block is read four entries per (broadcast) load.
         const int o = warp * 16, cc = lane & 15;
         float x[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             float s0 = (i == cc) ? 1.0f : 0.0f, s1 = 0.0f;
 #pragma unroll
-            for (int j = 0; j < i; ++j) {
-                const float aij = AT[(o + i) * LDT + o + j];
-                if (j & 1) s1 = fmaf(-aij, x[j], s1);
-                else s0 = fmaf(-aij, x[j], s0);
+            for (int j4 = 0; j4 < i; j4 += 4) {
+                const float4 a4 = *reinterpret_cast<const float4*>(AT + (o + i) * LDT + o + j4);
+                const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = j4 + e;
+                    if (j < i) {
+                        if (j & 1) s1 = fmaf(-av[e], x[j], s1);
+                        else s0 = fmaf(-av[e], x[j], s0);
+                    }
+                }
             }
             x[i] = s0 + s1;
         }
@@ -122,9 +132,14 @@ __device__ __forceinline__ void invert_unit_lower_inplace(float* AT, float* Xs, 
     }
     named_sync(bar_id, 128);
     const int g = lane >> 2, t = lane & 3;
-    float* X = Xs + warp * (16 * 24);
-    // 32 x 32 merges: warp 0 -> block (1, 0), warp 1 -> block (3, 2)
+    // Level A, warps 0-1: 32 x 32 merges, warp 0 -> block (1, 0), warp 1 -> block (3, 2),
+    // T_ba = -D_b (A_ba D_a).  Warps 2-3 meanwhile start block row r = warp of the
+    // lower-left X = A_21 T_11 from the diagonal blocks alone: P_r0 = A_r0 D_0 and
+    // X_r1 = A_r1 D_1 (kept in registers).
+    float pr0[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float xr1[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
     if (warp < 2) {
+        float* X = Xs + warp * (16 * 24);
         const int bo = warp ? 48 : 16, ao = warp ? 32 : 0;   // row block b, column block a
         float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         mma16x16_tf32(acc, AT + bo * LDT + ao, LDT, AT + ao * LDT + ao, LDT, 2, g, t);     // A_ba D_a
@@ -133,23 +148,31 @@ __device__ __forceinline__ void invert_unit_lower_inplace(float* AT, float* Xs, 
         float r[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         mma16x16_tf32(r, AT + bo * LDT + bo, LDT, X, 24, 2, g, t);                       // D_b (A_ba D_a)
         store16x16(AT + bo * LDT + ao, LDT, r, -1.0f, g, t);
+    } else {
+        const int r = warp;
+        mma16x16_tf32(pr0, AT + 16 * r * LDT, LDT, AT, LDT, 2, g, t);                    // A_r0 D_0
+        mma16x16_tf32(xr1, AT + 16 * r * LDT + 16, LDT, AT + 16 * LDT + 16, LDT, 2, g, t);  // A_r1 D_1
     }
     named_sync(bar_id, 128);
-    // 64 x 64 merge: warp w -> block (r, c) = (2 + w / 2, w % 2) of X = A_21 T_11, then T_21 = -T_22 X
+    // Level B: X_r0 = P_r0 + A_r1 T_10 (warps 2-3), X blocks to the scratch, slot 2 (r - 2) + c
+    if (warp >= 2) {
+        const int r = warp;
+        mma16x16_tf32(pr0, AT + 16 * r * LDT + 16, LDT, AT + 16 * LDT, LDT, 2, g, t);      // + A_r1 T_10
+        store16x16(Xs + (2 * (r - 2)) * (16 * 24), 24, pr0, 1.0f, g, t);
+        store16x16(Xs + (2 * (r - 2) + 1) * (16 * 24), 24, xr1, 1.0f, g, t);
+    }
+    named_sync(bar_id, 128);    // X blocks visible; every read of A_21 done
+    // then T_21 = -T_22 X, warp w -> block (r, c) = (2 + w / 2, w % 2)
     {
         const int r = 2 + (warp >> 1), c = warp & 1;
-        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        for (int m = c; m < 2; ++m)
-            mma16x16_tf32(acc, AT + 16 * r * LDT + 16 * m, LDT, AT + 16 * m * LDT + 16 * c, LDT, 2, g, t);
-        store16x16(X, 24, acc, 1.0f, g, t);
-        named_sync(bar_id, 128);    // X blocks visible; every read of A_21 done
         float rr[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        const float* X2c = Xs + c * (16 * 24);                   // X block (2, c), from warp c
+        const float* X2c = Xs + c * (16 * 24);
         if (r == 2) {
             mma16x16_tf32(rr, AT + 32 * LDT + 32, LDT, X2c, 24, 2, g, t);               // D_2 X_2c
         } else {
+            const float* X3c = Xs + (2 + c) * (16 * 24);
             mma16x16_tf32(rr, AT + 48 * LDT + 32, LDT, X2c, 24, 2, g, t);               // T_32 X_2c
-            mma16x16_tf32(rr, AT + 48 * LDT + 48, LDT, X, 24, 2, g, t);                 // D_3 X_3c
+            mma16x16_tf32(rr, AT + 48 * LDT + 48, LDT, X3c, 24, 2, g, t);               // D_3 X_3c
         }
         store16x16(AT + 16 * r * LDT + 16 * c, LDT, rr, -1.0f, g, t);
     }
@@ -158,29 +181,42 @@ __device__ __forceinline__ void invert_unit_lower_inplace(float* AT, float* Xs, 
 
 // From the inverse T (in place in AT, see above) write the bf16 operands
 // T diag(beta) -> tb and T diag(beta gamma) -> tbg, [j][j'] in 128-byte
-// swizzled rows.  tb / tbg may overlap AT: every thread reads its values
-// before the barrier and writes after it.
+// swizzled rows, with NTH threads (ltid < NTH) sharing barrier bar_id.
+// beta and gam are 16-byte aligned.
+// tb / tbg may overlap AT: every thread reads its values before the barrier
+// and writes after it.
+template <int NTH>
 __device__ __forceinline__ void write_scaled_t(const float* AT, const float* beta, const float* gam,
                                                uint8_t* tb, uint8_t* tbg, int ltid, uint32_t bar_id) {
-    const int j = ltid >> 1, half = ltid & 1;
-    float vb[32], vbg[32];
+    constexpr int PER = C * C / NTH;   // values of one row per thread
+    constexpr int TPR = C / PER;       // threads per row
+    static_assert(PER % 8 == 0 && TPR * PER == C, "whole 16-byte chunks per thread");
+    // thread -> (row j, column part): consecutive threads take consecutive rows, so
+    // the fp32 row loads (stride LDT) and the swizzled bf16 row stores are both
+    // free of bank conflicts, and a warp reads one set of gate factors
+    const int j = ltid % C, part = ltid / C;
+    float vb[PER], vbg[PER];
 #pragma unroll
-    for (int q = 0; q < 32; q += 4) {
-        const int col = half * 32 + q;
+    for (int q = 0; q < PER; q += 4) {
+        const int col = part * PER + q;
         float4 tt = make_float4(0.f, 0.f, 0.f, 0.f);
         if ((col >> 4) <= (j >> 4)) tt = *reinterpret_cast<const float4*>(AT + j * LDT + col);
+        const float4 b4 = *reinterpret_cast<const float4*>(beta + col);
+        const float4 g4 = *reinterpret_cast<const float4*>(gam + col);
         const float tv[4] = {tt.x, tt.y, tt.z, tt.w};
+        const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+        const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const float x = tv[e] * beta[col + e];
+            const float x = tv[e] * bv[e];
             vb[q + e] = x;
-            vbg[q + e] = x * gam[col + e];
+            vbg[q + e] = x * gv[e];
         }
     }
-    named_sync(bar_id, 128);
+    named_sync(bar_id, NTH);
 #pragma unroll
-    for (int ch = 0; ch < 4; ++ch) {
-        const int chunk = half * 4 + ch;
+    for (int ch = 0; ch < PER / 8; ++ch) {
+        const int chunk = part * (PER / 8) + ch;
         uint4 x, y;
         x.x = pack_bf16(vb[ch * 8 + 0], vb[ch * 8 + 1]);
         x.y = pack_bf16(vb[ch * 8 + 2], vb[ch * 8 + 3]);

@@ -24,10 +24,12 @@
 // small).  T is built from 16 x 16 diagonal inverses on CUDA cores and
 // warp-level tf32 tensor-core products for the blocks below the diagonal.
 //
-// Work: one CTA per (sequence, head) unit, 4 warps, chunks in order; the
+// Work: one CTA per (sequence, head) unit, 8 warps, chunks in order; the
 // next chunk's tiles stream in by TMA while the current chunk is computed.
-// Thread t owns TMEM lane t in every epilogue.  Replay: 96 KB of shared
-// memory and 256 TMEM columns, so two CTAs share an SM and overlap each
+// Warps w and w + 4 share TMEM lane quarter w (the only lanes a warp may
+// read) and split the 64 columns of every epilogue, so each thread moves 32
+// values per epilogue.  Replay: 96 KB of shared memory, 256 TMEM columns and
+// at most 128 registers per thread, so two CTAs share an SM and overlap each
 // other's serial chain.  Prefill adds the output path (184 KB, 512 columns).
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -41,7 +43,7 @@ namespace {
 using namespace sm100;
 using namespace chunk;
 
-constexpr int NT = 128;      // threads per CTA
+constexpr int NT = 256;      // threads per CTA
 
 // ---- shared memory map (byte offsets from a 1 KB aligned base) ----
 // Two tile slots (chunk c in slot c % 2, the next chunk prefetched by TMA),
@@ -103,6 +105,7 @@ struct Gates {
 };
 
 constexpr uint32_t BAR_GATES = 3;   // named barrier of warps 0-1
+constexpr uint32_t BAR_INV = 1;     // named barrier of warps 0-3 (the UT inverse)
 
 // Build the gate factors of one chunk from the fp32 gates of token `tid`
 // (identity transitions past the window).  Called by threads 0..63 only
@@ -155,7 +158,7 @@ __device__ __forceinline__ void issue_tiles(uint8_t* tile, uint64_t* bar, const 
 }
 
 template <bool REPLAY>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(NT, REPLAY ? 2 : 1)
 chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_q) {
     using L = Layout<REPLAY>;
@@ -169,6 +172,8 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
 
     const CallArgs& a = p.a;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wq = warp & 3, wh = warp >> 2;   // TMEM lane quarter; which 32 columns of an epilogue
+    const int row = wq * 32 + lane;            // this thread's TMEM lane
     constexpr uint32_t kTmemCols = REPLAY ? 256 : 512;
     const Unit u = a.unit_list[blockIdx.x];
     const int b = u.seq, h = u.head, H = a.num_heads;
@@ -199,7 +204,7 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = tmem_slot;
-    const uint32_t tlane = tbase + ((uint32_t)(warp * 32) << 16);   // this thread's lane, column 0
+    const uint32_t tlane = tbase + ((uint32_t)(wq * 32) << 16);   // this warp's lane quarter, column 0
     if (tid == 0 && nchunks > 0)
         issue_tiles<REPLAY>(sm + L::OFF_TILE, &bar_tile[0], &map_k, &map_v, &map_q, h, (int)w.row0);
 
@@ -209,15 +214,16 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     const uint32_t s_tb = smem_u32(sm + L::OFF_TB), s_tbg = smem_u32(sm + L::OFF_TBG);
     const uint32_t s_ub = smem_u32(sm + L::OFF_UB), s_mb = smem_u32(sm + L::OFF_MB), s_bq = smem_u32(sm + L::OFF_BQ);
 
-    // ---- initial state: TMEM lane dv = tid holds column dv of S (a row of S^T) ----
+    // ---- initial state: TMEM lane dv = row holds column dv of S (a row of S^T);
+    //      this thread fills key columns [64 wh, 64 wh + 64) ----
     const size_t state_base = ((size_t)b * H + h) * D * D;
     {
         float v[32];
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
+        for (int cb = 2 * wh; cb < 2 * wh + 2; ++cb) {
             if (!REPLAY && a.state_in) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = a.state_in[state_base + (size_t)(cb * 32 + i) * D + tid];
+                for (int i = 0; i < 32; ++i) v[i] = a.state_in[state_base + (size_t)(cb * 32 + i) * D + row];
             } else {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = 0.0f;
@@ -275,14 +281,13 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         }
     };
     auto write_outputs = [&](long long orow, int onc) {   // prefill: O of a finished chunk
-        float v[64];
-        tmem_ld32(tlane + TM_O, v);
-        tmem_ld32(tlane + TM_O + 32, v + 32);
+        float v[32];                                      // rows [32 wh, 32 wh + 32), value dim = row
+        tmem_ld32(tlane + TM_O + 32 * wh, v);
         tmem_wait_ld();
         __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o_out);
 #pragma unroll
-        for (int i = 0; i < C; ++i)
-            if (i < onc) o[((orow + i) * H + h) * (long long)D + tid] = __float2bfloat16_rn(v[i]);
+        for (int ii = 0; ii < 32; ++ii)
+            if (32 * wh + ii < onc) o[((orow + 32 * wh + ii) * H + h) * (long long)D + row] = __float2bfloat16_rn(v[ii]);
     };
 
     // ---- prologue: gates and K K^T of chunk 0 ----
@@ -292,11 +297,14 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     load_gates(1, al_nxt, be_nxt);
     if (nchunks > 0) {
         ok = tiles_ready(0);
-        if (ok && tid == 96) {
+        if (ok && (warp == 2 || warp == 3)) {
             tc_fence_after();
-            issue_kk(0);
+            if (elect_one()) {
+                if (warp == 3) issue_kk(0);
+                mma_commit(&bar_u);
+            }
+            __syncwarp();
         }
-        if (ok && (tid == 64 || tid == 96)) mma_commit(&bar_u);
         if (ok) {
             ok = wait_all(&bar_u, ph_u, a, 2);
             ph_u ^= 1;
@@ -326,86 +334,125 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
 
         // ---- epilogue 1: A = strict_tril(beta_i (gamma_i / gamma_j) K K^T) (fp32, in AT);
         //      prefill: M = tril((gamma_i / gamma_j) Q K^T) (bf16, MB) ----
-        {
-            float v[64];
-            tmem_ld32(tlane + TM_P, v);
-            tmem_ld32(tlane + TM_P + 32, v + 32);
+        if (REPLAY) {
+            // M = 64 accumulator: rows 16 wq .. 16 wq + 15 sit in the quarter's first 16 lanes.
+            // This thread takes rows i0 = 16 wq + lane / 4 and i0 + 8, columns
+            // 32 wh + 8 k + 2 (lane % 4) + {0, 1}, k = 0..3.
+            float v[16];
+            tmem_ld16x256b_x4(tlane + TM_P + 32 * wh, v);
             tmem_wait_ld();
-            const bool active = REPLAY ? (lane < 16) : true;
-            const bool krow = REPLAY ? true : (tid < C);
-            const int i = REPLAY ? warp * 16 + lane : (krow ? tid : tid - C);
-            if (active) {
-                const float gi = G.g2[i];
-                const float bi = krow ? G.beta[i] : 1.0f;
-                if (fast) {
-                    const float rowf = bi * G.gam[i];
-                    const float4* binv = reinterpret_cast<const float4*>(G.binv);
+            const int i0 = 16 * wq + (lane >> 2), jb = 32 * wh + 2 * (lane & 3);
 #pragma unroll
-                    for (int q = 0; q < C / 4; ++q) {
-                        const float4 bv = binv[q];
-                        v[4 * q] *= rowf * bv.x;
-                        v[4 * q + 1] *= rowf * bv.y;
-                        v[4 * q + 2] *= rowf * bv.z;
-                        v[4 * q + 3] *= rowf * bv.w;
+            for (int hf = 0; hf < 2; ++hf) {
+                const int i = i0 + 8 * hf;
+                const float gi = G.g2[i], bi = G.beta[i];
+                const float rowf = bi * G.gam[i];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int j = jb + 8 * k;
+                    float x0 = v[4 * k + 2 * hf], x1 = v[4 * k + 2 * hf + 1];
+                    if (fast) {
+                        const float2 bv = *reinterpret_cast<const float2*>(G.binv + j);
+                        x0 *= rowf * bv.x;
+                        x1 *= rowf * bv.y;
+                    } else {
+                        x0 *= bi * exp2f(gi - G.g2[j]);
+                        x1 *= bi * exp2f(gi - G.g2[j + 1]);
                     }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < C; ++j) v[j] *= bi * exp2f(gi - G.g2[j]);
+                    x0 = (j < i) ? x0 : 0.0f;
+                    x1 = (j + 1 < i) ? x1 : 0.0f;
+                    *reinterpret_cast<float2*>(AT + i * LDT + j) = make_float2(x0, x1);
                 }
-                if (krow) {
+            }
+        } else {
+            // [K; Q] K^T: lane r < 64 is K row r, lane r >= 64 is Q row r - 64; this thread
+            // takes columns [32 wh, 32 wh + 32) of its lane
+            float v[32];
+            tmem_ld32(tlane + TM_P + 32 * wh, v);
+            tmem_wait_ld();
+            const bool krow = row < C;
+            const int i = krow ? row : row - C;
+            const float gi = G.g2[i];
+            const float bi = krow ? G.beta[i] : 1.0f;
+            if (fast) {
+                const float rowf = bi * G.gam[i];
+                const float4* binv = reinterpret_cast<const float4*>(G.binv + 32 * wh);
 #pragma unroll
-                    for (int j = 0; j < C; ++j) v[j] = (j < i) ? v[j] : 0.0f;
-#pragma unroll
-                    for (int j = 0; j < C; j += 4)
-                        *reinterpret_cast<float4*>(AT + i * LDT + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-                } else {
-#pragma unroll
-                    for (int j = 0; j < C; ++j) v[j] = (j <= i) ? v[j] : 0.0f;
-                    write_row64_bf16(sm + L::OFF_MB, i, v);
+                for (int q = 0; q < 8; ++q) {
+                    const float4 bv = binv[q];
+                    v[4 * q] *= rowf * bv.x;
+                    v[4 * q + 1] *= rowf * bv.y;
+                    v[4 * q + 2] *= rowf * bv.z;
+                    v[4 * q + 3] *= rowf * bv.w;
                 }
+            } else {
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) v[jj] *= bi * exp2f(gi - G.g2[32 * wh + jj]);
+            }
+            if (krow) {
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) v[jj] = (32 * wh + jj < i) ? v[jj] : 0.0f;
+#pragma unroll
+                for (int jj = 0; jj < 32; jj += 4)
+                    *reinterpret_cast<float4*>(AT + i * LDT + 32 * wh + jj) =
+                        make_float4(v[jj], v[jj + 1], v[jj + 2], v[jj + 3]);
+            } else {
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) v[jj] = (32 * wh + jj <= i) ? v[jj] : 0.0f;
+                write_row32_bf16(sm + L::OFF_MB, i, 4 * wh, v);
             }
         }
         tc_fence_before();
         __syncthreads();
 
-        // ---- T = (I + A)^-1 in place, then T diag(beta) and T diag(beta gamma) in bf16 ----
-        invert_unit_lower_inplace(AT, Xs, tid, 0);
-        write_scaled_t(AT, G.beta, G.gam, sm + L::OFF_TB, sm + L::OFF_TBG, tid, 0);
+        // ---- T = (I + A)^-1 in place (warps 0-3).  Meanwhile warp 4 prefetches the next
+        //      chunk into the other slot, once the previous chunk's state update (the slot's
+        //      last reader) is done; a timeout there leaves the tiles unloaded and the wait
+        //      for them reports it ----
+        const uint32_t ph_s_prev = ph_s;   // replay: parity of the previous chunk's state update
+        if (REPLAY && c > 0) ph_s ^= 1;
+        if (warp < 4) {
+            invert_unit_lower_inplace(AT, Xs, tid, BAR_INV);
+        } else if (warp == 4) {
+            if (elect_one() && c + 1 < nchunks) {
+                bool slot_free = true;
+                if (REPLAY && c > 0) {   // prefill waited for it at the top of the chunk
+                    slot_free = mbar_wait_bounded(&bar_s, ph_s_prev, kWaitNs);
+                    if (!slot_free) report_timeout(a, 6);
+                }
+                if (slot_free)
+                    issue_tiles<REPLAY>(sm + L::OFF_TILE + (slot ^ 1) * L::TILE, &bar_tile[slot ^ 1], &map_k, &map_v,
+                                        &map_q, h, (int)(r0 + C));
+            }
+            __syncwarp();
+        }
+        __syncthreads();
+        // ---- T diag(beta) and T diag(beta gamma) in bf16 (all warps) ----
+        write_scaled_t<NT>(AT, G.beta, G.gam, sm + L::OFF_TB, sm + L::OFF_TBG, tid, 0);
         fence_proxy_async_smem();
         __syncthreads();
 
         // ---- W^T = K^T (T diag(beta gamma))^T -> TM_P and U'^T = V^T (T diag(beta))^T -> TM_U ----
-        const uint32_t ph_s_prev = ph_s;   // replay: parity of the previous chunk's state update
-        if (REPLAY && c > 0) ph_s ^= 1;
-        if (tid == 0) {
+        if (warp == 0) {
             tc_fence_after();
+            if (elect_one()) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tbase + TM_P, smem_desc_sw128(s_tile + kk * 2048, L::K_BLK, 1024),
-                            smem_desc_sw128(s_tbg + kk * 32, 16, 1024), id_w, kk > 0);
-            mma_commit(&bar_w);
-            // prefetch the next chunk into the other slot once the previous chunk's state
-            // update (its last reader) is done; a timeout here leaves the tiles unloaded
-            // and the wait for them reports it
-            if (REPLAY && c > 0) {
-                if (mbar_wait_bounded(&bar_s, ph_s_prev, kWaitNs)) {
-                    if (c + 1 < nchunks)
-                        issue_tiles<REPLAY>(sm + L::OFF_TILE + (slot ^ 1) * L::TILE, &bar_tile[slot ^ 1], &map_k,
-                                            &map_v, &map_q, h, (int)(r0 + C));
-                } else {
-                    report_timeout(a, 6);
-                }
-            } else if (c + 1 < nchunks) {
-                issue_tiles<REPLAY>(sm + L::OFF_TILE + (slot ^ 1) * L::TILE, &bar_tile[slot ^ 1], &map_k, &map_v,
-                                    &map_q, h, (int)(r0 + C));
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16_ss(tbase + TM_P, smem_desc_sw128(s_tile + kk * 2048, L::K_BLK, 1024),
+                                smem_desc_sw128(s_tbg + kk * 32, 16, 1024), id_w, kk > 0);
+                mma_commit(&bar_w);
             }
-        } else if (tid == 32) {
+            __syncwarp();
+        } else if (warp == 1) {
             tc_fence_after();
+            if (elect_one()) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tbase + TM_U, smem_desc_sw128(s_tile + L::V0 + kk * 2048, L::V_LBO, 1024),
-                            smem_desc_sw128(s_tb + kk * 32, 16, 1024), id_w, kk > 0);
-            mma_commit(&bar_w);
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16_ss(tbase + TM_U, smem_desc_sw128(s_tile + L::V0 + kk * 2048, L::V_LBO, 1024),
+                                smem_desc_sw128(s_tb + kk * 32, 16, 1024), id_w, kk > 0);
+                mma_commit(&bar_w);
+            }
+            __syncwarp();
         }
         ok = wait_all(&bar_w, ph_w, a, 3);
         ph_w ^= 1;
@@ -415,22 +462,23 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         // ---- epilogue 2: BU[j][dk] = -sigma W[j][dk] (fp32, K-major);
         //      prefill: BQ[i][dk] = sigma gamma_i Q[i][dk] ----
         {
-            float v[64];
-            tmem_ld32(tlane + TM_P, v);
-            tmem_ld32(tlane + TM_P + 32, v + 32);
+            float v[32];                                        // key dk = row, chunk rows [32 wh, 32 wh + 32)
+            tmem_ld32(tlane + TM_P + 32 * wh, v);
             tmem_wait_ld();
-            uint8_t* bu = sm + L::OFF_BU + (tid >> 5) * 8192;   // key block of this thread
-            const int kc = tid & 31;
+            uint8_t* bu = sm + L::OFF_BU + wq * 8192;           // key block of this thread's key
             const float ns = -sigma;
 #pragma unroll
-            for (int j = 0; j < C; ++j) *reinterpret_cast<float*>(bu + sw128_offset_f32(j, kc)) = ns * v[j];
+            for (int jj = 0; jj < 32; ++jj)
+                *reinterpret_cast<float*>(bu + sw128_offset_f32(32 * wh + jj, lane)) = ns * v[jj];
             if (!REPLAY) {
-                const int i = tid >> 1, half = tid & 1;   // row i, keys [64 half, 64 half + 64)
-                const uint8_t* qb = tile + L::Q0 + half * 16384;
+                const int i = tid >> 2, qk = tid & 3;           // row i, keys [32 qk, 32 qk + 32)
+                const uint8_t* qb = tile + L::Q0 + (qk >> 1) * 16384;
+                uint8_t* blk = sm + L::OFF_BQ + qk * 8192;
                 const float sg = sigma * G.gam[i];
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {       // 8 bf16 per 16-byte chunk of the Q row
-                    const uint4 raw = *reinterpret_cast<const uint4*>(qb + i * 128 + ((ch ^ (i & 7)) << 4));
+                for (int ch = 0; ch < 4; ++ch) {                // 8 bf16 per 16-byte chunk of the Q row
+                    const int cidx = (qk & 1) * 4 + ch;
+                    const uint4 raw = *reinterpret_cast<const uint4*>(qb + i * 128 + ((cidx ^ (i & 7)) << 4));
                     const uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
                     float f[8];
 #pragma unroll
@@ -438,17 +486,15 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                         f[2 * e] = sg * __uint_as_float(wds[e] << 16);
                         f[2 * e + 1] = sg * __uint_as_float(wds[e] & 0xffff0000u);
                     }
-                    const int col = half * 64 + ch * 8;                // key index of f[0]
-                    uint8_t* blk = sm + L::OFF_BQ + (col >> 5) * 8192;
-                    const int cc = col & 31;
-                    *reinterpret_cast<float4*>(blk + sw128_offset_f32(i, cc)) = make_float4(f[0], f[1], f[2], f[3]);
-                    *reinterpret_cast<float4*>(blk + sw128_offset_f32(i, cc + 4)) = make_float4(f[4], f[5], f[6], f[7]);
+                    *reinterpret_cast<float4*>(blk + sw128_offset_f32(i, 8 * ch)) = make_float4(f[0], f[1], f[2], f[3]);
+                    *reinterpret_cast<float4*>(blk + sw128_offset_f32(i, 8 * ch + 4)) =
+                        make_float4(f[4], f[5], f[6], f[7]);
                 }
             }
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        // the next chunk's tiles (prefetched since epilogue 1) must be in before its K K^T
+        // the next chunk's tiles (prefetched during the inverse) must be in before its K K^T
         if (c + 1 < nchunks) {
             ok = tiles_ready(c + 1);
             if (!ok) break;
@@ -456,25 +502,31 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             __syncthreads();
         }
 
-        // ---- the state product (tid 64) and the next chunk's K K^T (tid 96) go in together;
+        // ---- the state product (warp 2) and the next chunk's K K^T (warp 3) go in together;
         //      warps 0-1 build the next chunk's gate factors meanwhile ----
-        if (tid == 64) {
+        if (warp == 2) {
             tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 16; ++kk)
-                mma_tf32_ts(tbase + TM_U, tbase + TM_S + kk * 8,
-                            smem_desc_sw128(s_bu + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_u, 1u);
-            if (!REPLAY) {
+            if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < 16; ++kk)
-                    mma_tf32_ts(tbase + TM_O, tbase + TM_S + kk * 8,
-                                smem_desc_sw128(s_bq + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_u, kk > 0);
+                    mma_tf32_ts(tbase + TM_U, tbase + TM_S + kk * 8,
+                                smem_desc_sw128(s_bu + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_u, 1u);
+                if (!REPLAY) {
+#pragma unroll
+                    for (int kk = 0; kk < 16; ++kk)
+                        mma_tf32_ts(tbase + TM_O, tbase + TM_S + kk * 8,
+                                    smem_desc_sw128(s_bq + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_u, kk > 0);
+                }
+                mma_commit(&bar_u);
             }
-            mma_commit(&bar_u);
-        } else if (tid == 96) {
+            __syncwarp();
+        } else if (warp == 3) {
             tc_fence_after();
-            if (c + 1 < nchunks) issue_kk(c + 1);
-            mma_commit(&bar_u);
+            if (elect_one()) {
+                if (c + 1 < nchunks) issue_kk(c + 1);
+                mma_commit(&bar_u);
+            }
+            __syncwarp();
         } else if (tid < C && c + 1 < nchunks) {
             build_gates(s_gates[(c + 1) & 1], al_nxt, be_nxt, tid, lane);
         }
@@ -487,15 +539,14 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         // ---- epilogue U: U~ = diag(gamma_C / gamma) U / sigma_new into this chunk's V boxes
         //      (and U itself for the outputs) ----
         {
-            float v[64];
-            tmem_ld32(tlane + TM_U, v);
-            tmem_ld32(tlane + TM_U + 32, v + 32);
+            float v[32];                                        // value dv = row, chunk rows [32 wh, 32 wh + 32)
+            tmem_ld32(tlane + TM_U + 32 * wh, v);
             tmem_wait_ld();
-            if (!REPLAY) write_row64_bf16(sm + L::OFF_UB, tid, v);
+            if (!REPLAY) write_row32_bf16(sm + L::OFF_UB, row, 4 * wh, v);
             float snew = sigma * G.gam[C - 1];
             if (snew < kRenormBelow) {     // uniform: fold the scale into the TMEM state
 #pragma unroll
-                for (int cb = 0; cb < 4; ++cb) {
+                for (int cb = 2 * wh; cb < 2 * wh + 2; ++cb) {
                     float sv[32];
                     tmem_ld32(tlane + TM_S + cb * 32, sv);
                     tmem_wait_ld();
@@ -508,35 +559,38 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             }
             sigma = snew;
             const float inv = 1.0f / snew;
-            const float4* ev = reinterpret_cast<const float4*>(G.e);
+            const float4* ev = reinterpret_cast<const float4*>(G.e + 32 * wh);
 #pragma unroll
-            for (int q = 0; q < C / 4; ++q) {
+            for (int q = 0; q < 8; ++q) {
                 const float4 e4 = ev[q];
                 v[4 * q] *= e4.x * inv;
                 v[4 * q + 1] *= e4.y * inv;
                 v[4 * q + 2] *= e4.z * inv;
                 v[4 * q + 3] *= e4.w * inv;
             }
-            write_row64_bf16(tile + L::UT, tid, v);
+            write_row32_bf16(tile + L::UT, row, 4 * wh, v);
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
 
         // ---- S^T / sigma += U~^T K ;  prefill: O^T += U^T M^T ----
-        if (tid == 0) {
+        if (warp == 0) {
             tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tbase + TM_S, smem_desc_sw128(s_tile + L::UT + kk * 32, 16, 1024),
-                            smem_desc_sw128(s_tile + kk * 2048, L::K_BLK, 1024), id_s, 1u);
-            if (!REPLAY) {
+            if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ss(tbase + TM_O, smem_desc_sw128(s_ub + kk * 32, 16, 1024),
-                                smem_desc_sw128(s_mb + kk * 32, 16, 1024), id_o2, 1u);
+                    mma_bf16_ss(tbase + TM_S, smem_desc_sw128(s_tile + L::UT + kk * 32, 16, 1024),
+                                smem_desc_sw128(s_tile + kk * 2048, L::K_BLK, 1024), id_s, 1u);
+                if (!REPLAY) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ss(tbase + TM_O, smem_desc_sw128(s_ub + kk * 32, 16, 1024),
+                                    smem_desc_sw128(s_mb + kk * 32, 16, 1024), id_o2, 1u);
+                }
+                mma_commit(&bar_s);
             }
-            mma_commit(&bar_s);
+            __syncwarp();
         }
         o_r0 = r0;
         o_nc = nc;
@@ -548,15 +602,16 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         tc_fence_after();
         if (ok && !REPLAY) write_outputs(o_r0, o_nc);
     }
-    // ---- final state: S[dk][dv] = sigma * TMEM[lane dv][dk] ----
+    // ---- final state: S[dk][dv] = sigma * TMEM[lane dv][dk]; this thread writes keys
+    //      [64 wh, 64 wh + 64) of value column dv = row ----
     if (ok && a.state_out) {
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
+        for (int cb = 2 * wh; cb < 2 * wh + 2; ++cb) {
             float v[32];
             tmem_ld32(tlane + TM_S + cb * 32, v);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) a.state_out[state_base + (size_t)(cb * 32 + i) * D + tid] = sigma * v[i];
+            for (int i = 0; i < 32; ++i) a.state_out[state_base + (size_t)(cb * 32 + i) * D + row] = sigma * v[i];
         }
     }
     tc_fence_before();

@@ -153,12 +153,43 @@ __device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, ui
         : "memory");
 }
 
+// True in exactly one lane of a converged warp (elect.sync).  Single-thread
+// tcgen05.mma / TMA work is issued by the elected lane inside a warp-uniform
+// branch, so the operands stay warp-uniform; issuing from a `tid == 0` branch
+// instead measured about twice the cycles per MMA on sm_100a.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .b32 r;\n\t.reg .pred p;\n\t"
+        "elect.sync r|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 // Arrive once on `bar` when every tcgen05 operation this thread issued so far
 // has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                      smem_u32(bar))
                  : "memory");
+}
+
+// 16 lanes x 32 consecutive 32-bit columns spread over the whole warp
+// (shape 16x256b, four repeats): with t the thread's lane in the warp and q
+// the warp's lane-quarter base, register 4k + e holds lane q + t/4 + 8 (e/2),
+// column col + 8k + 2 (t%4) + (e%2).  This is the row layout of an M = 64
+// accumulator, whose rows sit in lanes 0..15 of each quarter.
+__device__ __forceinline__ void tmem_ld16x256b_x4(uint32_t taddr, float* v) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // 32 lanes x 32 consecutive 32-bit columns: thread i of the warp receives lane
