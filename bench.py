@@ -601,6 +601,117 @@ def bench_varlen(args):
              "data": "synthetic"}]
 
 
+def bench_decode(args):
+    """One decode step (the token after the prefill) of the 24-layer stack for 64 requests:
+    32 heads, d = 128, bf16 q/k/v/o, fp32 states updated in place.  The layers are folded into
+    the batch (24 x 64 = 1536 state slots, 6.4 GB of state, larger than L2), one launch."""
+    import gated_deltanet_state_tail_b200 as gdn
+    layers, B, H, d = 24, 64, 32, 128
+    nb = layers * B
+    t = inputs.draw_tensors(nb, H, d, d, "bf16", 0.9, 0.999, 7, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(8)
+    state = torch.randn((nb, H, d, d), generator=g, device="cuda") * 0.05
+    o = torch.empty((nb, H, d), dtype=torch.bfloat16, device="cuda")
+
+    def step():
+        gdn.gdn_decode_step(t["q"], t["k"], t["v"], t["alpha"], t["beta"], state, state, o)
+
+    for _ in range(args.warmup):
+        step()
+    ms = _time_ms(step, max(args.steps, 10))
+    nbytes = nb * H * (2 * d * d * 4 + 4 * d * 2 + 8)   # state read + write, q k v o, alpha beta
+    peaks = measured_peaks()
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return [{"metric": "GDN decode step (24 layers x 64 requests)", "value": ms, "unit": "ms",
+             "higher_is_better": False, "workload": "decode24-B64-H32-d128-bf16", "layers": layers,
+             "requests": B, "heads": H, "tokens_per_s": B / (ms / 1e3),
+             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                          "frac": gbs / peaks["hbm_gbs"], "traffic": None, "peak_source": peaks["source"],
+                          "bytes_per_launch": nbytes},
+             "l2": "6.4 GB of state per launch, larger than L2", "dtype": "bf16", "data": "synthetic"}]
+
+
+def bench_outputs(args):
+    """Replay with the window's outputs (layer chaining inside a replay group) against the
+    state-only replay, on one bench launch: 8 layers x 32 heads, R = 3277 rows each."""
+    import gated_deltanet_state_tail_b200 as gdn
+    layers, H, d, R = 8, 32, 128, 3277
+    t = inputs.draw_tensors(layers * R, H, d, d, "bf16", 0.9, 0.999, 9, device="cuda")
+    off = np.arange(layers + 1, dtype=np.int32) * R
+    plan = gdn.ReplayPlan(H, d, d, "bf16", off, [R] * layers, [R] * layers)
+    st = torch.empty((layers, H, d, d), device="cuda")
+    o = torch.empty((layers * R, H, d), dtype=torch.bfloat16, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    state_ms = _time_ms(lambda: plan.run(t["k"], t["v"], t["alpha"], t["beta"], st), 10, flush)
+    out_ms = _time_ms(lambda: plan.run_outputs(t["q"], t["k"], t["v"], t["alpha"], t["beta"], o,
+                                               state_out=st), 10, flush)
+    plan.check()
+    plan.close()
+    tokens = layers * R
+    return [{"metric": "replay with window outputs", "workload": "replay8-H32-d128-bf16-R3277",
+             "layers": layers, "heads": H, "R": R, "state_only_ms": state_ms, "with_outputs_ms": out_ms,
+             "with_outputs_tokens_per_s": tokens / (out_ms / 1e3), "dtype": "bf16", "data": "synthetic"}]
+
+
+def bench_overlap(args):
+    """Host-to-device copy of the full-attention layers' KV cache on a second stream while
+    the 24-layer tail replay runs on the first.  The pages give no FA-layer shape; the
+    8 FA layers of the 3:1 stack are taken as wide as the GDN layers (32 heads x 128,
+    K and V, bf16) at the 32K prefix: 8 x 32768 x 2 x 32 x 128 x 2 B = 4 GiB, pinned."""
+    import gated_deltanet_state_tail_b200 as gdn
+    wl = inputs.stack_workload(24)
+    data = StackData(wl, "cuda", compact=True)
+    rp, pp, state, o, st_out, _ = build_stack_runner(data, gdn.GDN_KERNEL_AUTO)
+    kv_bytes = 8 * wl.match_len[0] * 2 * wl.H * wl.dk * 2
+    host = torch.empty(kv_bytes, dtype=torch.uint8, pin_memory=True)
+    dev = torch.empty(kv_bytes, dtype=torch.uint8, device="cuda")
+    s_rep = torch.cuda.current_stream()
+    s_copy = torch.cuda.Stream()
+    per = data.per_launch
+
+    def replay():
+        for j, plan in enumerate(rp):
+            plan.run(data.k, data.v, data.alpha, data.beta, state[j * per:(j + 1) * per], stream=s_rep)
+
+    def timed(do_replay, do_copy):
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        er = torch.cuda.Event(enable_timing=True)
+        ec = torch.cuda.Event(enable_timing=True)
+        e0.record(s_rep)
+        s_copy.wait_event(e0)
+        if do_copy:
+            with torch.cuda.stream(s_copy):
+                dev.copy_(host, non_blocking=True)
+        ec.record(s_copy)
+        if do_replay:
+            replay()
+        er.record(s_rep)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(er), e0.elapsed_time(ec)
+
+    for _ in range(args.warmup):
+        timed(True, False)
+    timed(False, True)
+    reps = 5
+    t_rep = statistics.median(timed(True, False)[0] for _ in range(reps))
+    t_copy = statistics.median(timed(False, True)[1] for _ in range(reps))
+    both = [timed(True, True) for _ in range(reps)]
+    t_both = statistics.median(max(a, b) for a, b in both)
+    t_rep_in = statistics.median(a for a, _ in both)
+    for p in rp + pp:
+        p.check()
+        p.close()
+    hidden = max(0.0, min(1.0, (t_rep + t_copy - t_both) / min(t_rep, t_copy)))
+    return [{"metric": "transfer/replay overlap", "workload": "stack24 replay + FA-KV H2D (4 GiB)",
+             "fa_kv_bytes": kv_bytes, "replay_ms": t_rep, "copy_ms": t_copy, "both_ms": t_both,
+             "replay_ms_during_copy": t_rep_in, "h2d_gbs": kv_bytes / (t_copy / 1e3) / 1e9,
+             "hidden_fraction_of_shorter": hidden, "serial_ms": t_rep + t_copy,
+             "fa_kv_shape": "8 layers x 32768 tokens x (K, V) x 32 heads x 128 x bf16 (reading: FA layers "
+                            "as wide as the GDN layers, no head sharing)",
+             "dtype": "bf16", "data": "synthetic"}]
+
+
 # --------------------------------------------------------------------------
 # reference arm: the fp64 CPU oracle as it stands
 # --------------------------------------------------------------------------
@@ -640,8 +751,9 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="stack", choices=["stack", "sweep", "varlen"],
-                    help="stack = the bench line; sweep / varlen print auxiliary lines")
+    ap.add_argument("--workload", default="stack",
+                    choices=["stack", "sweep", "varlen", "decode", "outputs", "overlap"],
+                    help="stack = the bench line; the others print auxiliary lines")
     ap.add_argument("--layers", type=int, default=24,
                     help="GDN layers in the stack (a multiple of 3; 24 is the bench line, "
                          "fewer only for profiling captures)")
@@ -662,9 +774,11 @@ def main():
         return
 
     rank, world, local = dist_init(args.gpus)
-    if args.workload in ("sweep", "varlen"):
+    aux = {"sweep": bench_sweep, "varlen": bench_varlen, "decode": bench_decode, "outputs": bench_outputs,
+           "overlap": bench_overlap}
+    if args.workload in aux:
         if rank == 0:
-            for line in (bench_sweep(args) if args.workload == "sweep" else bench_varlen(args)):
+            for line in aux[args.workload](args):
                 print(json.dumps(line), flush=True)
         if world > 1:
             torch.distributed.destroy_process_group()

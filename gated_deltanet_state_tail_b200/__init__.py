@@ -6,7 +6,8 @@ memory and streams.  There is no CPU fallback: if the library is missing the
 import fails, and every call checks the status the library returns.
 
 The low-level names mirror the C entry points (``gdn_plan_create_replay``,
-``gdn_tail_replay_state``, ``gdn_chunk_prefill``, ...).  ``ReplayPlan`` and
+``gdn_tail_replay_state``, ``gdn_tail_replay_outputs``, ``gdn_chunk_prefill``,
+``gdn_decode_step``, ...).  ``ReplayPlan`` and
 ``PrefillPlan`` wrap a plan's lifetime; ``tail_replay_state`` and
 ``chunk_prefill`` are the one-call conveniences on torch tensors.
 """
@@ -30,6 +31,7 @@ EXPORTED = (
     "gdn_plan_window",
     "gdn_plan_info", "gdn_workspace_bytes", "gdn_tail_replay_state", "gdn_chunk_prefill",
     "gdn_workspace_status", "gdn_status_string", "gdn_version", "gdn_tail_replay_state_noalloc",
+    "gdn_tail_replay_outputs", "gdn_decode_step",
 )
 
 
@@ -73,6 +75,8 @@ def _load():
         "gdn_status_string": (ctypes.c_char_p, [I32]),
         "gdn_version": (I32, []),
         "gdn_tail_replay_state_noalloc": (I32, [pd, P, P, P, P, P, P, P, P, ctypes.POINTER(ctypes.c_uint32)]),
+        "gdn_tail_replay_outputs": (I32, [P, P, P, P, P, P, P, P, P, P, P, P, P]),
+        "gdn_decode_step": (I32, [I32, I32, I32, I32, I32, P, P, P, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -213,6 +217,27 @@ def gdn_tail_replay_state(handle, q, k, v, alpha, beta, seq_offsets, match_len, 
            "gdn_tail_replay_state")
 
 
+def gdn_tail_replay_outputs(handle, q, k, v, alpha, beta, seq_offsets, match_len, R, o_out, state_out,
+                            workspace, stream=None):
+    """Tail replay that also writes o_t = S_t^T q_t for every window row (rows of o_out
+    outside the windows are left untouched)."""
+    _check(_lib.gdn_tail_replay_outputs(handle, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+                                        _ptr(seq_offsets), _ptr(match_len), _ptr(R), _ptr(o_out),
+                                        _ptr(state_out), _ptr(workspace), _stream_handle(stream)),
+           "gdn_tail_replay_outputs")
+
+
+def gdn_decode_step(q, k, v, alpha, beta, state_in, state_out, o_out, stream=None):
+    """One decode step on dense [B, H, d] tensors (state [B, H, dk, dv] fp32; state_out may be
+    state_in for an in-place update)."""
+    B, H, dk = k.shape
+    dv = v.shape[2]
+    _check(_lib.gdn_decode_step(int(B), int(H), int(dk), int(dv), _dtype_code(k.dtype), _ptr(q), _ptr(k),
+                                _ptr(v), _ptr(alpha), _ptr(beta), _ptr(state_in), _ptr(state_out),
+                                _ptr(o_out), _stream_handle(stream)),
+           "gdn_decode_step")
+
+
 def gdn_chunk_prefill(handle, q, k, v, alpha, beta, cu_seqlens, state_in, o_out, state_out,
                       workspace, stream=None):
     _check(_lib.gdn_chunk_prefill(handle, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
@@ -283,6 +308,12 @@ class ReplayPlan(_Plan):
         gdn_tail_replay_state(self.handle, q, k, v, alpha, beta, seq_offsets, match_len, R,
                               state_out, self.workspace if workspace is None else workspace, stream)
 
+    def run_outputs(self, q, k, v, alpha, beta, o_out, state_out=None, seq_offsets=None, match_len=None,
+                    R=None, stream=None, workspace=None):
+        """Replay that also writes the window rows of o_out (see gdn_tail_replay_outputs)."""
+        gdn_tail_replay_outputs(self.handle, q, k, v, alpha, beta, seq_offsets, match_len, R, o_out,
+                                state_out, self.workspace if workspace is None else workspace, stream)
+
 
 class PrefillPlan(_Plan):
     """Plan of a chunked prefill over whole packed sequences (host cu_seqlens)."""
@@ -322,3 +353,14 @@ def chunk_prefill(q, k, v, alpha, beta, cu_seqlens, state_in=None, kernel=GDN_KE
     plan.check()
     plan.close()
     return o, st
+
+
+def decode_step(q, k, v, alpha, beta, state, o=None, in_place=True):
+    """One decode step on torch CUDA tensors ([B, H, d], state [B, H, dk, dv] fp32).
+    Updates `state` in place (or returns a new one) and returns (o, state)."""
+    import torch
+    if o is None:
+        o = torch.empty(v.shape, dtype=v.dtype, device=v.device)
+    out = state if in_place else torch.empty_like(state)
+    gdn_decode_step(q, k, v, alpha, beta, state, out, o)
+    return o, out

@@ -295,6 +295,74 @@ gdn_status gdn_tail_replay_state(gdn_plan_t plan, const void* q, const void* k, 
     return launch(plan, a, static_cast<cudaStream_t>(stream));
 }
 
+gdn_status gdn_tail_replay_outputs(gdn_plan_t plan, const void* q, const void* k, const void* v,
+                                   const float* alpha, const float* beta,
+                                   const int32_t* seq_offsets, const int32_t* match_len,
+                                   const int32_t* R, void* o_out, float* state_out, void* workspace,
+                                   void* stream) {
+    gdn_status s = check_call_common(plan, workspace);
+    if (s != GDN_OK) return s;
+    if (plan->kind != gdn::kReplay) return GDN_ERR_INVALID_ARG;
+    if (state_out && !aligned16(state_out)) return GDN_ERR_INVALID_ARG;
+    if (!o_out) return GDN_ERR_INVALID_ARG;   // selects the output-writing kernels
+    if (plan->total_tokens > 0) {
+        if (!q || !k || !v || !alpha || !beta) return GDN_ERR_INVALID_ARG;
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(alpha) || !aligned16(beta) ||
+            !aligned16(o_out))
+            return GDN_ERR_INVALID_ARG;
+    }
+    CallArgs a;
+    std::memset(&a, 0, sizeof a);
+    fill_common(plan, a, workspace);
+    a.chk_offsets = seq_offsets;
+    a.chk_match = match_len;
+    a.chk_budget = R;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.alpha = alpha;
+    a.beta = beta;
+    a.state_in = nullptr;
+    a.o_out = o_out;
+    a.state_out = state_out;
+    return launch(plan, a, static_cast<cudaStream_t>(stream));
+}
+
+gdn_status gdn_decode_step(int32_t batch, int32_t num_heads, int32_t d_k, int32_t d_v, int32_t dtype,
+                           const void* q, const void* k, const void* v, const float* alpha,
+                           const float* beta, const float* state_in, float* state_out, void* o_out,
+                           void* stream) {
+    if (batch < 0 || num_heads < 1) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
+    if ((d_k != 64 && d_k != 128) || (d_v != 64 && d_v != 128)) return GDN_ERR_UNSUPPORTED;
+    if ((long long)batch * num_heads > (1ll << 31) - 1) return GDN_ERR_INVALID_ARG;   // grid x
+    if (batch == 0) return GDN_OK;
+    if (!q || !k || !v || !alpha || !beta || !o_out) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(alpha) || !aligned16(beta) ||
+        !aligned16(o_out) || (state_in && !aligned16(state_in)) || (state_out && !aligned16(state_out)))
+        return GDN_ERR_INVALID_ARG;
+    gdn::DecodeArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.dtype = dtype;
+    a.num_heads = num_heads;
+    a.dk = d_k;
+    a.dv = d_v;
+    a.batch = batch;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.alpha = alpha;
+    a.beta = beta;
+    a.state_in = state_in;
+    a.state_out = state_out;
+    a.o_out = o_out;
+    if (gdn::launch_decode(a, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_CUDA;
+    }
+    return GDN_OK;
+}
+
 gdn_status gdn_chunk_prefill(gdn_plan_t plan, const void* q, const void* k, const void* v,
                              const float* alpha, const float* beta, const int32_t* cu_seqlens,
                              const float* state_in, void* o_out, float* state_out,
@@ -355,6 +423,6 @@ const char* gdn_status_string(gdn_status s) {
     return "unknown status";
 }
 
-int32_t gdn_version(void) { return 100; }
+int32_t gdn_version(void) { return 200; }
 
 }  // extern "C"

@@ -664,11 +664,17 @@ cudaError_t launch_chunk_tc(const CallArgs& a, cudaStream_t stream) {
     if (!chunk_tc_supported(a.dtype, a.dk, a.dv)) return cudaErrorInvalidValue;
     TcParams p;
     p.a = a;
-    const bool replay = a.kind == kReplay;
+    // the state-only instance unless outputs are asked for (a prefill, or a replay that
+    // also emits the window's outputs)
+    const bool replay = a.kind == kReplay && a.o_out == nullptr;
+    // a call with no rows to read (every window empty) still runs, to write the states;
+    // its tile maps are never read, so any aligned address stands in for a null buffer
+    const void* kb = a.k ? a.k : static_cast<const void*>(a.ws);
+    const void* vb = a.v ? a.v : static_cast<const void*>(a.ws);
+    const void* qb = replay ? kb : (a.q ? a.q : static_cast<const void*>(a.ws));
     CUtensorMap mk, mv, mq;
-    if (!a.k || !a.v || (!replay && !a.q)) return cudaErrorInvalidValue;
-    if (!make_tile_map(&mk, a.k, a.num_heads, a.rows_total) || !make_tile_map(&mv, a.v, a.num_heads, a.rows_total) ||
-        !make_tile_map(&mq, replay ? a.k : a.q, a.num_heads, a.rows_total))
+    if (!make_tile_map(&mk, kb, a.num_heads, a.rows_total) || !make_tile_map(&mv, vb, a.num_heads, a.rows_total) ||
+        !make_tile_map(&mq, qb, a.num_heads, a.rows_total))
         return cudaErrorInvalidValue;
     static bool attr_set[2] = {false, false};
     if (replay) {

@@ -64,7 +64,7 @@ struct CallArgs {
     const float* alpha;
     const float* beta;
     const float* state_in;  // null = zero state
-    void* o_out;            // null for replay
+    void* o_out;            // null = no outputs (the state-only replay)
     float* state_out;       // may be null for prefill
     WorkspaceHeader* ws;
 };
@@ -83,7 +83,25 @@ __device__ __forceinline__ bool window_agrees(const CallArgs& a, int b) {
     return true;
 }
 
+// One decode step over a dense batch (no plan): q, k [batch, H, dk]; v, o
+// [batch, H, dv]; alpha, beta [batch, H]; states [batch, H, dk, dv].
+struct DecodeArgs {
+    int dtype;              // 0 = fp32, 1 = bf16 (q, k, v, o)
+    int num_heads;
+    int dk, dv;
+    long long batch;
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* alpha;
+    const float* beta;
+    const float* state_in;  // null = zero state
+    float* state_out;       // may alias state_in; null = not written
+    void* o_out;
+};
+
 cudaError_t launch_recurrent(const CallArgs& a, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_chunk_tc(const CallArgs& a, cudaStream_t stream);
 bool chunk_tc_supported(int dtype, int dk, int dv);
 

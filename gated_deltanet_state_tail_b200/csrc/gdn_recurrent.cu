@@ -185,7 +185,7 @@ __global__ void __launch_bounds__(64 * (DK / 64), 3) recurrent_kernel(const Call
 template <typename T, int DK, int DV>
 cudaError_t launch_typed(const CallArgs& a, cudaStream_t stream) {
     dim3 grid((unsigned)a.units, DV / 64), block(64 * (DK / 64));
-    if (a.kind == kPrefill)
+    if (a.kind == kPrefill || a.o_out)   // outputs: a prefill, or a replay that emits them
         recurrent_kernel<T, DK, DV, true><<<grid, block, 0, stream>>>(a);
     else
         recurrent_kernel<T, DK, DV, false><<<grid, block, 0, stream>>>(a);

@@ -165,6 +165,53 @@ GDN_API gdn_status gdn_tail_replay_state(gdn_plan_t plan, const void* q, const v
                                  void* stream);
 
 /*
+ * Tail replay that also emits the replayed tokens' outputs: for every row t
+ * of sequence b's window, o_t = S_t^T q_t with S the state replayed from
+ * zero since the window's first row (the same states gdn_tail_replay_state
+ * rebuilds).  Within a group of GDN layers that Tail-Replay replays together
+ * ("Mecanismos Principais", item "Reconstrucao de Estado Independente": each
+ * group after a full-attention layer is rebuilt independently), these are
+ * the outputs a layer hands to the next one.
+ *   q            [rows, H, d_k] packed like k; required.
+ *   k, v, alpha, beta, seq_offsets, match_len, R
+ *                as for gdn_tail_replay_state.
+ *   o_out        [rows, H, d_v] in the plan's dtype, addressed like q: the
+ *                window rows are written, every other row is left untouched.
+ *   state_out    [batch, H, d_k, d_v] fp32, or NULL.
+ * It runs the output-writing kernels (the prefill ones, from a zero state),
+ * so it costs a prefill of the window rather than a state-only replay.
+ * Returns as gdn_tail_replay_state; INVALID_ARG for a prefill plan or a NULL
+ * o_out.
+ */
+GDN_API gdn_status gdn_tail_replay_outputs(gdn_plan_t plan, const void* q, const void* k, const void* v,
+                                           const float* alpha, const float* beta,
+                                           const int32_t* seq_offsets, const int32_t* match_len,
+                                           const int32_t* R, void* o_out, float* state_out,
+                                           void* workspace, void* stream);
+
+/*
+ * One decode step (the token after the prefill; the pages time the first
+ * one as TTFT, "Resultados"), for a dense batch with no plan:
+ *   S' = alpha (I - beta k k^T) S + beta k v^T,   o = S'^T q.
+ *   batch, num_heads, d_k, d_v, dtype
+ *                sizes (d in {64, 128}) and the element type of q, k, v, o.
+ *   q, k         [batch, H, d_k];  v, o_out: [batch, H, d_v]  (dtype).
+ *   alpha, beta  [batch, H] fp32.
+ *   state_in     [batch, H, d_k, d_v] fp32, or NULL for the zero state.
+ *   state_out    [batch, H, d_k, d_v] fp32, or NULL; may equal state_in
+ *                (updated in place).
+ *   stream       cudaStream_t.
+ * The step waits on nothing on the device, so it has no workspace and no
+ * device status.  batch = 0 launches nothing.  Returns GDN_OK,
+ * INVALID_ARG (null or misaligned pointers, batch < 0, H < 1), UNSUPPORTED
+ * (head dims or dtype) or CUDA.
+ */
+GDN_API gdn_status gdn_decode_step(int32_t batch, int32_t num_heads, int32_t d_k, int32_t d_v,
+                                   int32_t dtype, const void* q, const void* k, const void* v,
+                                   const float* alpha, const float* beta, const float* state_in,
+                                   float* state_out, void* o_out, void* stream);
+
+/*
  * Chunked prefill over each sequence of a prefill plan, continuing from
  * state_in, emitting o_t = S_t^T q_t for every row and the final state.
  *   q, k, v      packed rows, dtype of the plan.

@@ -95,6 +95,7 @@ def test_null_plan_calls_rejected():
     lib = gdn.library()
     assert lib.gdn_tail_replay_state(None, *([None] * 11)) == gdn.GDN_ERR_INVALID_ARG
     assert lib.gdn_chunk_prefill(None, *([None] * 11)) == gdn.GDN_ERR_INVALID_ARG
+    assert lib.gdn_tail_replay_outputs(None, *([None] * 12)) == gdn.GDN_ERR_INVALID_ARG
     assert lib.gdn_plan_window(None, 0, None, None) == gdn.GDN_ERR_INVALID_ARG
     assert lib.gdn_workspace_status(None, None) == gdn.GDN_ERR_INVALID_ARG
     lib.gdn_plan_destroy(None)
@@ -121,3 +122,24 @@ def test_replay_windows_edge_cases():
     assert list(row0) == [224, 256, 256] and list(ln) == [32, 0, 44]
     with pytest.raises(gdn.GdnError):
         gdn.gdn_replay_windows(off, [257, 0, 0], [1, 1, 1])
+
+
+@pytest.mark.parametrize("args,status", [
+    ((-1, 4, 128, 128, 1), "INVALID_ARG"),       # negative batch
+    ((2, 0, 128, 128, 1), "INVALID_ARG"),        # no heads
+    ((2, 4, 96, 128, 1), "UNSUPPORTED"),         # head dims
+    ((2, 4, 128, 32, 1), "UNSUPPORTED"),
+    ((2, 4, 128, 128, 5), "UNSUPPORTED"),        # dtype
+    ((2, 4, 128, 128, 1), "INVALID_ARG"),        # null buffers
+])
+def test_decode_step_rejected_before_any_device_work(args, status):
+    lib = gdn.library()
+    assert lib.gdn_decode_step(*args, *([None] * 9)) == getattr(gdn, "GDN_ERR_" + status)
+
+
+def test_decode_step_misaligned_rejected():
+    lib = gdn.library()
+    p = [4096] * 9
+    p[5] = 4100     # state_in not 16-byte aligned
+    assert lib.gdn_decode_step(2, 4, 128, 128, 1, *p) == gdn.GDN_ERR_INVALID_ARG
+    assert lib.gdn_decode_step(0, 4, 128, 128, 1, *([None] * 9)) == gdn.GDN_OK   # empty batch
