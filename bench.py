@@ -712,6 +712,46 @@ def bench_overlap(args):
              "dtype": "bf16", "data": "synthetic"}]
 
 
+def bench_fused(args):
+    """The 24-layer cache hit as 3 fused launches (replay window then suffix, 8 layers each)
+    against the 3 replay + 3 prefill launches of the bench line."""
+    import gated_deltanet_state_tail_b200 as gdn
+    wl = inputs.stack_workload(24)
+    data = StackData(wl, "cuda", compact=True)
+    rp, pp, state, o, st_out, _ = build_stack_runner(data, gdn.GDN_KERNEL_AUTO)
+    fp = []
+    for slots in data.launches:
+        off, ml, R = data.replay_desc(slots)
+        fp.append(gdn.FusedPlan(wl.H, wl.dk, wl.dv, wl.dtype, off, ml, R, data.suffix_cu(slots)))
+    per = data.per_launch
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    mid = torch.empty_like(state)
+
+    def separate():
+        run_step(data, rp, pp, state, o, st_out)
+
+    def fused():
+        for j, plan in enumerate(fp):
+            sl = slice(j * per, (j + 1) * per)
+            plan.run(data.k, data.v, data.alpha, data.beta, data.sq, data.sk, data.sv, data.sa, data.sb, o,
+                     st_out[sl], state_mid=mid[sl])
+
+    for _ in range(args.warmup):
+        separate()
+        fused()
+    sep_ms = _time_ms(separate, 10, flush)
+    ref = st_out.clone()
+    fused_ms = _time_ms(fused, 10, flush)
+    rel = float(((st_out - ref).norm() / ref.norm()).item())
+    for p in rp + pp + fp:
+        p.check()
+        p.close()
+    return [{"metric": "fused replay + suffix prefill", "workload": wl.name, "layers": wl.layers,
+             "separate_ms": sep_ms, "fused_ms": fused_ms, "launches_separate": 2 * len(data.launches),
+             "launches_fused": len(data.launches), "final_state_rel_diff_fused_vs_separate": rel,
+             "dtype": "bf16", "data": "synthetic"}]
+
+
 # --------------------------------------------------------------------------
 # reference arm: the fp64 CPU oracle as it stands
 # --------------------------------------------------------------------------
@@ -752,7 +792,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="stack",
-                    choices=["stack", "sweep", "varlen", "decode", "outputs", "overlap"],
+                    choices=["stack", "sweep", "varlen", "decode", "outputs", "overlap", "fused"],
                     help="stack = the bench line; the others print auxiliary lines")
     ap.add_argument("--layers", type=int, default=24,
                     help="GDN layers in the stack (a multiple of 3; 24 is the bench line, "
@@ -775,7 +815,7 @@ def main():
 
     rank, world, local = dist_init(args.gpus)
     aux = {"sweep": bench_sweep, "varlen": bench_varlen, "decode": bench_decode, "outputs": bench_outputs,
-           "overlap": bench_overlap}
+           "overlap": bench_overlap, "fused": bench_fused}
     if args.workload in aux:
         if rank == 0:
             for line in aux[args.workload](args):

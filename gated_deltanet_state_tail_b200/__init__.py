@@ -31,7 +31,7 @@ EXPORTED = (
     "gdn_plan_window",
     "gdn_plan_info", "gdn_workspace_bytes", "gdn_tail_replay_state", "gdn_chunk_prefill",
     "gdn_workspace_status", "gdn_status_string", "gdn_version", "gdn_tail_replay_state_noalloc",
-    "gdn_tail_replay_outputs", "gdn_decode_step",
+    "gdn_tail_replay_outputs", "gdn_decode_step", "gdn_plan_create_fused", "gdn_tail_replay_prefill",
 )
 
 
@@ -77,6 +77,8 @@ def _load():
         "gdn_tail_replay_state_noalloc": (I32, [pd, P, P, P, P, P, P, P, P, ctypes.POINTER(ctypes.c_uint32)]),
         "gdn_tail_replay_outputs": (I32, [P, P, P, P, P, P, P, P, P, P, P, P, P]),
         "gdn_decode_step": (I32, [I32, I32, I32, I32, I32, P, P, P, P, P, P, P, P, P]),
+        "gdn_plan_create_fused": (I32, [pd, P, P, P, ctypes.POINTER(P)]),
+        "gdn_tail_replay_prefill": (I32, [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -176,6 +178,19 @@ def gdn_plan_create_prefill(H, dk, dv, dtype, cu_seqlens, kernel=GDN_KERNEL_AUTO
     return h.value
 
 
+def gdn_plan_create_fused(H, dk, dv, dtype, seq_offsets, match_len, R, suffix_offsets,
+                          kernel=GDN_KERNEL_AUTO):
+    """Create a fused replay + suffix plan; returns the raw handle (int).  Host int arrays."""
+    off, ml, rr, so = _i32(seq_offsets), _i32(match_len), _i32(R), _i32(suffix_offsets)
+    if len(off) != len(ml) + 1 or len(rr) != len(ml) or len(so) != len(ml) + 1:
+        raise ValueError("seq_offsets and suffix_offsets need batch + 1 entries, match_len and R batch")
+    d = _make_desc(len(ml), H, dk, dv, dtype, kernel, off)
+    h = ctypes.c_void_p()
+    _check(_lib.gdn_plan_create_fused(ctypes.byref(d), ml.ctypes.data, rr.ctypes.data, so.ctypes.data,
+                                      ctypes.byref(h)), "gdn_plan_create_fused")
+    return h.value
+
+
 def gdn_replay_windows(seq_offsets, match_len, R):
     """Host-side replay windows: (row0 int64 [B], len int32 [B])."""
     off, ml, rr = _i32(seq_offsets), _i32(match_len), _i32(R)
@@ -225,6 +240,16 @@ def gdn_tail_replay_outputs(handle, q, k, v, alpha, beta, seq_offsets, match_len
                                         _ptr(seq_offsets), _ptr(match_len), _ptr(R), _ptr(o_out),
                                         _ptr(state_out), _ptr(workspace), _stream_handle(stream)),
            "gdn_tail_replay_outputs")
+
+
+def gdn_tail_replay_prefill(handle, k, v, alpha, beta, sq, sk, sv, salpha, sbeta, o_out, state_mid,
+                            state_out, workspace, stream=None):
+    """Fused rebuild of the states and prefill of the suffixes (one launch on the
+    tensor-core kernel)."""
+    _check(_lib.gdn_tail_replay_prefill(handle, _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(sq), _ptr(sk),
+                                        _ptr(sv), _ptr(salpha), _ptr(sbeta), _ptr(o_out), _ptr(state_mid),
+                                        _ptr(state_out), _ptr(workspace), _stream_handle(stream)),
+           "gdn_tail_replay_prefill")
 
 
 def gdn_decode_step(q, k, v, alpha, beta, state_in, state_out, o_out, stream=None):
@@ -326,6 +351,19 @@ class PrefillPlan(_Plan):
             stream=None, workspace=None):
         gdn_chunk_prefill(self.handle, q, k, v, alpha, beta, cu_seqlens, state_in, o_out, state_out,
                           self.workspace if workspace is None else workspace, stream)
+
+
+class FusedPlan(_Plan):
+    """Plan of a fused replay + suffix prefill (host int arrays)."""
+
+    def __init__(self, H, dk, dv, dtype, seq_offsets, match_len, R, suffix_offsets, kernel=GDN_KERNEL_AUTO):
+        h = gdn_plan_create_fused(H, dk, dv, dtype, seq_offsets, match_len, R, suffix_offsets, kernel)
+        super().__init__(h, H, dk, dv, dtype, len(match_len))
+
+    def run(self, k, v, alpha, beta, sq, sk, sv, salpha, sbeta, o_out, state_out, state_mid=None, stream=None,
+            workspace=None):
+        gdn_tail_replay_prefill(self.handle, k, v, alpha, beta, sq, sk, sv, salpha, sbeta, o_out, state_mid,
+                                state_out, self.workspace if workspace is None else workspace, stream)
 
 
 def tail_replay_state(k, v, alpha, beta, seq_offsets, match_len, R, kernel=GDN_KERNEL_AUTO):

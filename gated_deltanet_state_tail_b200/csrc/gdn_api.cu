@@ -25,12 +25,15 @@ struct gdn_plan {
     int kind;
     int batch, num_heads, dk, dv, dtype, kernel;
     int device;
-    std::vector<Window> windows;
+    std::vector<Window> windows;   // replay: the tail windows; prefill and fused: the (suffix) sequences
+    std::vector<Window> windows0;  // fused: the replay windows run before `windows`
     std::vector<Unit> units;
     long long total_tokens;
-    long long rows_total;     // seq_offsets[batch]
-    void* dev_block;          // windows then units
+    long long rows_total;     // rows the windows address (max end offset)
+    long long rows_total0;    // fused: rows the replay windows address
+    void* dev_block;          // windows, windows0, then units
     Window* d_windows;
+    Window* d_windows0;
     Unit* d_units;
 };
 
@@ -66,26 +69,36 @@ gdn_status finish_plan(gdn_plan* p, gdn_plan_t* out) {
     p->units.reserve((size_t)p->batch * p->num_heads);
     for (int b = 0; b < p->batch; ++b)
         for (int h = 0; h < p->num_heads; ++h) p->units.push_back(Unit{b, h});
-    std::stable_sort(p->units.begin(), p->units.end(), [p](const Unit& x, const Unit& y) {
-        return p->windows[x.seq].len > p->windows[y.seq].len;
-    });
+    auto unit_len = [p](int b) {
+        return (long long)p->windows[b].len + (p->windows0.empty() ? 0 : p->windows0[b].len);
+    };
+    std::stable_sort(p->units.begin(), p->units.end(),
+                     [&unit_len](const Unit& x, const Unit& y) { return unit_len(x.seq) > unit_len(y.seq); });
     p->total_tokens = 0;
     p->rows_total = 0;
+    p->rows_total0 = 0;
     for (const Window& w : p->windows) {
         p->total_tokens += w.len;
         p->rows_total = std::max(p->rows_total, (long long)w.expect_end);
     }
+    for (const Window& w : p->windows0) {
+        p->total_tokens += w.len;
+        p->rows_total0 = std::max(p->rows_total0, (long long)w.expect_end);
+    }
 
     if (cudaGetDevice(&p->device) != cudaSuccess) return GDN_ERR_CUDA;
     const size_t wbytes = sizeof(Window) * p->windows.size();
+    const size_t w0bytes = sizeof(Window) * p->windows0.size();
     const size_t ubytes = sizeof(Unit) * p->units.size();
-    if (cudaMalloc(&p->dev_block, wbytes + ubytes) != cudaSuccess) {
+    if (cudaMalloc(&p->dev_block, wbytes + w0bytes + ubytes) != cudaSuccess) {
         cudaGetLastError();
         return GDN_ERR_ALLOC;
     }
     p->d_windows = static_cast<Window*>(p->dev_block);
-    p->d_units = reinterpret_cast<Unit*>(static_cast<char*>(p->dev_block) + wbytes);
+    p->d_windows0 = w0bytes ? reinterpret_cast<Window*>(static_cast<char*>(p->dev_block) + wbytes) : nullptr;
+    p->d_units = reinterpret_cast<Unit*>(static_cast<char*>(p->dev_block) + wbytes + w0bytes);
     if (cudaMemcpy(p->d_windows, p->windows.data(), wbytes, cudaMemcpyHostToDevice) != cudaSuccess ||
+        (w0bytes && cudaMemcpy(p->d_windows0, p->windows0.data(), w0bytes, cudaMemcpyHostToDevice) != cudaSuccess) ||
         cudaMemcpy(p->d_units, p->units.data(), ubytes, cudaMemcpyHostToDevice) != cudaSuccess) {
         cudaFree(p->dev_block);
         p->dev_block = nullptr;
@@ -119,7 +132,38 @@ gdn_plan* new_plan(const gdn_varlen_desc* d, int kind) {
     p->dtype = d->dtype;
     p->kernel = resolve_kernel(d);
     p->dev_block = nullptr;
+    p->d_windows0 = nullptr;
     return p;
+}
+
+void fill_replay_windows(std::vector<Window>& win, int batch, const int32_t* off, const int32_t* match_len,
+                         const int32_t* R) {
+    win.resize(batch);
+    std::vector<int64_t> row0(batch);
+    std::vector<int32_t> len(batch);
+    gdn_replay_windows(batch, off, match_len, R, row0.data(), len.data());
+    for (int b = 0; b < batch; ++b) {
+        Window& w = win[b];
+        std::memset(&w, 0, sizeof w);
+        w.row0 = row0[b];   // R > L clamps to L; R = 0 is the Zero-Only state
+        w.len = len[b];
+        w.expect_off = off[b];
+        w.expect_end = off[b + 1];
+        w.expect_match = match_len[b];
+        w.expect_budget = R[b];
+    }
+}
+
+void fill_sequence_windows(std::vector<Window>& win, int batch, const int32_t* off) {
+    win.resize(batch);
+    for (int b = 0; b < batch; ++b) {
+        Window& w = win[b];
+        std::memset(&w, 0, sizeof w);
+        w.row0 = off[b];
+        w.len = off[b + 1] - off[b];
+        w.expect_off = off[b];
+        w.expect_end = off[b + 1];
+    }
 }
 
 gdn_status check_call_common(gdn_plan_t plan, void* workspace) {
@@ -178,21 +222,7 @@ gdn_status gdn_plan_create_replay(const gdn_varlen_desc* cache, const int32_t* m
         return GDN_ERR_UNSUPPORTED;
     gdn_plan* p = new_plan(cache, gdn::kReplay);
     if (!p) return GDN_ERR_ALLOC;
-    p->windows.resize(cache->batch);
-    std::vector<int64_t> row0(cache->batch);
-    std::vector<int32_t> len(cache->batch);
-    gdn_replay_windows(cache->batch, off, match_len_host, R_host, row0.data(), len.data());
-    for (int b = 0; b < cache->batch; ++b) {
-        const int L = match_len_host[b];
-        Window& w = p->windows[b];
-        std::memset(&w, 0, sizeof w);
-        w.row0 = row0[b];   // R > L clamps to L; R = 0 is the Zero-Only state
-        w.len = len[b];
-        w.expect_off = off[b];
-        w.expect_end = off[b + 1];
-        w.expect_match = L;
-        w.expect_budget = R_host[b];
-    }
+    fill_replay_windows(p->windows, cache->batch, off, match_len_host, R_host);
     s = finish_plan(p, out);
     if (s != GDN_OK) delete p;
     return s;
@@ -208,16 +238,33 @@ gdn_status gdn_plan_create_prefill(const gdn_varlen_desc* seqs, gdn_plan_t* out)
         return GDN_ERR_UNSUPPORTED;
     gdn_plan* p = new_plan(seqs, gdn::kPrefill);
     if (!p) return GDN_ERR_ALLOC;
-    const int32_t* off = seqs->seq_offsets_host;
-    p->windows.resize(seqs->batch);
-    for (int b = 0; b < seqs->batch; ++b) {
-        Window& w = p->windows[b];
-        std::memset(&w, 0, sizeof w);
-        w.row0 = off[b];
-        w.len = off[b + 1] - off[b];
-        w.expect_off = off[b];
-        w.expect_end = off[b + 1];
-    }
+    fill_sequence_windows(p->windows, seqs->batch, seqs->seq_offsets_host);
+    s = finish_plan(p, out);
+    if (s != GDN_OK) delete p;
+    return s;
+}
+
+gdn_status gdn_plan_create_fused(const gdn_varlen_desc* cache, const int32_t* match_len_host,
+                                 const int32_t* R_host, const int32_t* suffix_offsets_host, gdn_plan_t* out) {
+    if (!out) return GDN_ERR_INVALID_ARG;
+    *out = nullptr;
+    gdn_status s = check_desc(cache);
+    if (s != GDN_OK) return s;
+    if (!match_len_host || !R_host || !suffix_offsets_host) return GDN_ERR_INVALID_ARG;
+    const int32_t* off = cache->seq_offsets_host;
+    s = check_replay_arrays(cache->batch, off, match_len_host, R_host);
+    if (s != GDN_OK) return s;
+    gdn_varlen_desc suf = *cache;   // same batch, heads, dims, dtype and kernel; suffix offsets
+    suf.seq_offsets_host = suffix_offsets_host;
+    s = check_desc(&suf);
+    if (s != GDN_OK) return s;
+    if (resolve_kernel(cache) == GDN_KERNEL_CHUNKED_TC &&
+        !gdn::chunk_tc_supported(cache->dtype, cache->d_k, cache->d_v))
+        return GDN_ERR_UNSUPPORTED;
+    gdn_plan* p = new_plan(cache, gdn::kFused);
+    if (!p) return GDN_ERR_ALLOC;
+    fill_replay_windows(p->windows0, cache->batch, off, match_len_host, R_host);
+    fill_sequence_windows(p->windows, cache->batch, suffix_offsets_host);
     s = finish_plan(p, out);
     if (s != GDN_OK) delete p;
     return s;
@@ -246,8 +293,9 @@ void gdn_plan_destroy(gdn_plan_t plan) {
 
 gdn_status gdn_plan_window(gdn_plan_t plan, int32_t b, int64_t* row0, int32_t* len) {
     if (!plan || !row0 || !len || b < 0 || b >= plan->batch) return GDN_ERR_INVALID_ARG;
-    *row0 = plan->windows[b].row0;
-    *len = plan->windows[b].len;
+    const Window& w = plan->kind == gdn::kFused ? plan->windows0[b] : plan->windows[b];
+    *row0 = w.row0;
+    *len = w.len;
     return GDN_OK;
 }
 
@@ -391,6 +439,85 @@ gdn_status gdn_chunk_prefill(gdn_plan_t plan, const void* q, const void* k, cons
     a.o_out = o_out;
     a.state_out = state_out;
     return launch(plan, a, static_cast<cudaStream_t>(stream));
+}
+
+gdn_status gdn_tail_replay_prefill(gdn_plan_t plan, const void* k, const void* v, const float* alpha,
+                                   const float* beta, const void* sq, const void* sk, const void* sv,
+                                   const float* salpha, const float* sbeta, void* o_out, float* state_mid,
+                                   float* state_out, void* workspace, void* stream) {
+    gdn_status s = check_call_common(plan, workspace);
+    if (s != GDN_OK) return s;
+    if (plan->kind != gdn::kFused) return GDN_ERR_INVALID_ARG;
+    if (!state_out || !aligned16(state_out) || (state_mid && !aligned16(state_mid))) return GDN_ERR_INVALID_ARG;
+    long long win_tokens = 0, suf_tokens = 0;
+    for (const Window& w : plan->windows0) win_tokens += w.len;
+    for (const Window& w : plan->windows) suf_tokens += w.len;
+    if (win_tokens > 0) {
+        if (!k || !v || !alpha || !beta) return GDN_ERR_INVALID_ARG;
+        if (!aligned16(k) || !aligned16(v) || !aligned16(alpha) || !aligned16(beta)) return GDN_ERR_INVALID_ARG;
+    }
+    if (suf_tokens > 0) {
+        if (!sq || !sk || !sv || !salpha || !sbeta || !o_out) return GDN_ERR_INVALID_ARG;
+        if (!aligned16(sq) || !aligned16(sk) || !aligned16(sv) || !aligned16(salpha) || !aligned16(sbeta) ||
+            !aligned16(o_out))
+            return GDN_ERR_INVALID_ARG;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    CallArgs a;
+    std::memset(&a, 0, sizeof a);
+    fill_common(plan, a, workspace);
+    if (plan->kernel == GDN_KERNEL_CHUNKED_TC) {
+        // one launch: window chunks, then suffix chunks, the state kept on chip
+        a.kind = gdn::kFused;
+        a.q = sq;
+        a.k = sk;
+        a.v = sv;
+        a.alpha = salpha;
+        a.beta = sbeta;
+        a.o_out = o_out;
+        a.state_out = state_out;
+        a.windows0 = plan->d_windows0;
+        a.rows_total0 = plan->rows_total0;
+        a.k0 = k;
+        a.v0 = v;
+        a.alpha0 = alpha;
+        a.beta0 = beta;
+        a.state_mid = state_mid;
+        return launch(plan, a, st);
+    }
+    // the exact fp32 recurrent kernel: the same results as a replay launch then a prefill launch
+    if (cudaMemsetAsync(a.ws, 0, sizeof(WorkspaceHeader), st) != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_CUDA;
+    }
+    float* mid = state_mid ? state_mid : state_out;
+    a.kind = gdn::kReplay;
+    a.windows = plan->d_windows0;
+    a.rows_total = plan->rows_total0;
+    a.k = k;
+    a.v = v;
+    a.alpha = alpha;
+    a.beta = beta;
+    a.state_out = mid;
+    if (gdn::launch_recurrent(a, st) != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_CUDA;
+    }
+    fill_common(plan, a, workspace);
+    a.kind = gdn::kPrefill;
+    a.q = sq;
+    a.k = sk;
+    a.v = sv;
+    a.alpha = salpha;
+    a.beta = sbeta;
+    a.state_in = mid;
+    a.o_out = o_out;
+    a.state_out = state_out;
+    if (gdn::launch_recurrent(a, st) != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_CUDA;
+    }
+    return GDN_OK;
 }
 
 gdn_status gdn_workspace_status(const void* workspace, void* stream) {

@@ -142,16 +142,17 @@ __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, const C
     return ok;
 }
 
+// TMA of one chunk's tiles: K and V, and Q when the chunk writes outputs.
 template <bool REPLAY>
 __device__ __forceinline__ void issue_tiles(uint8_t* tile, uint64_t* bar, const CUtensorMap* mk, const CUtensorMap* mv,
-                                            const CUtensorMap* mq, int h, int r0) {
+                                            const CUtensorMap* mq, int h, int r0, bool with_q) {
     using L = Layout<REPLAY>;
-    mbar_arrive_expect_tx(bar, L::TILE);
+    mbar_arrive_expect_tx(bar, (!REPLAY && with_q) ? L::TILE : 32768u);
     tma_load_3d(tile, mk, bar, 0, h, r0);
     tma_load_3d(tile + L::K_BLK, mk, bar, 64, h, r0);
     tma_load_3d(tile + L::V0, mv, bar, 0, h, r0);
     tma_load_3d(tile + L::V0 + L::V_LBO, mv, bar, 64, h, r0);
-    if (!REPLAY) {
+    if (!REPLAY && with_q) {
         tma_load_3d(tile + L::Q0, mq, bar, 0, h, r0);
         tma_load_3d(tile + L::Q0 + 16384, mq, bar, 64, h, r0);
     }
@@ -160,7 +161,8 @@ __device__ __forceinline__ void issue_tiles(uint8_t* tile, uint64_t* bar, const 
 template <bool REPLAY>
 __global__ void __launch_bounds__(NT, REPLAY ? 2 : 1)
 chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
-                const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_q) {
+                const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_q,
+                const __grid_constant__ CUtensorMap map_k0, const __grid_constant__ CUtensorMap map_v0) {
     using L = Layout<REPLAY>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -182,8 +184,36 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         if (tid == 0) atomicOr(&a.ws->status, kStatusMismatch);
         return;
     }
+    // Chunk stream of this unit.  Prefill: the rows of a.windows[b], with outputs.  Fused
+    // replay + suffix: first the replay window a.windows0[b] (cache rows, no outputs), then
+    // the suffix a.windows[b] with outputs, the state staying in TMEM across the boundary.
     const Window w = a.windows[b];
-    const int nchunks = (w.len + C - 1) / C;
+    const bool fused = !REPLAY && a.windows0 != nullptr;
+    Window w0;
+    w0.row0 = 0;
+    w0.len = 0;
+    if (fused) w0 = a.windows0[b];
+    const int nA = (w0.len + C - 1) / C;                  // chunks without outputs (fused only)
+    const int nchunks = nA + (w.len + C - 1) / C;
+    struct ChunkSrc {
+        long long r0;   // first row
+        int nc;         // rows in the window (the rest are identity padding)
+        bool out;       // writes outputs (prefill rows)
+    };
+    auto chunk_src = [&](int cc) -> ChunkSrc {
+        if (cc < nA) return ChunkSrc{w0.row0 + (long long)cc * C, min(C, w0.len - cc * C), false};
+        const int k = cc - nA;
+        return ChunkSrc{w.row0 + (long long)k * C, min(C, w.len - k * C), !REPLAY};
+    };
+    auto issue_chunk = [&](int cc, int slot) {
+        const ChunkSrc cs = chunk_src(cc);
+        if (cs.out || REPLAY)
+            issue_tiles<REPLAY>(sm + L::OFF_TILE + slot * L::TILE, &bar_tile[slot], &map_k, &map_v, &map_q, h,
+                                (int)cs.r0, cs.out);
+        else
+            issue_tiles<REPLAY>(sm + L::OFF_TILE + slot * L::TILE, &bar_tile[slot], &map_k0, &map_v0, &map_q, h,
+                                (int)cs.r0, false);
+    };
 
     if (tid == 0) {
         mbar_init(&bar_tile[0], 1);
@@ -195,6 +225,10 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         tma_prefetch_desc(&map_k);
         tma_prefetch_desc(&map_v);
         if (!REPLAY) tma_prefetch_desc(&map_q);
+        if (fused) {
+            tma_prefetch_desc(&map_k0);
+            tma_prefetch_desc(&map_v0);
+        }
     }
     if (warp == 0) {
         tmem_alloc(&tmem_slot, kTmemCols);
@@ -205,8 +239,7 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     tc_fence_after();
     const uint32_t tbase = tmem_slot;
     const uint32_t tlane = tbase + ((uint32_t)(wq * 32) << 16);   // this warp's lane quarter, column 0
-    if (tid == 0 && nchunks > 0)
-        issue_tiles<REPLAY>(sm + L::OFF_TILE, &bar_tile[0], &map_k, &map_v, &map_q, h, (int)w.row0);
+    if (tid == 0 && nchunks > 0) issue_chunk(0, 0);
 
     float* AT = reinterpret_cast<float*>(sm + L::OFF_AT);
     float* Xs = reinterpret_cast<float*>(sm + L::OFF_X);
@@ -247,9 +280,14 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     auto load_gates = [&](int cc, float& al, float& be) {
         al = 1.0f;
         be = 0.0f;
-        if (tid < C && cc * C + tid < w.len) {
-            al = a.alpha[(w.row0 + (long long)cc * C + tid) * H + h];
-            be = a.beta[(w.row0 + (long long)cc * C + tid) * H + h];
+        if (tid < C && cc < nchunks) {
+            const ChunkSrc cs = chunk_src(cc);
+            if (tid < cs.nc) {
+                const float* pa = cc < nA ? a.alpha0 : a.alpha;
+                const float* pb = cc < nA ? a.beta0 : a.beta;
+                al = pa[(cs.r0 + tid) * H + h];
+                be = pb[(cs.r0 + tid) * H + h];
+            }
         }
     };
     // Wait for chunk cc's tiles and zero the rows past the window.
@@ -257,7 +295,7 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         const int slot = cc & 1;
         uint8_t* tile = sm + L::OFF_TILE + slot * L::TILE;
         if (!wait_all(&bar_tile[slot], (cc >> 1) & 1, a, 1)) return false;
-        const int ncc = min(C, w.len - cc * C);
+        const int ncc = chunk_src(cc).nc;
         if (ncc < C) {   // padded tokens are identity transitions: zero their rows
             const int nrows = C - ncc;
             const int nbox = REPLAY ? 4 : 6;
@@ -278,6 +316,18 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             const uint32_t off = (kk >> 2) * L::K_BLK + (kk & 3) * 32;
             mma_bf16_ss(tbase + TM_P, smem_desc_sw128(st + off, 16, 1024), smem_desc_sw128(st + off, 16, 1024),
                         id_kk, kk > 0);
+        }
+    };
+    // sigma * TMEM state -> dst[b][h] (fp32 [dk][dv]); this thread writes keys
+    // [64 wh, 64 wh + 64) of value column dv = row
+    auto write_state = [&](float* dst) {
+#pragma unroll
+        for (int cb = 2 * wh; cb < 2 * wh + 2; ++cb) {
+            float v[32];
+            tmem_ld32(tlane + TM_S + cb * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) dst[state_base + (size_t)(cb * 32 + i) * D + row] = sigma * v[i];
         }
     };
     auto write_outputs = [&](long long orow, int onc) {   // prefill: O of a finished chunk
@@ -312,11 +362,15 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     }
     long long o_r0 = 0;
     int o_nc = 0;
+    bool o_prev = false;   // the previous chunk wrote outputs
+    if (fused && nA == 0 && a.state_mid) write_state(a.state_mid);   // empty window: S at L is zero
 
     for (int c = 0; c < nchunks && ok; ++c) {
         const int slot = c & 1;
-        const long long r0 = w.row0 + (long long)c * C;
-        const int nc = min(C, w.len - c * C);
+        const ChunkSrc src = chunk_src(c);
+        const long long r0 = src.r0;
+        const int nc = src.nc;
+        const bool outc = !REPLAY && src.out;   // uniform: this chunk computes and writes outputs
         uint8_t* tile = sm + L::OFF_TILE + slot * L::TILE;
         const uint32_t s_tile = smem_u32(tile);
         Gates& G = s_gates[c & 1];
@@ -329,7 +383,8 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             ph_s ^= 1;
             if (!ok) break;
             tc_fence_after();
-            write_outputs(o_r0, o_nc);
+            if (o_prev) write_outputs(o_r0, o_nc);
+            if (fused && c == nA && a.state_mid) write_state(a.state_mid);   // the replayed state at L
         }
 
         // ---- epilogue 1: A = strict_tril(beta_i (gamma_i / gamma_j) K K^T) (fp32, in AT);
@@ -364,7 +419,7 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                     *reinterpret_cast<float2*>(AT + i * LDT + j) = make_float2(x0, x1);
                 }
             }
-        } else {
+        } else if (row < C || outc) {   // warp-uniform; Q rows only when the chunk writes outputs
             // [K; Q] K^T: lane r < 64 is K row r, lane r >= 64 is Q row r - 64; this thread
             // takes columns [32 wh, 32 wh + 32) of its lane
             float v[32];
@@ -420,9 +475,7 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                     slot_free = mbar_wait_bounded(&bar_s, ph_s_prev, kWaitNs);
                     if (!slot_free) report_timeout(a, 6);
                 }
-                if (slot_free)
-                    issue_tiles<REPLAY>(sm + L::OFF_TILE + (slot ^ 1) * L::TILE, &bar_tile[slot ^ 1], &map_k, &map_v,
-                                        &map_q, h, (int)(r0 + C));
+                if (slot_free) issue_chunk(c + 1, slot ^ 1);
             }
             __syncwarp();
         }
@@ -470,7 +523,7 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj)
                 *reinterpret_cast<float*>(bu + sw128_offset_f32(32 * wh + jj, lane)) = ns * v[jj];
-            if (!REPLAY) {
+            if (outc) {
                 const int i = tid >> 2, qk = tid & 3;           // row i, keys [32 qk, 32 qk + 32)
                 const uint8_t* qb = tile + L::Q0 + (qk >> 1) * 16384;
                 uint8_t* blk = sm + L::OFF_BQ + qk * 8192;
@@ -511,7 +564,7 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 for (int kk = 0; kk < 16; ++kk)
                     mma_tf32_ts(tbase + TM_U, tbase + TM_S + kk * 8,
                                 smem_desc_sw128(s_bu + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_u, 1u);
-                if (!REPLAY) {
+                if (outc) {
 #pragma unroll
                     for (int kk = 0; kk < 16; ++kk)
                         mma_tf32_ts(tbase + TM_O, tbase + TM_S + kk * 8,
@@ -542,7 +595,7 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             float v[32];                                        // value dv = row, chunk rows [32 wh, 32 wh + 32)
             tmem_ld32(tlane + TM_U + 32 * wh, v);
             tmem_wait_ld();
-            if (!REPLAY) write_row32_bf16(sm + L::OFF_UB, row, 4 * wh, v);
+            if (outc) write_row32_bf16(sm + L::OFF_UB, row, 4 * wh, v);
             float snew = sigma * G.gam[C - 1];
             if (snew < kRenormBelow) {     // uniform: fold the scale into the TMEM state
 #pragma unroll
@@ -582,7 +635,7 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 for (int kk = 0; kk < 4; ++kk)
                     mma_bf16_ss(tbase + TM_S, smem_desc_sw128(s_tile + L::UT + kk * 32, 16, 1024),
                                 smem_desc_sw128(s_tile + kk * 2048, L::K_BLK, 1024), id_s, 1u);
-                if (!REPLAY) {
+                if (outc) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_bf16_ss(tbase + TM_O, smem_desc_sw128(s_ub + kk * 32, 16, 1024),
@@ -594,26 +647,19 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         }
         o_r0 = r0;
         o_nc = nc;
+        o_prev = outc;
     }
 
     // ---- drain: the last state update (and outputs) ----
     if (ok && nchunks > 0) {
         ok = wait_all(&bar_s, ph_s, a, 5);
         tc_fence_after();
-        if (ok && !REPLAY) write_outputs(o_r0, o_nc);
+        if (ok && o_prev) write_outputs(o_r0, o_nc);
     }
-    // ---- final state: S[dk][dv] = sigma * TMEM[lane dv][dk]; this thread writes keys
-    //      [64 wh, 64 wh + 64) of value column dv = row ----
-    if (ok && a.state_out) {
-#pragma unroll
-        for (int cb = 2 * wh; cb < 2 * wh + 2; ++cb) {
-            float v[32];
-            tmem_ld32(tlane + TM_S + cb * 32, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) a.state_out[state_base + (size_t)(cb * 32 + i) * D + row] = sigma * v[i];
-        }
-    }
+    // fused with an empty suffix: the state at L is the final state
+    if (ok && fused && nA > 0 && nA == nchunks && a.state_mid) write_state(a.state_mid);
+    // ---- final state: S[dk][dv] = sigma * TMEM[lane dv][dk] ----
+    if (ok && a.state_out) write_state(a.state_out);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -676,6 +722,15 @@ cudaError_t launch_chunk_tc(const CallArgs& a, cudaStream_t stream) {
     if (!make_tile_map(&mk, kb, a.num_heads, a.rows_total) || !make_tile_map(&mv, vb, a.num_heads, a.rows_total) ||
         !make_tile_map(&mq, qb, a.num_heads, a.rows_total))
         return cudaErrorInvalidValue;
+    // fused replay + suffix: maps of the replayed cache rows (otherwise unused copies)
+    CUtensorMap mk0 = mk, mv0 = mv;
+    if (a.windows0) {
+        const void* kb0 = a.k0 ? a.k0 : static_cast<const void*>(a.ws);
+        const void* vb0 = a.v0 ? a.v0 : static_cast<const void*>(a.ws);
+        if (!make_tile_map(&mk0, kb0, a.num_heads, a.rows_total0) ||
+            !make_tile_map(&mv0, vb0, a.num_heads, a.rows_total0))
+            return cudaErrorInvalidValue;
+    }
     static bool attr_set[2] = {false, false};
     if (replay) {
         const uint32_t smem = Layout<true>::BYTES + 1024;
@@ -684,7 +739,7 @@ cudaError_t launch_chunk_tc(const CallArgs& a, cudaStream_t stream) {
             if (e != cudaSuccess) return e;
             attr_set[0] = true;
         }
-        chunk_tc_kernel<true><<<(unsigned)a.units, NT, smem, stream>>>(p, mk, mv, mq);
+        chunk_tc_kernel<true><<<(unsigned)a.units, NT, smem, stream>>>(p, mk, mv, mq, mk0, mv0);
     } else {
         const uint32_t smem = Layout<false>::BYTES + 1024;
         if (!attr_set[1]) {
@@ -692,7 +747,7 @@ cudaError_t launch_chunk_tc(const CallArgs& a, cudaStream_t stream) {
             if (e != cudaSuccess) return e;
             attr_set[1] = true;
         }
-        chunk_tc_kernel<false><<<(unsigned)a.units, NT, smem, stream>>>(p, mk, mv, mq);
+        chunk_tc_kernel<false><<<(unsigned)a.units, NT, smem, stream>>>(p, mk, mv, mq, mk0, mv0);
     }
     return cudaGetLastError();
 }

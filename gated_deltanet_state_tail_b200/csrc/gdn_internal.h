@@ -41,7 +41,8 @@ static_assert(sizeof(WorkspaceHeader) == 256, "header is 256 bytes");
 constexpr unsigned int kStatusMismatch = 1u;
 constexpr unsigned int kStatusTimeout = 2u;
 
-enum PlanKind { kReplay = 0, kPrefill = 1 };
+// kFused: the replay window of each sequence, then its suffix with outputs, in one launch
+enum PlanKind { kReplay = 0, kPrefill = 1, kFused = 2 };
 
 // Everything a kernel needs for one call.
 struct CallArgs {
@@ -67,6 +68,15 @@ struct CallArgs {
     void* o_out;            // null = no outputs (the state-only replay)
     float* state_out;       // may be null for prefill
     WorkspaceHeader* ws;
+    // fused replay + suffix (chunked kernel): a first segment of rows per sequence,
+    // replayed from the zero state without outputs before the rows of `windows`
+    const Window* windows0; // [batch] or null
+    long long rows_total0;  // rows of the buffers the first segment addresses
+    const void* k0;
+    const void* v0;
+    const float* alpha0;
+    const float* beta0;
+    float* state_mid;       // null, or [batch, H, dk, dv]: the state after the first segment
 };
 
 // Device-side check of one unit's window against the caller's descriptor

@@ -115,6 +115,22 @@ GDN_API gdn_status gdn_plan_create_replay(const gdn_varlen_desc* cache, const in
  */
 GDN_API gdn_status gdn_plan_create_prefill(const gdn_varlen_desc* seqs, gdn_plan_t* out);
 
+/*
+ * Build the schedule of a fused rebuild + suffix prefill: for each sequence,
+ * the replay window of gdn_plan_create_replay (from a zero state, no
+ * outputs), then the sequence's new suffix with outputs, continuing from the
+ * replayed state (the pages' cache hit: "Mecanismos Principais" rebuilds the
+ * state, "Resultados" times the suffix prefill that follows).
+ *   cache, match_len_host, R_host   as for gdn_plan_create_replay.
+ *   suffix_offsets_host             [batch + 1] row offsets of the suffixes in
+ *                                   their own packed buffers (non-decreasing).
+ * The suffix buffers share the cache descriptor's heads, dims, dtype and
+ * kernel choice.  gdn_plan_window reports the replay window.
+ */
+GDN_API gdn_status gdn_plan_create_fused(const gdn_varlen_desc* cache, const int32_t* match_len_host,
+                                         const int32_t* R_host, const int32_t* suffix_offsets_host,
+                                         gdn_plan_t* out);
+
 /* The replay windows a replay plan would use, computed on the host with no
  * device work: row0_out[b] = seq_offsets[b] + L_b - min(R_b, L_b) and
  * len_out[b] = min(R_b, L_b).  Same validation as gdn_plan_create_replay
@@ -128,8 +144,8 @@ GDN_API gdn_status gdn_replay_windows(int32_t batch, const int32_t* seq_offsets_
  * plan while a call that uses it may still be running. */
 GDN_API void gdn_plan_destroy(gdn_plan_t plan);
 
-/* First row and length of sequence b's work window (replay: the tail window;
- * prefill: the whole sequence).  For tests and schedulers. */
+/* First row and length of sequence b's work window (replay and fused: the
+ * tail window; prefill: the whole sequence).  For tests and schedulers. */
 GDN_API gdn_status gdn_plan_window(gdn_plan_t plan, int32_t b, int64_t* row0, int32_t* len);
 
 /* Number of (sequence, head) work units and the kernel the plan will run. */
@@ -227,6 +243,28 @@ GDN_API gdn_status gdn_chunk_prefill(gdn_plan_t plan, const void* q, const void*
                              const float* alpha, const float* beta, const int32_t* cu_seqlens,
                              const float* state_in, void* o_out, float* state_out,
                              void* workspace, void* stream);
+
+/*
+ * Fused rebuild + suffix prefill on a fused plan: equal (up to rounding
+ * order) to gdn_tail_replay_state followed by gdn_chunk_prefill from the
+ * rebuilt states.  With the tensor-core kernel it is one launch and the
+ * state never leaves the chip between the two phases; the fp32 recurrent
+ * kernel runs it as those two launches.
+ *   k, v, alpha, beta        the packed cache rows (as for the replay).
+ *   sq, sk, sv, salpha, sbeta
+ *                            the packed suffix rows (as for the prefill).
+ *   o_out                    [suffix rows, H, d_v] plan dtype; suffix rows written.
+ *   state_mid                [batch, H, d_k, d_v] fp32 or NULL: the rebuilt state
+ *                            at the end of the matched prefix.
+ *   state_out                [batch, H, d_k, d_v] fp32: the state after the suffix.
+ * No device descriptor arrays are checked.  Returns as gdn_chunk_prefill;
+ * INVALID_ARG for a plan that is not fused or a NULL state_out.
+ */
+GDN_API gdn_status gdn_tail_replay_prefill(gdn_plan_t plan, const void* k, const void* v,
+                                           const float* alpha, const float* beta, const void* sq,
+                                           const void* sk, const void* sv, const float* salpha,
+                                           const float* sbeta, void* o_out, float* state_mid,
+                                           float* state_out, void* workspace, void* stream);
 
 /*
  * Tail replay that allocates nothing (the pages describe no counterpart; this

@@ -96,6 +96,7 @@ def test_null_plan_calls_rejected():
     assert lib.gdn_tail_replay_state(None, *([None] * 11)) == gdn.GDN_ERR_INVALID_ARG
     assert lib.gdn_chunk_prefill(None, *([None] * 11)) == gdn.GDN_ERR_INVALID_ARG
     assert lib.gdn_tail_replay_outputs(None, *([None] * 12)) == gdn.GDN_ERR_INVALID_ARG
+    assert lib.gdn_tail_replay_prefill(None, *([None] * 14)) == gdn.GDN_ERR_INVALID_ARG
     assert lib.gdn_plan_window(None, 0, None, None) == gdn.GDN_ERR_INVALID_ARG
     assert lib.gdn_workspace_status(None, None) == gdn.GDN_ERR_INVALID_ARG
     lib.gdn_plan_destroy(None)
@@ -143,3 +144,19 @@ def test_decode_step_misaligned_rejected():
     p[5] = 4100     # state_in not 16-byte aligned
     assert lib.gdn_decode_step(2, 4, 128, 128, 1, *p) == gdn.GDN_ERR_INVALID_ARG
     assert lib.gdn_decode_step(0, 4, 128, 128, 1, *([None] * 9)) == gdn.GDN_OK   # empty batch
+
+
+def test_fused_plan_rejected_before_any_device_work():
+    lib = gdn.library()
+    d, off = _desc(batch=2, offsets=[0, 100, 150])
+    h = ctypes.c_void_p()
+    ml, rr = np.array([50, 10], np.int32), np.array([10, 1], np.int32)
+    bad_suffix = np.array([0, 20, 10], np.int32)       # decreasing suffix offsets
+    assert lib.gdn_plan_create_fused(ctypes.byref(d), ml.ctypes.data, rr.ctypes.data, bad_suffix.ctypes.data,
+                                     ctypes.byref(h)) == gdn.GDN_ERR_INVALID_ARG
+    assert lib.gdn_plan_create_fused(ctypes.byref(d), ml.ctypes.data, rr.ctypes.data, None,
+                                     ctypes.byref(h)) == gdn.GDN_ERR_INVALID_ARG
+    too_long = np.array([101, 10], np.int32)           # match longer than the cached entry
+    good_suffix = np.array([0, 20, 30], np.int32)
+    assert lib.gdn_plan_create_fused(ctypes.byref(d), too_long.ctypes.data, rr.ctypes.data,
+                                     good_suffix.ctypes.data, ctypes.byref(h)) == gdn.GDN_ERR_INVALID_ARG
