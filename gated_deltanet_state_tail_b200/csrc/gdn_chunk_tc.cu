@@ -24,13 +24,19 @@
 // small).  T is built from 16 x 16 diagonal inverses on CUDA cores and
 // warp-level tf32 tensor-core products for the blocks below the diagonal.
 //
-// Work: one CTA per (sequence, head) unit, 8 warps, chunks in order; the
+// Work: one CTA of 8 warps per (sequence, head) unit, chunks in order; the
 // next chunk's tiles stream in by TMA while the current chunk is computed.
 // Warps w and w + 4 share TMEM lane quarter w (the only lanes a warp may
-// read) and split the 64 columns of every epilogue, so each thread moves 32
-// values per epilogue.  Replay: 96 KB of shared memory, 256 TMEM columns and
-// at most 128 registers per thread, so two CTAs share an SM and overlap each
-// other's serial chain.  Prefill adds the output path (184 KB, 512 columns).
+// read).  Two kernels:
+//   replay_pipe_kernel  the state-only replay.  Two chunks are in flight:
+//                       warps 0-3 build A and T of chunk c + 1 while warps 4-7
+//                       finish chunk c's state chain.  96 KB of shared memory,
+//                       256 TMEM columns, at most 128 registers per thread, so
+//                       two CTAs share an SM.
+//   prefill_kernel      the prefill with outputs, and the fused replay +
+//                       suffix (the replay window's chunks first, without
+//                       outputs).  Warps w and w + 4 split the 64 columns of
+//                       every epilogue.  184 KB, 512 columns, one CTA per SM.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -158,12 +164,11 @@ __device__ __forceinline__ void issue_tiles(uint8_t* tile, uint64_t* bar, const 
     }
 }
 
-template <bool REPLAY>
-__global__ void __launch_bounds__(NT, REPLAY ? 2 : 1)
-chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
+__global__ void __launch_bounds__(NT, 1)
+prefill_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_q,
                 const __grid_constant__ CUtensorMap map_k0, const __grid_constant__ CUtensorMap map_v0) {
-    using L = Layout<REPLAY>;
+    using L = Layout<false>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     // bar_w: W and U' (two issuers); bar_u: the state product and the next
@@ -176,7 +181,7 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wq = warp & 3, wh = warp >> 2;   // TMEM lane quarter; which 32 columns of an epilogue
     const int row = wq * 32 + lane;            // this thread's TMEM lane
-    constexpr uint32_t kTmemCols = REPLAY ? 256 : 512;
+    constexpr uint32_t kTmemCols = 512;
     const Unit u = a.unit_list[blockIdx.x];
     const int b = u.seq, h = u.head, H = a.num_heads;
 
@@ -188,7 +193,7 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     // replay + suffix: first the replay window a.windows0[b] (cache rows, no outputs), then
     // the suffix a.windows[b] with outputs, the state staying in TMEM across the boundary.
     const Window w = a.windows[b];
-    const bool fused = !REPLAY && a.windows0 != nullptr;
+    const bool fused = a.windows0 != nullptr;
     Window w0;
     w0.row0 = 0;
     w0.len = 0;
@@ -203,16 +208,16 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     auto chunk_src = [&](int cc) -> ChunkSrc {
         if (cc < nA) return ChunkSrc{w0.row0 + (long long)cc * C, min(C, w0.len - cc * C), false};
         const int k = cc - nA;
-        return ChunkSrc{w.row0 + (long long)k * C, min(C, w.len - k * C), !REPLAY};
+        return ChunkSrc{w.row0 + (long long)k * C, min(C, w.len - k * C), true};
     };
     auto issue_chunk = [&](int cc, int slot) {
         const ChunkSrc cs = chunk_src(cc);
-        if (cs.out || REPLAY)
-            issue_tiles<REPLAY>(sm + L::OFF_TILE + slot * L::TILE, &bar_tile[slot], &map_k, &map_v, &map_q, h,
-                                (int)cs.r0, cs.out);
+        if (cs.out)
+            issue_tiles<false>(sm + L::OFF_TILE + slot * L::TILE, &bar_tile[slot], &map_k, &map_v, &map_q, h,
+                               (int)cs.r0, true);
         else
-            issue_tiles<REPLAY>(sm + L::OFF_TILE + slot * L::TILE, &bar_tile[slot], &map_k0, &map_v0, &map_q, h,
-                                (int)cs.r0, false);
+            issue_tiles<false>(sm + L::OFF_TILE + slot * L::TILE, &bar_tile[slot], &map_k0, &map_v0, &map_q, h,
+                               (int)cs.r0, false);
     };
 
     if (tid == 0) {
@@ -224,7 +229,7 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         mbar_fence_init();
         tma_prefetch_desc(&map_k);
         tma_prefetch_desc(&map_v);
-        if (!REPLAY) tma_prefetch_desc(&map_q);
+        tma_prefetch_desc(&map_q);
         if (fused) {
             tma_prefetch_desc(&map_k0);
             tma_prefetch_desc(&map_v0);
@@ -254,7 +259,7 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         float v[32];
 #pragma unroll
         for (int cb = 2 * wh; cb < 2 * wh + 2; ++cb) {
-            if (!REPLAY && a.state_in) {
+            if (a.state_in) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = a.state_in[state_base + (size_t)(cb * 32 + i) * D + row];
             } else {
@@ -267,8 +272,7 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     }
     float sigma = 1.0f;   // S = sigma * (TMEM state)
 
-    const uint32_t id_kk = REPLAY ? idesc_bf16(64, 64, false, false)    // K K^T; row r in lane 32 (r/16) + r%16
-                                  : idesc_bf16(128, 64, false, false);  // [K;Q] K^T
+    const uint32_t id_kk = idesc_bf16(128, 64, false, false);   // [K;Q] K^T
     const uint32_t id_w = idesc_bf16(128, 64, true, false);      // K^T (T..)^T, V^T (T..)^T
     const uint32_t id_u = idesc_tf32(128, 64, false, false);     // S^T (-sigma W^T), A in TMEM
     const uint32_t id_s = idesc_bf16(128, 128, false, true);     // U~^T K
@@ -298,7 +302,7 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         const int ncc = chunk_src(cc).nc;
         if (ncc < C) {   // padded tokens are identity transitions: zero their rows
             const int nrows = C - ncc;
-            const int nbox = REPLAY ? 4 : 6;
+            const int nbox = 6;
             for (int e = tid; e < nbox * nrows * 8; e += NT) {
                 const int t = e / (nrows * 8), rr = ncc + (e / 8) % nrows, ch = e % 8;
                 st_shared_v4(tile + t * 8192, (uint32_t)(rr * 128 + ch * 16), make_uint4(0, 0, 0, 0));
@@ -370,14 +374,14 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         const ChunkSrc src = chunk_src(c);
         const long long r0 = src.r0;
         const int nc = src.nc;
-        const bool outc = !REPLAY && src.out;   // uniform: this chunk computes and writes outputs
+        const bool outc = src.out;   // uniform: this chunk computes and writes outputs
         uint8_t* tile = sm + L::OFF_TILE + slot * L::TILE;
         const uint32_t s_tile = smem_u32(tile);
         Gates& G = s_gates[c & 1];
         const bool fast = G.g2[C - 1] >= kFastGateFloor;   // every partial product of gates is >= 2^-100
         tc_fence_after();
 
-        if (!REPLAY && c > 0) {
+        if (c > 0) {
             // the previous chunk's state update and outputs are complete before MB is rewritten
             ok = wait_all(&bar_s, ph_s, a, 6);
             ph_s ^= 1;
@@ -387,39 +391,9 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             if (fused && c == nA && a.state_mid) write_state(a.state_mid);   // the replayed state at L
         }
 
-        // ---- epilogue 1: A = strict_tril(beta_i (gamma_i / gamma_j) K K^T) (fp32, in AT);
-        //      prefill: M = tril((gamma_i / gamma_j) Q K^T) (bf16, MB) ----
-        if (REPLAY) {
-            // M = 64 accumulator: rows 16 wq .. 16 wq + 15 sit in the quarter's first 16 lanes.
-            // This thread takes rows i0 = 16 wq + lane / 4 and i0 + 8, columns
-            // 32 wh + 8 k + 2 (lane % 4) + {0, 1}, k = 0..3.
-            float v[16];
-            tmem_ld16x256b_x4(tlane + TM_P + 32 * wh, v);
-            tmem_wait_ld();
-            const int i0 = 16 * wq + (lane >> 2), jb = 32 * wh + 2 * (lane & 3);
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                const int i = i0 + 8 * hf;
-                const float gi = G.g2[i], bi = G.beta[i];
-                const float rowf = bi * G.gam[i];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int j = jb + 8 * k;
-                    float x0 = v[4 * k + 2 * hf], x1 = v[4 * k + 2 * hf + 1];
-                    if (fast) {
-                        const float2 bv = *reinterpret_cast<const float2*>(G.binv + j);
-                        x0 *= rowf * bv.x;
-                        x1 *= rowf * bv.y;
-                    } else {
-                        x0 *= bi * exp2f(gi - G.g2[j]);
-                        x1 *= bi * exp2f(gi - G.g2[j + 1]);
-                    }
-                    x0 = (j < i) ? x0 : 0.0f;
-                    x1 = (j + 1 < i) ? x1 : 0.0f;
-                    *reinterpret_cast<float2*>(AT + i * LDT + j) = make_float2(x0, x1);
-                }
-            }
-        } else if (row < C || outc) {   // warp-uniform; Q rows only when the chunk writes outputs
+        // ---- epilogue 1: A = strict_tril(beta_i (gamma_i / gamma_j) K K^T) (fp32, in AT) and
+        //      M = tril((gamma_i / gamma_j) Q K^T) (bf16, MB) ----
+        if (row < C || outc) {   // warp-uniform; Q rows only when the chunk writes outputs
             // [K; Q] K^T: lane r < 64 is K row r, lane r >= 64 is Q row r - 64; this thread
             // takes columns [32 wh, 32 wh + 32) of its lane
             float v[32];
@@ -461,22 +435,12 @@ chunk_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         __syncthreads();
 
         // ---- T = (I + A)^-1 in place (warps 0-3).  Meanwhile warp 4 prefetches the next
-        //      chunk into the other slot, once the previous chunk's state update (the slot's
-        //      last reader) is done; a timeout there leaves the tiles unloaded and the wait
-        //      for them reports it ----
-        const uint32_t ph_s_prev = ph_s;   // replay: parity of the previous chunk's state update
-        if (REPLAY && c > 0) ph_s ^= 1;
+        //      chunk into the other slot (its last reader, the previous chunk's state update,
+        //      was waited for at the top of this chunk) ----
         if (warp < 4) {
             invert_unit_lower_inplace(AT, Xs, tid, BAR_INV);
         } else if (warp == 4) {
-            if (elect_one() && c + 1 < nchunks) {
-                bool slot_free = true;
-                if (REPLAY && c > 0) {   // prefill waited for it at the top of the chunk
-                    slot_free = mbar_wait_bounded(&bar_s, ph_s_prev, kWaitNs);
-                    if (!slot_free) report_timeout(a, 6);
-                }
-                if (slot_free) issue_chunk(c + 1, slot ^ 1);
-            }
+            if (elect_one() && c + 1 < nchunks) issue_chunk(c + 1, slot ^ 1);
             __syncwarp();
         }
         __syncthreads();
@@ -1096,11 +1060,11 @@ cudaError_t launch_chunk_tc(const CallArgs& a, cudaStream_t stream) {
     } else {
         const uint32_t smem = Layout<false>::BYTES + 1024;
         if (!attr_set[1]) {
-            cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
             if (e != cudaSuccess) return e;
             attr_set[1] = true;
         }
-        chunk_tc_kernel<false><<<(unsigned)a.units, NT, smem, stream>>>(p, mk, mv, mq, mk0, mv0);
+        prefill_kernel<<<(unsigned)a.units, NT, smem, stream>>>(p, mk, mv, mq, mk0, mv0);
     }
     return cudaGetLastError();
 }
