@@ -3,7 +3,7 @@
 state from the last R tokens of the matched prefix, then prefill the suffix.
 
     python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
-                    [--workload stack|layer|varlen|tiny]
+                    [--workload stack|sweep|varlen|decode|outputs|overlap|fused]
 
 One JSON line on stdout (rank 0).  Default workload: the 24-layer stack, 32
 heads, d = 128, bf16, matched prefix L = 32768, replay R = 3277 (10%), suffix
@@ -43,15 +43,22 @@ GROUPS, GDN_PER_GROUP = 8, 3     # 24 GDN layers = 8 groups x 3
 # --------------------------------------------------------------------------
 # distributed plumbing
 # --------------------------------------------------------------------------
-def dist_init(n_gpus):
+def dist_init(n_gpus, backend=None):
+    """One process per GPU (torchrun env).  NCCL on GPUs; gloo covers the same host
+    logic on CPU.  Returns (rank, world, local rank)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
+        if backend is None:
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                                 device_id=torch.device("cuda", local))
+        else:
+            torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return rank, world, local
@@ -62,10 +69,14 @@ def barrier(world):
         torch.distributed.barrier()
 
 
+def _reduce_device():
+    return torch.device("cuda") if torch.distributed.get_backend() == "nccl" else torch.device("cpu")
+
+
 def max_over_ranks(x, world):
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=_reduce_device())
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
@@ -73,9 +84,15 @@ def max_over_ranks(x, world):
 def sum_over_ranks(x, world):
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=_reduce_device())
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
     return float(t.item())
+
+
+def replica_throughput(replayed_per_rank, world, t_rebuild_max_s):
+    """Whole-job replayed tokens/s of `world` independent replicas (no exchange step):
+    every rank replays the same count and the job lasts as long as its slowest rank."""
+    return replayed_per_rank * world / t_rebuild_max_s
 
 
 # --------------------------------------------------------------------------
@@ -351,8 +368,8 @@ def bench_ours(args, rank, world, local):
     t_rebuild = max_over_ranks(sum(rebuild_ms) / 1e3, world)
     t_step = max_over_ranks(sum(step_ms) / 1e3, world)
 
-    replayed = data.R * args.steps * world            # one request's tail through all 24 layers
-    value = replayed / t_rebuild
+    # one request's tail through all 24 layers, per step and per replica
+    value = replica_throughput(data.R * args.steps, world, t_rebuild)
 
     # roofline of the dominant kernel (the replay launch)
     peaks = measured_peaks()
