@@ -174,13 +174,17 @@ def measured_peaks():
             "source": "fallback", "sm_max_mhz": 1965.0}
 
 
+REPLAY_KERNEL_SOURCES = ("gdn_replay.cu", "gdn_chunk_common.h", "gdn_sm100.h", "gdn_internal.h")
+
+
 def kernel_source_sha():
+    """Hash of the sources that define the replay kernel (its DRAM traffic record in
+    profiles/traffic.txt is used only while this hash matches)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_deltanet_state_tail_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(f.read())
+    for name in REPLAY_KERNEL_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 

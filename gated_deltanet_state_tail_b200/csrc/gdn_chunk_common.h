@@ -6,10 +6,17 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <cuda.h>
+
 #include "gdn_internal.h"
 #include "gdn_sm100.h"
 
 namespace gdn {
+
+// [rows][H][128] bf16 viewed as (d, H, rows), box 64 x 1 x 64, 128-byte swizzle,
+// rows past `rows` read as zero (defined with the chunked prefill).
+bool make_tile_map(CUtensorMap* m, const void* base, int H, long long rows);
+
 namespace chunk {
 
 using namespace sm100;
@@ -229,6 +236,124 @@ __device__ __forceinline__ void write_scaled_t(const float* AT, const float* bet
         const uint32_t off = (uint32_t)(j * 128 + ((chunk ^ (j & 7)) << 4));
         st_shared_v4(tb, off, x);
         st_shared_v4(tbg, off, y);
+    }
+}
+
+// ---------------------------------------------------------------- kernel building blocks
+// Shared by the replay and prefill kernels of the chunked tensor-core path.
+
+constexpr int NT = 256;      // threads per CTA
+
+// ---- shared memory map (byte offsets from a 1 KB aligned base) ----
+// Two tile slots (chunk c in slot c % 2, the next chunk prefetched by TMA),
+// made of 8 KB boxes of 64 rows x 64 columns:
+//   replay : [K0 | K1 | V0 | V1]            (32 KB)
+//   prefill: [K0 | Q0 | K1 | Q1 | V0 | V1]  (48 KB; K block stride 16 KB so
+//            that [K; Q] is one 128-row operand)
+// Once W and U' of a chunk are done, its V boxes take the U tile
+// diag(gamma_C / gamma) U / sigma (bf16 [dv][j], 16 KB) that the state update
+// of the same chunk reads.
+// PREP (32 KB) is reused within a chunk, in this order:
+//   A -> T in place (fp32 64 x LDT) and the product scratch,
+//   T diag(beta), T diag(beta gamma) (bf16 [j][j'], 8 KB each),
+//   BU = -sigma W (fp32, K-major [j][dk], four 8 KB key blocks).
+// Prefill adds UB (bf16 U^T [dv][j]), MB (bf16 masked decayed Q K^T [i][j])
+// and BQ (fp32 sigma diag(gamma) Q, K-major [i][dk], four 8 KB blocks).
+template <bool REPLAY>
+struct Layout {
+    static constexpr uint32_t TILE = REPLAY ? 32768u : 49152u;
+    static constexpr uint32_t OFF_TILE = 0;
+    static constexpr uint32_t OFF_PREP = 2 * TILE;
+    static constexpr uint32_t OFF_AT = OFF_PREP;
+    static constexpr uint32_t OFF_X = OFF_PREP + 17408;
+    static constexpr uint32_t OFF_TB = OFF_PREP;
+    static constexpr uint32_t OFF_TBG = OFF_PREP + 8192;
+    static constexpr uint32_t OFF_BU = OFF_PREP;
+    static constexpr uint32_t OFF_UB = OFF_PREP + 32768;
+    static constexpr uint32_t OFF_MB = OFF_UB + 16384;
+    static constexpr uint32_t OFF_BQ = OFF_MB + 8192;
+    static constexpr uint32_t BYTES = REPLAY ? OFF_PREP + 32768 : OFF_BQ + 32768;
+    // offsets inside a tile slot
+    static constexpr uint32_t K_BLK = REPLAY ? 8192u : 16384u;   // stride of the two K blocks
+    static constexpr uint32_t Q0 = 8192;                          // prefill only
+    static constexpr uint32_t V0 = REPLAY ? 16384u : 32768u;
+    static constexpr uint32_t V_LBO = 8192;
+    static constexpr uint32_t UT = V0;
+};
+static_assert(Layout<true>::OFF_X + 4 * 16 * 24 * 4 <= Layout<true>::OFF_PREP + 32768, "prep scratch fits");
+
+// TMEM columns
+constexpr uint32_t TM_S = 0;      // 128 columns: fp32 S^T / sigma, lane = value row, column = key
+constexpr uint32_t TM_U = 128;    // 64 columns: U'^T then U^T, lane = value row
+constexpr uint32_t TM_P = 192;    // 64 columns: K K^T ([K;Q] K^T for prefill), then W^T (lane = key)
+constexpr uint32_t TM_O = 256;    // 64 columns (prefill): O^T, lane = value row
+
+struct TcParams {
+    CallArgs a;
+};
+
+// Per-chunk gate factors: beta, G = cumulative log2 decay, gamma = 2^G,
+// binv = 2^-G (when the chunk's total decay is >= 2^-100), e = 2^(G_C - G).
+struct Gates {
+    alignas(16) float beta[C];
+    alignas(16) float g2[C];
+    alignas(16) float gam[C];
+    alignas(16) float binv[C];
+    alignas(16) float e[C];
+    float scan;
+};
+
+constexpr uint32_t BAR_GATES = 3;   // named barrier of warps 0-1
+constexpr uint32_t BAR_INV = 1;     // named barrier of warps 0-3 (the UT inverse)
+
+// Build the gate factors of one chunk from the fp32 gates of token `tid`
+// (identity transitions past the window).  Called by threads 0..63 only
+// (warps 0 and 1, which share a named barrier).
+__device__ __forceinline__ void build_gates(Gates& G, float al, float be, int tid, int lane) {
+    {
+        float lg = al > 0.0f ? fmaxf(__log2f(al), kLog2Floor) : kLog2Floor;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            float y = __shfl_up_sync(0xffffffffu, lg, off);
+            if (lane >= off) lg += y;
+        }
+        if (tid == 31) G.scan = lg;
+        G.beta[tid] = be;
+        G.g2[tid] = lg;
+    }
+    named_sync(BAR_GATES, 64);
+    if (tid >= 32) G.g2[tid] += G.scan;
+    named_sync(BAR_GATES, 64);
+    {
+        const float g2C = G.g2[C - 1];
+        const float gj = G.g2[tid];
+        G.gam[tid] = exp2f(gj);
+        G.binv[tid] = g2C >= kFastGateFloor ? exp2f(-gj) : 0.0f;
+        G.e[tid] = exp2f(g2C - gj);
+    }
+}
+
+// Block-wide agreement after a bounded wait: every thread leaves together.
+__device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, const CallArgs& a, uint32_t where) {
+    bool ok = mbar_wait_bounded(bar, parity, kWaitNs);
+    ok = __syncthreads_and(ok) != 0;
+    if (!ok && threadIdx.x == 0) report_timeout(a, where);
+    return ok;
+}
+
+// TMA of one chunk's tiles: K and V, and Q when the chunk writes outputs.
+template <bool REPLAY>
+__device__ __forceinline__ void issue_tiles(uint8_t* tile, uint64_t* bar, const CUtensorMap* mk, const CUtensorMap* mv,
+                                            const CUtensorMap* mq, int h, int r0, bool with_q) {
+    using L = Layout<REPLAY>;
+    mbar_arrive_expect_tx(bar, (!REPLAY && with_q) ? L::TILE : 32768u);
+    tma_load_3d(tile, mk, bar, 0, h, r0);
+    tma_load_3d(tile + L::K_BLK, mk, bar, 64, h, r0);
+    tma_load_3d(tile + L::V0, mv, bar, 0, h, r0);
+    tma_load_3d(tile + L::V0 + L::V_LBO, mv, bar, 64, h, r0);
+    if (!REPLAY && with_q) {
+        tma_load_3d(tile + L::Q0, mq, bar, 0, h, r0);
+        tma_load_3d(tile + L::Q0 + 16384, mq, bar, 64, h, r0);
     }
 }
 
