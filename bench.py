@@ -306,9 +306,11 @@ def run_step(data, rp, pp, state, o, st_out, events=None, launch_events=None):
 # --------------------------------------------------------------------------
 # the CPU oracle as a bounded baseline
 # --------------------------------------------------------------------------
-def oracle_replay_sample(wl, seconds_hint=15.0):
-    """Time the fp64 oracle's replay of one layer (all heads) of the stack workload;
-    returns (tokens/s through the whole stack, cores, sample text)."""
+def oracle_replay_sample(wl, layers=1, min_seconds=0.0, max_reps=8):
+    """Time the fp64 oracle's replay of `layers` of the stack's layers (all heads, R tokens
+    each; one layer's inputs repeated, the oracle's cost does not depend on the values),
+    repeated until `min_seconds` have passed.  Returns (replayed tokens/s through the
+    whole stack, cores, sample text)."""
     import oracle
     R = wl.R[0]
     t = inputs.draw_tensors(R, wl.H, wl.dk, wl.dv, wl.dtype, wl.alpha_lo, wl.alpha_hi, 0,
@@ -316,17 +318,24 @@ def oracle_replay_sample(wl, seconds_hint=15.0):
 
     def bits(x):
         return x.contiguous().view(torch.int16).numpy().view(np.uint16) if x.dtype == torch.bfloat16 else x.numpy()
-    k, v = bits(t["k"]), bits(t["v"])
-    a, b = t["alpha"].numpy(), t["beta"].numpy()
-    off = np.array([0, R], np.int32)
-    heads = wl.H
+    k = np.concatenate([bits(t["k"])] * layers)
+    v = np.concatenate([bits(t["v"])] * layers)
+    a = np.concatenate([t["alpha"].numpy()] * layers)
+    b = np.concatenate([t["beta"].numpy()] * layers)
+    off = (np.arange(layers + 1) * R).astype(np.int32)
+    reps = 0
     t0 = time.perf_counter()
-    oracle.replay_state(k, v, a, b, off, [R], [R])
-    dt_layer = time.perf_counter() - t0
-    per_stack = dt_layer * wl.layers
+    while True:
+        oracle.replay_state(k, v, a, b, off, [R] * layers, [R] * layers)
+        reps += 1
+        elapsed = time.perf_counter() - t0
+        if elapsed >= min_seconds or reps >= max_reps:
+            break
+    per_stack = elapsed / (reps * layers) * wl.layers
+    scaled = "" if layers == wl.layers else f", scaled x{wl.layers / layers:g} to the {wl.layers}-layer stack"
     return (R / per_stack, oracle.num_threads(),
-            f"fp64 oracle replay of 1 of {wl.layers} layers ({heads} heads x {R} tokens, "
-            f"{dt_layer:.2f} s), scaled x{wl.layers} to the stack")
+            f"fp64 oracle replay of {layers} of {wl.layers} layers ({wl.H} heads x {R} tokens each), "
+            f"{reps} run(s) in {elapsed:.1f} s{scaled}")
 
 
 # --------------------------------------------------------------------------
@@ -425,7 +434,7 @@ def bench_ours(args, rank, world, local):
     if not args.no_e2e:
         result["e2e"] = e2e_host_buffers(data, kernel, args, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, sample = oracle_replay_sample(wl)
+        v, cores, sample = oracle_replay_sample(wl, layers=wl.layers, min_seconds=10.0)
         result["cpu_baseline"] = {"value": v, "unit": "replayed tokens/s", "cores": cores,
                                   "kind": "oracle", "sample": sample}
     return result
