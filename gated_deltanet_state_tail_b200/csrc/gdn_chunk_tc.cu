@@ -215,14 +215,26 @@ prefill_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             for (int i = 0; i < 32; ++i) dst[state_base + (size_t)(cb * 32 + i) * D + row] = sigma * v[i];
         }
     };
-    auto write_outputs = [&](long long orow, int onc) {   // prefill: O of a finished chunk
+    // Outputs of a finished chunk: O^T sits in TMEM with lane = value dim, so each thread
+    // holds one value column of 32 rows.  It is staged as bf16 rows [i][dv] in the UB
+    // region (free here: its last reader, the previous output product, is done) and
+    // written with 16-byte stores, 256 contiguous bytes per row.
+    auto write_outputs = [&](long long orow, int onc) {
         float v[32];                                      // rows [32 wh, 32 wh + 32), value dim = row
         tmem_ld32(tlane + TM_O + 32 * wh, v);
         tmem_wait_ld();
+        __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(sm + L::OFF_UB);
+#pragma unroll
+        for (int ii = 0; ii < 32; ++ii) stage[(32 * wh + ii) * D + row] = __float2bfloat16_rn(v[ii]);
+        __syncthreads();
         __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o_out);
 #pragma unroll
-        for (int ii = 0; ii < 32; ++ii)
-            if (32 * wh + ii < onc) o[((orow + 32 * wh + ii) * H + h) * (long long)D + row] = __float2bfloat16_rn(v[ii]);
+        for (int k = 0; k < (C * D / 8) / NT; ++k) {      // 16-byte pieces: 16 per row
+            const int idx = tid + k * NT, i = idx >> 4, ch = idx & 15;
+            if (i < onc)
+                *reinterpret_cast<uint4*>(o + ((orow + i) * H + h) * (long long)D + ch * 8) =
+                    *reinterpret_cast<const uint4*>(stage + i * D + ch * 8);
+        }
     };
 
     // ---- prologue: gates and K K^T of chunk 0 ----
