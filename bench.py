@@ -488,7 +488,8 @@ def full_prefill_comparator(data, kernel, rp, pp, state, o, st_out, iters=3):
 def e2e_host_buffers(data, kernel, args, world):
     """Same metric through the C ABI with host buffers: every step copies the
     tail windows and the suffix inputs from pinned host memory, runs the
-    replay and the suffix prefill, and reads states and outputs back."""
+    replay and the suffix prefill, and reads states and outputs back; the
+    copies of one launch group overlap the kernels of the previous one."""
     import gated_deltanet_state_tail_b200 as gdn
     wl = data.wl
     H, dk, dv = wl.H, wl.dk, wl.dv
@@ -516,16 +517,39 @@ def e2e_host_buffers(data, kernel, args, world):
         cu = np.array([s * N for s in slots] + [(j + 1) * per * N], np.int32)
         pp.append(gdn.PrefillPlan(H, dk, dv, wl.dtype, cu, kernel))
 
+    # The three launch groups are independent, so group j + 1's inputs cross PCIe while
+    # group j replays and prefills (copy-in stream, compute stream), and group j's states
+    # and outputs are read back on a third stream.
+    cur = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    n_groups = len(rp)
+    ev_in = [torch.cuda.Event() for _ in range(n_groups)]
+    ev_done = [torch.cuda.Event() for _ in range(n_groups)]
+
+    def rows_of(name, j):
+        per_rows = per * (R if name.startswith("t") else N)
+        return slice(j * per_rows, (j + 1) * per_rows)
+
     def step():
-        for k in dev:
-            dev[k].copy_(host[k], non_blocking=True)
-        for j in range(len(rp)):
-            rp[j].run(dev["tk"], dev["tv"], dev["talpha"], dev["tbeta"], state[j * per:(j + 1) * per])
-        for j in range(len(pp)):
+        s_in.wait_stream(cur)                  # the previous step no longer reads the inputs
+        with torch.cuda.stream(s_in):
+            for j in range(n_groups):
+                for k in dev:
+                    sl = rows_of(k, j)
+                    dev[k][sl].copy_(host[k][sl], non_blocking=True)
+                ev_in[j].record(s_in)
+        for j in range(n_groups):
+            cur.wait_event(ev_in[j])
+            gs, rs = slice(j * per, (j + 1) * per), slice(j * per * N, (j + 1) * per * N)
+            rp[j].run(dev["tk"], dev["tv"], dev["talpha"], dev["tbeta"], state[gs])
             pp[j].run(dev["sq"], dev["sk"], dev["sv"], dev["salpha"], dev["sbeta"], o,
-                      state_in=state[j * per:(j + 1) * per], state_out=st_out[j * per:(j + 1) * per])
-        h_state.copy_(st_out, non_blocking=True)
-        h_o.copy_(o, non_blocking=True)
+                      state_in=state[gs], state_out=st_out[gs])
+            ev_done[j].record(cur)
+            s_out.wait_event(ev_done[j])
+            with torch.cuda.stream(s_out):
+                h_state[gs].copy_(st_out[gs], non_blocking=True)
+                h_o[rs].copy_(o[rs], non_blocking=True)
+        cur.wait_stream(s_out)                 # the step ends with its results on the host
 
     steps = max(3, min(args.steps, 10))
     for _ in range(2):
