@@ -32,6 +32,7 @@ EXPORTED = (
     "gdn_plan_info", "gdn_workspace_bytes", "gdn_tail_replay_state", "gdn_chunk_prefill",
     "gdn_workspace_status", "gdn_status_string", "gdn_version", "gdn_tail_replay_state_noalloc",
     "gdn_tail_replay_outputs", "gdn_decode_step", "gdn_plan_create_fused", "gdn_tail_replay_prefill",
+    "gdn_selftest_bounded_wait",
 )
 
 
@@ -79,6 +80,7 @@ def _load():
         "gdn_decode_step": (I32, [I32, I32, I32, I32, I32, P, P, P, P, P, P, P, P, P]),
         "gdn_plan_create_fused": (I32, [pd, P, P, P, ctypes.POINTER(P)]),
         "gdn_tail_replay_prefill": (I32, [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P]),
+        "gdn_selftest_bounded_wait": (I32, [ctypes.c_uint64, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -286,6 +288,12 @@ def gdn_tail_replay_state_noalloc(H, dk, dv, dtype, seq_offsets, match_len, R, k
                                               ctypes.byref(st) if wait_status else None),
            "gdn_tail_replay_state_noalloc")
     return st.value if wait_status else None
+
+
+def gdn_selftest_bounded_wait(limit_ns, workspace, stream=None):
+    """Launch the failure-path self-test: a device wait bounded by limit_ns that runs out."""
+    _check(_lib.gdn_selftest_bounded_wait(int(limit_ns), _ptr(workspace), _stream_handle(stream)),
+           "gdn_selftest_bounded_wait")
 
 
 def gdn_workspace_status(workspace, stream=None) -> int:

@@ -1,0 +1,43 @@
+// gdn_selftest.cu -- self-test of the device-side failure path that every
+// kernel's bounded waits use: a wait that runs out sets kStatusTimeout and the
+// wait site in the workspace header, and the kernel returns instead of hanging
+// or trapping, so the context stays usable and the host reads the status with
+// gdn_workspace_status().
+#include <cuda_runtime.h>
+
+#include "gdn_internal.h"
+#include "gdn_sm100.h"
+#include "gdn_tail_replay.h"
+
+namespace gdn {
+namespace {
+
+constexpr unsigned int kSelftestWhere = 99u;   // wait-site code reported by the self-test
+
+// One thread waits, bounded by limit_ns, on an mbarrier that nothing arrives on.
+__global__ void bounded_wait_selftest_kernel(WorkspaceHeader* ws, unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    sm100::mbar_init(&bar, 1);
+    sm100::mbar_fence_init();
+    if (!sm100::mbar_wait_bounded(&bar, 0u, limit_ns)) {
+        atomicOr(&ws->status, kStatusTimeout);
+        atomicCAS(&ws->timeout_where, 0u, kSelftestWhere);
+    }
+}
+
+}  // namespace
+}  // namespace gdn
+
+extern "C" gdn_status gdn_selftest_bounded_wait(uint64_t limit_ns, void* workspace, void* stream) {
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 15u) != 0) return GDN_ERR_INVALID_ARG;
+    if (limit_ns == 0 || limit_ns > 1000000000ull) return GDN_ERR_INVALID_ARG;   // at most 1 s
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    auto* ws = static_cast<gdn::WorkspaceHeader*>(workspace);
+    if (cudaMemsetAsync(ws, 0, sizeof(gdn::WorkspaceHeader), st) != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_CUDA;
+    }
+    gdn::bounded_wait_selftest_kernel<<<1, 1, 0, st>>>(ws, (unsigned long long)limit_ns);
+    if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+    return GDN_OK;
+}

@@ -307,6 +307,19 @@ GDN_API gdn_status gdn_tail_replay_state_noalloc(const gdn_varlen_desc* cache,
  * GDN_ERR_MISMATCH), or GDN_ERR_CUDA if the stream itself failed. */
 GDN_API gdn_status gdn_workspace_status(const void* workspace, void* stream);
 
+/*
+ * Self-test of the failure path (the pages describe no counterpart).  Every
+ * kernel bounds its device waits; one that runs out records GDN_ERR_TIMEOUT
+ * and the wait site in the workspace and returns, so the context stays usable.
+ * This launches one thread that waits, for limit_ns nanoseconds (1 .. 1e9),
+ * on an mbarrier that nothing arrives on.  Afterwards gdn_workspace_status()
+ * returns GDN_ERR_TIMEOUT and the next call on the context works as usual.
+ *   workspace   >= 256 bytes of device memory, 16-byte aligned (its header
+ *               is cleared first).
+ * Returns GDN_OK, INVALID_ARG or CUDA.
+ */
+GDN_API gdn_status gdn_selftest_bounded_wait(uint64_t limit_ns, void* workspace, void* stream);
+
 /* Static description of a status code. */
 GDN_API const char* gdn_status_string(gdn_status s);
 

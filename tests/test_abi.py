@@ -160,3 +160,11 @@ def test_fused_plan_rejected_before_any_device_work():
     good_suffix = np.array([0, 20, 30], np.int32)
     assert lib.gdn_plan_create_fused(ctypes.byref(d), too_long.ctypes.data, rr.ctypes.data,
                                      good_suffix.ctypes.data, ctypes.byref(h)) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_selftest_arguments_rejected_before_launch():
+    lib = gdn.library()
+    assert lib.gdn_selftest_bounded_wait(1000, None, None) == gdn.GDN_ERR_INVALID_ARG
+    assert lib.gdn_selftest_bounded_wait(0, 4096, None) == gdn.GDN_ERR_INVALID_ARG          # no limit
+    assert lib.gdn_selftest_bounded_wait(2_000_000_000, 4096, None) == gdn.GDN_ERR_INVALID_ARG  # above 1 s
+    assert lib.gdn_selftest_bounded_wait(1000, 4100, None) == gdn.GDN_ERR_INVALID_ARG       # misaligned

@@ -227,3 +227,19 @@ def test_single_layer_full_size(kname):
     ref_o, ref_st2 = oracle_prefill(suf, [0, N], st)
     assert rel_err(o.float().cpu().numpy(), ref_o) <= TOL["bf16"]
     assert per_request_state_err(st2.cpu().numpy(), ref_st2) <= TOL["bf16"]
+
+
+def test_bounded_wait_timeout_is_reported_and_context_survives():
+    """The failure path every kernel's waits use: a wait on an mbarrier that nothing
+    arrives on runs out after 1 ms, the status word says GDN_ERR_TIMEOUT, and the
+    next call on the same context works."""
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    gdn.gdn_selftest_bounded_wait(1_000_000, ws)
+    assert gdn.gdn_workspace_status(ws) == gdn.GDN_ERR_TIMEOUT
+    header = ws.view(torch.int32).cpu().numpy()
+    assert header[2] == 99                                   # the wait site the self-test reports
+    # the context is still usable: a small replay runs and matches the oracle
+    t = make_cache([200], 2, 128, 128, "bf16", seed=3)
+    st = run_replay(t, np.array([0, 200], np.int32), [200], [150], gdn.GDN_KERNEL_AUTO, "bf16")
+    ref = oracle_replay(t, np.array([0, 200], np.int32), [200], [150])
+    assert per_request_state_err(st.cpu().numpy(), ref) <= TOL["bf16"]
