@@ -427,16 +427,26 @@ def bench_ours(args, rank, world, local):
         "wall_s_timed": wall,
     }
     result["clocks"] = clk.summary()
+    # tensor side of the same replay launch: 6 C d + 4 d^2 flops per token-head (chunk GEMMs)
+    flops_launch = units_per_launch * data.R * (6 * 64 * wl.dk + 4 * wl.dk * wl.dv)
+    result["replay_tflops"] = flops_launch / launch_s / 1e12
+    result["replay_tensor_frac"] = result["replay_tflops"] / peaks["bf16_tflops"]
+    if kernel_used == gdn.GDN_KERNEL_CHUNKED_TC:
+        result.update(launch_shapes(data, kernel))
 
     if not args.no_comparator:
         result.update(full_prefill_comparator(data, kernel, rp, pp, state, o, st_out))
         result["gdn_speedup_vs_full_prefill"] = result["full_prefill_ms"] / result["ms_per_step"]
+        result["gdn_speedup_token_ratio"] = (wl.match_len[0] + data.N) / (data.R + data.N)
     if not args.no_e2e:
         result["e2e"] = e2e_host_buffers(data, kernel, args, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, sample = oracle_replay_sample(wl, layers=wl.layers, min_seconds=10.0)
         result["cpu_baseline"] = {"value": v, "unit": "replayed tokens/s", "cores": cores,
                                   "kind": "oracle", "sample": sample}
+        sv, ssample = cpu_suffix_sample(wl)
+        result["cpu_suffix_prefill"] = {"value": sv, "unit": "suffix tokens/s", "cores": cores, "kind": "oracle",
+                                        "sample": ssample}
     return result
 
 
@@ -483,6 +493,55 @@ def full_prefill_comparator(data, kernel, rp, pp, state, o, st_out, iters=3):
             "gdn_speedup_vs_full_prefill": None,
             "replay_vs_full_state_rel_frob": {"mean": float(d_state.mean()), "max": float(d_state.max())},
             "replay_vs_full_suffix_out_rel_frob": float(d_o)}
+
+
+def launch_shapes(data, kernel, iters=5):
+    """The same 24-layer rebuild as one launch of all layers and as one launch per layer
+    (the bench line runs three launches of eight)."""
+    import gated_deltanet_state_tail_b200 as gdn
+    wl = data.wl
+    H, dk, dv = wl.H, wl.dk, wl.dv
+    state = torch.empty((data.layers, H, dk, dv), dtype=torch.float32, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    all_slots = list(range(data.layers))
+    off, ml, R = data.replay_desc(all_slots)
+    one = gdn.ReplayPlan(H, dk, dv, wl.dtype, off, ml, R, kernel)
+    per_layer = []
+    for s_ in all_slots:
+        o1, m1, r1 = data.replay_desc([s_])
+        per_layer.append(gdn.ReplayPlan(H, dk, dv, wl.dtype, o1, m1, r1, kernel))
+
+    def one_launch():
+        one.run(data.k, data.v, data.alpha, data.beta, state)
+
+    def per_layer_launches():
+        for s_, p in enumerate(per_layer):
+            p.run(data.k, data.v, data.alpha, data.beta, state[s_:s_ + 1])
+
+    t1 = _time_ms(one_launch, iters, flush)
+    t24 = _time_ms(per_layer_launches, iters, flush)
+    for p in [one] + per_layer:
+        p.check()
+        p.close()
+    return {"rebuild_1x24_ms": t1, "rebuild_24x1_ms": t24}
+
+
+def cpu_suffix_sample(wl):
+    """The fp64 oracle's suffix prefill (with outputs) of one layer: all heads, N tokens from
+    a random state; returns suffix tokens/s through the whole stack and the sample text."""
+    import oracle
+    N = wl.suffix_len[0]
+    t = inputs.draw_tensors(N, wl.H, wl.dk, wl.dv, wl.dtype, wl.alpha_lo, wl.alpha_hi, 1, device="cpu")
+
+    def bits(x):
+        return x.contiguous().view(torch.int16).numpy().view(np.uint16) if x.dtype == torch.bfloat16 else x.numpy()
+    si = np.random.default_rng(0).standard_normal((1, wl.H, wl.dk, wl.dv)) * 0.1
+    t0 = time.perf_counter()
+    oracle.prefill(bits(t["q"]), bits(t["k"]), bits(t["v"]), t["alpha"].numpy(), t["beta"].numpy(),
+                   np.array([0, N], np.int32), state_in=si)
+    dt = time.perf_counter() - t0
+    return N / (dt * wl.layers), f"fp64 oracle suffix prefill of 1 of {wl.layers} layers ({wl.H} heads x {N} tokens, " \
+                                 f"{dt:.2f} s), scaled x{wl.layers}"
 
 
 def e2e_host_buffers(data, kernel, args, world):
