@@ -31,8 +31,8 @@ using namespace chunk;
 // chain: the U epilogue, the state update on the tensor core, and the TMA of
 // chunk c + 2 into the tile slot that update frees.  Then all eight warps form
 // T diag(beta), W and U', and -sigma W of chunk c + 1 and start its state
-// product together with K K^T of chunk c + 2.  Same shared memory (97 KB) and
-// TMEM (256 columns) as the serial replay, so two CTAs still share an SM.
+// product together with K K^T of chunk c + 2.  97 KB of shared memory, 256
+// TMEM columns and at most 128 registers per thread, so two CTAs share an SM.
 constexpr uint32_t BAR_CHAIN = 2;   // named barrier of warps 4-7 (the state chain)
 
 __global__ void __launch_bounds__(NT, 2)
