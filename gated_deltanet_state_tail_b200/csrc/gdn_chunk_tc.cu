@@ -381,7 +381,9 @@ prefill_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             for (int jj = 0; jj < 32; ++jj)
                 *reinterpret_cast<float*>(bu + sw128_offset_f32(32 * wh + jj, lane)) = ns * v[jj];
             if (outc) {
-                const int i = tid >> 2, qk = tid & 3;           // row i, keys [32 qk, 32 qk + 32)
+                // row i, keys [32 qk, 32 qk + 32): consecutive threads take consecutive rows, so
+                // the swizzled 16-byte Q reads and BQ writes of a store phase hit distinct banks
+                const int i = tid & (C - 1), qk = tid >> 6;
                 const uint8_t* qb = tile + L::Q0 + (qk >> 1) * 16384;
                 uint8_t* blk = sm + L::OFF_BQ + qk * 8192;
                 const float sg = sigma * G.gam[i];
