@@ -534,16 +534,15 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapFloatOOBfill);
 
 EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
+    // resolved once (thread-safe static initialisation); null if the driver lacks it
+    static const EncodeTiledFn fn = [] {
         void* p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
+            return reinterpret_cast<EncodeTiledFn>(p);
+        return static_cast<EncodeTiledFn>(nullptr);
+    }();
     return fn;
 }
 
@@ -591,13 +590,10 @@ cudaError_t launch_chunk_tc(const CallArgs& a, cudaStream_t stream) {
             !make_tile_map(&mv0, vb0, a.num_heads, a.rows_total0))
             return cudaErrorInvalidValue;
     }
-    static bool attr_set = false;
+    static std::atomic<uint64_t> smem_set{0};
     const uint32_t smem = Layout<false>::BYTES + 1024;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    const cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(prefill_kernel), (int)smem, smem_set);
+    if (e != cudaSuccess) return e;
     prefill_kernel<<<(unsigned)a.units, NT, smem, stream>>>(p, mk, mv, mq, mk0, mv0);
     return cudaGetLastError();
 }

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace gdn {
 
 // Work window of one sequence, as validated on the host by the plan.
@@ -109,6 +111,19 @@ struct DecodeArgs {
     float* state_out;       // may alias state_in; null = not written
     void* o_out;
 };
+
+// Raise a kernel's dynamic shared-memory limit once per device (a kernel attribute
+// is per device); safe when several host threads launch at once.
+inline cudaError_t ensure_smem_limit(const void* kernel, int bytes, std::atomic<uint64_t>& done_devices) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (done_devices.load(std::memory_order_acquire) & bit) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done_devices.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+}
 
 cudaError_t launch_recurrent(const CallArgs& a, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);

@@ -389,13 +389,10 @@ cudaError_t launch_replay_tc(const CallArgs& a, cudaStream_t stream) {
     CUtensorMap mk, mv;
     if (!make_tile_map(&mk, kb, a.num_heads, a.rows_total) || !make_tile_map(&mv, vb, a.num_heads, a.rows_total))
         return cudaErrorInvalidValue;
-    static bool attr_set = false;
+    static std::atomic<uint64_t> smem_set{0};
     const uint32_t smem = Layout<true>::BYTES + 1024;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(replay_pipe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    const cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(replay_pipe_kernel), (int)smem, smem_set);
+    if (e != cudaSuccess) return e;
     replay_pipe_kernel<<<(unsigned)a.units, NT, smem, stream>>>(p, mk, mv);
     return cudaGetLastError();
 }
