@@ -243,3 +243,52 @@ def test_bounded_wait_timeout_is_reported_and_context_survives():
     st = run_replay(t, np.array([0, 200], np.int32), [200], [150], gdn.GDN_KERNEL_AUTO, "bf16")
     ref = oracle_replay(t, np.array([0, 200], np.int32), [200], [150])
     assert per_request_state_err(st.cpu().numpy(), ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("kname", ["recurrent", "chunked"])
+def test_random_varlen_batches(kname):
+    """Seeded random batches: request count, heads, cached length, match, budget and suffix
+    length drawn per batch (R = 0, R > L, L = 0 and partial chunks all occur); replay states,
+    suffix outputs and final states against the oracle."""
+    dtype, dk, dv = ("bf16", 128, 128) if kname == "chunked" else ("f32", 64, 128)
+    kernel = kernel_or_skip(kname, dtype, dk, dv)
+    rng = np.random.default_rng(2024)
+    for trial in range(12):
+        B = int(rng.integers(1, 6))
+        H = int(rng.integers(1, 4))
+        cached = rng.integers(0, 400, B)
+        ml = np.array([int(rng.integers(0, c + 1)) for c in cached])
+        R = np.array([int(rng.integers(0, m + 80)) for m in ml])           # R > L happens
+        slen = rng.integers(0, 200, B)
+        off = np.concatenate([[0], np.cumsum(cached)]).astype(np.int32)
+        cu = np.concatenate([[0], np.cumsum(slen)]).astype(np.int32)
+        seed = 1000 + trial
+        t = make_cache(list(cached) if off[-1] > 0 else [1], H, dk, dv, dtype, seed)
+        st = run_replay(t, off, ml, R, kernel, dtype)
+        ref = oracle_replay(t, off, ml, R)
+        assert per_request_state_err(st.cpu().numpy(), ref) <= TOL[dtype], f"trial {trial} replay"
+        if cu[-1] == 0:
+            continue
+        s = make_cache(list(slen), H, dk, dv, dtype, seed + 500)
+        o, st2 = run_prefill(s, cu, st, kernel, dtype)
+        ref_o, ref_st2 = oracle_prefill(s, cu, st)
+        assert per_request_rows_err(o.float().cpu().numpy(), ref_o, cu) <= TOL[dtype], f"trial {trial} outputs"
+        assert per_request_state_err(st2.cpu().numpy(), ref_st2) <= TOL[dtype], f"trial {trial} state"
+
+
+def test_longest_windows_against_oracle():
+    """The longest windows the workloads use, one head each: a full 32768-token replay (512
+    chunks through the tensor-core replay) and a 33792-token prefill from zero (the
+    full-prefill comparator's length), both against the fp64 oracle."""
+    kernel_or_skip("chunked", "bf16", 128, 128)
+    L = 32768
+    t = make_cache([L], 1, 128, 128, "bf16", seed=77, a_lo=0.97, a_hi=0.9999)
+    st = run_replay(t, np.array([0, L], np.int32), [L], [L], gdn.GDN_KERNEL_CHUNKED_TC, "bf16")
+    ref = oracle_replay(t, np.array([0, L], np.int32), [L], [L])
+    assert per_request_state_err(st.cpu().numpy(), ref) <= TOL["bf16"]
+    N = 33792
+    s = make_cache([N], 1, 128, 128, "bf16", seed=78, a_lo=0.97, a_hi=0.9999)
+    o, st2 = run_prefill(s, np.array([0, N], np.int32), None, gdn.GDN_KERNEL_CHUNKED_TC, "bf16")
+    ref_o, ref_st2 = oracle_prefill(s, np.array([0, N], np.int32), None)
+    assert rel_err(o.float().cpu().numpy(), ref_o) <= TOL["bf16"]
+    assert per_request_state_err(st2.cpu().numpy(), ref_st2) <= TOL["bf16"]
