@@ -26,13 +26,13 @@
 // small).  T is built from 16 x 16 diagonal inverses on CUDA cores and
 // warp-level tf32 tensor-core products for the blocks below the diagonal.
 //
-// Work: one CTA of 8 warps per (sequence, head) unit, chunks in order; the
-// next chunk's tiles stream in by TMA while the current chunk is computed.
+// Work: one CTA of 8 warps per (sequence, head) unit, chunks in order, two in
+// flight: warps 0-3 build A and M of chunk c + 1 and invert T while warps 4-7
+// finish chunk c (its state update, outputs and the next tile prefetch).
 // Warps w and w + 4 share TMEM lane quarter w (the only lanes a warp may
-// read) and split the 64 columns of every epilogue.  prefill_kernel runs
-// the prefill with outputs and the fused replay + suffix (the replay
-// window's chunks first, without outputs): 184 KB of shared memory, 512 TMEM
-// columns, one CTA per SM.
+// read).  prefill_pipe_kernel runs the prefill with outputs and the fused
+// replay + suffix (the replay window's chunks first, without outputs):
+// 192 KB of shared memory, 512 TMEM columns, one CTA per SM.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -45,60 +45,81 @@ namespace {
 using namespace sm100;
 using namespace chunk;
 
+// ---------------------------------------------------------------------------
+// Prefill (and fused replay + suffix) with two chunks in flight per CTA.
+//
+// Warps 0-3 form A and M of chunk c + 1 and invert T while warps 4-7 finish
+// chunk c: the U epilogue, the state update and O += U M^T on the tensor core,
+// then chunk c's outputs and the TMA of chunk c + 2 into the slot that frees.
+// M is double-buffered so chunk c + 1's can be written while chunk c's output
+// product reads its own.  192 KB of shared memory, 512 TMEM columns, one CTA
+// per SM.
+constexpr uint32_t BAR_CHAIN = 2;   // named barrier of warps 4-7
+struct PipeLayout {
+    static constexpr uint32_t TILE = Layout<false>::TILE;       // [K0 | Q0 | K1 | Q1 | V0 | V1]
+    static constexpr uint32_t OFF_TILE = 0;
+    static constexpr uint32_t OFF_PREP = 2 * TILE;              // A / T, T diag(..), -sigma W
+    static constexpr uint32_t OFF_AT = OFF_PREP;
+    static constexpr uint32_t OFF_X = OFF_PREP + 17408;
+    static constexpr uint32_t OFF_TB = OFF_PREP;
+    static constexpr uint32_t OFF_TBG = OFF_PREP + 8192;
+    static constexpr uint32_t OFF_BU = OFF_PREP;
+    static constexpr uint32_t OFF_UB = OFF_PREP + 32768;        // bf16 U^T [dv][j], then the output stage
+    static constexpr uint32_t OFF_MB = OFF_UB + 16384;          // two bf16 M [i][j], chunk c in c % 2
+    static constexpr uint32_t OFF_BQ = OFF_MB + 16384;          // fp32 sigma diag(gamma) Q, K-major
+    static constexpr uint32_t BYTES = OFF_BQ + 32768;
+};
+static_assert(PipeLayout::BYTES + 1024 <= 227 * 1024, "fits one CTA per SM");
+
 __global__ void __launch_bounds__(NT, 1)
-prefill_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
-                const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_q,
-                const __grid_constant__ CUtensorMap map_k0, const __grid_constant__ CUtensorMap map_v0) {
+prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
+                    const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_q,
+                    const __grid_constant__ CUtensorMap map_k0, const __grid_constant__ CUtensorMap map_v0) {
     using L = Layout<false>;
+    using PL = PipeLayout;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    // bar_w: W and U' (two issuers); bar_u: the state product and the next
-    // chunk's K K^T (two issuers); bar_s: the state update (one issuer)
     __shared__ uint64_t bar_tile[2], bar_w, bar_u, bar_s;
     __shared__ uint32_t tmem_slot;
-    __shared__ Gates s_gates[2];    // chunk c uses s_gates[c & 1]; chunk c + 1's are built during chunk c
+    __shared__ Gates s_gates[2];    // chunk c uses s_gates[c & 1]
 
     const CallArgs& a = p.a;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int wq = warp & 3, wh = warp >> 2;   // TMEM lane quarter; which 32 columns of an epilogue
-    const int row = wq * 32 + lane;            // this thread's TMEM lane
-    constexpr uint32_t kTmemCols = 512;
+    const int wq = warp & 3, wh = warp >> 2;
+    const int row = wq * 32 + lane;
     const Unit u = a.unit_list[blockIdx.x];
     const int b = u.seq, h = u.head, H = a.num_heads;
-
     if (!window_agrees(a, b)) {
         if (tid == 0) atomicOr(&a.ws->status, kStatusMismatch);
         return;
     }
-    // Chunk stream of this unit.  Prefill: the rows of a.windows[b], with outputs.  Fused
-    // replay + suffix: first the replay window a.windows0[b] (cache rows, no outputs), then
-    // the suffix a.windows[b] with outputs, the state staying in TMEM across the boundary.
+    // Chunk stream of this unit: the fused call's replay window first (cache rows, no
+    // outputs), then the sequence's rows with outputs.
     const Window w = a.windows[b];
     const bool fused = a.windows0 != nullptr;
     Window w0;
     w0.row0 = 0;
     w0.len = 0;
     if (fused) w0 = a.windows0[b];
-    const int nA = (w0.len + C - 1) / C;                  // chunks without outputs (fused only)
+    const int nA = (w0.len + C - 1) / C;
     const int nchunks = nA + (w.len + C - 1) / C;
     struct ChunkSrc {
-        long long r0;   // first row
-        int nc;         // rows in the window (the rest are identity padding)
-        bool out;       // writes outputs (prefill rows)
+        long long r0;
+        int nc;
+        bool out;
     };
     auto chunk_src = [&](int cc) -> ChunkSrc {
         if (cc < nA) return ChunkSrc{w0.row0 + (long long)cc * C, min(C, w0.len - cc * C), false};
         const int k = cc - nA;
         return ChunkSrc{w.row0 + (long long)k * C, min(C, w.len - k * C), true};
     };
-    auto issue_chunk = [&](int cc, int slot) {
+    auto tile_of = [&](int cc) { return sm + PL::OFF_TILE + (cc & 1) * PL::TILE; };
+    auto issue_chunk = [&](int cc) {
         const ChunkSrc cs = chunk_src(cc);
         if (cs.out)
-            issue_tiles<false>(sm + L::OFF_TILE + slot * L::TILE, &bar_tile[slot], &map_k, &map_v, &map_q, h,
-                               (int)cs.r0, true);
+            issue_tiles<false>(tile_of(cc), &bar_tile[cc & 1], &map_k, &map_v, &map_q, h, (int)cs.r0, true);
         else
-            issue_tiles<false>(sm + L::OFF_TILE + slot * L::TILE, &bar_tile[slot], &map_k0, &map_v0, &map_q, h,
-                               (int)cs.r0, false);
+            issue_tiles<false>(tile_of(cc), &bar_tile[cc & 1], &map_k0, &map_v0, &map_q, h, (int)cs.r0, false);
     };
 
     if (tid == 0) {
@@ -117,30 +138,29 @@ prefill_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         }
     }
     if (warp == 0) {
-        tmem_alloc(&tmem_slot, kTmemCols);
+        tmem_alloc(&tmem_slot, 512);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = tmem_slot;
-    const uint32_t tlane = tbase + ((uint32_t)(wq * 32) << 16);   // this warp's lane quarter, column 0
-    if (tid == 0 && nchunks > 0) issue_chunk(0, 0);
+    const uint32_t tlane = tbase + ((uint32_t)(wq * 32) << 16);
+    if (tid == 0) {   // both slots are free: chunks 0 and 1
+        for (int cc = 0; cc < 2 && cc < nchunks; ++cc) issue_chunk(cc);
+    }
 
-    float* AT = reinterpret_cast<float*>(sm + L::OFF_AT);
-    float* Xs = reinterpret_cast<float*>(sm + L::OFF_X);
-    const uint32_t s_bu = smem_u32(sm + L::OFF_BU);
-    const uint32_t s_tb = smem_u32(sm + L::OFF_TB), s_tbg = smem_u32(sm + L::OFF_TBG);
-    const uint32_t s_ub = smem_u32(sm + L::OFF_UB), s_mb = smem_u32(sm + L::OFF_MB), s_bq = smem_u32(sm + L::OFF_BQ);
-
-    // ---- initial state: TMEM lane dv = row holds column dv of S (a row of S^T);
-    //      this thread fills key columns [64 wh, 64 wh + 64) ----
+    float* AT = reinterpret_cast<float*>(sm + PL::OFF_AT);
+    float* Xs = reinterpret_cast<float*>(sm + PL::OFF_X);
+    const uint32_t s_bu = smem_u32(sm + PL::OFF_BU);
+    const uint32_t s_tb = smem_u32(sm + PL::OFF_TB), s_tbg = smem_u32(sm + PL::OFF_TBG);
+    const uint32_t s_ub = smem_u32(sm + PL::OFF_UB), s_bq = smem_u32(sm + PL::OFF_BQ);
     const size_t state_base = ((size_t)b * H + h) * D * D;
-    {
+    {   // initial state: TMEM lane dv holds column dv of S (a row of S^T)
         float v[32];
 #pragma unroll
         for (int cb = 2 * wh; cb < 2 * wh + 2; ++cb) {
-            if (a.state_in) {
+            if (a.state_in && !fused) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = a.state_in[state_base + (size_t)(cb * 32 + i) * D + row];
             } else {
@@ -151,17 +171,16 @@ prefill_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         }
         tmem_wait_st();
     }
-    float sigma = 1.0f;   // S = sigma * (TMEM state)
+    float sigma = 1.0f;
 
     const uint32_t id_kk = idesc_bf16(128, 64, false, false);   // [K;Q] K^T
-    const uint32_t id_w = idesc_bf16(128, 64, true, false);      // K^T (T..)^T, V^T (T..)^T
-    const uint32_t id_u = idesc_tf32(128, 64, false, false);     // S^T (-sigma W^T), A in TMEM
-    const uint32_t id_s = idesc_bf16(128, 128, false, true);     // U~^T K
-    const uint32_t id_o2 = idesc_bf16(128, 64, false, false);    // U^T M^T
-
+    const uint32_t id_w = idesc_bf16(128, 64, true, false);
+    const uint32_t id_u = idesc_tf32(128, 64, false, false);
+    const uint32_t id_s = idesc_bf16(128, 128, false, true);
+    const uint32_t id_o2 = idesc_bf16(128, 64, false, false);   // U^T M^T
     uint32_t ph_w = 0, ph_u = 0, ph_s = 0;
     bool ok = true;
-    // gates: registers hold the next chunk's alpha, beta (thread tid < 64 = token tid)
+
     auto load_gates = [&](int cc, float& al, float& be) {
         al = 1.0f;
         be = 0.0f;
@@ -175,16 +194,13 @@ prefill_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             }
         }
     };
-    // Wait for chunk cc's tiles and zero the rows past the window.
     auto tiles_ready = [&](int cc) -> bool {
-        const int slot = cc & 1;
-        uint8_t* tile = sm + L::OFF_TILE + slot * L::TILE;
-        if (!wait_all(&bar_tile[slot], (cc >> 1) & 1, a, 1)) return false;
+        uint8_t* tile = tile_of(cc);
+        if (!wait_all(&bar_tile[cc & 1], (cc >> 1) & 1, a, 1)) return false;
         const int ncc = chunk_src(cc).nc;
         if (ncc < C) {   // padded tokens are identity transitions: zero their rows
             const int nrows = C - ncc;
-            const int nbox = 6;
-            for (int e = tid; e < nbox * nrows * 8; e += NT) {
+            for (int e = tid; e < 6 * nrows * 8; e += NT) {
                 const int t = e / (nrows * 8), rr = ncc + (e / 8) % nrows, ch = e % 8;
                 st_shared_v4(tile + t * 8192, (uint32_t)(rr * 128 + ch * 16), make_uint4(0, 0, 0, 0));
             }
@@ -193,9 +209,8 @@ prefill_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         __syncthreads();
         return true;
     };
-    // K K^T (or [K; Q] K^T) of chunk cc into TM_P.
     auto issue_kk = [&](int cc) {
-        const uint32_t st = smem_u32(sm + L::OFF_TILE + (cc & 1) * L::TILE);
+        const uint32_t st = smem_u32(tile_of(cc));
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = (kk >> 2) * L::K_BLK + (kk & 3) * 32;
@@ -203,41 +218,14 @@ prefill_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                         id_kk, kk > 0);
         }
     };
-    // sigma * TMEM state -> dst[b][h] (fp32 [dk][dv]); this thread writes keys
-    // [64 wh, 64 wh + 64) of value column dv = row
-    auto write_state = [&](float* dst) {
+    if (fused && nA == 0 && a.state_mid) {   // empty window: the state at L is zero
 #pragma unroll
-        for (int cb = 2 * wh; cb < 2 * wh + 2; ++cb) {
-            float v[32];
-            tmem_ld32(tlane + TM_S + cb * 32, v);
-            tmem_wait_ld();
+        for (int cb = 2 * wh; cb < 2 * wh + 2; ++cb)
 #pragma unroll
-            for (int i = 0; i < 32; ++i) dst[state_base + (size_t)(cb * 32 + i) * D + row] = sigma * v[i];
-        }
-    };
-    // Outputs of a finished chunk: O^T sits in TMEM with lane = value dim, so each thread
-    // holds one value column of 32 rows.  It is staged as bf16 rows [i][dv] in the UB
-    // region (free here: its last reader, the previous output product, is done) and
-    // written with 16-byte stores, 256 contiguous bytes per row.
-    auto write_outputs = [&](long long orow, int onc) {
-        float v[32];                                      // rows [32 wh, 32 wh + 32), value dim = row
-        tmem_ld32(tlane + TM_O + 32 * wh, v);
-        tmem_wait_ld();
-        __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(sm + L::OFF_UB);
-#pragma unroll
-        for (int ii = 0; ii < 32; ++ii) stage[(32 * wh + ii) * D + row] = __float2bfloat16_rn(v[ii]);
-        __syncthreads();
-        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o_out);
-#pragma unroll
-        for (int k = 0; k < (C * D / 8) / NT; ++k) {      // 16-byte pieces: 16 per row
-            const int idx = tid + k * NT, i = idx >> 4, ch = idx & 15;
-            if (i < onc)
-                *reinterpret_cast<uint4*>(o + ((orow + i) * H + h) * (long long)D + ch * 8) =
-                    *reinterpret_cast<const uint4*>(stage + i * D + ch * 8);
-        }
-    };
+            for (int i = 0; i < 32; ++i) a.state_mid[state_base + (size_t)(cb * 32 + i) * D + row] = 0.0f;
+    }
 
-    // ---- prologue: gates and K K^T of chunk 0 ----
+    // ---- prologue: gates of chunk 0 (built) and 1 (registers), [K; Q] K^T of chunk 0 ----
     float al_nxt, be_nxt;
     load_gates(0, al_nxt, be_nxt);
     if (tid < C) build_gates(s_gates[0], al_nxt, be_nxt, tid, lane);
@@ -257,98 +245,188 @@ prefill_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             ph_u ^= 1;
         }
     }
-    long long o_r0 = 0;
-    int o_nc = 0;
-    bool o_prev = false;   // the previous chunk wrote outputs
-    if (fused && nA == 0 && a.state_mid) write_state(a.state_mid);   // empty window: S at L is zero
 
-    for (int c = 0; c < nchunks && ok; ++c) {
-        const int slot = c & 1;
-        const ChunkSrc src = chunk_src(c);
-        const long long r0 = src.r0;
-        const int nc = src.nc;
-        const bool outc = src.out;   // uniform: this chunk computes and writes outputs
-        uint8_t* tile = sm + L::OFF_TILE + slot * L::TILE;
-        const uint32_t s_tile = smem_u32(tile);
-        Gates& G = s_gates[c & 1];
-        const bool fast = G.g2[C - 1] >= kFastGateFloor;   // every partial product of gates is >= 2^-100
+    for (int c = -1; c < nchunks && ok; ++c) {
+        const int cn = c + 1;
+        const bool has_next = cn < nchunks;
+        bool xok = true;
         tc_fence_after();
-
-        if (c > 0) {
-            // the previous chunk's state update and outputs are complete before MB is rewritten
-            ok = wait_all(&bar_s, ph_s, a, 6);
-            ph_s ^= 1;
-            if (!ok) break;
-            tc_fence_after();
-            if (o_prev) write_outputs(o_r0, o_nc);
-            if (fused && c == nA && a.state_mid) write_state(a.state_mid);   // the replayed state at L
-        }
-
-        // ---- epilogue 1: A = strict_tril(beta_i (gamma_i / gamma_j) K K^T) (fp32, in AT) and
-        //      M = tril((gamma_i / gamma_j) Q K^T) (bf16, MB) ----
-        if (row < C || outc) {   // warp-uniform; Q rows only when the chunk writes outputs
-            // [K; Q] K^T: lane r < 64 is K row r, lane r >= 64 is Q row r - 64; this thread
-            // takes columns [32 wh, 32 wh + 32) of its lane
-            float v[32];
-            tmem_ld32(tlane + TM_P + 32 * wh, v);
-            tmem_wait_ld();
-            const bool krow = row < C;
-            const int i = krow ? row : row - C;
-            const float gi = G.g2[i];
-            const float bi = krow ? G.beta[i] : 1.0f;
-            if (fast) {
-                const float rowf = bi * G.gam[i];
-                const float4* binv = reinterpret_cast<const float4*>(G.binv + 32 * wh);
+        if (warp < 4) {
+            if (has_next) {
+                // ---- epilogue 1 of chunk cn: warps 0-1 hold K rows (lane = row), warps 2-3 the
+                //      Q rows; A = strict_tril(beta_i (gamma_i / gamma_j) K K^T) (fp32, in AT) and
+                //      M = tril((gamma_i / gamma_j) Q K^T) (bf16, MB[cn % 2]) ----
+                Gates& Gn = s_gates[cn & 1];
+                const bool outn = chunk_src(cn).out;
+                const bool krow = wq < 2;
+                if (krow || outn) {
+                    const bool fast = Gn.g2[C - 1] >= kFastGateFloor;
+                    const int i = krow ? row : row - C;
+                    const float gi = Gn.g2[i];
+                    const float bi = krow ? Gn.beta[i] : 1.0f;
+                    const float rowf = bi * Gn.gam[i];
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        float v[32];
+                        tmem_ld32(tlane + TM_P + 32 * hf, v);
+                        tmem_wait_ld();
+                        if (fast) {
+                            const float4* binv = reinterpret_cast<const float4*>(Gn.binv + 32 * hf);
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                const float4 bv = binv[q];
+                                v[4 * q] *= rowf * bv.x;
+                                v[4 * q + 1] *= rowf * bv.y;
+                                v[4 * q + 2] *= rowf * bv.z;
+                                v[4 * q + 3] *= rowf * bv.w;
+                            }
+                        } else {
+#pragma unroll
+                            for (int jj = 0; jj < 32; ++jj) v[jj] *= bi * exp2f(gi - Gn.g2[32 * hf + jj]);
+                        }
+                        if (krow) {
+#pragma unroll
+                            for (int jj = 0; jj < 32; ++jj) v[jj] = (32 * hf + jj < i) ? v[jj] : 0.0f;
+#pragma unroll
+                            for (int jj = 0; jj < 32; jj += 4)
+                                *reinterpret_cast<float4*>(AT + i * LDT + 32 * hf + jj) =
+                                    make_float4(v[jj], v[jj + 1], v[jj + 2], v[jj + 3]);
+                        } else {
+#pragma unroll
+                            for (int jj = 0; jj < 32; ++jj) v[jj] = (32 * hf + jj <= i) ? v[jj] : 0.0f;
+                            write_row32_bf16(sm + PL::OFF_MB + (cn & 1) * 8192, i, 4 * hf, v);
+                        }
+                    }
+                }
+                named_sync(BAR_INV, 128);   // every row of A is in before the inverse reads it
+                invert_unit_lower_inplace(AT, Xs, tid, BAR_INV);
+            }
+        } else if (c >= 0) {
+            // ---- chain of chunk c: U~ (and U^T for the outputs), the state update and
+            //      O += U M^T, then chunk c's outputs ----
+            Gates& G = s_gates[c & 1];
+            const ChunkSrc src = chunk_src(c);
+            const bool outc = src.out;
+            uint8_t* tile = tile_of(c);
+            float snew = sigma * G.gam[C - 1];
+            if (snew < kRenormBelow) {   // uniform
+#pragma unroll
+                for (int cb = 0; cb < 4; ++cb) {
+                    float sv[32];
+                    tmem_ld32(tlane + TM_S + cb * 32, sv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) sv[q] *= snew;
+                    tmem_st32(tlane + TM_S + cb * 32, sv);
+                }
+                tmem_wait_st();
+                snew = 1.0f;
+            }
+            const float inv = 1.0f / snew;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                float v[32];
+                tmem_ld32(tlane + TM_U + 32 * hf, v);
+                tmem_wait_ld();
+                if (outc) write_row32_bf16(sm + PL::OFF_UB, row, 4 * hf, v);
+                const float4* ev = reinterpret_cast<const float4*>(G.e + 32 * hf);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
-                    const float4 bv = binv[q];
-                    v[4 * q] *= rowf * bv.x;
-                    v[4 * q + 1] *= rowf * bv.y;
-                    v[4 * q + 2] *= rowf * bv.z;
-                    v[4 * q + 3] *= rowf * bv.w;
+                    const float4 e4 = ev[q];
+                    v[4 * q] *= e4.x * inv;
+                    v[4 * q + 1] *= e4.y * inv;
+                    v[4 * q + 2] *= e4.z * inv;
+                    v[4 * q + 3] *= e4.w * inv;
                 }
-            } else {
-#pragma unroll
-                for (int jj = 0; jj < 32; ++jj) v[jj] *= bi * exp2f(gi - G.g2[32 * wh + jj]);
+                write_row32_bf16(tile + L::UT, row, 4 * hf, v);
             }
-            if (krow) {
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_sync(BAR_CHAIN, 128);
+            if (warp == 4) {
+                tc_fence_after();
+                if (elect_one()) {
+                    const uint32_t s_tile = smem_u32(tile);
+                    const uint32_t s_mb = smem_u32(sm + PL::OFF_MB + (c & 1) * 8192);
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) v[jj] = (32 * wh + jj < i) ? v[jj] : 0.0f;
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ss(tbase + TM_S, smem_desc_sw128(s_tile + L::UT + kk * 32, 16, 1024),
+                                    smem_desc_sw128(s_tile + kk * 2048, L::K_BLK, 1024), id_s, 1u);
+                    if (outc) {
 #pragma unroll
-                for (int jj = 0; jj < 32; jj += 4)
-                    *reinterpret_cast<float4*>(AT + i * LDT + 32 * wh + jj) =
-                        make_float4(v[jj], v[jj + 1], v[jj + 2], v[jj + 3]);
-            } else {
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_bf16_ss(tbase + TM_O, smem_desc_sw128(s_ub + kk * 32, 16, 1024),
+                                        smem_desc_sw128(s_mb + kk * 32, 16, 1024), id_o2, 1u);
+                    }
+                    mma_commit(&bar_s);
+                    if (mbar_wait_bounded(&bar_s, ph_s, kWaitNs)) {
+                        if (c + 2 < nchunks) issue_chunk(c + 2);
+                    } else {
+                        report_timeout(a, 6);
+                        xok = false;
+                    }
+                }
+                __syncwarp();
+            }
+            sigma = snew;
+            named_sync(BAR_CHAIN, 128);   // the state update (and O) of chunk c are complete
+            tc_fence_after();
+            if (outc) {
+                // outputs: stage O as bf16 rows [i][dv] in UB (its last reader, O += U M^T, is
+                // done), then 16-byte stores of whole rows
+                __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(sm + PL::OFF_UB);
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) v[jj] = (32 * wh + jj <= i) ? v[jj] : 0.0f;
-                write_row32_bf16(sm + L::OFF_MB, i, 4 * wh, v);
+                for (int hf = 0; hf < 2; ++hf) {
+                    float v[32];   // O^T: value dim = row, chunk rows [32 hf, 32 hf + 32)
+                    tmem_ld32(tlane + TM_O + 32 * hf, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int ii = 0; ii < 32; ++ii) stage[(32 * hf + ii) * D + row] = __float2bfloat16_rn(v[ii]);
+                }
+                named_sync(BAR_CHAIN, 128);
+                __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o_out);
+                const int ct = tid - 128;   // this thread among the chain's 128
+#pragma unroll
+                for (int k = 0; k < (C * D / 8) / 128; ++k) {   // 16-byte pieces: 16 per row
+                    const int idx = ct + k * 128, i = idx >> 4, ch = idx & 15;
+                    if (i < src.nc)
+                        *reinterpret_cast<uint4*>(o + ((src.r0 + i) * H + h) * (long long)D + ch * 8) =
+                            *reinterpret_cast<const uint4*>(stage + i * D + ch * 8);
+                }
+            }
+            if (fused && c == nA - 1 && a.state_mid) {   // the state at L (chunk c is the window's last)
+#pragma unroll
+                for (int cb = 0; cb < 4; ++cb) {
+                    float v[32];
+                    tmem_ld32(tlane + TM_S + cb * 32, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) a.state_mid[state_base + (size_t)(cb * 32 + i) * D + row] = sigma * v[i];
+                }
             }
         }
-        tc_fence_before();
-        __syncthreads();
+        if (c >= 0) {   // every thread keeps the same running scale
+            const float snew = sigma * s_gates[c & 1].gam[C - 1];
+            if (warp < 4) sigma = snew < kRenormBelow ? 1.0f : snew;   // warps 4-7 updated it above
+            ph_s ^= 1;
+        }
+        ok = __syncthreads_and(xok) != 0;
+        if (!ok || !has_next) break;
 
-        // ---- T = (I + A)^-1 in place (warps 0-3).  Meanwhile warp 4 prefetches the next
-        //      chunk into the other slot (its last reader, the previous chunk's state update,
-        //      was waited for at the top of this chunk) ----
-        if (warp < 4) {
-            invert_unit_lower_inplace(AT, Xs, tid, BAR_INV);
-        } else if (warp == 4) {
-            if (elect_one() && c + 1 < nchunks) issue_chunk(c + 1, slot ^ 1);
-            __syncwarp();
-        }
-        __syncthreads();
-        // ---- T diag(beta) and T diag(beta gamma) in bf16 (all warps) ----
-        write_scaled_t<NT>(AT, G.beta, G.gam, sm + L::OFF_TB, sm + L::OFF_TBG, tid, 0);
+        // ---- phase Y, chunk cn ----
+        Gates& Gn = s_gates[cn & 1];
+        const ChunkSrc srcn = chunk_src(cn);
+        uint8_t* tile_n = tile_of(cn);
+        const uint32_t s_tile_n = smem_u32(tile_n);
+        write_scaled_t<NT>(AT, Gn.beta, Gn.gam, sm + PL::OFF_TB, sm + PL::OFF_TBG, tid, 0);
         fence_proxy_async_smem();
         __syncthreads();
-
-        // ---- W^T = K^T (T diag(beta gamma))^T -> TM_P and U'^T = V^T (T diag(beta))^T -> TM_U ----
         if (warp == 0) {
             tc_fence_after();
             if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ss(tbase + TM_P, smem_desc_sw128(s_tile + kk * 2048, L::K_BLK, 1024),
+                    mma_bf16_ss(tbase + TM_P, smem_desc_sw128(s_tile_n + kk * 2048, L::K_BLK, 1024),
                                 smem_desc_sw128(s_tbg + kk * 32, 16, 1024), id_w, kk > 0);
                 mma_commit(&bar_w);
             }
@@ -358,7 +436,7 @@ prefill_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ss(tbase + TM_U, smem_desc_sw128(s_tile + L::V0 + kk * 2048, L::V_LBO, 1024),
+                    mma_bf16_ss(tbase + TM_U, smem_desc_sw128(s_tile_n + L::V0 + kk * 2048, L::V_LBO, 1024),
                                 smem_desc_sw128(s_tb + kk * 32, 16, 1024), id_w, kk > 0);
                 mma_commit(&bar_w);
             }
@@ -368,27 +446,24 @@ prefill_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         ph_w ^= 1;
         if (!ok) break;
         tc_fence_after();
-
-        // ---- epilogue 2: BU[j][dk] = -sigma W[j][dk] (fp32, K-major);
-        //      prefill: BQ[i][dk] = sigma gamma_i Q[i][dk] ----
+        // ---- epilogue 2: BU = -sigma W (fp32, K-major); BQ = sigma diag(gamma) Q ----
         {
-            float v[32];                                        // key dk = row, chunk rows [32 wh, 32 wh + 32)
+            float v[32];
             tmem_ld32(tlane + TM_P + 32 * wh, v);
             tmem_wait_ld();
-            uint8_t* bu = sm + L::OFF_BU + wq * 8192;           // key block of this thread's key
+            uint8_t* bu = sm + PL::OFF_BU + wq * 8192;
             const float ns = -sigma;
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj)
                 *reinterpret_cast<float*>(bu + sw128_offset_f32(32 * wh + jj, lane)) = ns * v[jj];
-            if (outc) {
-                // row i, keys [32 qk, 32 qk + 32): consecutive threads take consecutive rows, so
-                // the swizzled 16-byte Q reads and BQ writes of a store phase hit distinct banks
+            if (srcn.out) {
+                // row i, keys [32 qk, 32 qk + 32): consecutive threads take consecutive rows
                 const int i = tid & (C - 1), qk = tid >> 6;
-                const uint8_t* qb = tile + L::Q0 + (qk >> 1) * 16384;
-                uint8_t* blk = sm + L::OFF_BQ + qk * 8192;
-                const float sg = sigma * G.gam[i];
+                const uint8_t* qb = tile_n + L::Q0 + (qk >> 1) * 16384;
+                uint8_t* blk = sm + PL::OFF_BQ + qk * 8192;
+                const float sg = sigma * Gn.gam[i];
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {                // 8 bf16 per 16-byte chunk of the Q row
+                for (int ch = 0; ch < 4; ++ch) {
                     const int cidx = (qk & 1) * 4 + ch;
                     const uint4 raw = *reinterpret_cast<const uint4*>(qb + i * 128 + ((cidx ^ (i & 7)) << 4));
                     const uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
@@ -406,16 +481,14 @@ prefill_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        // the next chunk's tiles (prefetched during the inverse) must be in before its K K^T
-        if (c + 1 < nchunks) {
-            ok = tiles_ready(c + 1);
+        if (cn + 1 < nchunks) {
+            ok = tiles_ready(cn + 1);
             if (!ok) break;
         } else {
             __syncthreads();
         }
-
-        // ---- the state product (warp 2) and the next chunk's K K^T (warp 3) go in together;
-        //      warps 0-1 build the next chunk's gate factors meanwhile ----
+        // ---- state product and O = sigma diag(gamma) Q S0 of chunk cn (warp 2), [K; Q] K^T of
+        //      chunk cn + 1 (warp 3); warps 0-1 build chunk cn + 1's gate factors ----
         if (warp == 2) {
             tc_fence_after();
             if (elect_one()) {
@@ -423,11 +496,12 @@ prefill_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 for (int kk = 0; kk < 16; ++kk)
                     mma_tf32_ts(tbase + TM_U, tbase + TM_S + kk * 8,
                                 smem_desc_sw128(s_bu + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_u, 1u);
-                if (outc) {
+                if (srcn.out) {
 #pragma unroll
                     for (int kk = 0; kk < 16; ++kk)
                         mma_tf32_ts(tbase + TM_O, tbase + TM_S + kk * 8,
-                                    smem_desc_sw128(s_bq + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_u, kk > 0);
+                                    smem_desc_sw128(s_bq + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_u,
+                                    kk > 0);
                 }
                 mma_commit(&bar_u);
             }
@@ -435,98 +509,37 @@ prefill_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         } else if (warp == 3) {
             tc_fence_after();
             if (elect_one()) {
-                if (c + 1 < nchunks) issue_kk(c + 1);
+                if (cn + 1 < nchunks) issue_kk(cn + 1);
                 mma_commit(&bar_u);
             }
             __syncwarp();
-        } else if (tid < C && c + 1 < nchunks) {
-            build_gates(s_gates[(c + 1) & 1], al_nxt, be_nxt, tid, lane);
+        } else if (tid < C && cn + 1 < nchunks) {
+            build_gates(s_gates[(cn + 1) & 1], al_nxt, be_nxt, tid, lane);
         }
-        if (c + 1 < nchunks) load_gates(c + 2, al_nxt, be_nxt);
+        if (cn + 1 < nchunks) load_gates(cn + 2, al_nxt, be_nxt);
         ok = wait_all(&bar_u, ph_u, a, 4);
         ph_u ^= 1;
-        if (!ok) break;
-        tc_fence_after();
-
-        // ---- epilogue U: U~ = diag(gamma_C / gamma) U / sigma_new into this chunk's V boxes
-        //      (and U itself for the outputs) ----
-        {
-            float v[32];                                        // value dv = row, chunk rows [32 wh, 32 wh + 32)
-            tmem_ld32(tlane + TM_U + 32 * wh, v);
-            tmem_wait_ld();
-            if (outc) write_row32_bf16(sm + L::OFF_UB, row, 4 * wh, v);
-            float snew = sigma * G.gam[C - 1];
-            if (snew < kRenormBelow) {     // uniform: fold the scale into the TMEM state
-#pragma unroll
-                for (int cb = 2 * wh; cb < 2 * wh + 2; ++cb) {
-                    float sv[32];
-                    tmem_ld32(tlane + TM_S + cb * 32, sv);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int q = 0; q < 32; ++q) sv[q] *= snew;
-                    tmem_st32(tlane + TM_S + cb * 32, sv);
-                }
-                tmem_wait_st();
-                snew = 1.0f;
-            }
-            sigma = snew;
-            const float inv = 1.0f / snew;
-            const float4* ev = reinterpret_cast<const float4*>(G.e + 32 * wh);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const float4 e4 = ev[q];
-                v[4 * q] *= e4.x * inv;
-                v[4 * q + 1] *= e4.y * inv;
-                v[4 * q + 2] *= e4.z * inv;
-                v[4 * q + 3] *= e4.w * inv;
-            }
-            write_row32_bf16(tile + L::UT, row, 4 * wh, v);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- S^T / sigma += U~^T K ;  prefill: O^T += U^T M^T ----
-        if (warp == 0) {
-            tc_fence_after();
-            if (elect_one()) {
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ss(tbase + TM_S, smem_desc_sw128(s_tile + L::UT + kk * 32, 16, 1024),
-                                smem_desc_sw128(s_tile + kk * 2048, L::K_BLK, 1024), id_s, 1u);
-                if (outc) {
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ss(tbase + TM_O, smem_desc_sw128(s_ub + kk * 32, 16, 1024),
-                                    smem_desc_sw128(s_mb + kk * 32, 16, 1024), id_o2, 1u);
-                }
-                mma_commit(&bar_s);
-            }
-            __syncwarp();
-        }
-        o_r0 = r0;
-        o_nc = nc;
-        o_prev = outc;
     }
 
-    // ---- drain: the last state update (and outputs) ----
-    if (ok && nchunks > 0) {
-        ok = wait_all(&bar_s, ph_s, a, 5);
-        tc_fence_after();
-        if (ok && o_prev) write_outputs(o_r0, o_nc);
-    }
-    // fused with an empty suffix: the state at L is the final state
-    if (ok && fused && nA > 0 && nA == nchunks && a.state_mid) write_state(a.state_mid);
     // ---- final state: S[dk][dv] = sigma * TMEM[lane dv][dk] ----
-    if (ok && a.state_out) write_state(a.state_out);
+    tc_fence_after();
+    if (ok && a.state_out) {
+#pragma unroll
+        for (int cb = 2 * wh; cb < 2 * wh + 2; ++cb) {
+            float v[32];
+            tmem_ld32(tlane + TM_S + cb * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) a.state_out[state_base + (size_t)(cb * 32 + i) * D + row] = sigma * v[i];
+        }
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tbase, kTmemCols);
+        tmem_dealloc(tbase, 512);
     }
 }
-
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
@@ -591,10 +604,10 @@ cudaError_t launch_chunk_tc(const CallArgs& a, cudaStream_t stream) {
             return cudaErrorInvalidValue;
     }
     static std::atomic<uint64_t> smem_set{0};
-    const uint32_t smem = Layout<false>::BYTES + 1024;
-    const cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(prefill_kernel), (int)smem, smem_set);
+    const uint32_t smem = PipeLayout::BYTES + 1024;
+    const cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(prefill_pipe_kernel), (int)smem, smem_set);
     if (e != cudaSuccess) return e;
-    prefill_kernel<<<(unsigned)a.units, NT, smem, stream>>>(p, mk, mv, mq, mk0, mv0);
+    prefill_pipe_kernel<<<(unsigned)a.units, NT, smem, stream>>>(p, mk, mv, mq, mk0, mv0);
     return cudaGetLastError();
 }
 
