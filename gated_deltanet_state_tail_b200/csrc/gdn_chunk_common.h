@@ -189,12 +189,16 @@ __device__ __forceinline__ void invert_unit_lower_inplace(float* AT, float* Xs, 
 // From the inverse T (in place in AT, see above) write the bf16 operands
 // T diag(beta) -> tb and T diag(beta gamma) -> tbg, [j][j'] in 128-byte
 // swizzled rows, with NTH threads (ltid < NTH) sharing barrier bar_id.
-// beta and gam are 16-byte aligned.
-// tb / tbg may overlap AT: every thread reads its values before the barrier
-// and writes after it.
-template <int NTH>
+// With rowe (the state-only replay), row j of both is also scaled by rowe[j]:
+// the products W and U' then carry the decay gamma_C / gamma_j that the state
+// update applies to row j of U.
+// beta, gam and rowe are 16-byte aligned.
+// IN_PLACE: tb / tbg overlap AT, so every thread reads its values before a
+// barrier and writes after it; otherwise there is no barrier.
+template <int NTH, bool IN_PLACE = true>
 __device__ __forceinline__ void write_scaled_t(const float* AT, const float* beta, const float* gam,
-                                               uint8_t* tb, uint8_t* tbg, int ltid, uint32_t bar_id) {
+                                               uint8_t* tb, uint8_t* tbg, int ltid, uint32_t bar_id,
+                                               const float* rowe = nullptr) {
     constexpr int PER = C * C / NTH;   // values of one row per thread
     constexpr int TPR = C / PER;       // threads per row
     static_assert(PER % 8 == 0 && TPR * PER == C, "whole 16-byte chunks per thread");
@@ -202,6 +206,7 @@ __device__ __forceinline__ void write_scaled_t(const float* AT, const float* bet
     // the fp32 row loads (stride LDT) and the swizzled bf16 row stores are both
     // free of bank conflicts, and a warp reads one set of gate factors
     const int j = ltid % C, part = ltid / C;
+    const float ej = rowe ? rowe[j] : 1.0f;
     float vb[PER], vbg[PER];
 #pragma unroll
     for (int q = 0; q < PER; q += 4) {
@@ -215,12 +220,12 @@ __device__ __forceinline__ void write_scaled_t(const float* AT, const float* bet
         const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const float x = tv[e] * bv[e];
+            const float x = tv[e] * bv[e] * ej;
             vb[q + e] = x;
             vbg[q + e] = x * gv[e];
         }
     }
-    named_sync(bar_id, NTH);
+    if (IN_PLACE) named_sync(bar_id, NTH);
 #pragma unroll
     for (int ch = 0; ch < PER / 8; ++ch) {
         const int chunk = part * (PER / 8) + ch;
@@ -253,9 +258,10 @@ constexpr int NT = 256;      // threads per CTA
 // Once W and U' of a chunk are done, its V boxes take the U tile
 // diag(gamma_C / gamma) U / sigma (bf16 [dv][j], 16 KB) that the state update
 // of the same chunk reads.
-// PREP (32 KB) is reused within a chunk, in this order:
+// PREP is reused within a chunk, in this order:
 //   A -> T in place (fp32 64 x LDT) and the product scratch,
-//   T diag(beta), T diag(beta gamma) (bf16 [j][j'], 8 KB each),
+//   T diag(beta), T diag(beta gamma) (bf16 [j][j'], 8 KB each; the replay
+//   keeps them past the end of T, 33 KB of PREP, the prefill over T, 32 KB),
 //   BU = -sigma W (fp32, K-major [j][dk], four 8 KB key blocks).
 // Prefill adds UB (bf16 U^T [dv][j]), MB (bf16 masked decayed Q K^T [i][j])
 // and BQ (fp32 sigma diag(gamma) Q, K-major [i][dk], four 8 KB blocks).
@@ -266,13 +272,13 @@ struct Layout {
     static constexpr uint32_t OFF_PREP = 2 * TILE;
     static constexpr uint32_t OFF_AT = OFF_PREP;
     static constexpr uint32_t OFF_X = OFF_PREP + 17408;
-    static constexpr uint32_t OFF_TB = OFF_PREP;
-    static constexpr uint32_t OFF_TBG = OFF_PREP + 8192;
+    static constexpr uint32_t OFF_TB = REPLAY ? OFF_PREP + 17408 : OFF_PREP;
+    static constexpr uint32_t OFF_TBG = OFF_TB + 8192;
     static constexpr uint32_t OFF_BU = OFF_PREP;
     static constexpr uint32_t OFF_UB = OFF_PREP + 32768;
     static constexpr uint32_t OFF_MB = OFF_UB + 16384;
     static constexpr uint32_t OFF_BQ = OFF_MB + 8192;
-    static constexpr uint32_t BYTES = REPLAY ? OFF_PREP + 32768 : OFF_BQ + 32768;
+    static constexpr uint32_t BYTES = REPLAY ? OFF_TBG + 8192 : OFF_BQ + 32768;
     // offsets inside a tile slot
     static constexpr uint32_t K_BLK = REPLAY ? 8192u : 16384u;   // stride of the two K blocks
     static constexpr uint32_t Q0 = 8192;                          // prefill only
@@ -281,6 +287,9 @@ struct Layout {
     static constexpr uint32_t UT = V0;
 };
 static_assert(Layout<true>::OFF_X + 4 * 16 * 24 * 4 <= Layout<true>::OFF_PREP + 32768, "prep scratch fits");
+static_assert(Layout<true>::OFF_TB >= Layout<true>::OFF_AT + C * LDT * 4 && Layout<true>::OFF_TB % 1024 == 0,
+              "replay T operands lie past T, 1 KB aligned");
+static_assert(2 * (Layout<true>::BYTES + 1024) <= 224 * 1024, "two replay CTAs per SM");
 
 // TMEM columns
 constexpr uint32_t TM_S = 0;      // 128 columns: fp32 S^T / sigma, lane = value row, column = key

@@ -11,6 +11,9 @@
 // chunk helpers): A_ij = beta_i (gamma_i / gamma_j) k_i.k_j, T = (I + A)^-1,
 // W = T diag(beta gamma) K, U' = T diag(beta) V, U = U' - W S0,
 // S_C = gamma_C S0 + K^T diag(gamma_C / gamma) U.
+// With E = diag(gamma_C / gamma), this kernel forms E W and E U' directly
+// (E scales the rows of the bf16 T operands), so U~ = E U = E U' - (E W) S0
+// reaches the state update without another pass over U.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -29,11 +32,13 @@ using namespace chunk;
 // The state-independent front of chunk c + 1 (A = strict_tril(...K K^T) and
 // the UT inverse) runs on warps 0-3 while warps 4-7 finish chunk c's state
 // chain: the U epilogue, the state update on the tensor core, and the TMA of
-// chunk c + 2 into the tile slot that update frees.  Then all eight warps form
-// T diag(beta), W and U', and -sigma W of chunk c + 1 and start its state
-// product together with K K^T of chunk c + 2.  97 KB of shared memory, 256
+// chunk c + 2 into the tile slot that update frees.  Warps 6-7 first write the
+// lower-right quarter of A, the only part of A outside columns 0-31.  Then all
+// eight warps form T diag(beta), W and U', and -sigma W of chunk c + 1 and start
+// its state product, then K K^T of chunk c + 2.  98 KB of shared memory, 256
 // TMEM columns and at most 128 registers per thread, so two CTAs share an SM.
 constexpr uint32_t BAR_CHAIN = 2;   // named barrier of warps 4-7 (the state chain)
+constexpr uint32_t BAR_A = 4;       // warps 6-7 -> warps 2-3: their part of A is written
 
 __global__ void __launch_bounds__(NT, 2)
 replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
@@ -141,6 +146,53 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         }
     };
 
+    // Epilogue 1 of chunk cc over the 32 columns [cb, cb + 32):
+    // A = strict_tril(beta_i (gamma_i / gamma_j) K K^T), fp32 into AT.  The M = 64
+    // accumulator keeps rows 16 wq .. 16 wq + 15 in the quarter's first 16 lanes; this
+    // thread takes rows i0 = 16 wq + lane / 4 and i0 + 8, columns cb + 8 k + 2 (lane % 4)
+    // + {0, 1}, k = 0..3.  Every gate factor is read before the first store to AT (a
+    // store through AT may alias them for the compiler, which would then serialise each
+    // load behind the previous store), and while the TMEM load is in flight.
+    auto epi1_half = [&](int cc, int cb) {
+        const Gates& Gn = s_gates[cc & 1];
+        const bool fast = Gn.g2[C - 1] >= kFastGateFloor;
+        float v[16];
+        tmem_ld16x256b_x4(tlane + TM_P + cb, v);
+        const int i0 = 16 * wq + (lane >> 2), jb = cb + 2 * (lane & 3);
+        const float* colf = fast ? Gn.binv : Gn.g2;   // column factor: 2^-G_j, or G_j
+        float2 cf[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) cf[k] = *reinterpret_cast<const float2*>(colf + jb + 8 * k);
+        float gi[2], bi[2], rowf[2];
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            const int i = i0 + 8 * hf;
+            gi[hf] = Gn.g2[i];
+            bi[hf] = Gn.beta[i];
+            rowf[hf] = bi[hf] * Gn.gam[i];
+        }
+        tmem_wait_ld();
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            const int i = i0 + 8 * hf;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int j = jb + 8 * k;
+                float x0 = v[4 * k + 2 * hf], x1 = v[4 * k + 2 * hf + 1];
+                if (fast) {
+                    x0 *= rowf[hf] * cf[k].x;
+                    x1 *= rowf[hf] * cf[k].y;
+                } else {
+                    x0 *= bi[hf] * exp2f(gi[hf] - cf[k].x);
+                    x1 *= bi[hf] * exp2f(gi[hf] - cf[k].y);
+                }
+                x0 = (j < i) ? x0 : 0.0f;
+                x1 = (j + 1 < i) ? x1 : 0.0f;
+                *reinterpret_cast<float2*>(AT + i * LDT + j) = make_float2(x0, x1);
+            }
+        }
+    };
+
     // ---- prologue: gates of chunk 0 (built) and 1 (registers), K K^T of chunk 0 ----
     float al_nxt, be_nxt;
     load_gates(0, al_nxt, be_nxt);
@@ -171,46 +223,27 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         tc_fence_after();
         if (warp < 4) {
             if (has_next) {
-                // ---- epilogue 1 of chunk cn: A = strict_tril(beta_i (gamma_i / gamma_j) K K^T).
-                //      M = 64 accumulator, rows 16 wq .. 16 wq + 15 in the quarter's first 16
-                //      lanes; this thread takes rows i0 = 16 wq + lane / 4 and i0 + 8, columns
-                //      8 k + 2 (lane % 4) + {0, 1}, k = 0..7 ----
-                Gates& Gn = s_gates[cn & 1];
-                const bool fast = Gn.g2[C - 1] >= kFastGateFloor;
-                float v[32];
-                tmem_ld16x256b_x8(tlane + TM_P, v);
-                tmem_wait_ld();
-                const int i0 = 16 * wq + (lane >> 2), jb = 2 * (lane & 3);
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    const int i = i0 + 8 * hf;
-                    const float gi = Gn.g2[i], bi = Gn.beta[i];
-                    const float rowf = bi * Gn.gam[i];
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const int j = jb + 8 * k;
-                        float x0 = v[4 * k + 2 * hf], x1 = v[4 * k + 2 * hf + 1];
-                        if (fast) {
-                            const float2 bv = *reinterpret_cast<const float2*>(Gn.binv + j);
-                            x0 *= rowf * bv.x;
-                            x1 *= rowf * bv.y;
-                        } else {
-                            x0 *= bi * exp2f(gi - Gn.g2[j]);
-                            x1 *= bi * exp2f(gi - Gn.g2[j + 1]);
-                        }
-                        x0 = (j < i) ? x0 : 0.0f;
-                        x1 = (j + 1 < i) ? x1 : 0.0f;
-                        *reinterpret_cast<float2*>(AT + i * LDT + j) = make_float2(x0, x1);
-                    }
-                }
-                // the diagonal solve of block wq reads only rows this warp wrote
+                // ---- epilogue 1 of chunk cn, columns 0-31 (warps 6-7 take rows 32-63 x
+                //      columns 32-63; rows 0-31 have no entries there) ----
+                epi1_half(cn, 0);
                 __syncwarp();
+                // the diagonal solve of block wq reads rows 16 wq .. 16 wq + 15; for wq >= 2
+                // their columns 32-63 come from warps 6-7 (the later stages of the inverse
+                // start after a barrier of warps 0-3 that follows this one)
+                if (wq >= 2) named_sync(BAR_A, 128);
                 // ---- T = (I + A)^-1 in place ----
                 invert_unit_lower_inplace(AT, Xs, tid, BAR_INV);
             }
-        } else if (c >= 0) {
+        } else {
+            if (has_next && warp >= 6) {
+                epi1_half(cn, 32);
+                named_arrive(BAR_A, 128);
+            }
+        }
+        if (warp >= 4 && c >= 0) {
             // ---- epilogue U of chunk c: U~ = diag(gamma_C / gamma) U / sigma_new into the
-            //      chunk's V boxes; the decay is folded into the TMEM state when sigma gets small ----
+            //      chunk's V boxes (the row decay is already in U, through the rows of the T
+            //      operands); the decay is folded into the TMEM state when sigma gets small ----
             Gates& G = s_gates[c & 1];
             uint8_t* tile = tile_of(c);
             float snew = sigma * G.gam[C - 1];
@@ -233,15 +266,8 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 float v[32];   // value dv = row, chunk rows [32 hf, 32 hf + 32)
                 tmem_ld32(tlane + TM_U + 32 * hf, v);
                 tmem_wait_ld();
-                const float4* ev = reinterpret_cast<const float4*>(G.e + 32 * hf);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 e4 = ev[q];
-                    v[4 * q] *= e4.x * inv;
-                    v[4 * q + 1] *= e4.y * inv;
-                    v[4 * q + 2] *= e4.z * inv;
-                    v[4 * q + 3] *= e4.w * inv;
-                }
+                for (int q = 0; q < 32; ++q) v[q] *= inv;
                 write_row32_bf16(tile + L::UT, row, 4 * hf, v);
             }
             fence_proxy_async_smem();
@@ -277,13 +303,13 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         ok = __syncthreads_and(xok) != 0;   // the state update of chunk c is done
         if (!ok || !has_next) break;
 
-        // ---- phase Y, chunk cn: T diag(beta), T diag(beta gamma) in bf16 ----
+        // ---- phase Y, chunk cn: E T diag(beta), E T diag(beta gamma) in bf16 ----
         Gates& Gn = s_gates[cn & 1];
         const uint32_t s_tile_n = smem_u32(tile_of(cn));
-        write_scaled_t<NT>(AT, Gn.beta, Gn.gam, sm + L::OFF_TB, sm + L::OFF_TBG, tid, 0);
+        write_scaled_t<NT, false>(AT, Gn.beta, Gn.gam, sm + L::OFF_TB, sm + L::OFF_TBG, tid, 0, Gn.e);
         fence_proxy_async_smem();
         __syncthreads();
-        // ---- W^T = K^T (T diag(beta gamma))^T -> TM_P and U'^T = V^T (T diag(beta))^T -> TM_U ----
+        // ---- (E W)^T = K^T (E T diag(beta gamma))^T -> TM_P and (E U')^T = V^T (E T diag(beta))^T -> TM_U ----
         if (warp == 0) {
             tc_fence_after();
             if (elect_one()) {
@@ -309,7 +335,7 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         ph_w ^= 1;
         if (!ok) break;
         tc_fence_after();
-        // ---- epilogue 2: BU[j][dk] = -sigma W[j][dk] (fp32, K-major) ----
+        // ---- epilogue 2: BU[j][dk] = -sigma (E W)[j][dk] (fp32, K-major) ----
         {
             float v[32];   // key dk = row, chunk rows [32 wh, 32 wh + 32)
             tmem_ld32(tlane + TM_P + 32 * wh, v);
@@ -322,14 +348,9 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        if (cn + 1 < nchunks) {
-            ok = tiles_ready(cn + 1);
-            if (!ok) break;
-        } else {
-            __syncthreads();
-        }
-        // ---- state product of chunk cn (warp 2) and K K^T of chunk cn + 1 (warp 3); warps 0-1
-        //      build chunk cn + 1's gate factors meanwhile ----
+        __syncthreads();
+        // ---- state product of chunk cn (warp 2) at once; K K^T of chunk cn + 1 (warp 3) once
+        //      its tiles are in, while warps 0-1 build chunk cn + 1's gate factors ----
         if (warp == 2) {
             tc_fence_after();
             if (elect_one()) {
@@ -340,18 +361,38 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 mma_commit(&bar_u);
             }
             __syncwarp();
-        } else if (warp == 3) {
+        }
+        // A full next chunk: warp 3 alone waits for its tiles (the next block-wide barrier
+        // orders them for every later reader).  A partial one: the block zero-pads it first.
+        // A tile timeout still waits for the state product below before the block leaves.
+        const bool has_nn = cn + 1 < nchunks;
+        const bool nn_partial = has_nn && w.len - (cn + 1) * C < C;   // uniform
+        bool tok = true;
+        if (nn_partial) tok = tiles_ready(cn + 1);
+        if (warp == 3) {
+            if (has_nn && !nn_partial) {
+                bool t = true;
+                if (lane == 0) {
+                    t = mbar_wait_bounded(&bar_tile[(cn + 1) & 1], ((cn + 1) >> 1) & 1, kWaitNs);
+                    if (!t) report_timeout(a, 1);
+                }
+                tok = __shfl_sync(0xffffffffu, (int)t, 0) != 0;
+            }
             tc_fence_after();
             if (elect_one()) {
-                if (cn + 1 < nchunks) issue_kk(cn + 1);
+                if (tok && has_nn) issue_kk(cn + 1);
                 mma_commit(&bar_u);
             }
             __syncwarp();
-        } else if (tid < C && cn + 1 < nchunks) {
+        } else if (tid < C && has_nn) {
             build_gates(s_gates[(cn + 1) & 1], al_nxt, be_nxt, tid, lane);
         }
-        if (cn + 1 < nchunks) load_gates(cn + 2, al_nxt, be_nxt);
-        ok = wait_all(&bar_u, ph_u, a, 4);
+        if (has_nn) load_gates(cn + 2, al_nxt, be_nxt);
+        {   // wait_all, with warp 3's tile flag in the same vote
+            const bool okw = mbar_wait_bounded(&bar_u, ph_u, kWaitNs);
+            ok = __syncthreads_and(okw && tok) != 0;
+            if (!ok && tid == 0) report_timeout(a, 4);
+        }
         ph_u ^= 1;
     }
 
