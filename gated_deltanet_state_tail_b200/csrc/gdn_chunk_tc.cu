@@ -481,14 +481,10 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        if (cn + 1 < nchunks) {
-            ok = tiles_ready(cn + 1);
-            if (!ok) break;
-        } else {
-            __syncthreads();
-        }
-        // ---- state product and O = sigma diag(gamma) Q S0 of chunk cn (warp 2), [K; Q] K^T of
-        //      chunk cn + 1 (warp 3); warps 0-1 build chunk cn + 1's gate factors ----
+        __syncthreads();
+        // ---- state product and O = sigma diag(gamma) Q S0 of chunk cn (warp 2) at once; [K; Q] K^T
+        //      of chunk cn + 1 (warp 3) once its tiles are in, while warps 0-1 build chunk cn + 1's
+        //      gate factors ----
         if (warp == 2) {
             tc_fence_after();
             if (elect_one()) {
@@ -506,18 +502,38 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 mma_commit(&bar_u);
             }
             __syncwarp();
-        } else if (warp == 3) {
+        }
+        // A full next chunk: warp 3 alone waits for its tiles (the next block-wide barrier
+        // orders them for every later reader).  A partial one: the block zero-pads it first.
+        // A tile timeout still waits for the state product below before the block leaves.
+        const bool has_nn = cn + 1 < nchunks;
+        const bool nn_partial = has_nn && chunk_src(cn + 1).nc < C;   // uniform
+        bool tok = true;
+        if (nn_partial) tok = tiles_ready(cn + 1);
+        if (warp == 3) {
+            if (has_nn && !nn_partial) {
+                bool t = true;
+                if (lane == 0) {
+                    t = mbar_wait_bounded(&bar_tile[(cn + 1) & 1], ((cn + 1) >> 1) & 1, kWaitNs);
+                    if (!t) report_timeout(a, 1);
+                }
+                tok = __shfl_sync(0xffffffffu, (int)t, 0) != 0;
+            }
             tc_fence_after();
             if (elect_one()) {
-                if (cn + 1 < nchunks) issue_kk(cn + 1);
+                if (tok && has_nn) issue_kk(cn + 1);
                 mma_commit(&bar_u);
             }
             __syncwarp();
-        } else if (tid < C && cn + 1 < nchunks) {
+        } else if (warp < 2 && tid < C && has_nn) {
             build_gates(s_gates[(cn + 1) & 1], al_nxt, be_nxt, tid, lane);
         }
-        if (cn + 1 < nchunks) load_gates(cn + 2, al_nxt, be_nxt);
-        ok = wait_all(&bar_u, ph_u, a, 4);
+        if (has_nn) load_gates(cn + 2, al_nxt, be_nxt);
+        {   // wait_all, with warp 3's tile flag in the same vote
+            const bool okw = mbar_wait_bounded(&bar_u, ph_u, kWaitNs);
+            ok = __syncthreads_and(okw && tok) != 0;
+            if (!ok && tid == 0) report_timeout(a, 4);
+        }
         ph_u ^= 1;
     }
 
