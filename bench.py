@@ -338,6 +338,55 @@ def oracle_replay_sample(wl, layers=1, min_seconds=0.0, max_reps=8):
             f"{reps} run(s) in {elapsed:.1f} s{scaled}")
 
 
+def _oracle_bits(x):
+    """bf16 tensors as their raw bits (the oracle's bf16 input form); fp32 as numpy."""
+    return x.contiguous().view(torch.int16).numpy().view(np.uint16) if x.dtype == torch.bfloat16 else x.numpy()
+
+
+def oracle_throughput(kind, dtype, H, dk, dv, tokens, alpha_lo, alpha_hi, seed=3, min_seconds=1.0,
+                      max_reps=20):
+    """Token-heads/s of the fp64 oracle on a bounded sample: one sequence of `tokens` rows
+    and `H` heads from a zero state, run until `min_seconds` have passed; kind "replay"
+    (state only) or "prefill" (with outputs).  The oracle runs its (sequence, head) units
+    in parallel, so H at least its thread count makes the figure stand for the whole
+    host.  Returns (token-heads/s, seconds)."""
+    import oracle
+    t = inputs.draw_tensors(tokens, H, dk, dv, dtype, alpha_lo, alpha_hi, seed, device="cpu",
+                            with_q=(kind == "prefill"))
+    off = np.array([0, tokens], np.int32)
+    k, v = _oracle_bits(t["k"]), _oracle_bits(t["v"])
+    a, b = t["alpha"].numpy(), t["beta"].numpy()
+    q = _oracle_bits(t["q"]) if kind == "prefill" else None
+    reps = 0
+    t0 = time.perf_counter()
+    while True:
+        if kind == "replay":
+            oracle.replay_state(k, v, a, b, off, [tokens], [tokens])
+        else:
+            oracle.prefill(q, k, v, a, b, off)
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= min_seconds or reps >= max_reps:
+            break
+    return reps * tokens * H / dt, dt
+
+
+def cpu_full_prefill_sample(wl, sample_tokens=2048):
+    """The fp64 oracle's full prefill (prefix ++ suffix from a zero state, with outputs) on
+    a bounded sample (as many heads as the oracle has threads, `sample_tokens` rows),
+    extrapolated by token-heads to the whole stack.  Returns (seconds per full prefill
+    of the stack, sample text)."""
+    import oracle
+    th = max(1, oracle.num_threads())
+    tps, dt = oracle_throughput("prefill", wl.dtype, th, wl.dk, wl.dv, sample_tokens, wl.alpha_lo,
+                                wl.alpha_hi)
+    full_tokens = wl.match_len[0] + wl.suffix_len[0]
+    secs = full_tokens * wl.H * wl.layers / tps
+    return secs, (f"fp64 oracle prefill with outputs of {th} heads x {sample_tokens} tokens (repeated for "
+                  f"{dt:.1f} s), "
+                  f"extrapolated by token-heads to {wl.layers} layers x {wl.H} heads x {full_tokens} tokens")
+
+
 # --------------------------------------------------------------------------
 # main benchmark (our kernels)
 # --------------------------------------------------------------------------
@@ -447,6 +496,11 @@ def bench_ours(args, rank, world, local):
         sv, ssample = cpu_suffix_sample(wl)
         result["cpu_suffix_prefill"] = {"value": sv, "unit": "suffix tokens/s", "cores": cores, "kind": "oracle",
                                         "sample": ssample}
+        fs, fsample = cpu_full_prefill_sample(wl)
+        result["cpu_full_prefill"] = {"value": fs, "unit": "s per full prefill of the stack (extrapolated)",
+                                      "cores": cores, "kind": "oracle", "sample": fsample}
+        # the same ratio as gdn_speedup_vs_full_prefill, on the host cores
+        result["cpu_gdn_speedup_vs_full_prefill"] = fs / (data.R / v + data.N / sv)
     return result
 
 
@@ -656,8 +710,16 @@ def bench_sweep(args):
     alpha ~ U[0.97, 0.9999]): replay latency, full-prefill latency, and the relative
     Frobenius distance of the replayed state to the state of the whole prefix."""
     import gated_deltanet_state_tail_b200 as gdn
+    import oracle
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
     lines = []
+    # the fp64 oracle's replay and full-prefill rates on the host cores (bounded samples),
+    # extrapolated by token-heads to every line below
+    th = max(1, oracle.num_threads())
+    rep_tps, rep_dt = oracle_throughput("replay", "bf16", th, 128, 128, 2048, 0.97, 0.9999)
+    pre_tps, pre_dt = oracle_throughput("prefill", "bf16", th, 128, 128, 2048, 0.97, 0.9999)
+    cpu_sample = (f"fp64 oracle on {th} heads x 2048 tokens, each kind repeated for at least 1 s (replay "
+                  f"{rep_dt:.1f} s, prefill with outputs {pre_dt:.1f} s); extrapolated by token-heads")
     for L in (8192, 16384, 32768):
         wl = [w for w in inputs.sweep_workloads() if w.match_len[0] == L]
         H = wl[0].H
@@ -680,6 +742,9 @@ def bench_sweep(args):
                           "replay_speedup_vs_full_prefill": full_ms / rep_ms,
                           "replayed_tokens_per_s": R / (rep_ms / 1e3),
                           "state_rel_frob": {"mean": float(e.mean()), "max": float(e.max())},
+                          "cpu_baseline": {"replay_ms": R * H / rep_tps * 1e3,
+                                           "full_prefill_ms": L * H / pre_tps * 1e3, "cores": th,
+                                           "kind": "oracle", "sample": cpu_sample},
                           "alpha": "U[0.97, 0.9999]", "heads": H, "dtype": "bf16", "data": "synthetic"})
             plan.close()
         pf.close()
@@ -706,12 +771,48 @@ def bench_varlen(args):
                                      state_in=st, state_out=st2), 10, flush)
     rp.check()
     pp.check()
+    cpu = cpu_varlen_sample(wl, off, cu, cache, suf)
     return [{"metric": "varlen replay + suffix", "workload": wl.name, "requests": wl.batch, "heads": H,
              "replayed_tokens": int(sum(min(r, l) for r, l in zip(wl.R, wl.match_len))),
              "suffix_tokens": int(sum(wl.suffix_len)), "replay_ms": rep_ms, "suffix_prefill_ms": suf_ms,
              "replayed_tokens_per_s": sum(min(r, l) for r, l in zip(wl.R, wl.match_len)) / (rep_ms / 1e3),
+             "suffix_tokens_per_s": sum(wl.suffix_len) / (suf_ms / 1e3), "cpu_baseline": cpu,
              "match_len": wl.match_len, "R": wl.R, "suffix_len": wl.suffix_len, "dtype": "bf16",
              "data": "synthetic"}]
+
+
+def varlen_tail_windows(wl, off, cache, nreq):
+    """The replay windows of the first `nreq` requests, copied to the host as sequences of
+    their own: (k, v, alpha, beta, offsets, lengths)."""
+    ml = [min(l, int(c)) for l, c in zip(wl.match_len[:nreq], np.diff(off)[:nreq])]
+    rr = [max(0, min(r, l)) for r, l in zip(wl.R[:nreq], ml)]
+    rows = torch.cat([torch.arange(int(off[b]) + ml[b] - rr[b], int(off[b]) + ml[b], dtype=torch.long)
+                      for b in range(nreq)]).to(cache["k"].device)
+    k, v = cache["k"][rows].cpu(), cache["v"][rows].cpu()
+    a, b_ = cache["alpha"][rows].cpu().numpy(), cache["beta"][rows].cpu().numpy()
+    woff = np.concatenate([[0], np.cumsum(rr)]).astype(np.int32)
+    return k, v, a, b_, woff, rr
+
+
+def cpu_varlen_sample(wl, off, cu, cache, suf, nreq=4):
+    """The fp64 oracle on the first `nreq` requests of the varlen batch (all heads): the
+    replay of their tails, then their suffix prefill from the replayed states.  The
+    tails are copied out as sequences of their own (a replay reads only its window)."""
+    import oracle
+    k, v, a, b_, woff, rr = varlen_tail_windows(wl, off, cache, nreq)
+    t0 = time.perf_counter()
+    states = oracle.replay_state(_oracle_bits(k), _oracle_bits(v), a, b_, woff, rr, rr)
+    t_rep = time.perf_counter() - t0
+    n_suf = int(cu[nreq])
+    sq, sk, sv = (suf[x][:n_suf].cpu() for x in ("q", "k", "v"))
+    t0 = time.perf_counter()
+    oracle.prefill(_oracle_bits(sq), _oracle_bits(sk), _oracle_bits(sv), suf["alpha"][:n_suf].cpu().numpy(),
+                   suf["beta"][:n_suf].cpu().numpy(), np.asarray(cu[:nreq + 1], np.int32), state_in=states)
+    t_suf = time.perf_counter() - t0
+    return {"replayed_tokens_per_s": sum(rr) / t_rep, "suffix_tokens_per_s": n_suf / t_suf,
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"fp64 oracle on requests 0-{nreq - 1} of {wl.batch} ({wl.H} heads): replay of "
+                      f"{sum(rr)} tail tokens {t_rep:.1f} s, suffix prefill of {n_suf} tokens {t_suf:.1f} s"}
 
 
 def bench_decode(args):
