@@ -212,6 +212,21 @@ def test_replay_then_suffix_equals_one_prefill(kname):
 
 
 @pytest.mark.parametrize("kname", ["recurrent", "chunked"])
+def test_full_window_replay_equals_prefill_state(kname):
+    """R = L: the replay kernel reproduces the state of a prefill from zero over the same
+    L tokens (the prefill kernel), and both match the oracle."""
+    kernel = kernel_or_skip(kname, "bf16", 128, 128)
+    L = 2000   # 31 full chunks and a ragged tail
+    t = make_cache([L], 4, 128, 128, "bf16", seed=23)
+    st = run_replay(t, [0, L], [L], [L], kernel, "bf16")
+    _, sp = run_prefill(t, [0, L], None, kernel, "bf16")
+    assert rel_err(st.cpu().numpy(), sp.cpu().numpy()) <= TOL["bf16"]
+    ref = oracle_replay(t, [0, L], [L], [L])
+    assert per_request_state_err(st.cpu().numpy(), ref) <= TOL["bf16"]
+    assert per_request_state_err(sp.cpu().numpy(), ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("kname", ["recurrent", "chunked"])
 def test_single_layer_full_size(kname):
     """One layer, 16 heads, d = 128, bf16: L = 8192, R = 410 (5%), N = 512, checked in full."""
     wl = inputs.single_layer_workload()
