@@ -226,6 +226,52 @@ def test_full_window_replay_equals_prefill_state(kname):
     assert per_request_state_err(sp.cpu().numpy(), ref) <= TOL["bf16"]
 
 
+def _gates(case, rows, H, seed, last_window_row):
+    """alpha, beta [rows, H] (fp32) for one gate regime."""
+    g = np.random.default_rng(seed)
+    a = g.uniform(0.9, 0.999, (rows, H))
+    b = 1.0 / (1.0 + np.exp(-g.standard_normal((rows, H))))
+    if case == "strong_decay":      # chunk decays far below 2^-100: the per-element exponent path
+        a = g.uniform(0.0, 0.3, (rows, H))
+    elif case == "zero_gates":      # alpha = 0 now and then, and on the window's last token
+        a[::37] = 0.0
+        a[last_window_row] = 0.0
+    elif case == "no_write":        # beta = 0: nothing is written, the state only decays
+        b[:] = 0.0
+    elif case == "identity":        # alpha = 1, beta = 0: every token is an identity transition
+        a[:] = 1.0
+        b[:] = 0.0
+    elif case == "mixed_heads":     # one launch, one head in each regime
+        a[:, 0] = g.uniform(0.0, 0.3, rows)
+    return torch.tensor(a, dtype=torch.float32), torch.tensor(b, dtype=torch.float32)
+
+
+@pytest.mark.parametrize("kname", ["recurrent", "chunked"])
+@pytest.mark.parametrize("case", ["strong_decay", "zero_gates", "no_write", "identity", "mixed_heads"])
+def test_gate_extremes(kname, case):
+    """Degenerate and extreme gates: the replay of a 500-token window and the suffix prefill
+    from a nonzero state, against the oracle.  Strong decay takes the kernels' per-element
+    exponent path and folds the running scale into the state every chunk; alpha = 0 at the
+    window's last token leaves beta k v^T; beta = 0 leaves a zero replay and a decayed
+    state_in; alpha = 1, beta = 0 carries state_in through unchanged."""
+    dtype, dk, dv = ("bf16", 128, 128) if kname == "chunked" else ("f32", 64, 128)
+    kernel = kernel_or_skip(kname, dtype, dk, dv)
+    L, R, N, H = 700, 500, 300, 2   # window of 7 chunks and a ragged tail; suffix of 4 and a tail
+    t = make_cache([L + N], H, dk, dv, dtype, seed=31)
+    a, b = _gates(case, L + N, H, 41, L - 1)
+    t["alpha"], t["beta"] = a.cuda(), b.cuda()
+    st = run_replay(t, [0, L + N], [L], [R], kernel, dtype)
+    ref = oracle_replay(t, [0, L + N], [L], [R])
+    assert per_request_state_err(st.cpu().numpy(), ref) <= TOL[dtype], "replay"
+    s = {k: x[L:] for k, x in t.items()}
+    gen = torch.Generator(device="cuda").manual_seed(5)
+    s0 = torch.randn((1, H, dk, dv), generator=gen, device="cuda") * 0.1
+    o, st2 = run_prefill(s, [0, N], s0, kernel, dtype)
+    ref_o, ref_st2 = oracle_prefill(s, [0, N], s0)
+    assert rel_err(o.float().cpu().numpy(), ref_o) <= TOL[dtype], "suffix outputs"
+    assert per_request_state_err(st2.cpu().numpy(), ref_st2) <= TOL[dtype], "suffix state"
+
+
 @pytest.mark.parametrize("kname", ["recurrent", "chunked"])
 def test_single_layer_full_size(kname):
     """One layer, 16 heads, d = 128, bf16: L = 8192, R = 410 (5%), N = 512, checked in full."""
