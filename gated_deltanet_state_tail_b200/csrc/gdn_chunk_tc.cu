@@ -511,20 +511,18 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         bool tok = true;
         if (nn_partial) tok = tiles_ready(cn + 1);
         if (warp == 3) {
-            if (has_nn && !nn_partial) {
-                bool t = true;
-                if (lane == 0) {
+            // the thread that sees the tiles arrive is the one that issues the MMA reading them
+            bool t = true;
+            if (elect_one()) {
+                if (has_nn && !nn_partial) {
                     t = mbar_wait_bounded(&bar_tile[(cn + 1) & 1], ((cn + 1) >> 1) & 1, kWaitNs);
                     if (!t) report_timeout(a, 1);
                 }
-                tok = __shfl_sync(0xffffffffu, (int)t, 0) != 0;
-            }
-            tc_fence_after();
-            if (elect_one()) {
-                if (tok && has_nn) issue_kk(cn + 1);
+                tc_fence_after();
+                if (t && tok && has_nn) issue_kk(cn + 1);
                 mma_commit(&bar_u);
             }
-            __syncwarp();
+            tok = __all_sync(0xffffffffu, t) && tok;
         } else if (warp < 2 && tid < C && has_nn) {
             build_gates(s_gates[(cn + 1) & 1], al_nxt, be_nxt, tid, lane);
         }
