@@ -137,12 +137,11 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         return true;
     };
     auto issue_kk = [&](int cc) {
-        const uint32_t st = smem_u32(tile_of(cc));
+        const uint64_t dk0 = smem_desc_sw128(smem_u32(tile_of(cc)), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * L::K_BLK + (kk & 3) * 32;
-            mma_bf16_ss(tbase + TM_P, smem_desc_sw128(st + off, 16, 1024), smem_desc_sw128(st + off, 16, 1024),
-                        id_kk, kk > 0);
+            const uint64_t d = desc_advance(dk0, (kk >> 2) * L::K_BLK + (kk & 3) * 32);
+            mma_bf16_ss(tbase + TM_P, d, d, id_kk, kk > 0);
         }
     };
 
@@ -278,10 +277,11 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 tc_fence_after();
                 if (elect_one()) {
                     const uint32_t s_tile = smem_u32(tile);
+                    const uint64_t da = smem_desc_sw128(s_tile + L::UT, 16, 1024);
+                    const uint64_t db = smem_desc_sw128(s_tile, L::K_BLK, 1024);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ss(tbase + TM_S, smem_desc_sw128(s_tile + L::UT + kk * 32, 16, 1024),
-                                    smem_desc_sw128(s_tile + kk * 2048, L::K_BLK, 1024), id_s, 1u);
+                        mma_bf16_ss(tbase + TM_S, desc_advance(da, kk * 32), desc_advance(db, kk * 2048), id_s, 1u);
                     mma_commit(&bar_s);
                     if (mbar_wait_bounded(&bar_s, ph_s, kWaitNs)) {
                         if (c + 2 < nchunks)
@@ -313,20 +313,22 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         if (warp == 0) {
             tc_fence_after();
             if (elect_one()) {
+                const uint64_t da = smem_desc_sw128(s_tile_n, L::K_BLK, 1024);
+                const uint64_t db = smem_desc_sw128(s_tbg, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ss(tbase + TM_P, smem_desc_sw128(s_tile_n + kk * 2048, L::K_BLK, 1024),
-                                smem_desc_sw128(s_tbg + kk * 32, 16, 1024), id_w, kk > 0);
+                    mma_bf16_ss(tbase + TM_P, desc_advance(da, kk * 2048), desc_advance(db, kk * 32), id_w, kk > 0);
                 mma_commit(&bar_w);
             }
             __syncwarp();
         } else if (warp == 1) {
             tc_fence_after();
             if (elect_one()) {
+                const uint64_t da = smem_desc_sw128(s_tile_n + L::V0, L::V_LBO, 1024);
+                const uint64_t db = smem_desc_sw128(s_tb, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ss(tbase + TM_U, smem_desc_sw128(s_tile_n + L::V0 + kk * 2048, L::V_LBO, 1024),
-                                smem_desc_sw128(s_tb + kk * 32, 16, 1024), id_w, kk > 0);
+                    mma_bf16_ss(tbase + TM_U, desc_advance(da, kk * 2048), desc_advance(db, kk * 32), id_w, kk > 0);
                 mma_commit(&bar_w);
             }
             __syncwarp();
@@ -354,10 +356,11 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         if (warp == 2) {
             tc_fence_after();
             if (elect_one()) {
+                const uint64_t db = smem_desc_sw128(s_bu, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < 16; ++kk)
                     mma_tf32_ts(tbase + TM_U, tbase + TM_S + kk * 8,
-                                smem_desc_sw128(s_bu + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_u, 1u);
+                                desc_advance(db, (kk >> 2) * 8192 + (kk & 3) * 32), id_u, 1u);
                 mma_commit(&bar_u);
             }
             __syncwarp();

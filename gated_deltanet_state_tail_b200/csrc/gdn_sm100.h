@@ -270,6 +270,13 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
     return d;
 }
 
+// The descriptor of the same operand `byte_offset` bytes further on: the start
+// address field holds the address in 16-byte units (14 bits, all of shared
+// memory), so stepping through a tile adds to it without touching the rest.
+__device__ __forceinline__ uint64_t desc_advance(uint64_t desc, uint32_t byte_offset) {
+    return desc + (uint64_t)(byte_offset >> 4);
+}
+
 // Instruction descriptor of kind::f16 with bf16 A/B and fp32 accumulation.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
     return (1u << 4)                          // D format: f32
