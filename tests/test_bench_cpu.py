@@ -61,3 +61,22 @@ def test_cpu_varlen_sample_reports_rates():
     assert r["kind"] == "oracle" and r["cores"] >= 1
     assert r["replayed_tokens_per_s"] > 0 and r["suffix_tokens_per_s"] > 0
     assert "requests 0-1 of 3" in r["sample"]
+
+
+def test_reference_arm_line():
+    """Rank 0 of `bench.py --impl reference` times the oracle on the host cores and
+    prints the same metric and config as our arm, with the fields the driver reads."""
+    class A:
+        warmup, steps = 3, 1
+    r = bench.bench_reference(A, 0, 1)
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in r, key
+    assert r["impl"] == "reference" and r["metric"] == bench.BENCH_METRIC
+    assert r["value"] > 0 and r["unit"] == "replayed tokens/s" and r["higher_is_better"] is True
+    assert r["config"]["workload"] == inputs.stack_workload(24).name
+    assert r["cpu_baseline"]["kind"] == "oracle" and r["cpu_baseline"]["value"] == r["value"]
+    assert r["cpu_baseline"]["cores"] >= 1
+    assert r["e2e"]["h2d_bytes_per_step"] == 0 and r["e2e"]["d2h_bytes_per_step"] == 0
+    assert bench.bench_reference(A, 1, 2) is None      # other ranks do no work
