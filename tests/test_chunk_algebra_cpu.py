@@ -11,9 +11,11 @@ chunk they
   * keep the state as S / sigma with a running scalar sigma, multiply the state
     product by -sigma, and fold sigma back into the state when sigma * gamma_C
     falls below 2^-40.
+The prefill keeps U unscaled for its outputs, O = sigma diag(gamma) Q (S / sigma)
++ M U, and applies E and 1 / sigma_new to U for the state update only.
 This test restates those steps (not the kernels' code) and shows that they
-reproduce the recurrence to fp64 rounding, including under strong and zero gates,
-so the kernels' parity rests on an exact reformulation."""
+reproduce the recurrence (states and outputs) to fp64 rounding, including under
+strong and zero gates, so the kernels' parity rests on an exact reformulation."""
 import numpy as np
 import pytest
 
@@ -104,3 +106,59 @@ def test_renormalisation_is_exercised():
     assert np.prod(a) < RENORM_BELOW
     _, _, a, _ = _inputs(64, 4, 4, "normal", seed=1)
     assert np.sum(np.log2(a)) >= FAST_FLOOR
+
+
+def chunk_algebra_prefill(q, k, v, alpha, beta, S0=None):
+    """The prefill's variant: U stays unscaled (the outputs use it); E and 1/sigma_new
+    are applied to U only for the state update.  Per chunk the outputs are
+    O = sigma diag(gamma) Q (S / sigma) + M U with M_ij = (q_i . k_j) 2^(G_i - G_j), j <= i."""
+    n, dk = k.shape
+    dv = v.shape[1]
+    St = np.zeros((dk, dv)) if S0 is None else np.array(S0, dtype=np.float64)
+    sigma = 1.0
+    o = np.zeros((n, dv))
+    for c0 in range(0, n, C):
+        qc = np.zeros((C, dk))
+        kc = np.zeros((C, dk))
+        vc = np.zeros((C, dv))
+        ac = np.ones(C)
+        bc = np.zeros(C)
+        m = min(C, n - c0)
+        qc[:m], kc[:m], vc[:m] = q[c0:c0 + m], k[c0:c0 + m], v[c0:c0 + m]
+        ac[:m], bc[:m] = alpha[c0:c0 + m], beta[c0:c0 + m]
+        lg = np.array([max(np.log2(a), LOG2_FLOOR) if a > 0 else LOG2_FLOOR for a in ac])
+        g2 = np.cumsum(lg)
+        gam = np.exp2(g2)
+        e = np.exp2(g2[-1] - g2)
+        if g2[-1] >= FAST_FLOOR:
+            ratio = gam[:, None] * np.exp2(-g2)[None, :]
+        else:
+            ratio = np.exp2(g2[:, None] - g2[None, :])
+        A = np.tril(bc[:, None] * ratio * (kc @ kc.T), -1)
+        Mq = np.tril(ratio * (qc @ kc.T))
+        T = np.linalg.inv(np.eye(C) + A)
+        U = (T * bc[None, :]) @ vc - sigma * ((T * (bc * gam)[None, :]) @ kc) @ St
+        O = sigma * (gam[:, None] * qc) @ St + Mq @ U
+        o[c0:c0 + m] = O[:m]
+        snew = sigma * gam[-1]
+        if snew < RENORM_BELOW:
+            St = St * snew
+            snew = 1.0
+        St = St + kc.T @ ((e[:, None] * U) / snew)
+        sigma = snew
+    return sigma * St, o
+
+
+@pytest.mark.parametrize("case", ["normal", "strong_decay", "zero_gates"])
+@pytest.mark.parametrize("n", [1, 64, 150])
+def test_prefill_chunk_algebra_matches_recurrence(case, n):
+    dk, dv = 16, 8
+    k, v, a, b = _inputs(n, dk, dv, case, seed=100 + n)
+    g = np.random.default_rng(200 + n)
+    q = g.standard_normal((n, dk))
+    q /= np.linalg.norm(q, axis=1, keepdims=True)
+    S0 = g.standard_normal((dk, dv))
+    S_ref, o_ref = oracle.recurrence(k, v, a, b, q=q, S0=S0)
+    S, o = chunk_algebra_prefill(q, k, v, a, b, S0=S0)
+    assert np.abs(S - S_ref).max() / np.abs(S_ref).max() <= 1e-10
+    assert np.abs(o - o_ref).max() / np.abs(o_ref).max() <= 1e-10
