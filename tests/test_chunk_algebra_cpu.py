@@ -162,3 +162,40 @@ def test_prefill_chunk_algebra_matches_recurrence(case, n):
     S, o = chunk_algebra_prefill(q, k, v, a, b, S0=S0)
     assert np.abs(S - S_ref).max() / np.abs(S_ref).max() <= 1e-10
     assert np.abs(o - o_ref).max() / np.abs(o_ref).max() <= 1e-10
+
+
+def blocked_unit_lower_inverse(A):
+    """(I + A)^-1 for strictly lower triangular 64 x 64 A by the kernels' block scheme:
+    16 x 16 diagonal inverses D_b, then T_10 = -D_1 A_10 D_0 and T_32 = -D_3 A_32 D_2,
+    X = A_21 T_11 by block rows (X_r0 = A_r0 D_0 + A_r1 T_10, X_r1 = A_r1 D_1), and
+    the lower-left 32 x 32 block T_21 = -T_22 X."""
+    B = 16
+    blk = lambda M, r, c: M[B * r:B * (r + 1), B * c:B * (c + 1)]
+    D = [np.linalg.inv(np.eye(B) + np.tril(blk(A, b, b), -1)) for b in range(4)]
+    T10 = -D[1] @ blk(A, 1, 0) @ D[0]
+    T32 = -D[3] @ blk(A, 3, 2) @ D[2]
+    X = {}
+    for r in (2, 3):
+        X[r, 0] = blk(A, r, 0) @ D[0] + blk(A, r, 1) @ T10
+        X[r, 1] = blk(A, r, 1) @ D[1]
+    T = np.zeros_like(A)
+    for b in range(4):
+        T[B * b:B * (b + 1), B * b:B * (b + 1)] = D[b]
+    T[B:2 * B, 0:B] = T10
+    T[3 * B:4 * B, 2 * B:3 * B] = T32
+    for c in (0, 1):
+        T[2 * B:3 * B, B * c:B * (c + 1)] = -D[2] @ X[2, c]
+        T[3 * B:4 * B, B * c:B * (c + 1)] = -(T32 @ X[2, c] + D[3] @ X[3, c])
+    return T
+
+
+@pytest.mark.parametrize("case", ["normal", "strong_decay"])
+def test_blocked_inverse_matches_dense_inverse(case):
+    g = np.random.default_rng(9)
+    for _ in range(5):
+        k, _, a, b = _inputs(C, 128, 1, case, seed=int(g.integers(1 << 30)))
+        g2 = np.cumsum(np.maximum(np.log2(np.maximum(a, 1e-300)), LOG2_FLOOR))
+        A = np.tril(b[:, None] * np.exp2(g2[:, None] - g2[None, :]) * (k @ k.T), -1)
+        ref = np.linalg.inv(np.eye(C) + A)
+        got = blocked_unit_lower_inverse(A)
+        assert np.abs(got - ref).max() / np.abs(ref).max() <= 1e-12
