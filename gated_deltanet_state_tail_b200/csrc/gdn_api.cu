@@ -54,6 +54,8 @@ gdn_status check_desc(const gdn_varlen_desc* d) {
     // element offsets are 64-bit on the device; rows * H * d must fit comfortably
     const long long rows = off[d->batch];
     if (rows * d->num_heads > (1ll << 40)) return GDN_ERR_INVALID_ARG;
+    // one CTA per (sequence, head) unit: the unit count is the grid's x extent
+    if ((long long)d->batch * d->num_heads > 0x7fffffffll) return GDN_ERR_INVALID_ARG;
     return GDN_OK;
 }
 
@@ -222,8 +224,12 @@ gdn_status gdn_plan_create_replay(const gdn_varlen_desc* cache, const int32_t* m
         return GDN_ERR_UNSUPPORTED;
     gdn_plan* p = new_plan(cache, gdn::kReplay);
     if (!p) return GDN_ERR_ALLOC;
-    fill_replay_windows(p->windows, cache->batch, off, match_len_host, R_host);
-    s = finish_plan(p, out);
+    try {   // host allocations report GDN_ERR_ALLOC instead of throwing across the C ABI
+        fill_replay_windows(p->windows, cache->batch, off, match_len_host, R_host);
+        s = finish_plan(p, out);
+    } catch (const std::bad_alloc&) {
+        s = GDN_ERR_ALLOC;
+    }
     if (s != GDN_OK) delete p;
     return s;
 }
@@ -238,8 +244,12 @@ gdn_status gdn_plan_create_prefill(const gdn_varlen_desc* seqs, gdn_plan_t* out)
         return GDN_ERR_UNSUPPORTED;
     gdn_plan* p = new_plan(seqs, gdn::kPrefill);
     if (!p) return GDN_ERR_ALLOC;
-    fill_sequence_windows(p->windows, seqs->batch, seqs->seq_offsets_host);
-    s = finish_plan(p, out);
+    try {
+        fill_sequence_windows(p->windows, seqs->batch, seqs->seq_offsets_host);
+        s = finish_plan(p, out);
+    } catch (const std::bad_alloc&) {
+        s = GDN_ERR_ALLOC;
+    }
     if (s != GDN_OK) delete p;
     return s;
 }
@@ -263,9 +273,13 @@ gdn_status gdn_plan_create_fused(const gdn_varlen_desc* cache, const int32_t* ma
         return GDN_ERR_UNSUPPORTED;
     gdn_plan* p = new_plan(cache, gdn::kFused);
     if (!p) return GDN_ERR_ALLOC;
-    fill_replay_windows(p->windows0, cache->batch, off, match_len_host, R_host);
-    fill_sequence_windows(p->windows, cache->batch, suffix_offsets_host);
-    s = finish_plan(p, out);
+    try {
+        fill_replay_windows(p->windows0, cache->batch, off, match_len_host, R_host);
+        fill_sequence_windows(p->windows, cache->batch, suffix_offsets_host);
+        s = finish_plan(p, out);
+    } catch (const std::bad_alloc&) {
+        s = GDN_ERR_ALLOC;
+    }
     if (s != GDN_OK) delete p;
     return s;
 }

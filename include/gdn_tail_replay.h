@@ -81,7 +81,7 @@ typedef enum gdn_kernel {
  * treating (layer, request) pairs as sequences of one packed batch. */
 typedef struct gdn_varlen_desc {
     int32_t batch;                    /* number of sequences, >= 1 */
-    int32_t num_heads;                /* H, >= 1 */
+    int32_t num_heads;                /* H, >= 1; batch * H <= 2^31 - 1 (one CTA per unit) */
     int32_t d_k;                      /* key head dim: 64 or 128 */
     int32_t d_v;                      /* value head dim: 64 or 128 */
     int32_t dtype;                    /* gdn_dtype of q, k, v, o */

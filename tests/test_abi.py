@@ -84,6 +84,18 @@ def test_replay_arrays_rejected():
     assert lib.gdn_plan_create_replay(ctypes.byref(d), None, None, None) == gdn.GDN_ERR_INVALID_ARG
 
 
+def test_unit_count_limited_to_the_grid():
+    """One CTA per (sequence, head) unit: batch * H above 2^31 - 1 is rejected before any
+    host or device allocation."""
+    batch, H = 1 << 16, 1 << 15                           # 2^31 units
+    zeros = np.zeros(batch + 1, np.int32)
+    d, off = _desc(batch=batch, H=H, offsets=zeros)
+    assert _create_replay(d, np.zeros(batch, np.int32), np.zeros(batch, np.int32)) == gdn.GDN_ERR_INVALID_ARG
+    lib = gdn.library()
+    h = ctypes.c_void_p()
+    assert lib.gdn_plan_create_prefill(ctypes.byref(d), ctypes.byref(h)) == gdn.GDN_ERR_INVALID_ARG
+
+
 def test_chunked_kernel_needs_bf16_d128():
     d, off = _desc(dtype=gdn.GDN_F32, kernel=gdn.GDN_KERNEL_CHUNKED_TC)
     assert _create_replay(d, [50], [10]) == gdn.GDN_ERR_UNSUPPORTED
