@@ -80,3 +80,28 @@ def test_reference_arm_line():
     assert r["cpu_baseline"]["cores"] >= 1
     assert r["e2e"]["h2d_bytes_per_step"] == 0 and r["e2e"]["d2h_bytes_per_step"] == 0
     assert bench.bench_reference(A, 1, 2) is None      # other ranks do no work
+
+
+def test_profiled_traffic_matches_the_committed_record(monkeypatch):
+    """roofline.traffic: the committed ncu record applies to the current replay sources,
+    scales by work units, and is dropped for another kernel or changed sources."""
+    rec = {}
+    with open(bench.os.path.join(bench.ROOT, "profiles", "traffic.txt")) as f:
+        for line in f:
+            if ":" in line and not line.lstrip().startswith("#"):
+                k, v = line.split(":", 1)
+                rec[k.strip()] = v.strip()
+    units = int(rec["units"])
+    if rec["source_sha"] != bench.kernel_source_sha():     # the kernel changed since the capture
+        assert bench.profiled_traffic(rec["kernel"], units) is None
+        return
+    full = bench.profiled_traffic(rec["kernel"], units)
+    assert full == float(rec["dram_bytes"])
+    assert bench.profiled_traffic(rec["kernel"], units // 2) == pytest.approx(full / 2)
+    # the bench launch's algorithmic bytes: the measured traffic is within a few percent
+    R, d, H, layers = 3277, 128, 32, 8
+    alg = layers * H * (R * (2 * d * 2 + 8) + d * d * 4)
+    assert units == layers * H and 0.95 <= full / alg <= 1.05
+    assert bench.profiled_traffic("recurrent", units) is None
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda: "0" * 16)
+    assert bench.profiled_traffic(rec["kernel"], units) is None
