@@ -19,10 +19,13 @@ import os
 import numpy as np
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libgdn_tail_replay.so")
+# GDN_DEBUG_BOUNDS=1 in the environment selects the debug build, whose kernels
+# check every global index against the plan and report GDN_ERR_BOUNDS.
+DEBUG_BOUNDS = os.environ.get("GDN_DEBUG_BOUNDS", "0") not in ("", "0")
+LIB_PATH = os.path.join(_PKG, "libgdn_tail_replay_debug.so" if DEBUG_BOUNDS else "libgdn_tail_replay.so")
 
 GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT, \
-    GDN_ERR_ALLOC, GDN_ERR_MISMATCH = range(7)
+    GDN_ERR_ALLOC, GDN_ERR_MISMATCH, GDN_ERR_BOUNDS = range(8)
 GDN_F32, GDN_BF16 = 0, 1
 GDN_KERNEL_AUTO, GDN_KERNEL_RECURRENT, GDN_KERNEL_CHUNKED_TC = 0, 1, 2
 
@@ -32,7 +35,8 @@ EXPORTED = (
     "gdn_plan_info", "gdn_workspace_bytes", "gdn_tail_replay_state", "gdn_chunk_prefill",
     "gdn_workspace_status", "gdn_status_string", "gdn_version", "gdn_tail_replay_state_noalloc",
     "gdn_tail_replay_outputs", "gdn_decode_step", "gdn_plan_create_fused", "gdn_tail_replay_prefill",
-    "gdn_selftest_bounded_wait",
+    "gdn_selftest_bounded_wait", "gdn_debug_fail_plan_allocations", "gdn_selftest_index_check",
+    "gdn_debug_bounds_enabled",
 )
 
 
@@ -51,6 +55,7 @@ class gdn_varlen_desc(ctypes.Structure):
         ("dtype", ctypes.c_int32),
         ("kernel", ctypes.c_int32),
         ("seq_offsets_host", ctypes.POINTER(ctypes.c_int32)),
+        ("row_stride_elems", ctypes.c_int64),
     ]
 
 
@@ -81,6 +86,9 @@ def _load():
         "gdn_plan_create_fused": (I32, [pd, P, P, P, ctypes.POINTER(P)]),
         "gdn_tail_replay_prefill": (I32, [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P]),
         "gdn_selftest_bounded_wait": (I32, [ctypes.c_uint64, P, P]),
+        "gdn_debug_fail_plan_allocations": (None, [I32]),
+        "gdn_selftest_index_check": (I32, [P, P]),
+        "gdn_debug_bounds_enabled": (I32, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -151,42 +159,58 @@ def _dtype_code(dtype) -> int:
     raise ValueError(f"unsupported dtype {dtype}")
 
 
-def _make_desc(batch, H, dk, dv, dtype, kernel, offsets: np.ndarray):
+def _make_desc(batch, H, dk, dv, dtype, kernel, offsets: np.ndarray, row_stride=0):
     d = gdn_varlen_desc()
     d.batch, d.num_heads, d.d_k, d.d_v = int(batch), int(H), int(dk), int(dv)
     d.dtype = _dtype_code(dtype)
     d.kernel = int(kernel)
     d.seq_offsets_host = offsets.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    d.row_stride_elems = int(row_stride)
     return d
 
 
-def gdn_plan_create_replay(H, dk, dv, dtype, seq_offsets, match_len, R, kernel=GDN_KERNEL_AUTO):
+def row_stride_of(*tensors) -> int:
+    """Row stride (elements) shared by [rows, H, d] views of q, k and v, or 0 when each
+    is packed.  Heads must be contiguous inside a row (strides (., d, 1))."""
+    ts = [t for t in tensors if t is not None]
+    for t in ts:
+        if t.dim() != 3 or t.stride(2) != 1 or t.stride(1) != t.shape[2]:
+            raise ValueError("q/k/v must be [rows, H, d] views with contiguous heads inside a row")
+    if all(t.stride(0) == t.shape[1] * t.shape[2] for t in ts):
+        return 0
+    rs = {t.stride(0) for t in ts}
+    if len(rs) != 1:
+        raise ValueError("q, k and v must share one row stride (or all be packed)")
+    return rs.pop()
+
+
+def gdn_plan_create_replay(H, dk, dv, dtype, seq_offsets, match_len, R, kernel=GDN_KERNEL_AUTO, row_stride=0):
     """Create a replay plan; returns the raw handle (int).  Host int arrays."""
     off, ml, rr = _i32(seq_offsets), _i32(match_len), _i32(R)
     if len(off) != len(ml) + 1 or len(rr) != len(ml):
         raise ValueError("seq_offsets must have batch + 1 entries, match_len and R batch entries")
-    d = _make_desc(len(ml), H, dk, dv, dtype, kernel, off)
+    d = _make_desc(len(ml), H, dk, dv, dtype, kernel, off, row_stride)
     h = ctypes.c_void_p()
     _check(_lib.gdn_plan_create_replay(ctypes.byref(d), ml.ctypes.data, rr.ctypes.data,
                                        ctypes.byref(h)), "gdn_plan_create_replay")
     return h.value
 
 
-def gdn_plan_create_prefill(H, dk, dv, dtype, cu_seqlens, kernel=GDN_KERNEL_AUTO):
+def gdn_plan_create_prefill(H, dk, dv, dtype, cu_seqlens, kernel=GDN_KERNEL_AUTO, row_stride=0):
     off = _i32(cu_seqlens)
-    d = _make_desc(len(off) - 1, H, dk, dv, dtype, kernel, off)
+    d = _make_desc(len(off) - 1, H, dk, dv, dtype, kernel, off, row_stride)
     h = ctypes.c_void_p()
     _check(_lib.gdn_plan_create_prefill(ctypes.byref(d), ctypes.byref(h)), "gdn_plan_create_prefill")
     return h.value
 
 
 def gdn_plan_create_fused(H, dk, dv, dtype, seq_offsets, match_len, R, suffix_offsets,
-                          kernel=GDN_KERNEL_AUTO):
+                          kernel=GDN_KERNEL_AUTO, row_stride=0):
     """Create a fused replay + suffix plan; returns the raw handle (int).  Host int arrays."""
     off, ml, rr, so = _i32(seq_offsets), _i32(match_len), _i32(R), _i32(suffix_offsets)
     if len(off) != len(ml) + 1 or len(rr) != len(ml) or len(so) != len(ml) + 1:
         raise ValueError("seq_offsets and suffix_offsets need batch + 1 entries, match_len and R batch")
-    d = _make_desc(len(ml), H, dk, dv, dtype, kernel, off)
+    d = _make_desc(len(ml), H, dk, dv, dtype, kernel, off, row_stride)
     h = ctypes.c_void_p()
     _check(_lib.gdn_plan_create_fused(ctypes.byref(d), ml.ctypes.data, rr.ctypes.data, so.ctypes.data,
                                       ctypes.byref(h)), "gdn_plan_create_fused")
@@ -274,13 +298,14 @@ def gdn_chunk_prefill(handle, q, k, v, alpha, beta, cu_seqlens, state_in, o_out,
 
 
 def gdn_tail_replay_state_noalloc(H, dk, dv, dtype, seq_offsets, match_len, R, k, v, alpha, beta,
-                                  state_out, kernel=GDN_KERNEL_AUTO, stream=None, wait_status=True):
+                                  state_out, kernel=GDN_KERNEL_AUTO, stream=None, wait_status=True,
+                                  row_stride=0):
     """Replay without any device allocation (schedule in the library's fixed
     device array).  Returns the device status word when wait_status is set."""
     off, ml, rr = _i32(seq_offsets), _i32(match_len), _i32(R)
     if len(off) != len(ml) + 1 or len(rr) != len(ml):
         raise ValueError("seq_offsets must have batch + 1 entries, match_len and R batch entries")
-    d = _make_desc(len(ml), H, dk, dv, dtype, kernel, off)
+    d = _make_desc(len(ml), H, dk, dv, dtype, kernel, off, row_stride)
     st = ctypes.c_uint32(0xFFFFFFFF)
     _check(_lib.gdn_tail_replay_state_noalloc(ctypes.byref(d), ml.ctypes.data, rr.ctypes.data,
                                               _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
@@ -294,6 +319,21 @@ def gdn_selftest_bounded_wait(limit_ns, workspace, stream=None):
     """Launch the failure-path self-test: a device wait bounded by limit_ns that runs out."""
     _check(_lib.gdn_selftest_bounded_wait(int(limit_ns), _ptr(workspace), _stream_handle(stream)),
            "gdn_selftest_bounded_wait")
+
+
+def gdn_selftest_index_check(workspace, stream=None):
+    """Debug build only: run one failing index check (access skipped); the workspace
+    status then reads GDN_ERR_BOUNDS."""
+    _check(_lib.gdn_selftest_index_check(_ptr(workspace), _stream_handle(stream)), "gdn_selftest_index_check")
+
+
+def gdn_debug_bounds_enabled() -> bool:
+    return bool(_lib.gdn_debug_bounds_enabled())
+
+
+def gdn_debug_fail_plan_allocations(count):
+    """Make the next `count` plan creations fail with GDN_ERR_ALLOC (0 clears it)."""
+    _lib.gdn_debug_fail_plan_allocations(int(count))
 
 
 def gdn_workspace_status(workspace, stream=None) -> int:
@@ -332,8 +372,8 @@ class _Plan:
 class ReplayPlan(_Plan):
     """Plan of a tail replay over a packed varlen cache (host int arrays)."""
 
-    def __init__(self, H, dk, dv, dtype, seq_offsets, match_len, R, kernel=GDN_KERNEL_AUTO):
-        h = gdn_plan_create_replay(H, dk, dv, dtype, seq_offsets, match_len, R, kernel)
+    def __init__(self, H, dk, dv, dtype, seq_offsets, match_len, R, kernel=GDN_KERNEL_AUTO, row_stride=0):
+        h = gdn_plan_create_replay(H, dk, dv, dtype, seq_offsets, match_len, R, kernel, row_stride)
         super().__init__(h, H, dk, dv, dtype, len(match_len))
 
     def run(self, k, v, alpha, beta, state_out, q=None, seq_offsets=None, match_len=None, R=None,
@@ -351,8 +391,8 @@ class ReplayPlan(_Plan):
 class PrefillPlan(_Plan):
     """Plan of a chunked prefill over whole packed sequences (host cu_seqlens)."""
 
-    def __init__(self, H, dk, dv, dtype, cu_seqlens, kernel=GDN_KERNEL_AUTO):
-        h = gdn_plan_create_prefill(H, dk, dv, dtype, cu_seqlens, kernel)
+    def __init__(self, H, dk, dv, dtype, cu_seqlens, kernel=GDN_KERNEL_AUTO, row_stride=0):
+        h = gdn_plan_create_prefill(H, dk, dv, dtype, cu_seqlens, kernel, row_stride)
         super().__init__(h, H, dk, dv, dtype, len(cu_seqlens) - 1)
 
     def run(self, q, k, v, alpha, beta, o_out, state_in=None, state_out=None, cu_seqlens=None,
@@ -364,8 +404,10 @@ class PrefillPlan(_Plan):
 class FusedPlan(_Plan):
     """Plan of a fused replay + suffix prefill (host int arrays)."""
 
-    def __init__(self, H, dk, dv, dtype, seq_offsets, match_len, R, suffix_offsets, kernel=GDN_KERNEL_AUTO):
-        h = gdn_plan_create_fused(H, dk, dv, dtype, seq_offsets, match_len, R, suffix_offsets, kernel)
+    def __init__(self, H, dk, dv, dtype, seq_offsets, match_len, R, suffix_offsets, kernel=GDN_KERNEL_AUTO,
+                 row_stride=0):
+        h = gdn_plan_create_fused(H, dk, dv, dtype, seq_offsets, match_len, R, suffix_offsets, kernel,
+                                  row_stride)
         super().__init__(h, H, dk, dv, dtype, len(match_len))
 
     def run(self, k, v, alpha, beta, sq, sk, sv, salpha, sbeta, o_out, state_out, state_mid=None, stream=None,
@@ -375,11 +417,12 @@ class FusedPlan(_Plan):
 
 
 def tail_replay_state(k, v, alpha, beta, seq_offsets, match_len, R, kernel=GDN_KERNEL_AUTO):
-    """One-shot replay on torch CUDA tensors; returns state [B, H, dk, dv] fp32."""
+    """One-shot replay on torch CUDA tensors; returns state [B, H, dk, dv] fp32.  k and v
+    may be row-strided views (e.g. slices of one fused projection buffer)."""
     import torch
     rows, H, dk = k.shape
     dv = v.shape[2]
-    plan = ReplayPlan(H, dk, dv, k.dtype, seq_offsets, match_len, R, kernel)
+    plan = ReplayPlan(H, dk, dv, k.dtype, seq_offsets, match_len, R, kernel, row_stride_of(k, v))
     out = torch.empty((plan.batch, H, dk, dv), dtype=torch.float32, device=k.device)
     plan.run(k, v, alpha, beta, out)
     plan.check()
@@ -388,11 +431,12 @@ def tail_replay_state(k, v, alpha, beta, seq_offsets, match_len, R, kernel=GDN_K
 
 
 def chunk_prefill(q, k, v, alpha, beta, cu_seqlens, state_in=None, kernel=GDN_KERNEL_AUTO):
-    """One-shot prefill on torch CUDA tensors; returns (o, state_out)."""
+    """One-shot prefill on torch CUDA tensors; returns (o, state_out).  q, k and v may be
+    row-strided views sharing one row stride; o is packed."""
     import torch
     rows, H, dk = k.shape
     dv = v.shape[2]
-    plan = PrefillPlan(H, dk, dv, k.dtype, cu_seqlens, kernel)
+    plan = PrefillPlan(H, dk, dv, k.dtype, cu_seqlens, kernel, row_stride_of(q, k, v))
     o = torch.empty((rows, H, dv), dtype=k.dtype, device=k.device)
     st = torch.empty((plan.batch, H, dk, dv), dtype=torch.float32, device=k.device)
     plan.run(q, k, v, alpha, beta, o, state_in=state_in, state_out=st)

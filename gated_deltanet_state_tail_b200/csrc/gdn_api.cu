@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <new>
@@ -24,6 +25,7 @@ using gdn::WorkspaceHeader;
 struct gdn_plan {
     int kind;
     int batch, num_heads, dk, dv, dtype, kernel;
+    long long rs_qk, rs_v;    // row strides (elements) of q/k and of v
     int device;
     std::vector<Window> windows;   // replay: the tail windows; prefill and fused: the (suffix) sequences
     std::vector<Window> windows0;  // fused: the replay windows run before `windows`
@@ -41,22 +43,50 @@ namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-gdn_status check_desc(const gdn_varlen_desc* d) {
+}  // namespace
+
+namespace gdn {
+
+gdn_status check_varlen_desc(const gdn_varlen_desc* d) {
     if (!d || !d->seq_offsets_host) return GDN_ERR_INVALID_ARG;
     if (d->batch < 1 || d->num_heads < 1) return GDN_ERR_INVALID_ARG;
     if (d->dtype != GDN_F32 && d->dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
     if ((d->d_k != 64 && d->d_k != 128) || (d->d_v != 64 && d->d_v != 128)) return GDN_ERR_UNSUPPORTED;
     if (d->kernel < GDN_KERNEL_AUTO || d->kernel > GDN_KERNEL_CHUNKED_TC) return GDN_ERR_INVALID_ARG;
+    // row stride: 0 = packed; otherwise every head of a row fits and rows start on 16 bytes
+    if (d->row_stride_elems != 0) {
+        const long long elem = d->dtype == GDN_BF16 ? 2 : 4;
+        const long long widest = (long long)d->num_heads * (d->d_k > d->d_v ? d->d_k : d->d_v);
+        if (d->row_stride_elems < widest || (d->row_stride_elems * elem) % 16 != 0) return GDN_ERR_INVALID_ARG;
+        if (d->row_stride_elems > (1ll << 40)) return GDN_ERR_INVALID_ARG;
+    }
     const int32_t* off = d->seq_offsets_host;
     if (off[0] < 0) return GDN_ERR_INVALID_ARG;
     for (int b = 0; b < d->batch; ++b)
         if (off[b + 1] < off[b]) return GDN_ERR_INVALID_ARG;
-    // element offsets are 64-bit on the device; rows * H * d must fit comfortably
+    // element offsets are 64-bit on the device; rows * row stride must fit comfortably
     const long long rows = off[d->batch];
-    if (rows * d->num_heads > (1ll << 40)) return GDN_ERR_INVALID_ARG;
+    const long long rs = row_stride_qk(d) > row_stride_v(d) ? row_stride_qk(d) : row_stride_v(d);
+    if (rows * d->num_heads > (1ll << 40) || rows * rs > (1ll << 46)) return GDN_ERR_INVALID_ARG;
     // one CTA per (sequence, head) unit: the unit count is the grid's x extent
     if ((long long)d->batch * d->num_heads > 0x7fffffffll) return GDN_ERR_INVALID_ARG;
     return GDN_OK;
+}
+
+}  // namespace gdn
+
+namespace {
+
+gdn_status check_desc(const gdn_varlen_desc* d) { return gdn::check_varlen_desc(d); }
+
+// Plan creations still to fail with GDN_ERR_ALLOC (gdn_debug_fail_plan_allocations).
+std::atomic<int> g_fail_plan_allocs{0};
+
+bool take_injected_alloc_failure() {
+    int pending = g_fail_plan_allocs.load(std::memory_order_relaxed);
+    while (pending > 0 && !g_fail_plan_allocs.compare_exchange_weak(pending, pending - 1)) {
+    }
+    return pending > 0;
 }
 
 int resolve_kernel(const gdn_varlen_desc* d) {
@@ -88,6 +118,8 @@ gdn_status finish_plan(gdn_plan* p, gdn_plan_t* out) {
         p->rows_total0 = std::max(p->rows_total0, (long long)w.expect_end);
     }
 
+    // an injected failure stands where the device allocation would fail
+    if (take_injected_alloc_failure()) return GDN_ERR_ALLOC;
     if (cudaGetDevice(&p->device) != cudaSuccess) return GDN_ERR_CUDA;
     const size_t wbytes = sizeof(Window) * p->windows.size();
     const size_t w0bytes = sizeof(Window) * p->windows0.size();
@@ -133,6 +165,8 @@ gdn_plan* new_plan(const gdn_varlen_desc* d, int kind) {
     p->dv = d->d_v;
     p->dtype = d->dtype;
     p->kernel = resolve_kernel(d);
+    p->rs_qk = gdn::row_stride_qk(d);
+    p->rs_v = gdn::row_stride_v(d);
     p->dev_block = nullptr;
     p->d_windows0 = nullptr;
     return p;
@@ -200,6 +234,8 @@ void fill_common(gdn_plan_t plan, CallArgs& a, void* workspace) {
     a.batch = plan->batch;
     a.units = (long long)plan->units.size();
     a.rows_total = plan->rows_total;
+    a.rs_qk = plan->rs_qk;
+    a.rs_v = plan->rs_v;
     a.windows = plan->d_windows;
     a.unit_list = plan->d_units;
     a.ws = static_cast<WorkspaceHeader*>(workspace);
@@ -547,8 +583,13 @@ gdn_status gdn_workspace_status(const void* workspace, void* stream) {
         return GDN_ERR_CUDA;
     }
     if (status & gdn::kStatusTimeout) return GDN_ERR_TIMEOUT;
+    if (status & gdn::kStatusBounds) return GDN_ERR_BOUNDS;
     if (status & gdn::kStatusMismatch) return GDN_ERR_MISMATCH;
     return GDN_OK;
+}
+
+void gdn_debug_fail_plan_allocations(int32_t count) {
+    g_fail_plan_allocs.store(count > 0 ? count : 0, std::memory_order_relaxed);
 }
 
 const char* gdn_status_string(gdn_status s) {
@@ -560,10 +601,11 @@ const char* gdn_status_string(gdn_status s) {
         case GDN_ERR_TIMEOUT: return "device wait timed out";
         case GDN_ERR_ALLOC: return "allocation failed";
         case GDN_ERR_MISMATCH: return "device descriptor arrays disagree with the plan";
+        case GDN_ERR_BOUNDS: return "device index outside the plan's extents (debug build)";
     }
     return "unknown status";
 }
 
-int32_t gdn_version(void) { return 200; }
+int32_t gdn_version(void) { return 300; }
 
 }  // extern "C"

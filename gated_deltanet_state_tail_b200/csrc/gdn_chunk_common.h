@@ -13,9 +13,10 @@
 
 namespace gdn {
 
-// [rows][H][128] bf16 viewed as (d, H, rows), box 64 x 1 x 64, 128-byte swizzle,
-// rows past `rows` read as zero (defined with the chunked prefill).
-bool make_tile_map(CUtensorMap* m, const void* base, int H, long long rows);
+// [rows][H][128] bf16 rows `row_stride` elements apart, viewed as (d, H, rows), box
+// 64 x 1 x 64, 128-byte swizzle, rows past `rows` read as zero (defined with the
+// chunked prefill).
+bool make_tile_map(CUtensorMap* m, const void* base, int H, long long rows, long long row_stride);
 
 namespace chunk {
 
@@ -351,6 +352,7 @@ __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, const C
 }
 
 // TMA of one chunk's tiles: K and V, and Q when the chunk writes outputs.
+// (Tile loads need no bounds check: TMA reads zeros past the map's extent.)
 template <bool REPLAY>
 __device__ __forceinline__ void issue_tiles(uint8_t* tile, uint64_t* bar, const CUtensorMap* mk, const CUtensorMap* mv,
                                             const CUtensorMap* mq, int h, int r0, bool with_q) {

@@ -103,6 +103,11 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     if (fused) w0 = a.windows0[b];
     const int nA = (w0.len + C - 1) / C;
     const int nchunks = nA + (w.len + C - 1) / C;
+    // debug build: the unit and its row ranges lie inside the plan's extents (uniform)
+    if (!index_ok(a.ws, b >= 0 && b < a.batch && h >= 0 && h < H && w.row0 >= 0 && w.len >= 0 &&
+                            w.row0 + w.len <= a.rows_total && w0.row0 >= 0 && w0.len >= 0 &&
+                            w0.row0 + w0.len <= (fused ? a.rows_total0 : 0)))
+        return;
     struct ChunkSrc {
         long long r0;
         int nc;
@@ -189,8 +194,11 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             if (tid < cs.nc) {
                 const float* pa = cc < nA ? a.alpha0 : a.alpha;
                 const float* pb = cc < nA ? a.beta0 : a.beta;
-                al = pa[(cs.r0 + tid) * H + h];
-                be = pb[(cs.r0 + tid) * H + h];
+                const long long r = cs.r0 + tid;
+                if (index_ok(a.ws, r < (cc < nA ? a.rows_total0 : a.rows_total))) {
+                    al = pa[r * H + h];
+                    be = pb[r * H + h];
+                }
             }
         }
     };
@@ -390,7 +398,7 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
 #pragma unroll
                 for (int k = 0; k < (C * D / 8) / 128; ++k) {   // 16-byte pieces: 16 per row
                     const int idx = ct + k * 128, i = idx >> 4, ch = idx & 15;
-                    if (i < src.nc)
+                    if (i < src.nc && index_ok(a.ws, src.r0 + i < a.rows_total))
                         *reinterpret_cast<uint4*>(o + ((src.r0 + i) * H + h) * (long long)D + ch * 8) =
                             *reinterpret_cast<const uint4*>(stage + i * D + ch * 8);
                 }
@@ -579,13 +587,14 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-// [rows][H][128] bf16, box = 64 columns x 1 head x 64 rows, 128-byte swizzle.
-bool make_tile_map(CUtensorMap* m, const void* base, int H, long long rows) {
+// [rows][H][128] bf16 with rows row_stride elements apart, box = 64 columns x 1 head
+// x 64 rows, 128-byte swizzle.
+bool make_tile_map(CUtensorMap* m, const void* base, int H, long long rows, long long row_stride) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     if (rows < 1) rows = 1;
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
-    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)row_stride * 2};
     cuuint32_t box[3] = {64, 1, 64};
     cuuint32_t es[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
@@ -609,16 +618,17 @@ cudaError_t launch_chunk_tc(const CallArgs& a, cudaStream_t stream) {
     const void* vb = a.v ? a.v : static_cast<const void*>(a.ws);
     const void* qb = a.q ? a.q : static_cast<const void*>(a.ws);
     CUtensorMap mk, mv, mq;
-    if (!make_tile_map(&mk, kb, a.num_heads, a.rows_total) || !make_tile_map(&mv, vb, a.num_heads, a.rows_total) ||
-        !make_tile_map(&mq, qb, a.num_heads, a.rows_total))
+    if (!make_tile_map(&mk, kb, a.num_heads, a.rows_total, a.rs_qk) ||
+        !make_tile_map(&mv, vb, a.num_heads, a.rows_total, a.rs_v) ||
+        !make_tile_map(&mq, qb, a.num_heads, a.rows_total, a.rs_qk))
         return cudaErrorInvalidValue;
     // fused replay + suffix: maps of the replayed cache rows (otherwise unused copies)
     CUtensorMap mk0 = mk, mv0 = mv;
     if (a.windows0) {
         const void* kb0 = a.k0 ? a.k0 : static_cast<const void*>(a.ws);
         const void* vb0 = a.v0 ? a.v0 : static_cast<const void*>(a.ws);
-        if (!make_tile_map(&mk0, kb0, a.num_heads, a.rows_total0) ||
-            !make_tile_map(&mv0, vb0, a.num_heads, a.rows_total0))
+        if (!make_tile_map(&mk0, kb0, a.num_heads, a.rows_total0, a.rs_qk) ||
+            !make_tile_map(&mv0, vb0, a.num_heads, a.rows_total0, a.rs_v))
             return cudaErrorInvalidValue;
     }
     static std::atomic<uint64_t> smem_set{0};

@@ -7,6 +7,8 @@
 
 #include <atomic>
 
+#include "gdn_tail_replay.h"
+
 namespace gdn {
 
 // Work window of one sequence, as validated on the host by the plan.
@@ -34,14 +36,30 @@ struct Unit {
 // Per-call device scratch at the start of the caller's workspace.
 struct WorkspaceHeader {
     unsigned int status;        // bit set of kStatus*
-    unsigned int next_unit;     // dynamic scheduler counter
     unsigned int timeout_where; // first wait that gave up (kernel-defined code)
-    unsigned int pad[61];
+    unsigned int pad[62];
 };
 static_assert(sizeof(WorkspaceHeader) == 256, "header is 256 bytes");
 
 constexpr unsigned int kStatusMismatch = 1u;
 constexpr unsigned int kStatusTimeout = 2u;
+constexpr unsigned int kStatusBounds = 4u;   // a checked index fell outside the plan (debug build)
+
+// Index checks of the debug build (compiled with -DGDN_DEBUG_BOUNDS).  Each
+// computed global row, head, column and state index is compared with the
+// extents the plan validated on the host; a failing check sets kStatusBounds
+// and the access is skipped (no trap, no out-of-range access).  In the release
+// build every check is the constant `true` and compiles away.
+#ifdef GDN_DEBUG_BOUNDS
+constexpr bool kDebugBounds = true;
+__device__ __forceinline__ bool index_ok(WorkspaceHeader* ws, bool cond) {
+    if (!cond) atomicOr(&ws->status, kStatusBounds);
+    return cond;
+}
+#else
+constexpr bool kDebugBounds = false;
+__device__ __forceinline__ bool index_ok(WorkspaceHeader*, bool) { return true; }
+#endif
 
 // kFused: the replay window of each sequence, then its suffix with outputs, in one launch
 enum PlanKind { kReplay = 0, kPrefill = 1, kFused = 2 };
@@ -55,6 +73,8 @@ struct CallArgs {
     int batch;
     long long units;
     long long rows_total;   // rows of the packed buffers the plan addresses (max offset)
+    long long rs_qk;        // elements between consecutive rows of q and k (H * dk when packed)
+    long long rs_v;         // elements between consecutive rows of v (H * dv when packed)
     const Window* windows;  // [batch], plan-owned device memory
     const Unit* unit_list;  // [units], longest first
     // optional device descriptor arrays to check against the plan
@@ -123,6 +143,18 @@ inline cudaError_t ensure_smem_limit(const void* kernel, int bytes, std::atomic<
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e == cudaSuccess) done_devices.fetch_or(bit, std::memory_order_acq_rel);
     return e;
+}
+
+// Host validation of a varlen descriptor shared by every entry point that takes
+// one: sizes, dtype, kernel choice, offsets, row stride and the 64-bit extent bound.
+gdn_status check_varlen_desc(const gdn_varlen_desc* d);
+
+// Row strides (elements) of q/k and of v that a descriptor implies.
+inline long long row_stride_qk(const gdn_varlen_desc* d) {
+    return d->row_stride_elems ? d->row_stride_elems : (long long)d->num_heads * d->d_k;
+}
+inline long long row_stride_v(const gdn_varlen_desc* d) {
+    return d->row_stride_elems ? d->row_stride_elems : (long long)d->num_heads * d->d_v;
 }
 
 cudaError_t launch_recurrent(const CallArgs& a, cudaStream_t stream);

@@ -8,7 +8,9 @@
 // schedule table and the status word live in one file-scope __device__
 // array of fixed size, which every GPU that loads this library holds until
 // the process exits.  Nothing here calls cudaMalloc, cudaFree or any
-// allocating routine; the host-side schedule is built in a stack buffer.
+// allocating routine; the host-side schedule is built in a per-thread static
+// buffer (not on the stack: the callers this serves may run on threads with
+// small stacks).
 //
 // The array is shared by every call on a device and keeps the last call's
 // contents: each call rewrites the schedule and clears the status word
@@ -16,7 +18,6 @@
 // (different streams, or several host threads at once) race on it.
 #include <cuda_runtime.h>
 
-#include <atomic>
 #include <cstdint>
 #include <cstring>
 
@@ -28,22 +29,24 @@ namespace {
 constexpr size_t kScratchBytes = 64 * 1024;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::atomic<void*> g_scratch_addr[kMaxDevices];
-
-// Device address of the scratch array on the current device (resolved once
-// per device; the first call on a device does it).
-void* scratch_address(int dev) {
-    if (dev < 0 || dev >= kMaxDevices) return nullptr;
-    void* p = g_scratch_addr[dev].load(std::memory_order_acquire);
-    if (p) return p;
+// Device address of the scratch array in the current device's context.  It is
+// resolved on every call (a cheap host lookup once the module is loaded): a
+// cached address would go stale if the context were destroyed and recreated
+// (cudaDeviceReset), since the array can then land elsewhere.  The first call
+// on a device also loads this library's device code there.
+void* scratch_address() {
+    void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
         cudaGetLastError();
         return nullptr;
     }
-    g_scratch_addr[dev].store(p, std::memory_order_release);
     return p;
 }
+
+// Host staging of the schedule, one buffer per host thread.  cudaMemcpyAsync
+// from pageable memory has read the source by the time it returns, so the
+// next call on the same thread may overwrite it at once.
+thread_local unsigned char t_host_stage[kScratchBytes] __attribute__((aligned(16)));
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -59,12 +62,10 @@ extern "C" gdn_status gdn_tail_replay_state_noalloc(const gdn_varlen_desc* cache
     using gdn::Unit;
     using gdn::Window;
     using gdn::WorkspaceHeader;
-    if (!cache || !cache->seq_offsets_host || !match_len_host || !R_host) return GDN_ERR_INVALID_ARG;
-    if (cache->batch < 1 || cache->num_heads < 1) return GDN_ERR_INVALID_ARG;
-    if (cache->dtype != GDN_F32 && cache->dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
-    if ((cache->d_k != 64 && cache->d_k != 128) || (cache->d_v != 64 && cache->d_v != 128))
-        return GDN_ERR_UNSUPPORTED;
-    if (cache->kernel < GDN_KERNEL_AUTO || cache->kernel > GDN_KERNEL_CHUNKED_TC) return GDN_ERR_INVALID_ARG;
+    // the same descriptor checks a replay plan makes
+    gdn_status s0 = gdn::check_varlen_desc(cache);
+    if (s0 != GDN_OK) return s0;
+    if (!match_len_host || !R_host) return GDN_ERR_INVALID_ARG;
     const int batch = cache->batch, H = cache->num_heads;
     const size_t need = sizeof(WorkspaceHeader) + sizeof(Window) * (size_t)batch +
                         sizeof(Unit) * (size_t)batch * (size_t)H;
@@ -78,7 +79,7 @@ extern "C" gdn_status gdn_tail_replay_state_noalloc(const gdn_varlen_desc* cache
     // Temporaries (window rows and lengths, sequence order) sit after it.
     const size_t tmp_bytes = (sizeof(int64_t) + 2 * sizeof(int32_t)) * (size_t)batch;
     if (need + tmp_bytes > kScratchBytes) return GDN_ERR_UNSUPPORTED;
-    alignas(16) unsigned char host[kScratchBytes];
+    unsigned char* host = t_host_stage;
     Window* win = reinterpret_cast<Window*>(host + sizeof(WorkspaceHeader));
     Unit* units = reinterpret_cast<Unit*>(host + sizeof(WorkspaceHeader) + sizeof(Window) * batch);
     int64_t* row0 = reinterpret_cast<int64_t*>(host + ((need + 15) & ~size_t(15)));
@@ -123,15 +124,10 @@ extern "C" gdn_status gdn_tail_replay_state_noalloc(const gdn_varlen_desc* cache
         }
         if (!state_out || !aligned16(state_out)) return GDN_ERR_INVALID_ARG;
 
-        int dev = -1;
-        if (cudaGetDevice(&dev) != cudaSuccess) {
-            cudaGetLastError();
-            return GDN_ERR_CUDA;
-        }
-        unsigned char* scratch = static_cast<unsigned char*>(scratch_address(dev));
+        unsigned char* scratch = static_cast<unsigned char*>(scratch_address());
         if (!scratch) return GDN_ERR_CUDA;
         cudaStream_t st = static_cast<cudaStream_t>(stream);
-        std::memset(host, 0, sizeof(WorkspaceHeader));   // status word and counters start at zero
+        std::memset(host, 0, sizeof(WorkspaceHeader));   // status word and wait site start at zero
         if (cudaMemcpyAsync(scratch, host, need, cudaMemcpyHostToDevice, st) != cudaSuccess) {
             cudaGetLastError();
             return GDN_ERR_CUDA;
@@ -146,6 +142,8 @@ extern "C" gdn_status gdn_tail_replay_state_noalloc(const gdn_varlen_desc* cache
         a.batch = batch;
         a.units = (long long)batch * H;
         a.rows_total = rows_total;
+        a.rs_qk = gdn::row_stride_qk(cache);
+        a.rs_v = gdn::row_stride_v(cache);
         a.windows = reinterpret_cast<const Window*>(scratch + sizeof(WorkspaceHeader));
         a.unit_list = reinterpret_cast<const Unit*>(scratch + sizeof(WorkspaceHeader) + sizeof(Window) * batch);
         a.k = k;

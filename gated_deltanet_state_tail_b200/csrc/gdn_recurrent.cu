@@ -49,8 +49,8 @@ __device__ __forceinline__ void store1(float* p, float x) { *p = x; }
 __device__ __forceinline__ void store1(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
 
 // Stage rows [t0, t0 + n) of one head (n <= kStageTokens) into shared memory
-// as fp32.  Element loads are 4-wide vectors; all row strides are multiples
-// of 4 elements because d_k, d_v are multiples of 64.
+// as fp32.  Element loads are 4-wide vectors: every row stride is a multiple
+// of 16 bytes (the host checks it) and d_k, d_v are multiples of 64.
 template <typename T, int DK, int DV, bool OUT>
 __device__ __forceinline__ void stage_rows(const CallArgs& a, long long row0, int t0, int n, int h,
                                            float* sk, float* sv, float* sq, float* sa, float* sb) {
@@ -60,16 +60,19 @@ __device__ __forceinline__ void stage_rows(const CallArgs& a, long long row0, in
     const T* q = static_cast<const T*>(a.q);
     for (int e = threadIdx.x * 4; e < n * DK; e += blockDim.x * 4) {
         int j = e / DK, i = e % DK;
-        long long g = ((row0 + t0 + j) * H + h) * (long long)DK + i;
+        if (!index_ok(a.ws, row0 + t0 + j < a.rows_total)) continue;
+        long long g = (row0 + t0 + j) * a.rs_qk + (long long)h * DK + i;
         load4<T>(k + g, sk + e);
         if (OUT) load4<T>(q + g, sq + e);
     }
     for (int e = threadIdx.x * 4; e < n * DV; e += blockDim.x * 4) {
         int j = e / DV, i = e % DV;
-        long long g = ((row0 + t0 + j) * H + h) * (long long)DV + i;
+        if (!index_ok(a.ws, row0 + t0 + j < a.rows_total)) continue;
+        long long g = (row0 + t0 + j) * a.rs_v + (long long)h * DV + i;
         load4<T>(v + g, sv + e);
     }
     for (int j = threadIdx.x; j < n; j += blockDim.x) {
+        if (!index_ok(a.ws, row0 + t0 + j < a.rows_total)) continue;
         long long g = (row0 + t0 + j) * H + h;
         sa[j] = a.alpha[g];
         sb[j] = a.beta[g];
@@ -98,6 +101,10 @@ __global__ void __launch_bounds__(64 * (DK / 64), 3) recurrent_kernel(const Call
     }
     const Window w = a.windows[b];
     const size_t state_base = ((size_t)b * a.num_heads + h) * DK * DV;
+    // debug build: the unit, its column block and its window lie inside the plan (uniform)
+    if (!index_ok(a.ws, b >= 0 && b < a.batch && h >= 0 && h < a.num_heads && blockIdx.y * COLS + COLS <= DV &&
+                            w.row0 >= 0 && w.len >= 0 && w.row0 + w.len <= a.rows_total))
+        return;
 
     float s[KR];
     float sigma = 1.0f;
@@ -171,7 +178,7 @@ __global__ void __launch_bounds__(64 * (DK / 64), 3) recurrent_kernel(const Call
                 }
                 float ov = ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
                 if (KS == 2) ov += __shfl_xor_sync(0xffffffffu, ov, 1);
-                if (part == 0)
+                if (part == 0 && index_ok(a.ws, w.row0 + t0 + j < a.rows_total))
                     store1(o + ((w.row0 + t0 + j) * a.num_heads + h) * (long long)DV + c, sigma * ov);
             }
         }

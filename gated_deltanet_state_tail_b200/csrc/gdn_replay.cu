@@ -64,6 +64,10 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     }
     const Window w = a.windows[b];
     const int nchunks = (w.len + C - 1) / C;
+    // debug build: the unit and its window lie inside the plan's extents (uniform)
+    if (!index_ok(a.ws, b >= 0 && b < a.batch && h >= 0 && h < H && w.row0 >= 0 && w.len >= 0 &&
+                            w.row0 + w.len <= a.rows_total))
+        return;
 
     if (tid == 0) {
         mbar_init(&bar_tile[0], 1);
@@ -117,8 +121,11 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         al = 1.0f;
         be = 0.0f;
         if (tid < C && cc * C + tid < w.len) {
-            al = a.alpha[(w.row0 + (long long)cc * C + tid) * H + h];
-            be = a.beta[(w.row0 + (long long)cc * C + tid) * H + h];
+            const long long r = w.row0 + (long long)cc * C + tid;
+            if (index_ok(a.ws, r < a.rows_total)) {
+                al = a.alpha[r * H + h];
+                be = a.beta[r * H + h];
+            }
         }
     };
     auto tiles_ready = [&](int cc) -> bool {
@@ -429,7 +436,8 @@ cudaError_t launch_replay_tc(const CallArgs& a, cudaStream_t stream) {
     const void* kb = a.k ? a.k : static_cast<const void*>(a.ws);
     const void* vb = a.v ? a.v : static_cast<const void*>(a.ws);
     CUtensorMap mk, mv;
-    if (!make_tile_map(&mk, kb, a.num_heads, a.rows_total) || !make_tile_map(&mv, vb, a.num_heads, a.rows_total))
+    if (!make_tile_map(&mk, kb, a.num_heads, a.rows_total, a.rs_qk) ||
+        !make_tile_map(&mv, vb, a.num_heads, a.rows_total, a.rs_v))
         return cudaErrorInvalidValue;
     static std::atomic<uint64_t> smem_set{0};
     const uint32_t smem = Layout<true>::BYTES + 1024;

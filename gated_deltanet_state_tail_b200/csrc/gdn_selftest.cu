@@ -1,8 +1,9 @@
-// gdn_selftest.cu -- self-test of the device-side failure path that every
-// kernel's bounded waits use: a wait that runs out sets kStatusTimeout and the
+// gdn_selftest.cu -- self-tests of the device-side failure paths.  Every
+// kernel's bounded waits: a wait that runs out sets kStatusTimeout and the
 // wait site in the workspace header, and the kernel returns instead of hanging
 // or trapping, so the context stays usable and the host reads the status with
-// gdn_workspace_status().
+// gdn_workspace_status().  The debug build's index checks: a failing check
+// sets kStatusBounds and skips the access it guards.
 #include <cuda_runtime.h>
 
 #include "gdn_internal.h"
@@ -25,6 +26,15 @@ __global__ void bounded_wait_selftest_kernel(WorkspaceHeader* ws, unsigned long 
     }
 }
 
+// The debug build's index check on an index one past a stated 4-element extent:
+// the check records kStatusBounds and skips the store it guards.  (The index
+// is still inside the header's pad array, so even an unchecked store would
+// stay in the caller's workspace.)
+__global__ void index_check_selftest_kernel(WorkspaceHeader* ws) {
+    const long long extent = 4, idx = extent;   // one past the end
+    if (index_ok(ws, idx < extent)) ws->pad[idx] = 1u;
+}
+
 }  // namespace
 }  // namespace gdn
 
@@ -41,3 +51,19 @@ extern "C" gdn_status gdn_selftest_bounded_wait(uint64_t limit_ns, void* workspa
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     return GDN_OK;
 }
+
+extern "C" gdn_status gdn_selftest_index_check(void* workspace, void* stream) {
+    if (!gdn::kDebugBounds) return GDN_ERR_UNSUPPORTED;   // the release build has no index checks
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 15u) != 0) return GDN_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    auto* ws = static_cast<gdn::WorkspaceHeader*>(workspace);
+    if (cudaMemsetAsync(ws, 0, sizeof(gdn::WorkspaceHeader), st) != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_CUDA;
+    }
+    gdn::index_check_selftest_kernel<<<1, 1, 0, st>>>(ws);
+    if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+    return GDN_OK;
+}
+
+extern "C" int32_t gdn_debug_bounds_enabled(void) { return gdn::kDebugBounds ? 1 : 0; }

@@ -20,10 +20,13 @@
  *
  * Conventions shared by every call
  * --------------------------------
- *  Layout.  q, k: [rows, H, d_k]; v, o: [rows, H, d_v]; token-major packed
- *    rows, contiguous (row stride H*d elements).  alpha, beta: [rows, H]
- *    fp32 always (bf16 would round 0.999 to 1).  States: [batch, H, d_k,
- *    d_v] fp32, row-major, key dimension first.
+ *  Layout.  q, k: [rows, H, d_k]; v, o: [rows, H, d_v]; token-major rows,
+ *    heads contiguous inside a row.  The rows of q, k and v are
+ *    gdn_varlen_desc.row_stride_elems elements apart (0 = packed: H*d_k for
+ *    q and k, H*d_v for v), so q, k and v may be slices of one fused
+ *    projection buffer; o is always packed (row stride H*d_v).  alpha, beta:
+ *    [rows, H] fp32 always (bf16 would round 0.999 to 1), packed.  States:
+ *    [batch, H, d_k, d_v] fp32, row-major, key dimension first.
  *  dtype.  q, k, v and o share one element type: GDN_F32 or GDN_BF16.
  *  Ownership.  The caller owns every buffer.  The library allocates device
  *    memory only inside gdn_plan_create_* (a small schedule table) and frees
@@ -63,7 +66,8 @@ typedef enum gdn_status {
     GDN_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
     GDN_ERR_TIMEOUT = 4,      /* a device-side wait gave up (reported via the workspace) */
     GDN_ERR_ALLOC = 5,        /* plan creation could not allocate */
-    GDN_ERR_MISMATCH = 6      /* device descriptor arrays disagree with the plan */
+    GDN_ERR_MISMATCH = 6,     /* device descriptor arrays disagree with the plan */
+    GDN_ERR_BOUNDS = 7        /* debug build: a device index fell outside the plan's extents */
 } gdn_status;
 
 typedef enum gdn_dtype { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
@@ -77,8 +81,14 @@ typedef enum gdn_kernel {
 } gdn_kernel;
 
 /* Varlen batch descriptor.  Sequence b occupies rows [seq_offsets[b],
- * seq_offsets[b+1]) of the packed buffers.  Layer stacks are folded in by
- * treating (layer, request) pairs as sequences of one packed batch. */
+ * seq_offsets[b+1]) of the row buffers.  Layer stacks are folded in by
+ * treating (layer, request) pairs as sequences of one batch.
+ * row_stride_elems: elements from one row of q, k or v to the next; 0 means
+ * packed.  Otherwise it must be >= H * max(d_k, d_v) and a multiple of 16
+ * bytes (8 bf16 or 4 fp32 elements: the tensor-core kernel reads rows with
+ * TMA, whose strides are 16-byte multiples).  A fused [rows, 3, H, d]
+ * projection buffer, for example, gives q, k and v with row stride 3*H*d.
+ * rows * row stride must stay below 2^40 elements. */
 typedef struct gdn_varlen_desc {
     int32_t batch;                    /* number of sequences, >= 1 */
     int32_t num_heads;                /* H, >= 1; batch * H <= 2^31 - 1 (one CTA per unit) */
@@ -87,6 +97,7 @@ typedef struct gdn_varlen_desc {
     int32_t dtype;                    /* gdn_dtype of q, k, v, o */
     int32_t kernel;                   /* gdn_kernel; 0 = AUTO */
     const int32_t* seq_offsets_host;  /* [batch + 1] host copy; non-decreasing, [0] >= 0 */
+    int64_t row_stride_elems;         /* q/k/v row stride in elements; 0 = packed */
 } gdn_varlen_desc;
 
 typedef struct gdn_plan* gdn_plan_t;
@@ -95,7 +106,7 @@ typedef struct gdn_plan* gdn_plan_t;
  * Build the schedule of a tail replay ("Mecanismos Principais", item
  * "Reconstrucao de Estado Independente": the last k tokens of the matched
  * prefix, replayed from a zero state).
- *   cache          descriptor of the packed prefix cache; the cached entry of
+ *   cache          descriptor of the prefix cache rows; the cached entry of
  *                  sequence b may be longer than its match.
  *   match_len_host [batch] matched prefix length L_b, 0 <= L_b <= cached length.
  *   R_host         [batch] replay budget R_b >= 0; R_b > L_b is clamped to L_b,
@@ -123,9 +134,9 @@ GDN_API gdn_status gdn_plan_create_prefill(const gdn_varlen_desc* seqs, gdn_plan
  * state, "Resultados" times the suffix prefill that follows).
  *   cache, match_len_host, R_host   as for gdn_plan_create_replay.
  *   suffix_offsets_host             [batch + 1] row offsets of the suffixes in
- *                                   their own packed buffers (non-decreasing).
- * The suffix buffers share the cache descriptor's heads, dims, dtype and
- * kernel choice.  gdn_plan_window reports the replay window.
+ *                                   their own row buffers (non-decreasing).
+ * The suffix buffers share the cache descriptor's heads, dims, dtype, row
+ * stride and kernel choice.  gdn_plan_window reports the replay window.
  */
 GDN_API gdn_status gdn_plan_create_fused(const gdn_varlen_desc* cache, const int32_t* match_len_host,
                                          const int32_t* R_host, const int32_t* suffix_offsets_host,
@@ -160,7 +171,7 @@ GDN_API size_t gdn_workspace_bytes(gdn_plan_t plan);
 /*
  * Tail replay: rebuild the state at the end of each matched prefix.
  *   q            unused by the state-only replay; may be NULL.
- *   k, v         packed cache rows, dtype of the plan.
+ *   k, v         cache rows (row stride of the plan), dtype of the plan.
  *   alpha, beta  [rows, H] fp32 gates of the cached rows.
  *   seq_offsets, match_len, R
  *                device copies of the arrays given to the plan ([batch+1],
@@ -188,7 +199,7 @@ GDN_API gdn_status gdn_tail_replay_state(gdn_plan_t plan, const void* q, const v
  * ("Mecanismos Principais", item "Reconstrucao de Estado Independente": each
  * group after a full-attention layer is rebuilt independently), these are
  * the outputs a layer hands to the next one.
- *   q            [rows, H, d_k] packed like k; required.
+ *   q            [rows, H, d_k] with the row stride of k; required.
  *   k, v, alpha, beta, seq_offsets, match_len, R
  *                as for gdn_tail_replay_state.
  *   o_out        [rows, H, d_v] in the plan's dtype, addressed like q: the
@@ -230,7 +241,7 @@ GDN_API gdn_status gdn_decode_step(int32_t batch, int32_t num_heads, int32_t d_k
 /*
  * Chunked prefill over each sequence of a prefill plan, continuing from
  * state_in, emitting o_t = S_t^T q_t for every row and the final state.
- *   q, k, v      packed rows, dtype of the plan.
+ *   q, k, v      rows (row stride of the plan), dtype of the plan.
  *   alpha, beta  [rows, H] fp32.
  *   cu_seqlens   device copy of the plan's offsets ([batch+1] int32) or NULL;
  *                checked like the replay's descriptor arrays.
@@ -250,9 +261,9 @@ GDN_API gdn_status gdn_chunk_prefill(gdn_plan_t plan, const void* q, const void*
  * rebuilt states.  With the tensor-core kernel it is one launch and the
  * state never leaves the chip between the two phases; the fp32 recurrent
  * kernel runs it as those two launches.
- *   k, v, alpha, beta        the packed cache rows (as for the replay).
+ *   k, v, alpha, beta        the cache rows (as for the replay).
  *   sq, sk, sv, salpha, sbeta
- *                            the packed suffix rows (as for the prefill).
+ *                            the suffix rows (as for the prefill).
  *   o_out                    [suffix rows, H, d_v] plan dtype; suffix rows written.
  *   state_mid                [batch, H, d_k, d_v] fp32 or NULL: the rebuilt state
  *                            at the end of the matched prefix.
@@ -277,9 +288,10 @@ GDN_API gdn_status gdn_tail_replay_prefill(gdn_plan_t plan, const void* k, const
  * and the status word live in one fixed 64 KB __device__ array inside the
  * library, which every GPU that loads the library holds until the process
  * exits.  The call validates like gdn_plan_create_replay, builds the
- * schedule in a host stack buffer, copies it into that array on `stream`,
- * clears the status word and launches the same kernel a plan would.  No
- * cudaMalloc, cudaFree or other allocating routine is called.
+ * schedule in a per-thread static host buffer (not on the caller's stack),
+ * copies it into that array on `stream`, clears the status word and
+ * launches the same kernel a plan would.  No cudaMalloc, cudaFree or other
+ * allocating routine is called.
  *   cache, match_len_host, R_host   as for gdn_plan_create_replay.
  *   k, v, alpha, beta, state_out    as for gdn_tail_replay_state.
  *   stream                          cudaStream_t.
@@ -290,10 +302,12 @@ GDN_API gdn_status gdn_tail_replay_prefill(gdn_plan_t plan, const void* k, const
  * Limit: 256 + 32 * batch + 8 * batch * num_heads bytes (plus 16 * batch of
  * host temporaries) must fit in 64 KB; larger batches return
  * GDN_ERR_UNSUPPORTED before anything is launched.
- * The first call on a device resolves the array's device address; make that
- * first call before any stream capture.  Every call on a device shares the
- * array, which keeps the last call's contents, so calls whose work overlaps
- * on the GPU (different streams, or several host threads) race.
+ * Every call looks up the array's device address on the current device
+ * (so a recreated context is handled); the first call on a device also loads
+ * the library's device code there, so make that first call before any stream
+ * capture.  Every call on a device shares the array, which keeps the last
+ * call's contents, so calls whose work overlaps on the GPU (different
+ * streams, or several host threads) race.
  */
 GDN_API gdn_status gdn_tail_replay_state_noalloc(const gdn_varlen_desc* cache,
                                                  const int32_t* match_len_host,
@@ -303,8 +317,9 @@ GDN_API gdn_status gdn_tail_replay_state_noalloc(const gdn_varlen_desc* cache,
                                                  void* stream, uint32_t* status_out);
 
 /* Synchronise `stream`, then return the status the device recorded in
- * `workspace` during the last call (GDN_OK, GDN_ERR_TIMEOUT or
- * GDN_ERR_MISMATCH), or GDN_ERR_CUDA if the stream itself failed. */
+ * `workspace` during the last call (GDN_OK, GDN_ERR_TIMEOUT, GDN_ERR_BOUNDS
+ * or GDN_ERR_MISMATCH, in that order of precedence), or GDN_ERR_CUDA if the
+ * stream itself failed. */
 GDN_API gdn_status gdn_workspace_status(const void* workspace, void* stream);
 
 /*
@@ -319,6 +334,33 @@ GDN_API gdn_status gdn_workspace_status(const void* workspace, void* stream);
  * Returns GDN_OK, INVALID_ARG or CUDA.
  */
 GDN_API gdn_status gdn_selftest_bounded_wait(uint64_t limit_ns, void* workspace, void* stream);
+
+/*
+ * Test aid for callers' failure paths (the pages describe no counterpart):
+ * the next `count` plan creations in this process (gdn_plan_create_*) fail
+ * with GDN_ERR_ALLOC at the point where they would allocate their device
+ * schedule table, before any device call, and free what they built on the
+ * host.  count <= 0 clears a pending injection.  Thread-safe; meant for
+ * tests, so that an out-of-memory path can be exercised without exhausting
+ * the device.
+ */
+GDN_API void gdn_debug_fail_plan_allocations(int32_t count);
+
+/*
+ * Debug build (libgdn_tail_replay_debug.so, compiled with -DGDN_DEBUG_BOUNDS;
+ * the pages describe no counterpart).  Every kernel that has a workspace
+ * checks each global row, head, column and state index it computes against
+ * the extents the plan validated on the host.  A failing check skips the
+ * access and sets GDN_ERR_BOUNDS in the workspace status; nothing traps.
+ * The decode step has no workspace: its indices come from its grid alone.
+ * gdn_debug_bounds_enabled() returns 1 in the debug build, 0 otherwise.
+ * gdn_selftest_index_check() runs one failing check (on an index one past a
+ * 4-element extent, access skipped) so that gdn_workspace_status() then
+ * returns GDN_ERR_BOUNDS; the release build returns GDN_ERR_UNSUPPORTED.
+ *   workspace   >= 256 bytes of device memory, 16-byte aligned (cleared first).
+ */
+GDN_API int32_t gdn_debug_bounds_enabled(void);
+GDN_API gdn_status gdn_selftest_index_check(void* workspace, void* stream);
 
 /* Static description of a status code. */
 GDN_API const char* gdn_status_string(gdn_status s);

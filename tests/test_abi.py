@@ -34,17 +34,18 @@ def test_every_declared_symbol_is_exported():
 
 def test_version_and_status_strings():
     assert gdn.gdn_version() >= 100
-    for s in range(7):
+    for s in range(8):
         assert gdn.gdn_status_string(s)
     assert gdn.gdn_status_string(0) == "ok"
     assert "unknown" in gdn.gdn_status_string(99)
 
 
-def _desc(batch=1, H=2, dk=128, dv=128, dtype=gdn.GDN_BF16, kernel=0, offsets=None):
+def _desc(batch=1, H=2, dk=128, dv=128, dtype=gdn.GDN_BF16, kernel=0, offsets=None, row_stride=0):
     off = np.asarray(offsets if offsets is not None else [0, 100], np.int32)
     d = gdn.gdn_varlen_desc()
     d.batch, d.num_heads, d.d_k, d.d_v, d.dtype, d.kernel = batch, H, dk, dv, dtype, kernel
     d.seq_offsets_host = off.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    d.row_stride_elems = row_stride
     return d, off
 
 
@@ -64,6 +65,11 @@ def _create_replay(d, ml, R):
     (dict(H=0), gdn.GDN_ERR_INVALID_ARG),
     (dict(kernel=9), gdn.GDN_ERR_INVALID_ARG),
     (dict(offsets=[-1, 100]), gdn.GDN_ERR_INVALID_ARG),
+    (dict(row_stride=255), gdn.GDN_ERR_INVALID_ARG),              # below H * d = 256
+    (dict(row_stride=260), gdn.GDN_ERR_INVALID_ARG),              # 520 bytes: not a 16-byte multiple
+    (dict(row_stride=-768), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dtype=gdn.GDN_F32, kernel=1, row_stride=258), gdn.GDN_ERR_INVALID_ARG),   # 1032 bytes
+    (dict(dk=64, dv=128, kernel=1, row_stride=200), gdn.GDN_ERR_INVALID_ARG),      # below H * max(dk, dv)
 ])
 def test_descriptor_rejected_before_any_device_work(kw, status):
     d, off = _desc(**kw)
@@ -180,3 +186,88 @@ def test_selftest_arguments_rejected_before_launch():
     assert lib.gdn_selftest_bounded_wait(0, 4096, None) == gdn.GDN_ERR_INVALID_ARG          # no limit
     assert lib.gdn_selftest_bounded_wait(2_000_000_000, 4096, None) == gdn.GDN_ERR_INVALID_ARG  # above 1 s
     assert lib.gdn_selftest_bounded_wait(1000, 4100, None) == gdn.GDN_ERR_INVALID_ARG       # misaligned
+
+
+def test_row_stride_accepted_up_to_plan_allocation():
+    """A valid row stride passes every host check: with an allocation failure injected the
+    plan stops exactly where it would allocate its device table (no device needed)."""
+    lib = gdn.library()
+    h = ctypes.c_void_p()
+    for stride, dtype in ((3 * 2 * 128, gdn.GDN_BF16), (264, gdn.GDN_BF16), (260, gdn.GDN_F32)):
+        d, off = _desc(row_stride=stride, dtype=dtype, kernel=1)
+        gdn.gdn_debug_fail_plan_allocations(1)
+        assert _create_replay(d, [50], [10]) == gdn.GDN_ERR_ALLOC
+    gdn.gdn_debug_fail_plan_allocations(0)
+
+
+def test_injected_allocation_failure_reports_alloc_for_every_plan_kind():
+    """The host-side fault injection: each plan creator returns GDN_ERR_ALLOC at its device
+    allocation, leaves *out NULL, and the injection is used up one creation at a time."""
+    lib = gdn.library()
+    d, off = _desc(batch=2, offsets=[0, 100, 150])
+    ml, rr = np.array([50, 10], np.int32), np.array([10, 1], np.int32)
+    suffix = np.array([0, 20, 30], np.int32)
+    gdn.gdn_debug_fail_plan_allocations(3)
+    h = ctypes.c_void_p(1234)
+    assert lib.gdn_plan_create_replay(ctypes.byref(d), ml.ctypes.data, rr.ctypes.data,
+                                      ctypes.byref(h)) == gdn.GDN_ERR_ALLOC
+    assert h.value is None
+    assert lib.gdn_plan_create_prefill(ctypes.byref(d), ctypes.byref(h)) == gdn.GDN_ERR_ALLOC
+    assert lib.gdn_plan_create_fused(ctypes.byref(d), ml.ctypes.data, rr.ctypes.data, suffix.ctypes.data,
+                                     ctypes.byref(h)) == gdn.GDN_ERR_ALLOC
+    assert h.value is None
+    # used up: the next creation gets past the injection point (here, without a device, it
+    # then fails at the device query; with one it succeeds)
+    st = lib.gdn_plan_create_prefill(ctypes.byref(d), ctypes.byref(h))
+    assert st != gdn.GDN_ERR_ALLOC
+    if st == gdn.GDN_OK:
+        lib.gdn_plan_destroy(h)
+    # a cleared injection does not fire; invalid arguments are still reported first
+    gdn.gdn_debug_fail_plan_allocations(5)
+    gdn.gdn_debug_fail_plan_allocations(0)
+    st = lib.gdn_plan_create_prefill(ctypes.byref(d), ctypes.byref(h))
+    assert st != gdn.GDN_ERR_ALLOC
+    if st == gdn.GDN_OK:
+        lib.gdn_plan_destroy(h)
+    gdn.gdn_debug_fail_plan_allocations(1)
+    bad, _ = _desc(batch=0)
+    assert lib.gdn_plan_create_prefill(ctypes.byref(bad), ctypes.byref(h)) == gdn.GDN_ERR_INVALID_ARG
+    gdn.gdn_debug_fail_plan_allocations(0)
+
+
+def test_python_plan_surfaces_injected_alloc_failure():
+    gdn.gdn_debug_fail_plan_allocations(1)
+    try:
+        with pytest.raises(gdn.GdnError) as e:
+            gdn.gdn_plan_create_replay(2, 128, 128, "bf16", [0, 100], [50], [10])
+        assert e.value.status == gdn.GDN_ERR_ALLOC
+    finally:
+        gdn.gdn_debug_fail_plan_allocations(0)
+
+
+def test_noalloc_rejects_descriptor_over_the_extent_bound():
+    """The allocation-free entry applies the plan's descriptor checks, including
+    rows * H <= 2^40, before touching the device."""
+    lib = gdn.library()
+    rows = (1 << 31) - 1
+    d, off = _desc(batch=1, H=1024, offsets=[0, rows], kernel=1)
+    ml, rr = np.array([rows], np.int32), np.array([10], np.int32)
+    st = ctypes.c_uint32(0)
+    assert lib.gdn_tail_replay_state_noalloc(ctypes.byref(d), ml.ctypes.data, rr.ctypes.data, 4096, 4096,
+                                             4096, 4096, 4096, None, ctypes.byref(st)) == gdn.GDN_ERR_INVALID_ARG
+    d, off = _desc(batch=1, H=2, offsets=[0, 100], row_stride=100, kernel=1)   # stride below H * d
+    assert lib.gdn_tail_replay_state_noalloc(ctypes.byref(d), ml.ctypes.data, rr.ctypes.data, 4096, 4096,
+                                             4096, 4096, 4096, None, ctypes.byref(st)) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_row_stride_of_views():
+    import torch
+    x = torch.zeros(10, 3, 4, 64)
+    q, k, v = x[:, 0], x[:, 1], x[:, 2]
+    assert gdn.row_stride_of(q, k, v) == 3 * 4 * 64
+    p = torch.zeros(10, 4, 64)
+    assert gdn.row_stride_of(p, p.clone()) == 0
+    with pytest.raises(ValueError):
+        gdn.row_stride_of(q, p)                 # one strided, one packed
+    with pytest.raises(ValueError):
+        gdn.row_stride_of(torch.zeros(10, 64, 4).transpose(1, 2))   # heads not contiguous

@@ -77,38 +77,37 @@ def test_varlen_batch_full_size_sampled():
 
 @pytest.mark.parametrize("L", [8192, 32768])
 def test_replay_budget_sweep_error_curve(L):
-    """The replay's distance to the full-prefix state shrinks as R grows (the
-    gated updates attenuate older inputs), reaches the kernel's rounding at
-    R = L, and tracks the oracle's curve on sampled heads."""
+    """The replay-budget sweep (slow decay, alpha ~ U[0.97, 0.9999]) on sampled heads:
+
+    * at every budget R/L in {1, 2, 5, 10, 25, 100}% the GPU's replayed state
+      matches the fp64 oracle's replay of the same window element by element;
+    * the truncation error ||S_R - S_L|| / ||S_L||, taken from the oracle alone
+      (fp64, no kernel rounding in it), shrinks as R grows (gated updates
+      attenuate older inputs), is exactly 0 at R = L, and falls below the
+      kernel's own rounding error once the window is long enough."""
     H = 32
     t = inputs.draw_tensors(L, H, 128, 128, "bf16", 0.97, 0.9999, 7, device="cuda", with_q=False)
-    full_plan = gdn.ReplayPlan(H, 128, 128, "bf16", [0, L], [L], [L])
-    full = torch.empty((1, H, 128, 128), device="cuda")
-    full_plan.run(t["k"], t["v"], t["alpha"], t["beta"], full)
-    assert full_plan.status() == gdn.GDN_OK
-    full_plan.close()
-    errs = []
-    pcts = (1, 2, 5, 10, 25, 100)
-    for pct in pcts:
+    heads = [0, 17]
+    sub = {n: oracle_view(t[n][:, heads]) for n in ("k", "v", "alpha", "beta")}
+    S_full = oracle.replay_state(sub["k"], sub["v"], sub["alpha"], sub["beta"], [0, L], [L], [L])[0]
+    trunc, kern = [], []
+    for pct in (1, 2, 5, 10, 25, 100):
         R = inputs.ceil_budget(L, pct, 100)
         plan = gdn.ReplayPlan(H, 128, 128, "bf16", [0, L], [L], [R])
-        st = torch.empty_like(full)
+        st = torch.empty((1, H, 128, 128), device="cuda")
         plan.run(t["k"], t["v"], t["alpha"], t["beta"], st)
         assert plan.status() == gdn.GDN_OK
         plan.close()
-        e = ((st - full).flatten(2).norm(dim=2) / full.flatten(2).norm(dim=2))[0]
-        errs.append(e.cpu().numpy())
-    means = [float(e.mean()) for e in errs]
-    assert means[-1] <= 1e-2                       # R = L: same state up to rounding
-    for a_, b_ in zip(means, means[1:]):
-        assert b_ <= a_ + 1e-2                     # non-increasing up to rounding
-    assert means[0] > means[-1]
-    # oracle curve on two heads at the two smallest budgets
-    for hh in (0, 17):
-        sub = {n: oracle_view(t[n][:, hh:hh + 1]) for n in ("k", "v", "alpha", "beta")}
-        S_full = oracle.replay_state(sub["k"], sub["v"], sub["alpha"], sub["beta"], [0, L], [L], [L])[0, 0]
-        for k, pct in enumerate(pcts[:2]):
-            R = inputs.ceil_budget(L, pct, 100)
-            S_rep = oracle.replay_state(sub["k"], sub["v"], sub["alpha"], sub["beta"], [0, L], [L], [R])[0, 0]
-            e_ref = np.linalg.norm(S_rep - S_full) / np.linalg.norm(S_full)
-            assert abs(errs[k][hh] - e_ref) <= 2e-2, f"pct {pct} head {hh}: {errs[k][hh]} vs {e_ref}"
+        S_rep = oracle.replay_state(sub["k"], sub["v"], sub["alpha"], sub["beta"], [0, L], [L], [R])[0]
+        got = st[0, heads].cpu().numpy()
+        for i, hh in enumerate(heads):
+            e = rel_err(got[i], S_rep[i])
+            assert e <= TOL["bf16"], f"L {L} R {R} head {hh}: {e}"
+            kern.append(e)
+        trunc.append([np.linalg.norm(S_rep[i] - S_full[i]) / np.linalg.norm(S_full[i]) for i in range(len(heads))])
+    trunc = np.array(trunc)
+    assert np.all(trunc[-1] == 0.0)                       # R = L replays the whole prefix
+    assert np.all(np.diff(trunc, axis=0) <= 1e-12)        # non-increasing in R
+    assert np.all(trunc[0] > 1e-4)                        # 1% of the prefix is a visible truncation
+    floor = max(kern)
+    assert np.all(trunc[4] < floor), f"25% budget: truncation {trunc[4]} vs kernel rounding {floor}"

@@ -1,7 +1,9 @@
 """The allocation-free replay entry point, for callers that cannot call
 cudaMalloc (a memory pool that owns the whole device heap, or a runtime that
-only hands out its own buffers): its output must match the plan-based entry
-point's, on two calls in a row.  This file is collected last on purpose."""
+only hands out its own buffers): on two calls in a row its output must equal
+the plan-based entry point's bit for bit (both run the same kernel on the same
+schedule), and match the fp64 oracle within the parity tolerance.  This file
+is collected last on purpose."""
 import ctypes
 
 import numpy as np
@@ -10,7 +12,8 @@ import torch
 
 import gated_deltanet_state_tail_b200 as gdn
 from gated_deltanet_state_tail_b200 import inputs
-from helpers import TOL, rel_err
+import oracle
+from helpers import TOL, oracle_view, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -45,8 +48,12 @@ def test_noalloc_matches_plan_entry_point_twice(dtype, dk, dv):
                                                    t["alpha"], t["beta"], out)
         assert status == 0, f"call {call}: device status {status}"
         torch.cuda.synchronize()
+        assert torch.equal(out, ref), f"call {call}: differs from the plan entry point"
+        want = oracle.replay_state(oracle_view(t["k"]), oracle_view(t["v"]), oracle_view(t["alpha"]),
+                                   oracle_view(t["beta"]), off, ml, R)
+        got = out.cpu().numpy()
         for b in range(len(ml)):
-            assert rel_err(out[b].cpu().numpy(), ref[b].cpu().numpy()) <= TOL[dtype], f"call {call} request {b}"
+            assert rel_err(got[b], want[b]) <= TOL[dtype], f"call {call} request {b}"
 
 
 def test_noalloc_rejects_batches_beyond_its_scratch():
