@@ -491,6 +491,16 @@ def bench_ours(args, rank, world, local):
         result["gdn_speedup_token_ratio"] = (wl.match_len[0] + data.N) / (data.R + data.N)
     if not args.no_e2e:
         result["e2e"] = e2e_host_buffers(data, kernel, args, world)
+    R_stack, N_stack = data.R, data.N
+    if world == 1 and not args.no_extras:
+        # the other workloads of the hot path, one GPU: the single layer at 8K (5%), the
+        # ragged 64-request batch and the replay-budget sweep
+        for p_ in rp + pp:
+            p_.close()
+        del data, rp, pp, state, o, st_out
+        torch.cuda.empty_cache()
+        result["workloads"] = {"layer": workload_layer(flush, peaks), "varlen": workload_varlen(flush, peaks),
+                               "sweep": workload_sweep(flush, peaks)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, sample = oracle_replay_sample(wl, layers=wl.layers, min_seconds=10.0)
         result["cpu_baseline"] = {"value": v, "unit": "replayed tokens/s", "cores": cores,
@@ -502,7 +512,7 @@ def bench_ours(args, rank, world, local):
         result["cpu_full_prefill"] = {"value": fs, "unit": "s per full prefill of the stack (extrapolated)",
                                       "cores": cores, "kind": "oracle", "sample": fsample}
         # the same ratio as gdn_speedup_vs_full_prefill, on the host cores
-        result["cpu_gdn_speedup_vs_full_prefill"] = fs / (data.R / v + data.N / sv)
+        result["cpu_gdn_speedup_vs_full_prefill"] = fs / (R_stack / v + N_stack / sv)
     return result
 
 
@@ -707,54 +717,81 @@ def _time_ms(fn, iters=5, flush=None):
     return statistics.median(ts)
 
 
-def bench_sweep(args):
-    """Replay budget R/L in {1, 2, 5, 10, 25, 100}% at L = 8K, 16K, 32K (one layer, 32 heads,
-    alpha ~ U[0.97, 0.9999]): replay latency, full-prefill latency, and the relative
-    Frobenius distance of the replayed state to the state of the whole prefix."""
+def replay_bytes(H, dk, dv, R_list):
+    """Algorithmic HBM bytes of a bf16 replay launch: per (sequence, head) unit the k and v
+    rows of its window (2 x d x 2 B per token) and the fp32 gates (8 B per token), plus the
+    fp32 state written (dk x dv x 4 B)."""
+    return sum(H * (r * (dk * 2 + dv * 2 + 8) + dk * dv * 4) for r in R_list)
+
+
+def _hbm_roofline(nbytes, ms, peaks):
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": gbs / peaks["hbm_gbs"], "bytes_per_launch": nbytes, "peak_source": peaks["source"]}
+
+
+def _oracle_timed(fn, min_seconds=1.0, max_reps=50):
+    """Run fn() until min_seconds have passed; returns (seconds per run, runs, result)."""
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        out = fn()
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= min_seconds or reps >= max_reps:
+            return dt / reps, reps, out
+
+
+def workload_layer(flush, peaks, iters=20):
+    """One GDN layer, 16 heads, d = 128, bf16: matched prefix L = 8192, replay R = 410 (5%),
+    suffix N = 512.  Rebuild and suffix prefill (one launch each), the full prefill of
+    L + N as the GPU comparator, and the fp64 oracle's rebuild and suffix prefill on the
+    host cores (the whole workload, repeated for at least 1 s each)."""
     import gated_deltanet_state_tail_b200 as gdn
     import oracle
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
-    lines = []
-    # the fp64 oracle's replay and full-prefill rates on the host cores (bounded samples),
-    # extrapolated by token-heads to every line below
-    th = max(1, oracle.num_threads())
-    rep_tps, rep_dt = oracle_throughput("replay", "bf16", th, 128, 128, 2048, 0.97, 0.9999)
-    pre_tps, pre_dt = oracle_throughput("prefill", "bf16", th, 128, 128, 2048, 0.97, 0.9999)
-    cpu_sample = (f"fp64 oracle on {th} heads x 2048 tokens, each kind repeated for at least 1 s (replay "
-                  f"{rep_dt:.1f} s, prefill with outputs {pre_dt:.1f} s); extrapolated by token-heads")
-    for L in (8192, 16384, 32768):
-        wl = [w for w in inputs.sweep_workloads() if w.match_len[0] == L]
-        H = wl[0].H
-        t = inputs.draw_tensors(L, H, 128, 128, "bf16", 0.97, 0.9999, 0, device="cuda")
-        full_state = torch.empty((1, H, 128, 128), device="cuda")
-        pf = gdn.PrefillPlan(H, 128, 128, "bf16", [0, L])
-        o = torch.empty((L, H, 128), dtype=torch.bfloat16, device="cuda")
-        full_ms = _time_ms(lambda: pf.run(t["q"], t["k"], t["v"], t["alpha"], t["beta"], o,
-                                          state_out=full_state), flush=flush)
-        pf.check()
-        for w in wl:
-            R = w.R[0]
-            plan = gdn.ReplayPlan(H, 128, 128, "bf16", [0, L], [L], [R])
-            st = torch.empty_like(full_state)
-            rep_ms = _time_ms(lambda: plan.run(t["k"], t["v"], t["alpha"], t["beta"], st), flush=flush)
-            plan.check()
-            e = ((st - full_state).flatten(2).norm(dim=2) / full_state.flatten(2).norm(dim=2))[0]
-            lines.append({"metric": "replay-budget sweep", "workload": w.name, "L": L, "pct": w.extra["pct"],
-                          "R": R, "replay_ms": rep_ms, "full_prefill_ms": full_ms,
-                          "replay_speedup_vs_full_prefill": full_ms / rep_ms,
-                          "replayed_tokens_per_s": R / (rep_ms / 1e3),
-                          "state_rel_frob": {"mean": float(e.mean()), "max": float(e.max())},
-                          "cpu_baseline": {"replay_ms": R * H / rep_tps * 1e3,
-                                           "full_prefill_ms": L * H / pre_tps * 1e3, "cores": th,
-                                           "kind": "oracle", "sample": cpu_sample},
-                          "alpha": "U[0.97, 0.9999]", "heads": H, "dtype": "bf16", "data": "synthetic"})
-            plan.close()
-        pf.close()
-    return lines
+    wl = inputs.single_layer_workload()
+    H, L, R, N = wl.H, wl.match_len[0], wl.R[0], wl.suffix_len[0]
+    t = inputs.draw_tensors(L + N, H, 128, 128, "bf16", wl.alpha_lo, wl.alpha_hi, wl.seeds[0], device="cuda")
+    rp = gdn.ReplayPlan(H, 128, 128, "bf16", [0, L + N], [L], [R])
+    pp = gdn.PrefillPlan(H, 128, 128, "bf16", [0, N])
+    fp = gdn.PrefillPlan(H, 128, 128, "bf16", [0, L + N])
+    st = torch.empty((1, H, 128, 128), device="cuda")
+    st2 = torch.empty_like(st)
+    o = torch.empty((N, H, 128), dtype=torch.bfloat16, device="cuda")
+    of = torch.empty((L + N, H, 128), dtype=torch.bfloat16, device="cuda")
+    s = {n: t[n][L:] for n in t}
+    rep_ms = _time_ms(lambda: rp.run(t["k"], t["v"], t["alpha"], t["beta"], st), iters, flush)
+    suf_ms = _time_ms(lambda: pp.run(s["q"], s["k"], s["v"], s["alpha"], s["beta"], o, state_in=st,
+                                     state_out=st2), iters, flush)
+    full_ms = _time_ms(lambda: fp.run(t["q"], t["k"], t["v"], t["alpha"], t["beta"], of, state_out=st2),
+                       5, flush)
+    for p_ in (rp, pp, fp):
+        p_.check()
+        p_.close()
+    # the oracle on the same workload: the rebuild (R rows x H heads), then the suffix
+    win = {n: _oracle_bits(t[n][L - R:L].cpu()) for n in ("k", "v", "alpha", "beta")}
+    sh = {n: _oracle_bits(s[n].cpu()) for n in ("q", "k", "v", "alpha", "beta")}
+    cpu_rep_s, nr, S = _oracle_timed(lambda: oracle.replay_state(win["k"], win["v"], win["alpha"], win["beta"],
+                                                                 [0, R], [R], [R]))
+    cpu_suf_s, ns, _ = _oracle_timed(lambda: oracle.prefill(sh["q"], sh["k"], sh["v"], sh["alpha"], sh["beta"],
+                                                            [0, N], state_in=S))
+    units = H
+    return {"workload": wl.name, "heads": H, "matched_prefix": L, "replay": R, "suffix": N,
+            "rebuild_ms": rep_ms, "suffix_prefill_ms": suf_ms, "full_prefill_ms": full_ms,
+            "replayed_tokens_per_s": R / (rep_ms / 1e3),
+            "gdn_speedup_vs_full_prefill": full_ms / (rep_ms + suf_ms),
+            "ctas_per_launch": units,
+            "roofline": _hbm_roofline(replay_bytes(H, 128, 128, [R]), rep_ms, peaks),
+            "cpu_baseline": {"value": R / cpu_rep_s, "unit": "replayed tokens/s", "rebuild_ms": cpu_rep_s * 1e3,
+                             "suffix_prefill_ms": cpu_suf_s * 1e3, "cores": oracle.num_threads(),
+                             "kind": "oracle",
+                             "sample": f"the whole workload: fp64 oracle rebuild ({H} heads x {R} tokens, "
+                                       f"{nr} runs) and suffix prefill ({H} heads x {N} tokens, {ns} runs)"},
+            "timing": f"median of {iters} launches, 256 MB L2 flush before each"}
 
 
-def bench_varlen(args):
-    """64 ragged requests (16 heads): replay of every tail, then every suffix."""
+def workload_varlen(flush, peaks, iters=10):
+    """64 ragged requests, 16 heads: every tail replayed, then every suffix prefilled (one
+    launch each).  The fp64 oracle runs requests 0-3 on the host cores."""
     import gated_deltanet_state_tail_b200 as gdn
     wl = inputs.varlen_workload(64, seed=0)
     off, cu = wl.seq_offsets(), wl.suffix_cu()
@@ -767,20 +804,103 @@ def bench_varlen(args):
     st = torch.empty((wl.batch, H, 128, 128), device="cuda")
     st2 = torch.empty_like(st)
     o = torch.empty((int(cu[-1]), H, 128), dtype=torch.bfloat16, device="cuda")
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
-    rep_ms = _time_ms(lambda: rp.run(cache["k"], cache["v"], cache["alpha"], cache["beta"], st), 10, flush)
+    rep_ms = _time_ms(lambda: rp.run(cache["k"], cache["v"], cache["alpha"], cache["beta"], st), iters, flush)
     suf_ms = _time_ms(lambda: pp.run(suf["q"], suf["k"], suf["v"], suf["alpha"], suf["beta"], o,
-                                     state_in=st, state_out=st2), 10, flush)
+                                     state_in=st, state_out=st2), iters, flush)
     rp.check()
     pp.check()
+    rp.close()
+    pp.close()
+    Reff = [min(r, l) for r, l in zip(wl.R, wl.match_len)]
     cpu = cpu_varlen_sample(wl, off, cu, cache, suf)
-    return [{"metric": "varlen replay + suffix", "workload": wl.name, "requests": wl.batch, "heads": H,
-             "replayed_tokens": int(sum(min(r, l) for r, l in zip(wl.R, wl.match_len))),
-             "suffix_tokens": int(sum(wl.suffix_len)), "replay_ms": rep_ms, "suffix_prefill_ms": suf_ms,
-             "replayed_tokens_per_s": sum(min(r, l) for r, l in zip(wl.R, wl.match_len)) / (rep_ms / 1e3),
-             "suffix_tokens_per_s": sum(wl.suffix_len) / (suf_ms / 1e3), "cpu_baseline": cpu,
-             "match_len": wl.match_len, "R": wl.R, "suffix_len": wl.suffix_len, "dtype": "bf16",
-             "data": "synthetic"}]
+    del cache, suf
+    return {"workload": wl.name, "requests": wl.batch, "heads": H,
+            "replayed_tokens": int(sum(Reff)), "suffix_tokens": int(sum(wl.suffix_len)),
+            "rebuild_ms": rep_ms, "suffix_prefill_ms": suf_ms,
+            "replayed_tokens_per_s": sum(Reff) / (rep_ms / 1e3),
+            "suffix_tokens_per_s": sum(wl.suffix_len) / (suf_ms / 1e3),
+            "longest_window": int(max(Reff)),
+            "roofline": _hbm_roofline(replay_bytes(H, 128, 128, Reff), rep_ms, peaks),
+            "cpu_baseline": cpu, "timing": f"median of {iters} launches, 256 MB L2 flush before each",
+            "match_len": wl.match_len, "R": wl.R, "suffix_len": wl.suffix_len}
+
+
+def workload_sweep(flush, peaks, sample_heads=(0, 17), iters=5):
+    """Replay budget R/L in {1, 2, 5, 10, 25, 100}% at L = 8K, 16K, 32K (one layer, 32 heads,
+    slow decay alpha ~ U[0.97, 0.9999]).  Per point: the replay's latency and roofline
+    fraction, the full prefill of L (per L), and on sampled heads
+
+    * `truncation_rel_frob`: ||S_R - S_L|| / ||S_L|| from the fp64 oracle alone, the
+      state error that replaying only the tail causes (no kernel rounding in it);
+    * `kernel_vs_oracle`: the GPU replay's own error against the oracle's replay of the
+      same window (max|err| / max|ref| and relative Frobenius), its rounding floor.
+
+    The oracle's host time per point is extrapolated by token-heads from bounded samples."""
+    import gated_deltanet_state_tail_b200 as gdn
+    import oracle
+    th = max(1, oracle.num_threads())
+    rep_tps, rep_dt = oracle_throughput("replay", "bf16", th, 128, 128, 2048, 0.97, 0.9999)
+    pre_tps, pre_dt = oracle_throughput("prefill", "bf16", th, 128, 128, 2048, 0.97, 0.9999)
+    cpu_sample = (f"fp64 oracle on {th} heads x 2048 tokens, each kind repeated for at least 1 s (replay "
+                  f"{rep_dt:.1f} s, prefill with outputs {pre_dt:.1f} s); extrapolated by token-heads")
+    heads = list(sample_heads)
+    points = []
+    for L in (8192, 16384, 32768):
+        wls = [w for w in inputs.sweep_workloads() if w.match_len[0] == L]
+        H = wls[0].H
+        t = inputs.draw_tensors(L, H, 128, 128, "bf16", 0.97, 0.9999, 0, device="cuda")
+        full_state = torch.empty((1, H, 128, 128), device="cuda")
+        pf = gdn.PrefillPlan(H, 128, 128, "bf16", [0, L])
+        o = torch.empty((L, H, 128), dtype=torch.bfloat16, device="cuda")
+        full_ms = _time_ms(lambda: pf.run(t["q"], t["k"], t["v"], t["alpha"], t["beta"], o,
+                                          state_out=full_state), iters, flush)
+        pf.check()
+        pf.close()
+        sub = {n: _oracle_bits(t[n][:, heads].cpu()) for n in ("k", "v", "alpha", "beta")}
+        S_full = oracle.replay_state(sub["k"], sub["v"], sub["alpha"], sub["beta"], [0, L], [L], [L])[0]
+        for w in wls:
+            R = w.R[0]
+            plan = gdn.ReplayPlan(H, 128, 128, "bf16", [0, L], [L], [R])
+            st = torch.empty_like(full_state)
+            rep_ms = _time_ms(lambda: plan.run(t["k"], t["v"], t["alpha"], t["beta"], st), iters, flush)
+            plan.check()
+            plan.close()
+            S_rep = oracle.replay_state(sub["k"], sub["v"], sub["alpha"], sub["beta"], [0, L], [L], [R])[0]
+            got = st[0, heads].double().cpu().numpy()
+            trunc = [float(np.linalg.norm(S_rep[i] - S_full[i]) / np.linalg.norm(S_full[i]))
+                     for i in range(len(heads))]
+            k_max = [float(np.max(np.abs(got[i] - S_rep[i])) / np.max(np.abs(S_rep[i]))) for i in range(len(heads))]
+            k_frob = [float(np.linalg.norm(got[i] - S_rep[i]) / np.linalg.norm(S_rep[i])) for i in range(len(heads))]
+            points.append({"L": L, "pct": w.extra["pct"], "R": R, "replay_ms": rep_ms, "full_prefill_ms": full_ms,
+                           "replay_speedup_vs_full_prefill": full_ms / rep_ms,
+                           "replayed_tokens_per_s": R / (rep_ms / 1e3),
+                           "roofline_frac": _hbm_roofline(replay_bytes(H, 128, 128, [R]), rep_ms, peaks)["frac"],
+                           "truncation_rel_frob": {"mean": float(np.mean(trunc)), "max": float(np.max(trunc))},
+                           "kernel_vs_oracle": {"max_err_over_max_ref": float(np.max(k_max)),
+                                                "rel_frob": float(np.max(k_frob))},
+                           "cpu_baseline_ms": {"replay": R * H / rep_tps * 1e3, "full_prefill": L * H / pre_tps * 1e3}})
+        del t
+    return {"workload": "sweep-H32-d128-bf16-L8K16K32K-alpha0.97-0.9999", "heads": 32,
+            "sampled_heads": heads, "points": points,
+            "cpu_baseline": {"cores": th, "kind": "oracle", "sample": cpu_sample},
+            "timing": f"median of {iters} launches, 256 MB L2 flush before each"}
+
+
+def bench_sweep(args):
+    """The replay-budget sweep as one auxiliary line per point."""
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    sw = workload_sweep(flush, measured_peaks())
+    return [dict(p, metric="replay-budget sweep", workload=f"sweep-L{p['L']}-p{p['pct']}", heads=sw["heads"],
+                 sampled_heads=sw["sampled_heads"], alpha="U[0.97, 0.9999]", dtype="bf16", data="synthetic",
+                 cpu_sample=sw["cpu_baseline"]["sample"])
+            for p in sw["points"]]
+
+
+def bench_varlen(args):
+    """64 ragged requests (16 heads): replay of every tail, then every suffix."""
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    v = workload_varlen(flush, measured_peaks())
+    return [dict(v, metric="varlen replay + suffix", dtype="bf16", data="synthetic")]
 
 
 def varlen_tail_windows(wl, off, cache, nreq):
@@ -1024,6 +1144,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-comparator", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the single-layer, varlen and sweep workloads of the bench line")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

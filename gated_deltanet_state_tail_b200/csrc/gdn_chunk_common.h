@@ -256,16 +256,15 @@ constexpr int NT = 256;      // threads per CTA
 //   replay : [K0 | K1 | V0 | V1]            (32 KB)
 //   prefill: [K0 | Q0 | K1 | Q1 | V0 | V1]  (48 KB; K block stride 16 KB so
 //            that [K; Q] is one 128-row operand)
-// Once W and U' of a chunk are done, its V boxes take the U tile
-// diag(gamma_C / gamma) U / sigma (bf16 [dv][j], 16 KB) that the state update
-// of the same chunk reads.
 // PREP is reused within a chunk, in this order:
 //   A -> T in place (fp32 64 x LDT) and the product scratch,
 //   T diag(beta), T diag(beta gamma) (bf16 [j][j'], 8 KB each; the replay
 //   keeps them past the end of T, 33 KB of PREP, the prefill over T, 32 KB),
 //   BU = -sigma W (fp32, K-major [j][dk], four 8 KB key blocks).
-// Prefill adds UB (bf16 U^T [dv][j]), MB (bf16 masked decayed Q K^T [i][j])
-// and BQ (fp32 sigma diag(gamma) Q, K-major [i][dk], four 8 KB blocks).
+// Prefill adds UB (the bf16 output stage [i][dv]), MB (bf16 masked decayed
+// Q K^T [i][j]) and BQ (fp32 sigma diag(gamma) Q, K-major [i][dk], four 8 KB
+// blocks).  Both kernels keep the bf16 U tiles the state update (and the
+// prefill's output product) read in TMEM, not in the tile slot.
 template <bool REPLAY>
 struct Layout {
     static constexpr uint32_t TILE = REPLAY ? 32768u : 49152u;
@@ -285,7 +284,6 @@ struct Layout {
     static constexpr uint32_t Q0 = 8192;                          // prefill only
     static constexpr uint32_t V0 = REPLAY ? 16384u : 32768u;
     static constexpr uint32_t V_LBO = 8192;
-    static constexpr uint32_t UT = V0;
 };
 static_assert(Layout<true>::OFF_X + 4 * 16 * 24 * 4 <= Layout<true>::OFF_PREP + 32768, "prep scratch fits");
 static_assert(Layout<true>::OFF_TB >= Layout<true>::OFF_AT + C * LDT * 4 && Layout<true>::OFF_TB % 1024 == 0,
@@ -294,9 +292,12 @@ static_assert(2 * (Layout<true>::BYTES + 1024) <= 224 * 1024, "two replay CTAs p
 
 // TMEM columns
 constexpr uint32_t TM_S = 0;      // 128 columns: fp32 S^T / sigma, lane = value row, column = key
-constexpr uint32_t TM_U = 128;    // 64 columns: U'^T then U^T, lane = value row
+constexpr uint32_t TM_U = 128;    // 64 columns: U'^T then U^T, lane = value row (replay: then U~^T in
+                                  // bf16, two chunk rows per column, in its first 32 columns)
 constexpr uint32_t TM_P = 192;    // 64 columns: K K^T ([K;Q] K^T for prefill), then W^T (lane = key)
 constexpr uint32_t TM_O = 256;    // 64 columns (prefill): O^T, lane = value row
+constexpr uint32_t TM_UB = 320;   // 32 columns (prefill): U^T in bf16, two chunk rows per column
+constexpr uint32_t TM_UT = 352;   // 32 columns (prefill): U~^T = U^T diag(e) / sigma in bf16
 
 struct TcParams {
     CallArgs a;

@@ -64,7 +64,7 @@ struct PipeLayout {
     static constexpr uint32_t OFF_TB = OFF_PREP;
     static constexpr uint32_t OFF_TBG = OFF_PREP + 8192;
     static constexpr uint32_t OFF_BU = OFF_PREP;
-    static constexpr uint32_t OFF_UB = OFF_PREP + 32768;        // bf16 U^T [dv][j], then the output stage
+    static constexpr uint32_t OFF_UB = OFF_PREP + 32768;        // the output stage, bf16 O [i][dv]
     static constexpr uint32_t OFF_MB = OFF_UB + 16384;          // two bf16 M [i][j], chunk c in c % 2
     static constexpr uint32_t OFF_BQ = OFF_MB + 16384;          // fp32 sigma diag(gamma) Q, K-major
     static constexpr uint32_t BYTES = OFF_BQ + 32768;
@@ -159,7 +159,7 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     float* Xs = reinterpret_cast<float*>(sm + PL::OFF_X);
     const uint32_t s_bu = smem_u32(sm + PL::OFF_BU);
     const uint32_t s_tb = smem_u32(sm + PL::OFF_TB), s_tbg = smem_u32(sm + PL::OFF_TBG);
-    const uint32_t s_ub = smem_u32(sm + PL::OFF_UB), s_bq = smem_u32(sm + PL::OFF_BQ);
+    const uint32_t s_bq = smem_u32(sm + PL::OFF_BQ);
     const size_t state_base = ((size_t)b * H + h) * D * D;
     {   // initial state: TMEM lane dv holds column dv of S (a row of S^T)
         float v[32];
@@ -182,7 +182,7 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     const uint32_t id_w = idesc_bf16(128, 64, true, false);
     const uint32_t id_u = idesc_tf32(128, 64, false, false);
     const uint32_t id_s = idesc_bf16(128, 128, false, true);
-    const uint32_t id_o2 = idesc_bf16(128, 64, false, false);   // U^T M^T
+    const uint32_t id_o2 = idesc_bf16(128, 64, false, false);   // U^T M^T, A (U^T) in TMEM
     uint32_t ph_w = 0, ph_u = 0, ph_s = 0;
     bool ok = true;
 
@@ -330,24 +330,29 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 snew = 1.0f;
             }
             const float inv = 1.0f / snew;
+            // U^T (for the outputs) and U~^T = U^T diag(e) / sigma (for the state update) as
+            // bf16 in TMEM, two chunk rows per 32-bit column: the A operands of both MMAs
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 float v[32];
                 tmem_ld32(tlane + TM_U + 32 * hf, v);
                 tmem_wait_ld();
-                if (outc) write_row32_bf16(sm + PL::OFF_UB, row, 4 * hf, v);
+                uint32_t pk[16];
+                if (outc) {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) pk[q] = pack_bf16(v[2 * q], v[2 * q + 1]);
+                    tmem_st16(tlane + TM_UB + 16 * hf, pk);
+                }
                 const float4* ev = reinterpret_cast<const float4*>(G.e + 32 * hf);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     const float4 e4 = ev[q];
-                    v[4 * q] *= e4.x * inv;
-                    v[4 * q + 1] *= e4.y * inv;
-                    v[4 * q + 2] *= e4.z * inv;
-                    v[4 * q + 3] *= e4.w * inv;
+                    pk[2 * q] = pack_bf16(v[4 * q] * (e4.x * inv), v[4 * q + 1] * (e4.y * inv));
+                    pk[2 * q + 1] = pack_bf16(v[4 * q + 2] * (e4.z * inv), v[4 * q + 3] * (e4.w * inv));
                 }
-                write_row32_bf16(tile + L::UT, row, 4 * hf, v);
+                tmem_st16(tlane + TM_UT + 16 * hf, pk);
             }
-            fence_proxy_async_smem();
+            tmem_wait_st();
             tc_fence_before();
             named_sync(BAR_CHAIN, 128);
             if (warp == 4) {
@@ -355,17 +360,15 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 if (elect_one()) {
                     const uint32_t s_tile = smem_u32(tile);
                     const uint32_t s_mb = smem_u32(sm + PL::OFF_MB + (c & 1) * 8192);
-                    const uint64_t da = smem_desc_sw128(s_tile + L::UT, 16, 1024);
                     const uint64_t db = smem_desc_sw128(s_tile, L::K_BLK, 1024);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ss(tbase + TM_S, desc_advance(da, kk * 32), desc_advance(db, kk * 2048), id_s, 1u);
+                        mma_bf16_ts(tbase + TM_S, tbase + TM_UT + kk * 8, desc_advance(db, kk * 2048), id_s, 1u);
                     if (outc) {
-                        const uint64_t dua = smem_desc_sw128(s_ub, 16, 1024);
                         const uint64_t dmb = smem_desc_sw128(s_mb, 16, 1024);
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            mma_bf16_ss(tbase + TM_O, desc_advance(dua, kk * 32), desc_advance(dmb, kk * 32), id_o2, 1u);
+                            mma_bf16_ts(tbase + TM_O, tbase + TM_UB + kk * 8, desc_advance(dmb, kk * 32), id_o2, 1u);
                     }
                     mma_commit(&bar_s);
                     if (mbar_wait_bounded(&bar_s, ph_s, kWaitNs)) {
@@ -381,8 +384,8 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             named_sync(BAR_CHAIN, 128);   // the state update (and O) of chunk c are complete
             tc_fence_after();
             if (outc) {
-                // outputs: stage O as bf16 rows [i][dv] in UB (its last reader, O += U M^T, is
-                // done), then 16-byte stores of whole rows
+                // outputs: stage O as bf16 rows [i][dv] in the UB region, then 16-byte stores of
+                // whole rows
                 __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(sm + PL::OFF_UB);
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {

@@ -13,7 +13,9 @@
 // S_C = gamma_C S0 + K^T diag(gamma_C / gamma) U.
 // With E = diag(gamma_C / gamma), this kernel forms E W and E U' directly
 // (E scales the rows of the bf16 T operands), so U~ = E U = E U' - (E W) S0
-// reaches the state update without another pass over U.
+// reaches the state update without another pass over U.  U~ stays in tensor
+// memory: the U epilogue writes it back as bf16 over its own columns, and the
+// state update reads it from there as the A operand.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -31,8 +33,8 @@ using namespace chunk;
 //
 // The state-independent front of chunk c + 1 (A = strict_tril(...K K^T) and
 // the UT inverse) runs on warps 0-3 while warps 4-7 finish chunk c's state
-// chain: the U epilogue, the state update on the tensor core, and the TMA of
-// chunk c + 2 into the tile slot that update frees.  Warps 6-7 first write the
+// chain: the U epilogue (U~ to bf16 in TMEM), the state update on the tensor
+// core, and the TMA of chunk c + 2 into the tile slot that update frees.  Warps 6-7 first write the
 // lower-right quarter of A, the only part of A outside columns 0-31.  Then all
 // eight warps form T diag(beta), W and U', and -sigma W of chunk c + 1 and start
 // its state product, then K K^T of chunk c + 2.  98 KB of shared memory, 256
@@ -113,7 +115,7 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     const uint32_t id_kk = idesc_bf16(64, 64, false, false);   // K K^T; row r in lane 32 (r/16) + r%16
     const uint32_t id_w = idesc_bf16(128, 64, true, false);    // K^T (T..)^T, V^T (T..)^T
     const uint32_t id_u = idesc_tf32(128, 64, false, false);   // S^T (-sigma W^T), A in TMEM
-    const uint32_t id_s = idesc_bf16(128, 128, false, true);   // U~^T K
+    const uint32_t id_s = idesc_bf16(128, 128, false, true);   // U~^T K, A (U~^T) in TMEM
     uint32_t ph_w = 0, ph_u = 0, ph_s = 0;
     bool ok = true;
 
@@ -267,16 +269,21 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 snew = 1.0f;
             }
             const float inv = 1.0f / snew;
+            // U~^T as bf16 back into TMEM, two chunk rows per 32-bit column, over the first 32
+            // columns of TM_U (half hf lands on columns 16 hf .. 16 hf + 15, which this thread
+            // has read already): the A operand of the state update, with no trip through
+            // shared memory
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 float v[32];   // value dv = row, chunk rows [32 hf, 32 hf + 32)
                 tmem_ld32(tlane + TM_U + 32 * hf, v);
                 tmem_wait_ld();
+                uint32_t pk[16];
 #pragma unroll
-                for (int q = 0; q < 32; ++q) v[q] *= inv;
-                write_row32_bf16(tile + L::UT, row, 4 * hf, v);
+                for (int q = 0; q < 16; ++q) pk[q] = pack_bf16(v[2 * q] * inv, v[2 * q + 1] * inv);
+                tmem_st16(tlane + TM_U + 16 * hf, pk);
             }
-            fence_proxy_async_smem();
+            tmem_wait_st();
             tc_fence_before();
             named_sync(BAR_CHAIN, 128);
             // ---- S^T / sigma += U~^T K of chunk c; once it is done the slot takes chunk c + 2 ----
@@ -284,11 +291,10 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 tc_fence_after();
                 if (elect_one()) {
                     const uint32_t s_tile = smem_u32(tile);
-                    const uint64_t da = smem_desc_sw128(s_tile + L::UT, 16, 1024);
                     const uint64_t db = smem_desc_sw128(s_tile, L::K_BLK, 1024);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ss(tbase + TM_S, desc_advance(da, kk * 32), desc_advance(db, kk * 2048), id_s, 1u);
+                        mma_bf16_ts(tbase + TM_S, tbase + TM_U + kk * 8, desc_advance(db, kk * 2048), id_s, 1u);
                     mma_commit(&bar_s);
                     if (mbar_wait_bounded(&bar_s, ph_s, kWaitNs)) {
                         if (c + 2 < nchunks)
