@@ -62,6 +62,52 @@ def chunk_algebra_state(k, v, alpha, beta, S0=None):
     return sigma * St
 
 
+def chunk_algebra_state_grouped(k, v, alpha, beta):
+    """The replay kernel's grouping of the state term: P = K_c (S / sigma) is formed
+    right after the previous chunk's state update, from the chunk's own keys (rows past
+    the window as zeros), and E U = E T diag(beta) V + (-sigma E T diag(beta gamma)) P,
+    both products into one accumulator.  From a zero state (the replay), so the first
+    chunk has no P term."""
+    n, dk = k.shape
+    dv = v.shape[1]
+    St = np.zeros((dk, dv))
+    sigma = 1.0
+    chunks = []
+    for c0 in range(0, n, C):
+        m = min(C, n - c0)
+        kc = np.zeros((C, dk))
+        vc = np.zeros((C, dv))
+        ac = np.ones(C)
+        bc = np.zeros(C)
+        kc[:m], vc[:m], ac[:m], bc[:m] = k[c0:c0 + m], v[c0:c0 + m], alpha[c0:c0 + m], beta[c0:c0 + m]
+        chunks.append((kc, vc, ac, bc))
+    P = None
+    for ci, (kc, vc, ac, bc) in enumerate(chunks):
+        lg = np.array([max(np.log2(a), LOG2_FLOOR) if a > 0 else LOG2_FLOOR for a in ac])
+        g2 = np.cumsum(lg)
+        gam = np.exp2(g2)
+        e = np.exp2(g2[-1] - g2)
+        if g2[-1] >= FAST_FLOOR:
+            decay = (bc * gam)[:, None] * np.exp2(-g2)[None, :]
+        else:
+            decay = bc[:, None] * np.exp2(g2[:, None] - g2[None, :])
+        T = np.linalg.inv(np.eye(C) + np.tril(decay * (kc @ kc.T), -1))
+        tb = e[:, None] * T * bc[None, :]                      # E T diag(beta), bf16 operand
+        b2 = -sigma * tb * gam[None, :]                        # -sigma E T diag(beta gamma), fp32 operand
+        EU = tb @ vc
+        if P is not None:
+            EU = EU + b2 @ P
+        snew = sigma * gam[-1]
+        if snew < RENORM_BELOW:
+            St = St * snew
+            snew = 1.0
+        St = St + kc.T @ (EU / snew)
+        sigma = snew
+        if ci + 1 < len(chunks):
+            P = chunks[ci + 1][0] @ St                         # next chunk's keys times S / sigma
+    return sigma * St
+
+
 def _inputs(n, dk, dv, case, seed):
     g = np.random.default_rng(seed)
     k = g.standard_normal((n, dk))
@@ -88,6 +134,42 @@ def test_chunk_algebra_matches_recurrence(case, n):
     S = chunk_algebra_state(k, v, a, b)
     scale = max(np.abs(S_ref).max(), 1e-300)
     assert np.abs(S - S_ref).max() / scale <= 1e-10
+
+
+@pytest.mark.parametrize("case", ["normal", "strong_decay", "zero_gates", "slow_decay"])
+@pytest.mark.parametrize("n", [1, 63, 64, 65, 200])
+def test_grouped_state_term_matches_recurrence(case, n):
+    dk, dv = 16, 8
+    k, v, a, b = _inputs(n, dk, dv, case, seed=300 + n)
+    S_ref, _ = oracle.recurrence(k, v, a, b)
+    S = chunk_algebra_state_grouped(k, v, a, b)
+    scale = max(np.abs(S_ref).max(), 1e-300)
+    assert np.abs(S - S_ref).max() / scale <= 1e-10
+
+
+def test_grouped_state_term_needs_the_updated_state():
+    """Planted mistake: P taken from the state before the previous chunk's update."""
+    dk, dv, n = 16, 8, 200
+    k, v, a, b = _inputs(n, dk, dv, "normal", seed=7)
+    S_ref, _ = oracle.recurrence(k, v, a, b)
+    # restate with the stale state: the P of chunk c + 1 from S before chunk c's update
+    St = np.zeros((dk, dv))
+    sigma, P, prev = 1.0, None, np.zeros((dk, dv))
+    for c0 in range(0, n, C):
+        m = min(C, n - c0)
+        kc = np.zeros((C, dk)); vc = np.zeros((C, dv)); ac = np.ones(C); bc = np.zeros(C)
+        kc[:m], vc[:m], ac[:m], bc[:m] = k[c0:c0 + m], v[c0:c0 + m], a[c0:c0 + m], b[c0:c0 + m]
+        g2 = np.cumsum(np.log2(ac))
+        gam = np.exp2(g2)
+        e = np.exp2(g2[-1] - g2)
+        T = np.linalg.inv(np.eye(C) + np.tril(bc[:, None] * np.exp2(g2[:, None] - g2[None, :]) * (kc @ kc.T), -1))
+        tb = e[:, None] * T * bc[None, :]
+        EU = tb @ vc + (0 if c0 == 0 else (-sigma * tb * gam[None, :]) @ (kc @ prev))
+        prev = St.copy()
+        snew = sigma * gam[-1]
+        St = St + kc.T @ (EU / snew)
+        sigma = snew
+    assert np.abs(sigma * St - S_ref).max() / np.abs(S_ref).max() > 1e-3
 
 
 def test_chunk_algebra_from_a_nonzero_state():

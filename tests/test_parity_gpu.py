@@ -298,7 +298,7 @@ def test_bounded_wait_timeout_is_reported_and_context_survives():
     gdn.gdn_selftest_bounded_wait(1_000_000, ws)
     assert gdn.gdn_workspace_status(ws) == gdn.GDN_ERR_TIMEOUT
     header = ws.view(torch.int32).cpu().numpy()
-    assert header[2] == 99                                   # the wait site the self-test reports
+    assert header[1] == 99                                   # the wait site the self-test reports
     # the context is still usable: a small replay runs and matches the oracle
     t = make_cache([200], 2, 128, 128, "bf16", seed=3)
     st = run_replay(t, np.array([0, 200], np.int32), [200], [150], gdn.GDN_KERNEL_AUTO, "bf16")
