@@ -9,13 +9,18 @@
 //   S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T.
 // The replay runs 64 tokens at a time in the chunkwise WY / UT form (see the
 // chunk helpers): A_ij = beta_i (gamma_i / gamma_j) k_i.k_j, T = (I + A)^-1,
-// W = T diag(beta gamma) K, U' = T diag(beta) V, U = U' - W S0,
+// U' = T diag(beta) V, U = U' - T diag(beta gamma) K S0,
 // S_C = gamma_C S0 + K^T diag(gamma_C / gamma) U.
-// With E = diag(gamma_C / gamma), this kernel forms E W and E U' directly
-// (E scales the rows of the bf16 T operands), so U~ = E U = E U' - (E W) S0
-// reaches the state update without another pass over U.  U~ stays in tensor
-// memory: the U epilogue writes it back as bf16 over its own columns, and the
-// state update reads it from there as the A operand.
+//
+// This kernel groups the state-dependent term as T diag(beta gamma) (K S0):
+// with E = diag(gamma_C / gamma), the state S = sigma S~ and P = K S~0,
+//   E U = E U' - sigma (E T diag(beta gamma)) P,
+//   S~_C = S~0 + K^T (E U) / (sigma gamma_C).
+// P needs only the chunk's keys and the state, so it is formed on the tensor
+// core as soon as the previous chunk's state update is done, while the
+// chunk's T is still being built; once T is ready, E U is two MMAs into one
+// accumulator (E U' from V, then the P term).  The serial part of a chunk is
+// therefore: T operands -> U MMAs -> U epilogue -> state update -> P.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -28,29 +33,139 @@ namespace {
 using namespace sm100;
 using namespace chunk;
 
-// ---------------------------------------------------------------------------
-// Tail replay with two chunks in flight inside the CTA.
-//
-// The state-independent front of chunk c + 1 (A = strict_tril(...K K^T) and
-// the UT inverse) runs on warps 0-3 while warps 4-7 finish chunk c's state
-// chain: the U epilogue (U~ to bf16 in TMEM), the state update on the tensor
-// core, and the TMA of chunk c + 2 into the tile slot that update frees.  Warps 6-7 first write the
-// lower-right quarter of A, the only part of A outside columns 0-31.  Then all
-// eight warps form T diag(beta), W and U', and -sigma W of chunk c + 1 and start
-// its state product, then K K^T of chunk c + 2.  98 KB of shared memory, 256
-// TMEM columns and at most 128 registers per thread, so two CTAs share an SM.
+// ---- shared memory (byte offsets from a 1 KB aligned base) ----
+// K of a chunk stays from its K K^T until its state update (two slots); V only
+// until its U' MMA (one slot).  K32 holds the next chunk's keys in fp32, the B
+// operand of P.  AT holds A, then T in place, then the fp32 operand
+// -sigma E T diag(beta gamma) in place; TB holds the bf16 E T diag(beta), and
+// the inverse's scratch before it.
+struct ReplayLayout {
+    static constexpr uint32_t BOX = 8192;                   // 64 rows x 64 bf16 (128-byte swizzle)
+    static constexpr uint32_t K_SLOT = 2 * BOX;             // [dk 0-63 | dk 64-127]
+    static constexpr uint32_t OFF_K = 0;                    // chunk c in slot c % 2
+    static constexpr uint32_t OFF_V = OFF_K + 2 * K_SLOT;   // [dv 0-63 | dv 64-127]
+    static constexpr uint32_t OFF_K32 = OFF_V + 2 * BOX;    // fp32 [j][dk], four 8 KB blocks of 32 columns
+    static constexpr uint32_t OFF_AT = OFF_K32 + 32768;     // fp32 64 x LDT
+    static constexpr uint32_t OFF_TB = OFF_AT + C * LDT * 4;
+    static constexpr uint32_t OFF_X = OFF_TB;
+    static constexpr uint32_t BYTES = OFF_TB + 8192;
+};
+static_assert(ReplayLayout::OFF_TB % 1024 == 0 && ReplayLayout::OFF_AT % 1024 == 0, "operands on 1 KB");
+static_assert(4 * 16 * 24 * 4 <= 8192, "inverse scratch fits the T operand's space");
+static_assert(2 * 8192 <= C * LDT * 4, "the fp32 T operand fits over T");
+static_assert(2 * (ReplayLayout::BYTES + 1024 + 4096) <= 228 * 1024, "two replay CTAs per SM");
+
+// TMEM columns: the state S~^T (lane = value row), then two 64-column regions
+// that alternate between chunks.  Region c % 2 holds K K^T of chunk c (M = 64),
+// then E U of chunk c (M = 128, lane = value row) and U~ = E U / sigma in bf16
+// over its first 32 columns; after chunk c's state update it holds P of chunk
+// c + 1 (P^T, lane = value row, fp32).
+constexpr uint32_t TM_R0 = 128;
+
 constexpr uint32_t BAR_CHAIN = 2;   // named barrier of warps 4-7 (the state chain)
 constexpr uint32_t BAR_A = 4;       // warps 6-7 -> warps 2-3: their part of A is written
 
+// From T (fp32, in place in AT) write the two T operands of a chunk, with
+// 256 threads (thread -> row j = tid % 64, columns 16 part .. 16 part + 15):
+//   tb : E T diag(beta), bf16 [j][j'] in 128-byte swizzled rows (U' = that V);
+//   AT : -sigma E T diag(beta gamma), fp32 K-major [j][j'] in two 8 KB blocks of
+//        32 columns (128-byte swizzled), over T itself: every thread reads its
+//        values, the block meets at a barrier, then writes.
+// Consecutive threads take consecutive rows, so the row reads (stride LDT) and
+// the swizzled stores are free of bank conflicts.
+__device__ __forceinline__ void write_t_operands(float* AT, const Gates& G, float sigma, uint8_t* tb, int tid) {
+    const int j = tid & (C - 1), part = tid >> 6;
+    const float ej = G.e[j];
+    const float nsj = -sigma * ej;
+    float vb[16], vg[16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int col = part * 16 + 4 * q;
+        float4 tt = make_float4(0.f, 0.f, 0.f, 0.f);
+        if ((col >> 4) <= (j >> 4)) tt = *reinterpret_cast<const float4*>(AT + j * LDT + col);
+        const float4 b4 = *reinterpret_cast<const float4*>(G.beta + col);
+        const float4 g4 = *reinterpret_cast<const float4*>(G.gam + col);
+        const float tv[4] = {tt.x, tt.y, tt.z, tt.w};
+        const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+        const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float tbv = tv[e] * bv[e];
+            vb[4 * q + e] = tbv * ej;
+            vg[4 * q + e] = tbv * gv[e] * nsj;
+        }
+    }
+    __syncthreads();   // every read of T is done before the fp32 operand overwrites it
+#pragma unroll
+    for (int ch = 0; ch < 2; ++ch) {
+        uint4 x;
+        x.x = pack_bf16(vb[ch * 8 + 0], vb[ch * 8 + 1]);
+        x.y = pack_bf16(vb[ch * 8 + 2], vb[ch * 8 + 3]);
+        x.z = pack_bf16(vb[ch * 8 + 4], vb[ch * 8 + 5]);
+        x.w = pack_bf16(vb[ch * 8 + 6], vb[ch * 8 + 7]);
+        st_shared_v4(tb, (uint32_t)(j * 128 + (((2 * part + ch) ^ (j & 7)) << 4)), x);
+    }
+    uint8_t* blk = reinterpret_cast<uint8_t*>(AT) + (part >> 1) * 8192 + j * 128;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<float4*>(blk + (((4 * (part & 1) + q) ^ (j & 7)) << 4)) =
+            make_float4(vg[4 * q], vg[4 * q + 1], vg[4 * q + 2], vg[4 * q + 3]);
+}
+
+// Keys of one chunk (bf16 K slot: two 8 KB boxes of 64 rows x 64 columns,
+// 128-byte swizzled) to fp32, K-major [j][dk] in four 8 KB blocks of 32 columns
+// (128-byte swizzled); rows j >= nrows are written as zeros.  128 threads:
+// thread ct -> row j = ct % 64, columns 64 h .. 64 h + 63 with h = ct / 64.
+__device__ __forceinline__ void convert_k_f32(const uint8_t* kslot, uint8_t* k32, int ct, int nrows) {
+    const int j = ct & (C - 1), h = ct >> 6;
+    const uint8_t* src = kslot + h * 8192 + j * 128;
+    const bool live = j < nrows;
+    // every load before the first store (the stores may alias the loads for the compiler)
+    uint4 raw[8];
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch)
+        raw[ch] = live ? *reinterpret_cast<const uint4*>(src + ((ch ^ (j & 7)) << 4)) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {   // columns 64 h + 8 ch .. + 7
+        const uint32_t wds[4] = {raw[ch].x, raw[ch].y, raw[ch].z, raw[ch].w};
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            f[2 * e] = __uint_as_float(wds[e] << 16);
+            f[2 * e + 1] = __uint_as_float(wds[e] & 0xffff0000u);
+        }
+        uint8_t* blk = k32 + (2 * h + (ch >> 2)) * 8192 + j * 128;
+        *reinterpret_cast<float4*>(blk + (((2 * (ch & 3)) ^ (j & 7)) << 4)) = make_float4(f[0], f[1], f[2], f[3]);
+        *reinterpret_cast<float4*>(blk + (((2 * (ch & 3) + 1) ^ (j & 7)) << 4)) = make_float4(f[4], f[5], f[6], f[7]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Tail replay, two chunks in flight inside the CTA.  Iteration c:
+//   phase X  warps 0-3: A of chunk c + 1 (columns 0-31; its K K^T was issued in the
+//                       last phase Y), then T = (I + A)^-1;
+//            warps 4-7: chunk c's chain: the U epilogue (U~ to bf16 in TMEM), the
+//                       state update, then P of chunk c + 1 and the TMA of chunk
+//                       c + 2's keys (warp 4); warps 6-7 first write the lower-right
+//                       quarter of A.
+//   phase Y  all warps: the T operands of chunk c + 1; then warp 2 issues the P term
+//                       and U' of chunk c + 1 into one accumulator, and K K^T of
+//                       chunk c + 2 once the P term has read its region; warps 4-7
+//                       turn chunk c + 2's keys into fp32 once P of chunk c + 1 is
+//                       done with them; warps 0-1 build the gates of chunk c + 2;
+//                       then the TMA of chunk c + 2's values.
+// 106 KB of shared memory, 256 TMEM columns and at most 128 registers per
+// thread, so two CTAs share an SM.
 __global__ void __launch_bounds__(NT, 2)
 replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                    const __grid_constant__ CUtensorMap map_v) {
-    using L = Layout<true>;
+    using RL = ReplayLayout;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    // bar_w: W and U' (two issuers); bar_u: the state product and the next chunk's
-    // K K^T (two issuers); bar_s: the state update (one issuer)
-    __shared__ uint64_t bar_tile[2], bar_w, bar_u, bar_s;
+    // bar_k: keys of chunk c (slot c % 2); bar_v: values; bar_kk: K K^T; bar_s: the
+    // state update; bar_p: P; bar_x: the P term of E U; bar_u: E U (the P term and U').
+    // One issuer each.
+    __shared__ uint64_t bar_k[2], bar_v, bar_kk, bar_s, bar_p, bar_x, bar_u;
     __shared__ uint32_t tmem_slot;
     __shared__ Gates s_gates[2];    // chunk c uses s_gates[c & 1]
 
@@ -72,11 +187,14 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         return;
 
     if (tid == 0) {
-        mbar_init(&bar_tile[0], 1);
-        mbar_init(&bar_tile[1], 1);
-        mbar_init(&bar_w, 2);
-        mbar_init(&bar_u, 2);
+        mbar_init(&bar_k[0], 1);
+        mbar_init(&bar_k[1], 1);
+        mbar_init(&bar_v, 1);
+        mbar_init(&bar_kk, 1);
         mbar_init(&bar_s, 1);
+        mbar_init(&bar_p, 1);
+        mbar_init(&bar_x, 1);
+        mbar_init(&bar_u, 1);
         mbar_fence_init();
         tma_prefetch_desc(&map_k);
         tma_prefetch_desc(&map_v);
@@ -90,17 +208,30 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     tc_fence_after();
     const uint32_t tbase = tmem_slot;
     const uint32_t tlane = tbase + ((uint32_t)(wq * 32) << 16);
-    auto tile_of = [&](int cc) { return sm + L::OFF_TILE + (cc & 1) * L::TILE; };
-    if (tid == 0) {   // both slots are free: chunks 0 and 1
-        for (int cc = 0; cc < 2 && cc < nchunks; ++cc)
-            issue_tiles<true>(tile_of(cc), &bar_tile[cc & 1], &map_k, &map_v, &map_k, h,
-                              (int)(w.row0 + (long long)cc * C), false);
+    auto region = [](int cc) -> uint32_t { return TM_R0 + (uint32_t)(cc & 1) * 64u; };
+    auto kslot = [&](int cc) { return sm + RL::OFF_K + (cc & 1) * RL::K_SLOT; };
+    auto issue_k = [&](int cc) {
+        uint8_t* dst = kslot(cc);
+        const int r0 = (int)(w.row0 + (long long)cc * C);
+        mbar_arrive_expect_tx(&bar_k[cc & 1], RL::K_SLOT);
+        tma_load_3d(dst, &map_k, &bar_k[cc & 1], 0, h, r0);
+        tma_load_3d(dst + RL::BOX, &map_k, &bar_k[cc & 1], 64, h, r0);
+    };
+    auto issue_v = [&](int cc) {
+        const int r0 = (int)(w.row0 + (long long)cc * C);
+        mbar_arrive_expect_tx(&bar_v, 2 * RL::BOX);
+        tma_load_3d(sm + RL::OFF_V, &map_v, &bar_v, 0, h, r0);
+        tma_load_3d(sm + RL::OFF_V + RL::BOX, &map_v, &bar_v, 64, h, r0);
+    };
+    if (tid == 0) {
+        for (int cc = 0; cc < 2 && cc < nchunks; ++cc) issue_k(cc);
+        if (nchunks > 0) issue_v(0);
     }
 
-    float* AT = reinterpret_cast<float*>(sm + L::OFF_AT);
-    float* Xs = reinterpret_cast<float*>(sm + L::OFF_X);
-    const uint32_t s_bu = smem_u32(sm + L::OFF_BU);
-    const uint32_t s_tb = smem_u32(sm + L::OFF_TB), s_tbg = smem_u32(sm + L::OFF_TBG);
+    float* AT = reinterpret_cast<float*>(sm + RL::OFF_AT);
+    float* Xs = reinterpret_cast<float*>(sm + RL::OFF_X);
+    const uint32_t s_at = smem_u32(sm + RL::OFF_AT), s_tb = smem_u32(sm + RL::OFF_TB);
+    const uint32_t s_k32 = smem_u32(sm + RL::OFF_K32), s_v = smem_u32(sm + RL::OFF_V);
     const size_t state_base = ((size_t)b * H + h) * D * D;
     {   // zero state: TMEM lane dv holds column dv of S / sigma (a row of S^T)
         float v[32];
@@ -113,10 +244,9 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     float sigma = 1.0f;
 
     const uint32_t id_kk = idesc_bf16(64, 64, false, false);   // K K^T; row r in lane 32 (r/16) + r%16
-    const uint32_t id_w = idesc_bf16(128, 64, true, false);    // K^T (T..)^T, V^T (T..)^T
-    const uint32_t id_u = idesc_tf32(128, 64, false, false);   // S^T (-sigma W^T), A in TMEM
+    const uint32_t id_w = idesc_bf16(128, 64, true, false);    // V^T (E T diag(beta))^T
+    const uint32_t id_t = idesc_tf32(128, 64, false, false);   // P^T = S~^T K^T; P^T (-sigma E T..)^T; A in TMEM
     const uint32_t id_s = idesc_bf16(128, 128, false, true);   // U~^T K, A (U~^T) in TMEM
-    uint32_t ph_w = 0, ph_u = 0, ph_s = 0;
     bool ok = true;
 
     auto load_gates = [&](int cc, float& al, float& be) {
@@ -130,31 +260,9 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             }
         }
     };
-    auto tiles_ready = [&](int cc) -> bool {
-        uint8_t* tile = tile_of(cc);
-        if (!wait_all(&bar_tile[cc & 1], (cc >> 1) & 1, a, 1)) return false;
-        const int ncc = min(C, w.len - cc * C);
-        if (ncc < C) {   // padded tokens are identity transitions: zero their rows
-            const int nrows = C - ncc;
-            for (int e = tid; e < 4 * nrows * 8; e += NT) {
-                const int t = e / (nrows * 8), rr = ncc + (e / 8) % nrows, ch = e % 8;
-                st_shared_v4(tile + t * 8192, (uint32_t)(rr * 128 + ch * 16), make_uint4(0, 0, 0, 0));
-            }
-            fence_proxy_async_smem();
-        }
-        __syncthreads();
-        return true;
-    };
-    auto issue_kk = [&](int cc) {
-        const uint64_t dk0 = smem_desc_sw128(smem_u32(tile_of(cc)), 16, 1024);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t d = desc_advance(dk0, (kk >> 2) * L::K_BLK + (kk & 3) * 32);
-            mma_bf16_ss(tbase + TM_P, d, d, id_kk, kk > 0);
-        }
-    };
+    auto nrows_of = [&](int cc) { return min(C, w.len - cc * C); };
 
-    // Epilogue 1 of chunk cc over the 32 columns [cb, cb + 32):
+    // Epilogue 1 of chunk cc over the 32 columns [cb, cb + 32) of its K K^T:
     // A = strict_tril(beta_i (gamma_i / gamma_j) K K^T), fp32 into AT.  The M = 64
     // accumulator keeps rows 16 wq .. 16 wq + 15 in the quarter's first 16 lanes; this
     // thread takes rows i0 = 16 wq + lane / 4 and i0 + 8, columns cb + 8 k + 2 (lane % 4)
@@ -165,7 +273,7 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         const Gates& Gn = s_gates[cc & 1];
         const bool fast = Gn.g2[C - 1] >= kFastGateFloor;
         float v[16];
-        tmem_ld16x256b_x4(tlane + TM_P + cb, v);
+        tmem_ld16x256b_x4(tlane + region(cc) + cb, v);
         const int i0 = 16 * wq + (lane >> 2), jb = cb + 2 * (lane & 3);
         const float* colf = fast ? Gn.binv : Gn.g2;   // column factor: 2^-G_j, or G_j
         float2 cf[4];
@@ -200,6 +308,31 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             }
         }
     };
+    // wait for K K^T of chunk cc (every thread that reads it); false if the wait ran out
+    auto kk_ready = [&](int cc) -> bool {
+        const bool t = mbar_wait_bounded(&bar_kk, cc & 1, kWaitNs);
+        if (!t) report_timeout(a, 2);
+        tc_fence_after();
+        return t;
+    };
+
+    // zero the rows past the window of a partial chunk's key (bx = 0) or value slot;
+    // every thread takes part, after the tile has arrived
+    auto zero_tail_rows = [&](uint8_t* slot, int nrows) {
+        const int nz = C - nrows;
+        for (int e = tid; e < 2 * nz * 8; e += NT) {
+            const int bx = e / (nz * 8), rr = nrows + (e / 8) % nz, ch = e % 8;
+            st_shared_v4(slot + bx * RL::BOX, (uint32_t)(rr * 128 + ch * 16), make_uint4(0, 0, 0, 0));
+        }
+    };
+    auto issue_kk = [&](int cc) {
+        const uint64_t dk0 = smem_desc_sw128(smem_u32(kslot(cc)), 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t d = desc_advance(dk0, (kk >> 2) * RL::BOX + (kk & 3) * 32);
+            mma_bf16_ss(tbase + region(cc), d, d, id_kk, kk > 0);
+        }
+    };
 
     // ---- prologue: gates of chunk 0 (built) and 1 (registers), K K^T of chunk 0 ----
     float al_nxt, be_nxt;
@@ -207,32 +340,40 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     if (tid < C) build_gates(s_gates[0], al_nxt, be_nxt, tid, lane);
     load_gates(1, al_nxt, be_nxt);
     if (nchunks > 0) {
-        ok = tiles_ready(0);
-        if (ok && (warp == 2 || warp == 3)) {
-            tc_fence_after();
+        bool t = true;
+        if (nrows_of(0) < C) {
+            t = mbar_wait_bounded(&bar_k[0], 0, kWaitNs);
+            if (t) zero_tail_rows(kslot(0), nrows_of(0));
+            else report_timeout(a, 1);
+            fence_proxy_async_smem();
+        }
+        ok = __syncthreads_and(t) != 0;
+        if (ok && warp == 0) {
+            bool tw = true;
             if (elect_one()) {
-                if (warp == 3) issue_kk(0);
-                mma_commit(&bar_u);
+                if (nrows_of(0) == C) {
+                    tw = mbar_wait_bounded(&bar_k[0], 0, kWaitNs);
+                    if (!tw) report_timeout(a, 1);
+                }
+                tc_fence_after();
+                if (tw) issue_kk(0);
+                mma_commit(&bar_kk);
             }
             __syncwarp();
         }
-        if (ok) {
-            ok = wait_all(&bar_u, ph_u, a, 2);
-            ph_u ^= 1;
-        }
     }
+    __syncthreads();
 
-    // Iteration c: phase X overlaps chunk c's chain (c >= 0) with chunk c + 1's front;
-    // phase Y finishes chunk c + 1's state-independent part and starts its state product.
     for (int c = -1; c < nchunks && ok; ++c) {
         const int cn = c + 1;
         const bool has_next = cn < nchunks;
         bool xok = true;
-        tc_fence_after();
+        // =============================== phase X ===============================
         if (warp < 4) {
             if (has_next) {
                 // ---- epilogue 1 of chunk cn, columns 0-31 (warps 6-7 take rows 32-63 x
                 //      columns 32-63; rows 0-31 have no entries there) ----
+                xok = kk_ready(cn) && xok;
                 epi1_half(cn, 0);
                 __syncwarp();
                 // the diagonal solve of block wq reads rows 16 wq .. 16 wq + 15; for wq >= 2
@@ -244,170 +385,187 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             }
         } else {
             if (has_next && warp >= 6) {
+                xok = kk_ready(cn) && xok;
                 epi1_half(cn, 32);
                 named_arrive(BAR_A, 128);
             }
-        }
-        if (warp >= 4 && c >= 0) {
-            // ---- epilogue U of chunk c: U~ = diag(gamma_C / gamma) U / sigma_new into the
-            //      chunk's V boxes (the row decay is already in U, through the rows of the T
-            //      operands); the decay is folded into the TMEM state when sigma gets small ----
-            Gates& G = s_gates[c & 1];
-            uint8_t* tile = tile_of(c);
-            float snew = sigma * G.gam[C - 1];
-            if (snew < kRenormBelow) {   // uniform
+            if (c >= 0) {
+                // ---- epilogue U of chunk c: U~ = E U / sigma_new, bf16 back into TMEM over the
+                //      first 32 columns of its region (half hf lands on columns 16 hf .. 16 hf +
+                //      15, which this thread has read already); the decay is folded into the
+                //      TMEM state when sigma gets small ----
+                Gates& G = s_gates[c & 1];
+                float snew = sigma * G.gam[C - 1];
+                if (snew < kRenormBelow) {   // uniform
 #pragma unroll
-                for (int cb = 0; cb < 4; ++cb) {
-                    float sv[32];
-                    tmem_ld32(tlane + TM_S + cb * 32, sv);
+                    for (int cb = 0; cb < 4; ++cb) {
+                        float sv[32];
+                        tmem_ld32(tlane + TM_S + cb * 32, sv);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) sv[q] *= snew;
+                        tmem_st32(tlane + TM_S + cb * 32, sv);
+                    }
+                    snew = 1.0f;
+                }
+                const float inv = 1.0f / snew;
+                const uint32_t ru = region(c);
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    float v[32];   // value dv = row, chunk rows [32 hf, 32 hf + 32)
+                    tmem_ld32(tlane + ru + 32 * hf, v);
                     tmem_wait_ld();
+                    uint32_t pk[16];
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) sv[q] *= snew;
-                    tmem_st32(tlane + TM_S + cb * 32, sv);
+                    for (int q = 0; q < 16; ++q) pk[q] = pack_bf16(v[2 * q] * inv, v[2 * q + 1] * inv);
+                    tmem_st16(tlane + ru + 16 * hf, pk);
                 }
                 tmem_wait_st();
-                snew = 1.0f;
-            }
-            const float inv = 1.0f / snew;
-            // U~^T as bf16 back into TMEM, two chunk rows per 32-bit column, over the first 32
-            // columns of TM_U (half hf lands on columns 16 hf .. 16 hf + 15, which this thread
-            // has read already): the A operand of the state update, with no trip through
-            // shared memory
+                tc_fence_before();
+                xok = named_sync_and(BAR_CHAIN, 128, xok);
+                // ---- S~^T += U~^T K of chunk c; then P^T of chunk cn = S~^T K_cn^T into the same
+                //      region (its keys are in fp32 since the last phase Y), and the keys of
+                //      chunk c + 2 into the slot chunk c frees ----
+                if (warp == 4) {
+                    tc_fence_after();
+                    bool t = xok;
+                    if (elect_one()) {
+                        if (t) {
+                            const uint64_t db = smem_desc_sw128(smem_u32(kslot(c)), RL::BOX, 1024);
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                float v[32];   // value dv = row, chunk rows [32 hf, 32 hf + 32)
-                tmem_ld32(tlane + TM_U + 32 * hf, v);
-                tmem_wait_ld();
-                uint32_t pk[16];
+                            for (int kk = 0; kk < 4; ++kk)
+                                mma_bf16_ts(tbase + TM_S, tbase + ru + kk * 8, desc_advance(db, kk * 2048), id_s, 1u);
+                        }
+                        mma_commit(&bar_s);
+                        if (mbar_wait_bounded(&bar_s, c & 1, kWaitNs)) {
+                            tc_fence_after();
+                            if (t && has_next) {
+                                const uint64_t dk = smem_desc_sw128(s_k32, 16, 1024);
 #pragma unroll
-                for (int q = 0; q < 16; ++q) pk[q] = pack_bf16(v[2 * q] * inv, v[2 * q + 1] * inv);
-                tmem_st16(tlane + TM_U + 16 * hf, pk);
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            named_sync(BAR_CHAIN, 128);
-            // ---- S^T / sigma += U~^T K of chunk c; once it is done the slot takes chunk c + 2 ----
-            if (warp == 4) {
-                tc_fence_after();
-                if (elect_one()) {
-                    const uint32_t s_tile = smem_u32(tile);
-                    const uint64_t db = smem_desc_sw128(s_tile, L::K_BLK, 1024);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ts(tbase + TM_S, tbase + TM_U + kk * 8, desc_advance(db, kk * 2048), id_s, 1u);
-                    mma_commit(&bar_s);
-                    if (mbar_wait_bounded(&bar_s, ph_s, kWaitNs)) {
-                        if (c + 2 < nchunks)
-                            issue_tiles<true>(tile, &bar_tile[c & 1], &map_k, &map_v, &map_k, h,
-                                              (int)(w.row0 + (long long)(c + 2) * C), false);
-                    } else {
-                        report_timeout(a, 6);
-                        xok = false;
+                                for (int kk = 0; kk < 16; ++kk)
+                                    mma_tf32_ts(tbase + ru, tbase + TM_S + kk * 8,
+                                                desc_advance(dk, (kk >> 2) * 8192 + (kk & 3) * 32), id_t, kk > 0);
+                            }
+                            if (has_next) mma_commit(&bar_p);
+                            if (t && c + 2 < nchunks) issue_k(c + 2);
+                        } else {
+                            report_timeout(a, 6);
+                            t = false;
+                        }
                     }
+                    xok = __all_sync(0xffffffffu, t) && xok;
                 }
-                __syncwarp();
             }
         }
         if (c >= 0) {   // every thread keeps the same running scale
             const float snew = sigma * s_gates[c & 1].gam[C - 1];
             sigma = snew < kRenormBelow ? 1.0f : snew;
-            ph_s ^= 1;
         }
-        ok = __syncthreads_and(xok) != 0;   // the state update of chunk c is done
+        tc_fence_before();
+        ok = __syncthreads_and(xok) != 0;   // T of chunk cn is in AT; chunk c's state update is done
         if (!ok || !has_next) break;
-
-        // ---- phase Y, chunk cn: E T diag(beta), E T diag(beta gamma) in bf16 ----
-        Gates& Gn = s_gates[cn & 1];
-        const uint32_t s_tile_n = smem_u32(tile_of(cn));
-        write_scaled_t<NT, false>(AT, Gn.beta, Gn.gam, sm + L::OFF_TB, sm + L::OFF_TBG, tid, 0, Gn.e);
-        fence_proxy_async_smem();
-        __syncthreads();
-        // ---- (E W)^T = K^T (E T diag(beta gamma))^T -> TM_P and (E U')^T = V^T (E T diag(beta))^T -> TM_U ----
-        if (warp == 0) {
-            tc_fence_after();
-            if (elect_one()) {
-                const uint64_t da = smem_desc_sw128(s_tile_n, L::K_BLK, 1024);
-                const uint64_t db = smem_desc_sw128(s_tbg, 16, 1024);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ss(tbase + TM_P, desc_advance(da, kk * 2048), desc_advance(db, kk * 32), id_w, kk > 0);
-                mma_commit(&bar_w);
-            }
-            __syncwarp();
-        } else if (warp == 1) {
-            tc_fence_after();
-            if (elect_one()) {
-                const uint64_t da = smem_desc_sw128(s_tile_n + L::V0, L::V_LBO, 1024);
-                const uint64_t db = smem_desc_sw128(s_tb, 16, 1024);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ss(tbase + TM_U, desc_advance(da, kk * 2048), desc_advance(db, kk * 32), id_w, kk > 0);
-                mma_commit(&bar_w);
-            }
-            __syncwarp();
-        }
-        ok = wait_all(&bar_w, ph_w, a, 3);
-        ph_w ^= 1;
-        if (!ok) break;
         tc_fence_after();
-        // ---- epilogue 2: BU[j][dk] = -sigma (E W)[j][dk] (fp32, K-major) ----
-        {
-            float v[32];   // key dk = row, chunk rows [32 wh, 32 wh + 32)
-            tmem_ld32(tlane + TM_P + 32 * wh, v);
-            tmem_wait_ld();
-            uint8_t* bu = sm + L::OFF_BU + wq * 8192;
-            const float ns = -sigma;
-#pragma unroll
-            for (int jj = 0; jj < 32; ++jj)
-                *reinterpret_cast<float*>(bu + sw128_offset_f32(32 * wh + jj, lane)) = ns * v[jj];
+
+        // =============================== phase Y ===============================
+        // ---- T operands of chunk cn: E T diag(beta) (bf16) and -sigma E T diag(beta gamma)
+        //      (fp32, over T); partial tiles get their rows past the window zeroed first ----
+        const Gates& Gn = s_gates[cn & 1];
+        const int ncn = nrows_of(cn);
+        const bool has_nn = cn + 1 < nchunks;
+        const int nnn = has_nn ? nrows_of(cn + 1) : C;
+        bool tok = true;
+        if (ncn < C) {   // values of chunk cn
+            const bool t = mbar_wait_bounded(&bar_v, cn & 1, kWaitNs);
+            if (t) zero_tail_rows(sm + RL::OFF_V, ncn);
+            else report_timeout(a, 1);
+            tok = tok && t;
         }
+        if (nnn < C) {   // keys of chunk cn + 1 (its K K^T is issued below)
+            const bool t = mbar_wait_bounded(&bar_k[(cn + 1) & 1], ((cn + 1) >> 1) & 1, kWaitNs);
+            if (t) zero_tail_rows(kslot(cn + 1), nnn);
+            else report_timeout(a, 1);
+            tok = tok && t;
+        }
+        write_t_operands(AT, Gn, sigma, sm + RL::OFF_TB, tid);
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();
-        // ---- state product of chunk cn (warp 2) at once; K K^T of chunk cn + 1 (warp 3) once
-        //      its tiles are in, while warps 0-1 build chunk cn + 1's gate factors ----
+        tok = __syncthreads_and(tok) != 0;
         if (warp == 2) {
+            // ---- (E U)^T of chunk cn into its region: P^T (-sigma E T diag(beta gamma))^T, then
+            //      + V^T (E T diag(beta))^T; then K K^T of chunk cn + 1 into the region the P
+            //      term has just read ----
             tc_fence_after();
+            bool t = tok;
             if (elect_one()) {
-                const uint64_t db = smem_desc_sw128(s_bu, 16, 1024);
-#pragma unroll
-                for (int kk = 0; kk < 16; ++kk)
-                    mma_tf32_ts(tbase + TM_U, tbase + TM_S + kk * 8,
-                                desc_advance(db, (kk >> 2) * 8192 + (kk & 3) * 32), id_u, 1u);
-                mma_commit(&bar_u);
-            }
-            __syncwarp();
-        }
-        // A full next chunk: warp 3 alone waits for its tiles (the next block-wide barrier
-        // orders them for every later reader).  A partial one: the block zero-pads it first.
-        // A tile timeout still waits for the state product below before the block leaves.
-        const bool has_nn = cn + 1 < nchunks;
-        const bool nn_partial = has_nn && w.len - (cn + 1) * C < C;   // uniform
-        bool tok = true;
-        if (nn_partial) tok = tiles_ready(cn + 1);
-        if (warp == 3) {
-            // the thread that sees the tiles arrive is the one that issues the MMA reading them
-            bool t = true;
-            if (elect_one()) {
-                if (has_nn && !nn_partial) {
-                    t = mbar_wait_bounded(&bar_tile[(cn + 1) & 1], ((cn + 1) >> 1) & 1, kWaitNs);
+                const uint32_t rn = region(cn);
+                if (t && ncn == C) {
+                    t = mbar_wait_bounded(&bar_v, cn & 1, kWaitNs);
                     if (!t) report_timeout(a, 1);
                 }
+                if (t && cn > 0) {   // the state is zero before chunk 0
+                    t = mbar_wait_bounded(&bar_p, (cn - 1) & 1, kWaitNs);
+                    if (!t) report_timeout(a, 3);
+                }
                 tc_fence_after();
-                if (t && tok && has_nn) issue_kk(cn + 1);
+                if (t) {
+                    if (cn > 0) {
+                        const uint64_t d2 = smem_desc_sw128(s_at, 16, 1024);
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            mma_tf32_ts(tbase + rn, tbase + region(c) + kk * 8,
+                                        desc_advance(d2, (kk >> 2) * 8192 + (kk & 3) * 32), id_t, kk > 0);
+                        mma_commit(&bar_x);
+                    }
+                    const uint64_t dv = smem_desc_sw128(s_v, RL::BOX, 1024);
+                    const uint64_t dt = smem_desc_sw128(s_tb, 16, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ss(tbase + rn, desc_advance(dv, kk * 2048), desc_advance(dt, kk * 32), id_w,
+                                    (cn > 0 || kk > 0) ? 1u : 0u);
+                }
                 mma_commit(&bar_u);
+                if (has_nn) {
+                    if (t && nnn == C) {
+                        t = mbar_wait_bounded(&bar_k[(cn + 1) & 1], ((cn + 1) >> 1) & 1, kWaitNs);
+                        if (!t) report_timeout(a, 1);
+                    }
+                    if (t && cn > 0) {   // the P term is done reading region (cn + 1) % 2
+                        t = mbar_wait_bounded(&bar_x, (cn - 1) & 1, kWaitNs);
+                        if (!t) report_timeout(a, 5);
+                    }
+                    tc_fence_after();
+                    if (t) issue_kk(cn + 1);
+                    mma_commit(&bar_kk);
+                }
             }
             tok = __all_sync(0xffffffffu, t) && tok;
+        } else if (warp >= 4) {
+            // ---- keys of chunk cn + 1 to fp32 (the B operand of its P), once P of chunk cn
+            //      is done reading them ----
+            if (has_nn) {
+                const int ct = tid - 128;
+                bool t = true;
+                if (cn > 0) t = mbar_wait_bounded(&bar_p, (cn - 1) & 1, kWaitNs);
+                if (t) t = mbar_wait_bounded(&bar_k[(cn + 1) & 1], ((cn + 1) >> 1) & 1, kWaitNs);
+                if (t) convert_k_f32(kslot(cn + 1), sm + RL::OFF_K32, ct, nnn);
+                else report_timeout(a, 7);
+                fence_proxy_async_smem();
+                tok = tok && t;
+            }
         } else if (tid < C && has_nn) {
             build_gates(s_gates[(cn + 1) & 1], al_nxt, be_nxt, tid, lane);
         }
         if (has_nn) load_gates(cn + 2, al_nxt, be_nxt);
-        {   // wait_all, with warp 3's tile flag in the same vote
-            const bool okw = mbar_wait_bounded(&bar_u, ph_u, kWaitNs);
+        {
+            const bool okw = mbar_wait_bounded(&bar_u, cn & 1, kWaitNs);
             ok = __syncthreads_and(okw && tok) != 0;
             if (!ok && tid == 0) report_timeout(a, 4);
         }
-        ph_u ^= 1;
+        // U' of chunk cn is done with the value slot: the values of chunk cn + 1 go there
+        if (ok && warp == 2 && has_nn) {
+            if (elect_one()) issue_v(cn + 1);
+            __syncwarp();
+        }
     }
 
     // ---- final state: S[dk][dv] = sigma * TMEM[lane dv][dk] ----
@@ -446,7 +604,7 @@ cudaError_t launch_replay_tc(const CallArgs& a, cudaStream_t stream) {
         !make_tile_map(&mv, vb, a.num_heads, a.rows_total, a.rs_v))
         return cudaErrorInvalidValue;
     static std::atomic<uint64_t> smem_set{0};
-    const uint32_t smem = Layout<true>::BYTES + 1024;
+    const uint32_t smem = ReplayLayout::BYTES + 1024;
     const cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(replay_pipe_kernel), (int)smem, smem_set);
     if (e != cudaSuccess) return e;
     replay_pipe_kernel<<<(unsigned)a.units, NT, smem, stream>>>(p, mk, mv);
