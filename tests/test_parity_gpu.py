@@ -353,3 +353,29 @@ def test_longest_windows_against_oracle():
     ref_o, ref_st2 = oracle_prefill(s, np.array([0, N], np.int32), None)
     assert rel_err(o.float().cpu().numpy(), ref_o) <= TOL["bf16"]
     assert per_request_state_err(st2.cpu().numpy(), ref_st2) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("kname", ["recurrent", "chunked"])
+def test_chunk_boundary_window_lengths(kname):
+    """Windows of 1, 63, 64, 65, 127, 128, 129, 191, 192 and 193 rows in one launch: one to
+    four chunks, with and without a partial last chunk (whose key and value rows past the
+    window are zeroed in shared memory), so every iteration shape of the two-chunk
+    schedule runs.  The cached entries are longer than their windows, so the rows past
+    a window hold real data that must not leak in.  Replay, then a prefill of suffixes
+    of the same lengths from the replayed states."""
+    kernel = kernel_or_skip(kname, "bf16", 128, 128)
+    lens = [1, 63, 64, 65, 127, 128, 129, 191, 192, 193]
+    H = 2
+    cached = [n + 37 for n in lens]
+    ml = [n + 5 for n in lens]
+    off = np.concatenate([[0], np.cumsum(cached)]).astype(np.int32)
+    t = make_cache(cached, H, 128, 128, "bf16", seed=91)
+    st = run_replay(t, off, ml, lens, kernel, "bf16")
+    ref = oracle_replay(t, off, ml, lens)
+    assert per_request_state_err(st.cpu().numpy(), ref) <= TOL["bf16"]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    s = make_cache(lens, H, 128, 128, "bf16", seed=92)
+    o, st2 = run_prefill(s, cu, st, kernel, "bf16")
+    ref_o, ref_st2 = oracle_prefill(s, cu, st)
+    assert per_request_rows_err(o.float().cpu().numpy(), ref_o, cu) <= TOL["bf16"]
+    assert per_request_state_err(st2.cpu().numpy(), ref_st2) <= TOL["bf16"]
