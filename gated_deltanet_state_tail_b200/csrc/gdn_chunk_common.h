@@ -189,17 +189,13 @@ __device__ __forceinline__ void invert_unit_lower_inplace(float* AT, float* Xs, 
 
 // From the inverse T (in place in AT, see above) write the bf16 operands
 // T diag(beta) -> tb and T diag(beta gamma) -> tbg, [j][j'] in 128-byte
-// swizzled rows, with NTH threads (ltid < NTH) sharing barrier bar_id.
-// With rowe (the state-only replay), row j of both is also scaled by rowe[j]:
-// the products W and U' then carry the decay gamma_C / gamma_j that the state
-// update applies to row j of U.
-// beta, gam and rowe are 16-byte aligned.
-// IN_PLACE: tb / tbg overlap AT, so every thread reads its values before a
-// barrier and writes after it; otherwise there is no barrier.
-template <int NTH, bool IN_PLACE = true>
+// swizzled rows, with NTH threads (ltid < NTH) sharing barrier bar_id (the
+// prefill's W and U' operands).  beta and gam are 16-byte aligned.  tb / tbg
+// overlap AT, so every thread reads its values before a barrier and writes
+// after it.
+template <int NTH>
 __device__ __forceinline__ void write_scaled_t(const float* AT, const float* beta, const float* gam,
-                                               uint8_t* tb, uint8_t* tbg, int ltid, uint32_t bar_id,
-                                               const float* rowe = nullptr) {
+                                               uint8_t* tb, uint8_t* tbg, int ltid, uint32_t bar_id) {
     constexpr int PER = C * C / NTH;   // values of one row per thread
     constexpr int TPR = C / PER;       // threads per row
     static_assert(PER % 8 == 0 && TPR * PER == C, "whole 16-byte chunks per thread");
@@ -207,7 +203,6 @@ __device__ __forceinline__ void write_scaled_t(const float* AT, const float* bet
     // the fp32 row loads (stride LDT) and the swizzled bf16 row stores are both
     // free of bank conflicts, and a warp reads one set of gate factors
     const int j = ltid % C, part = ltid / C;
-    const float ej = rowe ? rowe[j] : 1.0f;
     float vb[PER], vbg[PER];
 #pragma unroll
     for (int q = 0; q < PER; q += 4) {
@@ -221,12 +216,12 @@ __device__ __forceinline__ void write_scaled_t(const float* AT, const float* bet
         const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const float x = tv[e] * bv[e] * ej;
+            const float x = tv[e] * bv[e];
             vb[q + e] = x;
             vbg[q + e] = x * gv[e];
         }
     }
-    if (IN_PLACE) named_sync(bar_id, NTH);
+    named_sync(bar_id, NTH);
 #pragma unroll
     for (int ch = 0; ch < PER / 8; ++ch) {
         const int chunk = part * (PER / 8) + ch;
@@ -250,51 +245,24 @@ __device__ __forceinline__ void write_scaled_t(const float* AT, const float* bet
 
 constexpr int NT = 256;      // threads per CTA
 
-// ---- shared memory map (byte offsets from a 1 KB aligned base) ----
-// Two tile slots (chunk c in slot c % 2, the next chunk prefetched by TMA),
-// made of 8 KB boxes of 64 rows x 64 columns:
-//   replay : [K0 | K1 | V0 | V1]            (32 KB)
-//   prefill: [K0 | Q0 | K1 | Q1 | V0 | V1]  (48 KB; K block stride 16 KB so
-//            that [K; Q] is one 128-row operand)
-// PREP is reused within a chunk, in this order:
-//   A -> T in place (fp32 64 x LDT) and the product scratch,
-//   T diag(beta), T diag(beta gamma) (bf16 [j][j'], 8 KB each; the replay
-//   keeps them past the end of T, 33 KB of PREP, the prefill over T, 32 KB),
-//   BU = -sigma W (fp32, K-major [j][dk], four 8 KB key blocks).
-// Prefill adds UB (the bf16 output stage [i][dv]), MB (bf16 masked decayed
-// Q K^T [i][j]) and BQ (fp32 sigma diag(gamma) Q, K-major [i][dk], four 8 KB
-// blocks).  Both kernels keep the bf16 U tiles the state update (and the
-// prefill's output product) read in TMEM, not in the tile slot.
-template <bool REPLAY>
-struct Layout {
-    static constexpr uint32_t TILE = REPLAY ? 32768u : 49152u;
-    static constexpr uint32_t OFF_TILE = 0;
-    static constexpr uint32_t OFF_PREP = 2 * TILE;
-    static constexpr uint32_t OFF_AT = OFF_PREP;
-    static constexpr uint32_t OFF_X = OFF_PREP + 17408;
-    static constexpr uint32_t OFF_TB = REPLAY ? OFF_PREP + 17408 : OFF_PREP;
-    static constexpr uint32_t OFF_TBG = OFF_TB + 8192;
-    static constexpr uint32_t OFF_BU = OFF_PREP;
-    static constexpr uint32_t OFF_UB = OFF_PREP + 32768;
-    static constexpr uint32_t OFF_MB = OFF_UB + 16384;
-    static constexpr uint32_t OFF_BQ = OFF_MB + 8192;
-    static constexpr uint32_t BYTES = REPLAY ? OFF_TBG + 8192 : OFF_BQ + 32768;
-    // offsets inside a tile slot
-    static constexpr uint32_t K_BLK = REPLAY ? 8192u : 16384u;   // stride of the two K blocks
-    static constexpr uint32_t Q0 = 8192;                          // prefill only
-    static constexpr uint32_t V0 = REPLAY ? 16384u : 32768u;
+// ---- the prefill's tile slot (byte offsets inside a slot of 48 KB) ----
+// Two slots (chunk c in slot c % 2, the next chunk prefetched by TMA), made of
+// 8 KB boxes of 64 rows x 64 columns: [K0 | Q0 | K1 | Q1 | V0 | V1], the K block
+// stride 16 KB so that [K; Q] is one 128-row operand.  (The replay keeps its own
+// map in gdn_replay.cu.)
+struct TileLayout {
+    static constexpr uint32_t TILE = 49152;
+    static constexpr uint32_t K_BLK = 16384;   // stride of the two K blocks
+    static constexpr uint32_t Q0 = 8192;
+    static constexpr uint32_t V0 = 32768;
     static constexpr uint32_t V_LBO = 8192;
 };
-static_assert(Layout<true>::OFF_X + 4 * 16 * 24 * 4 <= Layout<true>::OFF_PREP + 32768, "prep scratch fits");
-static_assert(Layout<true>::OFF_TB >= Layout<true>::OFF_AT + C * LDT * 4 && Layout<true>::OFF_TB % 1024 == 0,
-              "replay T operands lie past T, 1 KB aligned");
-static_assert(2 * (Layout<true>::BYTES + 1024) <= 224 * 1024, "two replay CTAs per SM");
 
-// TMEM columns
+// TMEM columns (the state in both kernels; the rest is the prefill's map, the
+// replay keeps its own regions in gdn_replay.cu)
 constexpr uint32_t TM_S = 0;      // 128 columns: fp32 S^T / sigma, lane = value row, column = key
-constexpr uint32_t TM_U = 128;    // 64 columns: U'^T then U^T, lane = value row (replay: then U~^T in
-                                  // bf16, two chunk rows per column, in its first 32 columns)
-constexpr uint32_t TM_P = 192;    // 64 columns: K K^T ([K;Q] K^T for prefill), then W^T (lane = key)
+constexpr uint32_t TM_U = 128;    // 64 columns: U'^T then U^T, lane = value row
+constexpr uint32_t TM_P = 192;    // 64 columns: [K;Q] K^T, then W^T (lane = key)
 constexpr uint32_t TM_O = 256;    // 64 columns (prefill): O^T, lane = value row
 constexpr uint32_t TM_UB = 320;   // 32 columns (prefill): U^T in bf16, two chunk rows per column
 constexpr uint32_t TM_UT = 352;   // 32 columns (prefill): U~^T = U^T diag(e) / sigma in bf16
@@ -352,18 +320,17 @@ __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, const C
     return ok;
 }
 
-// TMA of one chunk's tiles: K and V, and Q when the chunk writes outputs.
+// TMA of one prefill chunk's tiles: K and V, and Q when the chunk writes outputs.
 // (Tile loads need no bounds check: TMA reads zeros past the map's extent.)
-template <bool REPLAY>
 __device__ __forceinline__ void issue_tiles(uint8_t* tile, uint64_t* bar, const CUtensorMap* mk, const CUtensorMap* mv,
                                             const CUtensorMap* mq, int h, int r0, bool with_q) {
-    using L = Layout<REPLAY>;
-    mbar_arrive_expect_tx(bar, (!REPLAY && with_q) ? L::TILE : 32768u);
+    using L = TileLayout;
+    mbar_arrive_expect_tx(bar, with_q ? L::TILE : 32768u);
     tma_load_3d(tile, mk, bar, 0, h, r0);
     tma_load_3d(tile + L::K_BLK, mk, bar, 64, h, r0);
     tma_load_3d(tile + L::V0, mv, bar, 0, h, r0);
     tma_load_3d(tile + L::V0 + L::V_LBO, mv, bar, 64, h, r0);
-    if (!REPLAY && with_q) {
+    if (with_q) {
         tma_load_3d(tile + L::Q0, mq, bar, 0, h, r0);
         tma_load_3d(tile + L::Q0 + 16384, mq, bar, 64, h, r0);
     }

@@ -56,7 +56,7 @@ using namespace chunk;
 // per SM.
 constexpr uint32_t BAR_CHAIN = 2;   // named barrier of warps 4-7
 struct PipeLayout {
-    static constexpr uint32_t TILE = Layout<false>::TILE;       // [K0 | Q0 | K1 | Q1 | V0 | V1]
+    static constexpr uint32_t TILE = TileLayout::TILE;       // [K0 | Q0 | K1 | Q1 | V0 | V1]
     static constexpr uint32_t OFF_TILE = 0;
     static constexpr uint32_t OFF_PREP = 2 * TILE;              // A / T, T diag(..), -sigma W
     static constexpr uint32_t OFF_AT = OFF_PREP;
@@ -75,7 +75,7 @@ __global__ void __launch_bounds__(NT, 1)
 prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_q,
                     const __grid_constant__ CUtensorMap map_k0, const __grid_constant__ CUtensorMap map_v0) {
-    using L = Layout<false>;
+    using L = TileLayout;
     using PL = PipeLayout;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -122,9 +122,9 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     auto issue_chunk = [&](int cc) {
         const ChunkSrc cs = chunk_src(cc);
         if (cs.out)
-            issue_tiles<false>(tile_of(cc), &bar_tile[cc & 1], &map_k, &map_v, &map_q, h, (int)cs.r0, true);
+            issue_tiles(tile_of(cc), &bar_tile[cc & 1], &map_k, &map_v, &map_q, h, (int)cs.r0, true);
         else
-            issue_tiles<false>(tile_of(cc), &bar_tile[cc & 1], &map_k0, &map_v0, &map_q, h, (int)cs.r0, false);
+            issue_tiles(tile_of(cc), &bar_tile[cc & 1], &map_k0, &map_v0, &map_q, h, (int)cs.r0, false);
     };
 
     if (tid == 0) {
