@@ -96,8 +96,9 @@ __device__ __forceinline__ void store16x16(float* D, int ldd, const float acc[2]
 // A (entries on and above the diagonal are ignored); on exit it holds
 // T = (I + A)^-1 on and below the diagonal 16 x 16 blocks (the upper
 // triangles of the diagonal blocks are written as zeros; the blocks above
-// them are left untouched and must be read as zero).  Xs is scratch of
-// 4 x 16 x 24 floats.
+// them are left untouched and must be read as zero).  Xs holds the merges'
+// four 16 x 16 scratch blocks: block s at Xs + (s / 2) XHI + (s % 2) XLO, row
+// stride LDX (see the placements below).
 //
 // Diagonal blocks: forward substitution on CUDA cores, warp w solves block w
 // with one lane per column.  Then recursive doubling with
@@ -107,8 +108,11 @@ __device__ __forceinline__ void store16x16(float* D, int ldd, const float acc[2]
 // block -T_22 X (warp (r, c) computes 16 x 16 block (r, c)).  ltid is the
 // thread's index among the 128 threads that run it; bar_id names the barrier
 // those threads share.
+template <int LDX, int XHI, int XLO>
 __device__ __forceinline__ void invert_unit_lower_inplace(float* AT, float* Xs, int ltid, uint32_t bar_id) {
     const int warp = ltid >> 5, lane = ltid & 31;
+    // scratch block s (16 x 16, row stride LDX) of the merges
+    auto xslot = [&](int s) { return Xs + (s >> 1) * XHI + (s & 1) * XLO; };
     {
         // every lane computes; lanes 16..31 repeat lanes 0..15 and do not store.
         // Row i of the block is read four entries per (broadcast) load.
@@ -147,14 +151,14 @@ __device__ __forceinline__ void invert_unit_lower_inplace(float* AT, float* Xs, 
     float pr0[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
     float xr1[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
     if (warp < 2) {
-        float* X = Xs + warp * (16 * 24);
+        float* X = xslot(warp);
         const int bo = warp ? 48 : 16, ao = warp ? 32 : 0;   // row block b, column block a
         float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         mma16x16_tf32(acc, AT + bo * LDT + ao, LDT, AT + ao * LDT + ao, LDT, 2, g, t);     // A_ba D_a
-        store16x16(X, 24, acc, 1.0f, g, t);
+        store16x16(X, LDX, acc, 1.0f, g, t);
         __syncwarp();
         float r[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        mma16x16_tf32(r, AT + bo * LDT + bo, LDT, X, 24, 2, g, t);                       // D_b (A_ba D_a)
+        mma16x16_tf32(r, AT + bo * LDT + bo, LDT, X, LDX, 2, g, t);                      // D_b (A_ba D_a)
         store16x16(AT + bo * LDT + ao, LDT, r, -1.0f, g, t);
     } else {
         const int r = warp;
@@ -166,26 +170,32 @@ __device__ __forceinline__ void invert_unit_lower_inplace(float* AT, float* Xs, 
     if (warp >= 2) {
         const int r = warp;
         mma16x16_tf32(pr0, AT + 16 * r * LDT + 16, LDT, AT + 16 * LDT, LDT, 2, g, t);      // + A_r1 T_10
-        store16x16(Xs + (2 * (r - 2)) * (16 * 24), 24, pr0, 1.0f, g, t);
-        store16x16(Xs + (2 * (r - 2) + 1) * (16 * 24), 24, xr1, 1.0f, g, t);
+        store16x16(xslot(2 * (r - 2)), LDX, pr0, 1.0f, g, t);
+        store16x16(xslot(2 * (r - 2) + 1), LDX, xr1, 1.0f, g, t);
     }
     named_sync(bar_id, 128);    // X blocks visible; every read of A_21 done
     // then T_21 = -T_22 X, warp w -> block (r, c) = (2 + w / 2, w % 2)
     {
         const int r = 2 + (warp >> 1), c = warp & 1;
         float rr[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        const float* X2c = Xs + c * (16 * 24);
+        const float* X2c = xslot(c);
         if (r == 2) {
-            mma16x16_tf32(rr, AT + 32 * LDT + 32, LDT, X2c, 24, 2, g, t);               // D_2 X_2c
+            mma16x16_tf32(rr, AT + 32 * LDT + 32, LDT, X2c, LDX, 2, g, t);              // D_2 X_2c
         } else {
-            const float* X3c = Xs + (2 + c) * (16 * 24);
-            mma16x16_tf32(rr, AT + 48 * LDT + 32, LDT, X2c, 24, 2, g, t);               // T_32 X_2c
-            mma16x16_tf32(rr, AT + 48 * LDT + 48, LDT, X3c, 24, 2, g, t);               // D_3 X_3c
+            const float* X3c = xslot(2 + c);
+            mma16x16_tf32(rr, AT + 48 * LDT + 32, LDT, X2c, LDX, 2, g, t);              // T_32 X_2c
+            mma16x16_tf32(rr, AT + 48 * LDT + 48, LDT, X3c, LDX, 2, g, t);              // D_3 X_3c
         }
         store16x16(AT + 16 * r * LDT + 16 * c, LDT, rr, -1.0f, g, t);
     }
     named_sync(bar_id, 128);
 }
+
+// The scratch placements of the inverse: a separate buffer of four 16 x 24
+// blocks, or the upper-right 32 x 32 quarter of AT itself (rows 0-31, columns
+// 32-63), which neither A nor T uses.
+#define GDN_INV_SCRATCH_SEPARATE 24, 2 * 16 * 24, 16 * 24
+#define GDN_INV_SCRATCH_IN_AT LDT, 16 * LDT, 16
 
 // From the inverse T (in place in AT, see above) write the bf16 operands
 // T diag(beta) -> tb and T diag(beta gamma) -> tbg, [j][j'] in 128-byte

@@ -1,7 +1,7 @@
 // gdn_chunk_tc.cu -- chunked gated-delta-rule prefill on tcgen05 tensor cores
 // (bf16 q/k/v, d_k = d_v = 128, fp32 state in tensor memory), the fused
 // replay + suffix, and the dispatch of the chunked path (the state-only
-// replay kernel is in gdn_replay.cu).
+// replay kernels are in gdn_replay.cu and gdn_replay_ws.cu).
 //
 // The recurrence (Gated DeltaNet, replayed by Tail-Replay: "Tail-Replay:
 // Escaping the Curse of Linear Attention in Prefix Caching for Hybrid LLMs",
@@ -33,6 +33,8 @@
 // read).  prefill_pipe_kernel runs the prefill with outputs and the fused
 // replay + suffix (the replay window's chunks first, without outputs):
 // 192 KB of shared memory, 512 TMEM columns, one CTA per SM.
+#include <atomic>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -306,7 +308,7 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                     }
                 }
                 named_sync(BAR_INV, 128);   // every row of A is in before the inverse reads it
-                invert_unit_lower_inplace(AT, Xs, tid, BAR_INV);
+                invert_unit_lower_inplace<GDN_INV_SCRATCH_SEPARATE>(AT, Xs, tid, BAR_INV);
             }
         } else if (c >= 0) {
             // ---- chain of chunk c: U~ (and U^T for the outputs), the state update and
@@ -607,12 +609,27 @@ bool make_tile_map(CUtensorMap* m, const void* base, int H, long long rows, long
 
 bool chunk_tc_supported(int dtype, int dk, int dv) { return dtype == 1 && dk == 128 && dv == 128; }
 
+// SMs of the current device, looked up once per device (0 if the query fails).
+static int device_sm_count() {
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    int v = cache[dev].load(std::memory_order_relaxed);
+    if (v > 0) return v;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev].store(v, std::memory_order_relaxed);
+    return v;
+}
+
 cudaError_t launch_chunk_tc(const CallArgs& a, cudaStream_t stream) {
     if (a.units == 0) return cudaSuccess;
     if (!chunk_tc_supported(a.dtype, a.dk, a.dv)) return cudaErrorInvalidValue;
-    // the state-only replay kernel unless outputs are asked for (a prefill, a fused replay
-    // + suffix, or a replay that also emits the window's outputs)
-    if (a.kind == kReplay && a.o_out == nullptr) return launch_replay_tc(a, stream);
+    // the state-only replay kernels unless outputs are asked for (a prefill, a fused replay
+    // + suffix, or a replay that also emits the window's outputs): with at most one unit
+    // per SM the warp-specialised kernel (one CTA per SM, the front of a unit's chunks
+    // decoupled from its state chain); otherwise the two-chunk kernel, two CTAs per SM
+    if (a.kind == kReplay && a.o_out == nullptr)
+        return a.units <= (long long)device_sm_count() ? launch_replay_ws(a, stream) : launch_replay_tc(a, stream);
     TcParams p;
     p.a = a;
     // a call with no rows to read (every window empty) still runs, to write the states;

@@ -161,6 +161,7 @@ cudaError_t launch_recurrent(const CallArgs& a, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_chunk_tc(const CallArgs& a, cudaStream_t stream);   // dispatches the replay below
 cudaError_t launch_replay_tc(const CallArgs& a, cudaStream_t stream);
+cudaError_t launch_replay_ws(const CallArgs& a, cudaStream_t stream);
 bool chunk_tc_supported(int dtype, int dk, int dv);
 
 }  // namespace gdn

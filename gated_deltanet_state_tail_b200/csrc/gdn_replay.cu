@@ -381,7 +381,7 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 // start after a barrier of warps 0-3 that follows this one)
                 if (wq >= 2) named_sync(BAR_A, 128);
                 // ---- T = (I + A)^-1 in place ----
-                invert_unit_lower_inplace(AT, Xs, tid, BAR_INV);
+                invert_unit_lower_inplace<GDN_INV_SCRATCH_SEPARATE>(AT, Xs, tid, BAR_INV);
             }
         } else {
             if (has_next && warp >= 6) {

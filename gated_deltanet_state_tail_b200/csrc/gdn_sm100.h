@@ -293,6 +293,22 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
     return d;
 }
 
+// Shared-memory matrix descriptor for an MN-major 32-bit (tf32) operand, the
+// one swizzle tcgen05 takes for it: 128-byte rows (32 elements along MN, one
+// row per K index), 32-byte chunks, the chunk index inside a row XORed with the
+// row index modulo 4 (a 512-byte atom of 4 rows).
+//   lbo = byte stride between 32-element MN blocks, sbo = byte stride between
+//   4-row groups along K.
+__device__ __forceinline__ uint64_t smem_desc_sw128_32b(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;   // descriptor version for tcgen05
+    d |= (uint64_t)1 << 61;   // swizzle mode: 128-byte rows with 32-byte atoms
+    return d;
+}
+
 // The descriptor of the same operand `byte_offset` bytes further on: the start
 // address field holds the address in 16-byte units (14 bits, all of shared
 // memory), so stepping through a tile adds to it without touching the rest.
