@@ -108,6 +108,63 @@ def chunk_algebra_state_grouped(k, v, alpha, beta):
     return sigma * St
 
 
+def chunk_algebra_state_prescaled(k, v, alpha, beta, zero_fold_is_none=False):
+    """The warp-specialised replay's form: the running sigma and the fold decision come
+    from the gates alone (before any state arithmetic), and both T operands carry the
+    scales, so U~ = E U / sigma' leaves the product ready for the state update:
+        U~ = (E T diag(beta) / sigma') V + (-(sigma / sigma') E T diag(beta gamma)) P,
+        S~ <- fold * S~ (when sigma gamma_C < 2^-40; then sigma' = 1),  S~ += K^T U~.
+    zero_fold_is_none plants a mistake (a fold factor of exactly 0 read as 'no fold')."""
+    n, dk = k.shape
+    dv = v.shape[1]
+    chunks = []
+    for c0 in range(0, n, C):
+        m = min(C, n - c0)
+        kc = np.zeros((C, dk))
+        vc = np.zeros((C, dv))
+        ac = np.ones(C)
+        bc = np.zeros(C)
+        kc[:m], vc[:m], ac[:m], bc[:m] = k[c0:c0 + m], v[c0:c0 + m], alpha[c0:c0 + m], beta[c0:c0 + m]
+        chunks.append((kc, vc, ac, bc))
+    # the gate side: per chunk (sigma, sigma', fold factor or None)
+    scales, sigma = [], 1.0
+    for kc, vc, ac, bc in chunks:
+        g2C = sum(max(np.log2(a), LOG2_FLOOR) if a > 0 else LOG2_FLOOR for a in ac)
+        snew, fold = sigma * np.exp2(g2C), None
+        if snew < RENORM_BELOW:
+            fold, snew = snew, 1.0
+        if zero_fold_is_none and fold == 0.0:
+            fold = None
+        scales.append((sigma, snew, fold))
+        sigma = snew
+    St = np.zeros((dk, dv))
+    P = None
+    for ci, (kc, vc, ac, bc) in enumerate(chunks):
+        lg = np.array([max(np.log2(a), LOG2_FLOOR) if a > 0 else LOG2_FLOOR for a in ac])
+        g2 = np.cumsum(lg)
+        gam = np.exp2(g2)
+        e = np.exp2(g2[-1] - g2)
+        if g2[-1] >= FAST_FLOOR:
+            decay = (bc * gam)[:, None] * np.exp2(-g2)[None, :]
+        else:
+            # only i > j is used (G is non-increasing there); the upper triangle is clamped
+            decay = bc[:, None] * np.exp2(np.minimum(g2[:, None] - g2[None, :], 0.0))
+        T = np.linalg.inv(np.eye(C) + np.tril(decay * (kc @ kc.T), -1))
+        sg, snew, fold = scales[ci]
+        tbv = T * bc[None, :]
+        tb = (e / snew)[:, None] * tbv                          # bf16 operand
+        tbg = (-(sg / snew) * e)[:, None] * tbv * gam[None, :]  # fp32 operand
+        Ut = tb @ vc
+        if P is not None:
+            Ut = Ut + tbg @ P
+        if fold is not None:
+            St = St * fold
+        St = St + kc.T @ Ut
+        if ci + 1 < len(chunks):
+            P = chunks[ci + 1][0] @ St
+    return (scales[-1][1] if scales else 1.0) * St
+
+
 def _inputs(n, dk, dv, case, seed):
     g = np.random.default_rng(seed)
     k = g.standard_normal((n, dk))
@@ -145,6 +202,32 @@ def test_grouped_state_term_matches_recurrence(case, n):
     S = chunk_algebra_state_grouped(k, v, a, b)
     scale = max(np.abs(S_ref).max(), 1e-300)
     assert np.abs(S - S_ref).max() / scale <= 1e-10
+
+
+@pytest.mark.parametrize("case", ["normal", "strong_decay", "zero_gates", "slow_decay"])
+@pytest.mark.parametrize("n", [1, 63, 64, 65, 200])
+def test_prescaled_operands_match_recurrence(case, n):
+    dk, dv = 16, 8
+    k, v, a, b = _inputs(n, dk, dv, case, seed=600 + n)
+    S_ref, _ = oracle.recurrence(k, v, a, b)
+    S = chunk_algebra_state_prescaled(k, v, a, b)
+    scale = max(np.abs(S_ref).max(), 1e-300)
+    assert np.abs(S - S_ref).max() / scale <= 1e-10
+
+
+def test_prescaled_fold_of_zero_is_still_a_fold():
+    """Planted mistake: a chunk of zero gates makes the fold factor exactly 0 (the kernel's
+    fp32 arithmetic already reaches 0 for chunks whose decay is below about 2^-150);
+    reading that as 'no fold' keeps the old state and fails against the recurrence."""
+    dk, dv, n = 16, 8, 200
+    k, v, a, b = _inputs(n, dk, dv, "normal", seed=11)
+    a[64:128] = 0.0
+    S_ref, _ = oracle.recurrence(k, v, a, b)
+    good = chunk_algebra_state_prescaled(k, v, a, b)
+    bad = chunk_algebra_state_prescaled(k, v, a, b, zero_fold_is_none=True)
+    scale = np.abs(S_ref).max()
+    assert np.abs(good - S_ref).max() / scale <= 1e-10
+    assert np.abs(bad - S_ref).max() / scale > 1e-3
 
 
 def test_grouped_state_term_needs_the_updated_state():
