@@ -34,18 +34,16 @@ using namespace sm100;
 using namespace chunk;
 
 // ---- shared memory (byte offsets from a 1 KB aligned base) ----
-// K of a chunk stays from its K K^T until its state update (two slots); V only
-// until its U' MMA (one slot).  K32 holds the next chunk's keys in fp32, the B
-// operand of P.  AT holds A, then T in place, then the fp32 operand
-// -sigma E T diag(beta gamma) in place; TB holds the bf16 E T diag(beta), and
-// the inverse's scratch before it.
+// K of a chunk stays from its K K^T until its state update (two slots; P of
+// the chunk reads them too); V only until its U' MMA (one slot).  AT holds A,
+// then T in place, then the fp32 operand -sigma E T diag(beta gamma) in place;
+// TB holds the bf16 E T diag(beta), and the inverse's scratch before it.
 struct ReplayLayout {
     static constexpr uint32_t BOX = 8192;                   // 64 rows x 64 bf16 (128-byte swizzle)
     static constexpr uint32_t K_SLOT = 2 * BOX;             // [dk 0-63 | dk 64-127]
     static constexpr uint32_t OFF_K = 0;                    // chunk c in slot c % 2
     static constexpr uint32_t OFF_V = OFF_K + 2 * K_SLOT;   // [dv 0-63 | dv 64-127]
-    static constexpr uint32_t OFF_K32 = OFF_V + 2 * BOX;    // fp32 [j][dk], four 8 KB blocks of 32 columns
-    static constexpr uint32_t OFF_AT = OFF_K32 + 32768;     // fp32 64 x LDT
+    static constexpr uint32_t OFF_AT = OFF_V + 2 * BOX;     // fp32 64 x LDT
     static constexpr uint32_t OFF_TB = OFF_AT + C * LDT * 4;
     static constexpr uint32_t OFF_X = OFF_TB;
     static constexpr uint32_t BYTES = OFF_TB + 8192;
@@ -55,15 +53,19 @@ static_assert(4 * 16 * 24 * 4 <= 8192, "inverse scratch fits the T operand's spa
 static_assert(2 * 8192 <= C * LDT * 4, "the fp32 T operand fits over T");
 static_assert(2 * (ReplayLayout::BYTES + 1024 + 4096) <= 228 * 1024, "two replay CTAs per SM");
 
-// TMEM columns: the state S~^T (lane = value row), then two 64-column regions
-// that alternate between chunks.  Region c % 2 holds K K^T of chunk c (M = 64),
-// then E U of chunk c (M = 128, lane = value row) and U~ = E U / sigma in bf16
-// over its first 32 columns; after chunk c's state update it holds P of chunk
-// c + 1 (P^T, lane = value row, fp32).
-constexpr uint32_t TM_R0 = 128;
+// TMEM columns: the state S~^T (fp32, lane = value row), then two 64-column
+// regions with fixed roles.  TM_X holds E U of chunk c (M = 128, lane = value
+// row), then U~ = E U / sigma in bf16 over its first 32 columns, and after
+// chunk c's state update a bf16 copy of S~^T (two keys per column), the A
+// operand of P.  TM_Y holds K K^T of chunk c + 1 (M = 64), then, once its A
+// epilogue has read it, P^T of chunk c + 1 = S~^T K^T (fp32, lane = value row),
+// the A operand of the P term.
+constexpr uint32_t TM_X = 128;
+constexpr uint32_t TM_Y = 192;
 
 constexpr uint32_t BAR_CHAIN = 2;   // named barrier of warps 4-7 (the state chain)
 constexpr uint32_t BAR_A = 4;       // warps 6-7 -> warps 2-3: their part of A is written
+constexpr uint32_t BAR_KK = 5;      // warps 0-3 -> warp 4: K K^T in TM_Y is read, P may overwrite it
 
 // From T (fp32, in place in AT) write the two T operands of a chunk, with
 // 256 threads (thread -> row j = tid % 64, columns 16 part .. 16 part + 15):
@@ -112,49 +114,21 @@ __device__ __forceinline__ void write_t_operands(float* AT, const Gates& G, floa
             make_float4(vg[4 * q], vg[4 * q + 1], vg[4 * q + 2], vg[4 * q + 3]);
 }
 
-// Keys of one chunk (bf16 K slot: two 8 KB boxes of 64 rows x 64 columns,
-// 128-byte swizzled) to fp32, K-major [j][dk] in four 8 KB blocks of 32 columns
-// (128-byte swizzled); rows j >= nrows are written as zeros.  128 threads:
-// thread ct -> row j = ct % 64, columns 64 h .. 64 h + 63 with h = ct / 64.
-__device__ __forceinline__ void convert_k_f32(const uint8_t* kslot, uint8_t* k32, int ct, int nrows) {
-    const int j = ct & (C - 1), h = ct >> 6;
-    const uint8_t* src = kslot + h * 8192 + j * 128;
-    const bool live = j < nrows;
-    // every load before the first store (the stores may alias the loads for the compiler)
-    uint4 raw[8];
-#pragma unroll
-    for (int ch = 0; ch < 8; ++ch)
-        raw[ch] = live ? *reinterpret_cast<const uint4*>(src + ((ch ^ (j & 7)) << 4)) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {   // columns 64 h + 8 ch .. + 7
-        const uint32_t wds[4] = {raw[ch].x, raw[ch].y, raw[ch].z, raw[ch].w};
-        float f[8];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            f[2 * e] = __uint_as_float(wds[e] << 16);
-            f[2 * e + 1] = __uint_as_float(wds[e] & 0xffff0000u);
-        }
-        uint8_t* blk = k32 + (2 * h + (ch >> 2)) * 8192 + j * 128;
-        *reinterpret_cast<float4*>(blk + (((2 * (ch & 3)) ^ (j & 7)) << 4)) = make_float4(f[0], f[1], f[2], f[3]);
-        *reinterpret_cast<float4*>(blk + (((2 * (ch & 3) + 1) ^ (j & 7)) << 4)) = make_float4(f[4], f[5], f[6], f[7]);
-    }
-}
-
 // ---------------------------------------------------------------------------
 // Tail replay, two chunks in flight inside the CTA.  Iteration c:
 //   phase X  warps 0-3: A of chunk c + 1 (columns 0-31; its K K^T was issued in the
 //                       last phase Y), then T = (I + A)^-1;
 //            warps 4-7: chunk c's chain: the U epilogue (U~ to bf16 in TMEM), the
-//                       state update, then P of chunk c + 1 and the TMA of chunk
-//                       c + 2's keys (warp 4); warps 6-7 first write the lower-right
-//                       quarter of A.
+//                       state update, a bf16 copy of the new state in TMEM, then P
+//                       of chunk c + 1 from that copy and the chunk's bf16 keys, and
+//                       the TMA of chunk c + 2's keys (warp 4); warps 6-7 first
+//                       write the lower-right quarter of A.
 //   phase Y  all warps: the T operands of chunk c + 1; then warp 2 issues the P term
 //                       and U' of chunk c + 1 into one accumulator, and K K^T of
-//                       chunk c + 2 once the P term has read its region; warps 4-7
-//                       turn chunk c + 2's keys into fp32 once P of chunk c + 1 is
-//                       done with them; warps 0-1 build the gates of chunk c + 2;
-//                       then the TMA of chunk c + 2's values.
-// 106 KB of shared memory, 256 TMEM columns and at most 128 registers per
+//                       chunk c + 2 once the P term has read its region; warps 0-1
+//                       build the gates of chunk c + 2; then the TMA of chunk
+//                       c + 2's values.
+// 74 KB of shared memory, 256 TMEM columns and at most 128 registers per
 // thread, so two CTAs share an SM.
 __global__ void __launch_bounds__(NT, 2)
 replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
@@ -208,7 +182,6 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     tc_fence_after();
     const uint32_t tbase = tmem_slot;
     const uint32_t tlane = tbase + ((uint32_t)(wq * 32) << 16);
-    auto region = [](int cc) -> uint32_t { return TM_R0 + (uint32_t)(cc & 1) * 64u; };
     auto kslot = [&](int cc) { return sm + RL::OFF_K + (cc & 1) * RL::K_SLOT; };
     auto issue_k = [&](int cc) {
         uint8_t* dst = kslot(cc);
@@ -231,7 +204,7 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     float* AT = reinterpret_cast<float*>(sm + RL::OFF_AT);
     float* Xs = reinterpret_cast<float*>(sm + RL::OFF_X);
     const uint32_t s_at = smem_u32(sm + RL::OFF_AT), s_tb = smem_u32(sm + RL::OFF_TB);
-    const uint32_t s_k32 = smem_u32(sm + RL::OFF_K32), s_v = smem_u32(sm + RL::OFF_V);
+    const uint32_t s_v = smem_u32(sm + RL::OFF_V);
     const size_t state_base = ((size_t)b * H + h) * D * D;
     {   // zero state: TMEM lane dv holds column dv of S / sigma (a row of S^T)
         float v[32];
@@ -245,7 +218,8 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
 
     const uint32_t id_kk = idesc_bf16(64, 64, false, false);   // K K^T; row r in lane 32 (r/16) + r%16
     const uint32_t id_w = idesc_bf16(128, 64, true, false);    // V^T (E T diag(beta))^T
-    const uint32_t id_t = idesc_tf32(128, 64, false, false);   // P^T = S~^T K^T; P^T (-sigma E T..)^T; A in TMEM
+    const uint32_t id_t = idesc_tf32(128, 64, false, false);   // P^T (-sigma E T diag(beta gamma))^T, A in TMEM
+    const uint32_t id_p = idesc_bf16(128, 64, false, false);   // P^T = S~^T K^T, A (bf16 S~^T) in TMEM
     const uint32_t id_s = idesc_bf16(128, 128, false, true);   // U~^T K, A (U~^T) in TMEM
     bool ok = true;
 
@@ -273,7 +247,7 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         const Gates& Gn = s_gates[cc & 1];
         const bool fast = Gn.g2[C - 1] >= kFastGateFloor;
         float v[16];
-        tmem_ld16x256b_x4(tlane + region(cc) + cb, v);
+        tmem_ld16x256b_x4(tlane + TM_Y + cb, v);
         const int i0 = 16 * wq + (lane >> 2), jb = cb + 2 * (lane & 3);
         const float* colf = fast ? Gn.binv : Gn.g2;   // column factor: 2^-G_j, or G_j
         float2 cf[4];
@@ -330,7 +304,7 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
             const uint64_t d = desc_advance(dk0, (kk >> 2) * RL::BOX + (kk & 3) * 32);
-            mma_bf16_ss(tbase + region(cc), d, d, id_kk, kk > 0);
+            mma_bf16_ss(tbase + TM_Y, d, d, id_kk, kk > 0);
         }
     };
 
@@ -376,6 +350,10 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 xok = kk_ready(cn) && xok;
                 epi1_half(cn, 0);
                 __syncwarp();
+                if (c >= 0) {   // K K^T of chunk cn is read: P of chunk cn may take TM_Y
+                    tc_fence_before();
+                    named_arrive(BAR_KK, 160);
+                }
                 // the diagonal solve of block wq reads rows 16 wq .. 16 wq + 15; for wq >= 2
                 // their columns 32-63 come from warps 6-7 (the later stages of the inverse
                 // start after a barrier of warps 0-3 that follows this one)
@@ -391,9 +369,9 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             }
             if (c >= 0) {
                 // ---- epilogue U of chunk c: U~ = E U / sigma_new, bf16 back into TMEM over the
-                //      first 32 columns of its region (half hf lands on columns 16 hf .. 16 hf +
-                //      15, which this thread has read already); the decay is folded into the
-                //      TMEM state when sigma gets small ----
+                //      first 32 columns of TM_X (half hf lands on columns 16 hf .. 16 hf + 15,
+                //      which this thread has read already); the decay is folded into the TMEM
+                //      state when sigma gets small ----
                 Gates& G = s_gates[c & 1];
                 float snew = sigma * G.gam[C - 1];
                 if (snew < kRenormBelow) {   // uniform
@@ -409,51 +387,70 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                     snew = 1.0f;
                 }
                 const float inv = 1.0f / snew;
-                const uint32_t ru = region(c);
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     float v[32];   // value dv = row, chunk rows [32 hf, 32 hf + 32)
-                    tmem_ld32(tlane + ru + 32 * hf, v);
+                    tmem_ld32(tlane + TM_X + 32 * hf, v);
                     tmem_wait_ld();
                     uint32_t pk[16];
 #pragma unroll
                     for (int q = 0; q < 16; ++q) pk[q] = pack_bf16(v[2 * q] * inv, v[2 * q + 1] * inv);
-                    tmem_st16(tlane + ru + 16 * hf, pk);
+                    tmem_st16(tlane + TM_X + 16 * hf, pk);
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 xok = named_sync_and(BAR_CHAIN, 128, xok);
-                // ---- S~^T += U~^T K of chunk c; then P^T of chunk cn = S~^T K_cn^T into the same
-                //      region (its keys are in fp32 since the last phase Y), and the keys of
-                //      chunk c + 2 into the slot chunk c frees ----
+                // ---- S~^T += U~^T K of chunk c ----
                 if (warp == 4) {
                     tc_fence_after();
-                    bool t = xok;
                     if (elect_one()) {
-                        if (t) {
+                        if (xok) {
                             const uint64_t db = smem_desc_sw128(smem_u32(kslot(c)), RL::BOX, 1024);
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk)
-                                mma_bf16_ts(tbase + TM_S, tbase + ru + kk * 8, desc_advance(db, kk * 2048), id_s, 1u);
+                                mma_bf16_ts(tbase + TM_S, tbase + TM_X + kk * 8, desc_advance(db, kk * 2048), id_s, 1u);
                         }
                         mma_commit(&bar_s);
-                        if (mbar_wait_bounded(&bar_s, c & 1, kWaitNs)) {
-                            tc_fence_after();
-                            if (t && has_next) {
-                                const uint64_t dk = smem_desc_sw128(s_k32, 16, 1024);
-#pragma unroll
-                                for (int kk = 0; kk < 16; ++kk)
-                                    mma_tf32_ts(tbase + ru, tbase + TM_S + kk * 8,
-                                                desc_advance(dk, (kk >> 2) * 8192 + (kk & 3) * 32), id_t, kk > 0);
-                            }
-                            if (has_next) mma_commit(&bar_p);
-                            if (t && c + 2 < nchunks) issue_k(c + 2);
-                        } else {
-                            report_timeout(a, 6);
-                            t = false;
-                        }
                     }
-                    xok = __all_sync(0xffffffffu, t) && xok;
+                    __syncwarp();
+                }
+                // ---- every chain thread waits for the update; then the bf16 copy of its
+                //      lane of S~^T into TM_X (U~ is read), two keys per column ----
+                bool t = xok && mbar_wait_bounded(&bar_s, c & 1, kWaitNs);
+                if (xok && !t) report_timeout(a, 6);
+                tc_fence_after();
+                if (t && has_next) {
+#pragma unroll
+                    for (int cb = 0; cb < 4; ++cb) {
+                        float sv[32];
+                        tmem_ld32(tlane + TM_S + cb * 32, sv);
+                        tmem_wait_ld();
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) pk[q] = pack_bf16(sv[2 * q], sv[2 * q + 1]);
+                        tmem_st16(tlane + TM_X + cb * 16, pk);
+                    }
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                xok = named_sync_and(BAR_CHAIN, 128, t) && xok;
+                // ---- P^T of chunk cn = S~^T K_cn^T into TM_Y once warps 0-3 have read K K^T
+                //      there, and the keys of chunk c + 2 into the slot chunk c frees ----
+                if (warp == 4) {
+                    if (has_next) named_sync(BAR_KK, 160);
+                    tc_fence_after();
+                    if (elect_one()) {
+                        if (xok && has_next) {
+                            const uint64_t dk = smem_desc_sw128(smem_u32(kslot(cn)), 16, 1024);
+#pragma unroll
+                            for (int kk = 0; kk < 8; ++kk)
+                                mma_bf16_ts(tbase + TM_Y, tbase + TM_X + kk * 8,
+                                            desc_advance(dk, (kk >> 2) * RL::BOX + (kk & 3) * 32), id_p, kk > 0);
+                        }
+                        if (has_next) mma_commit(&bar_p);
+                        if (xok && c + 2 < nchunks) issue_k(c + 2);
+                    }
+                    __syncwarp();
                 }
             }
         }
@@ -491,13 +488,12 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         tc_fence_before();
         tok = __syncthreads_and(tok) != 0;
         if (warp == 2) {
-            // ---- (E U)^T of chunk cn into its region: P^T (-sigma E T diag(beta gamma))^T, then
-            //      + V^T (E T diag(beta))^T; then K K^T of chunk cn + 1 into the region the P
-            //      term has just read ----
+            // ---- (E U)^T of chunk cn into TM_X: P^T (-sigma E T diag(beta gamma))^T, then
+            //      + V^T (E T diag(beta))^T; then K K^T of chunk cn + 1 into TM_Y once the P
+            //      term has read it ----
             tc_fence_after();
             bool t = tok;
             if (elect_one()) {
-                const uint32_t rn = region(cn);
                 if (t && ncn == C) {
                     t = mbar_wait_bounded(&bar_v, cn & 1, kWaitNs);
                     if (!t) report_timeout(a, 1);
@@ -512,7 +508,7 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                         const uint64_t d2 = smem_desc_sw128(s_at, 16, 1024);
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
-                            mma_tf32_ts(tbase + rn, tbase + region(c) + kk * 8,
+                            mma_tf32_ts(tbase + TM_X, tbase + TM_Y + kk * 8,
                                         desc_advance(d2, (kk >> 2) * 8192 + (kk & 3) * 32), id_t, kk > 0);
                         mma_commit(&bar_x);
                     }
@@ -520,7 +516,7 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                     const uint64_t dt = smem_desc_sw128(s_tb, 16, 1024);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ss(tbase + rn, desc_advance(dv, kk * 2048), desc_advance(dt, kk * 32), id_w,
+                        mma_bf16_ss(tbase + TM_X, desc_advance(dv, kk * 2048), desc_advance(dt, kk * 32), id_w,
                                     (cn > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(&bar_u);
@@ -529,7 +525,7 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                         t = mbar_wait_bounded(&bar_k[(cn + 1) & 1], ((cn + 1) >> 1) & 1, kWaitNs);
                         if (!t) report_timeout(a, 1);
                     }
-                    if (t && cn > 0) {   // the P term is done reading region (cn + 1) % 2
+                    if (t && cn > 0) {   // the P term is done reading TM_Y
                         t = mbar_wait_bounded(&bar_x, (cn - 1) & 1, kWaitNs);
                         if (!t) report_timeout(a, 5);
                     }
@@ -539,19 +535,6 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 }
             }
             tok = __all_sync(0xffffffffu, t) && tok;
-        } else if (warp >= 4) {
-            // ---- keys of chunk cn + 1 to fp32 (the B operand of its P), once P of chunk cn
-            //      is done reading them ----
-            if (has_nn) {
-                const int ct = tid - 128;
-                bool t = true;
-                if (cn > 0) t = mbar_wait_bounded(&bar_p, (cn - 1) & 1, kWaitNs);
-                if (t) t = mbar_wait_bounded(&bar_k[(cn + 1) & 1], ((cn + 1) >> 1) & 1, kWaitNs);
-                if (t) convert_k_f32(kslot(cn + 1), sm + RL::OFF_K32, ct, nnn);
-                else report_timeout(a, 7);
-                fence_proxy_async_smem();
-                tok = tok && t;
-            }
         } else if (tid < C && has_nn) {
             build_gates(s_gates[(cn + 1) & 1], al_nxt, be_nxt, tid, lane);
         }
