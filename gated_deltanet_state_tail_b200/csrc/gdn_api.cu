@@ -25,6 +25,7 @@ using gdn::WorkspaceHeader;
 struct gdn_plan {
     int kind;
     int batch, num_heads, dk, dv, dtype, kernel;
+    int replay_variant;       // gdn::ReplayVariant (chunked kernel, state-only replay)
     long long rs_qk, rs_v;    // row strides (elements) of q/k and of v
     int device;
     std::vector<Window> windows;   // replay: the tail windows; prefill and fused: the (suffix) sequences
@@ -52,7 +53,7 @@ gdn_status check_varlen_desc(const gdn_varlen_desc* d) {
     if (d->batch < 1 || d->num_heads < 1) return GDN_ERR_INVALID_ARG;
     if (d->dtype != GDN_F32 && d->dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
     if ((d->d_k != 64 && d->d_k != 128) || (d->d_v != 64 && d->d_v != 128)) return GDN_ERR_UNSUPPORTED;
-    if (d->kernel < GDN_KERNEL_AUTO || d->kernel > GDN_KERNEL_CHUNKED_TC) return GDN_ERR_INVALID_ARG;
+    if (d->kernel < GDN_KERNEL_AUTO || d->kernel > GDN_KERNEL_CHUNKED_TC_WARP_SPEC) return GDN_ERR_INVALID_ARG;
     // row stride: 0 = packed; otherwise every head of a row fits and rows start on 16 bytes
     if (d->row_stride_elems != 0) {
         const long long elem = d->dtype == GDN_BF16 ? 2 : 4;
@@ -90,7 +91,7 @@ bool take_injected_alloc_failure() {
 }
 
 int resolve_kernel(const gdn_varlen_desc* d) {
-    if (d->kernel != GDN_KERNEL_AUTO) return d->kernel;
+    if (d->kernel != GDN_KERNEL_AUTO) return gdn::kernel_family_of(d->kernel);
     return gdn::chunk_tc_supported(d->dtype, d->d_k, d->d_v) ? GDN_KERNEL_CHUNKED_TC
                                                               : GDN_KERNEL_RECURRENT;
 }
@@ -165,6 +166,7 @@ gdn_plan* new_plan(const gdn_varlen_desc* d, int kind) {
     p->dv = d->d_v;
     p->dtype = d->dtype;
     p->kernel = resolve_kernel(d);
+    p->replay_variant = gdn::replay_variant_of(d->kernel);
     p->rs_qk = gdn::row_stride_qk(d);
     p->rs_v = gdn::row_stride_v(d);
     p->dev_block = nullptr;
@@ -239,6 +241,7 @@ void fill_common(gdn_plan_t plan, CallArgs& a, void* workspace) {
     a.windows = plan->d_windows;
     a.unit_list = plan->d_units;
     a.ws = static_cast<WorkspaceHeader*>(workspace);
+    a.replay_variant = plan->replay_variant;
 }
 
 }  // namespace

@@ -108,8 +108,21 @@ __device__ __forceinline__ void store16x16(float* D, int ldd, const float acc[2]
 // block -T_22 X (warp (r, c) computes 16 x 16 block (r, c)).  ltid is the
 // thread's index among the 128 threads that run it; bar_id names the barrier
 // those threads share.
-template <int LDX, int XHI, int XLO>
-__device__ __forceinline__ void invert_unit_lower_inplace(float* AT, float* Xs, int ltid, uint32_t bar_id) {
+//
+// emit sees each 16 x 16 block of T once it is final: emit.diagonal(AT, q)
+// runs on 64 threads (q = 0..63, warps 0-1, while warps 2-3 merge) once the four
+// diagonal blocks are in AT (zeros above their diagonals); emit.block(r0, c0,
+// acc, scale, g, t) gets block (r0 / 16, c0 / 16) below the diagonal from the
+// registers of the warp that computed it, as scale times an m16n8 fragment pair
+// (T[r0 + g + 8 h][c0 + 8 nt + 2 t + e] = scale * acc[nt][2 h + e]).
+struct NoEmit {
+    __device__ __forceinline__ void diagonal(const float*, int) const {}
+    __device__ __forceinline__ void block(int, int, const float (&)[2][4], float, int, int) const {}
+};
+
+template <int LDX, int XHI, int XLO, class Emit = NoEmit>
+__device__ __forceinline__ void invert_unit_lower_inplace(float* AT, float* Xs, int ltid, uint32_t bar_id,
+                                                          const Emit& emit = Emit()) {
     const int warp = ltid >> 5, lane = ltid & 31;
     // scratch block s (16 x 16, row stride LDX) of the merges
     auto xslot = [&](int s) { return Xs + (s >> 1) * XHI + (s & 1) * XLO; };
@@ -160,6 +173,7 @@ __device__ __forceinline__ void invert_unit_lower_inplace(float* AT, float* Xs, 
         float r[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         mma16x16_tf32(r, AT + bo * LDT + bo, LDT, X, LDX, 2, g, t);                      // D_b (A_ba D_a)
         store16x16(AT + bo * LDT + ao, LDT, r, -1.0f, g, t);
+        emit.block(bo, ao, r, -1.0f, g, t);
     } else {
         const int r = warp;
         mma16x16_tf32(pr0, AT + 16 * r * LDT, LDT, AT, LDT, 2, g, t);                    // A_r0 D_0
@@ -172,6 +186,8 @@ __device__ __forceinline__ void invert_unit_lower_inplace(float* AT, float* Xs, 
         mma16x16_tf32(pr0, AT + 16 * r * LDT + 16, LDT, AT + 16 * LDT, LDT, 2, g, t);      // + A_r1 T_10
         store16x16(xslot(2 * (r - 2)), LDX, pr0, 1.0f, g, t);
         store16x16(xslot(2 * (r - 2) + 1), LDX, xr1, 1.0f, g, t);
+    } else {
+        emit.diagonal(AT, ltid);
     }
     named_sync(bar_id, 128);    // X blocks visible; every read of A_21 done
     // then T_21 = -T_22 X, warp w -> block (r, c) = (2 + w / 2, w % 2)
@@ -187,6 +203,7 @@ __device__ __forceinline__ void invert_unit_lower_inplace(float* AT, float* Xs, 
             mma16x16_tf32(rr, AT + 48 * LDT + 48, LDT, X3c, LDX, 2, g, t);              // D_3 X_3c
         }
         store16x16(AT + 16 * r * LDT + 16 * c, LDT, rr, -1.0f, g, t);
+        emit.block(16 * r, 16 * c, rr, -1.0f, g, t);
     }
     named_sync(bar_id, 128);
 }

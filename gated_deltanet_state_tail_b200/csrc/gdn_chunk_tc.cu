@@ -629,7 +629,10 @@ cudaError_t launch_chunk_tc(const CallArgs& a, cudaStream_t stream) {
     // per SM the warp-specialised kernel (one CTA per SM, the front of a unit's chunks
     // decoupled from its state chain); otherwise the two-chunk kernel, two CTAs per SM
     if (a.kind == kReplay && a.o_out == nullptr)
-        return a.units <= (long long)device_sm_count() ? launch_replay_ws(a, stream) : launch_replay_tc(a, stream);
+        return (a.replay_variant == kReplayWarpSpec ||
+                (a.replay_variant == kReplayBySize && a.units <= (long long)device_sm_count()))
+                   ? launch_replay_ws(a, stream)
+                   : launch_replay_tc(a, stream);
     TcParams p;
     p.a = a;
     // a call with no rows to read (every window empty) still runs, to write the states;

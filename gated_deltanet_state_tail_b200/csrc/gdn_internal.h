@@ -99,7 +99,26 @@ struct CallArgs {
     const float* alpha0;
     const float* beta0;
     float* state_mid;       // null, or [batch, H, dk, dv]: the state after the first segment
+    int replay_variant;     // ReplayVariant: which chunked kernel runs the state-only replay
 };
+
+// The chunked path's state-only replay kernel: chosen by launch size, or pinned by
+// the descriptor's kernel field (GDN_KERNEL_CHUNKED_TC_TWO_CTA / _WARP_SPEC).
+enum ReplayVariant { kReplayBySize = 0, kReplayTwoCta = 1, kReplayWarpSpec = 2 };
+
+inline int replay_variant_of(int kernel) {
+    return kernel == GDN_KERNEL_CHUNKED_TC_TWO_CTA    ? kReplayTwoCta
+           : kernel == GDN_KERNEL_CHUNKED_TC_WARP_SPEC ? kReplayWarpSpec
+                                                        : kReplayBySize;
+}
+
+// The kernel family a descriptor's kernel field names (the pinned replay variants
+// are the chunked kernel).
+inline int kernel_family_of(int kernel) {
+    return (kernel == GDN_KERNEL_CHUNKED_TC_TWO_CTA || kernel == GDN_KERNEL_CHUNKED_TC_WARP_SPEC)
+               ? GDN_KERNEL_CHUNKED_TC
+               : kernel;
+}
 
 // Device-side check of one unit's window against the caller's descriptor
 // arrays.  Returns true if the unit may run.

@@ -70,7 +70,7 @@ extern "C" gdn_status gdn_tail_replay_state_noalloc(const gdn_varlen_desc* cache
     const size_t need = sizeof(WorkspaceHeader) + sizeof(Window) * (size_t)batch +
                         sizeof(Unit) * (size_t)batch * (size_t)H;
     if (need > kScratchBytes) return GDN_ERR_UNSUPPORTED;   // beyond the fixed scratch
-    int kernel = cache->kernel;
+    int kernel = gdn::kernel_family_of(cache->kernel);
     const bool tc_ok = gdn::chunk_tc_supported(cache->dtype, cache->d_k, cache->d_v);
     if (kernel == GDN_KERNEL_AUTO) kernel = tc_ok ? GDN_KERNEL_CHUNKED_TC : GDN_KERNEL_RECURRENT;
     if (kernel == GDN_KERNEL_CHUNKED_TC && !tc_ok) return GDN_ERR_UNSUPPORTED;
@@ -152,6 +152,7 @@ extern "C" gdn_status gdn_tail_replay_state_noalloc(const gdn_varlen_desc* cache
         a.beta = beta;
         a.state_out = state_out;
         a.ws = reinterpret_cast<WorkspaceHeader*>(scratch);
+        a.replay_variant = gdn::replay_variant_of(cache->kernel);
         cudaError_t e = kernel == GDN_KERNEL_CHUNKED_TC ? gdn::launch_chunk_tc(a, st) : gdn::launch_recurrent(a, st);
         if (e != cudaSuccess) {
             cudaGetLastError();

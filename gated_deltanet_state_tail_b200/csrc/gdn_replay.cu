@@ -36,21 +36,23 @@ using namespace chunk;
 // ---- shared memory (byte offsets from a 1 KB aligned base) ----
 // K of a chunk stays from its K K^T until its state update (two slots; P of
 // the chunk reads them too); V only until its U' MMA (one slot).  AT holds A,
-// then T in place, then the fp32 operand -sigma E T diag(beta gamma) in place;
-// TB holds the bf16 E T diag(beta), and the inverse's scratch before it.
+// then T in place, with the inverse's scratch in its unused upper-right
+// quarter.  The inverse writes the T operands as their blocks become final: TB
+// the bf16 E T diag(beta) (the B operand of U'), TG the fp32 -sigma' E T
+// diag(beta gamma) (the B operand of the P term); the blocks above the
+// diagonal are zeroed once and never written.
 struct ReplayLayout {
     static constexpr uint32_t BOX = 8192;                   // 64 rows x 64 bf16 (128-byte swizzle)
     static constexpr uint32_t K_SLOT = 2 * BOX;             // [dk 0-63 | dk 64-127]
     static constexpr uint32_t OFF_K = 0;                    // chunk c in slot c % 2
     static constexpr uint32_t OFF_V = OFF_K + 2 * K_SLOT;   // [dv 0-63 | dv 64-127]
     static constexpr uint32_t OFF_AT = OFF_V + 2 * BOX;     // fp32 64 x LDT
-    static constexpr uint32_t OFF_TB = OFF_AT + C * LDT * 4;
-    static constexpr uint32_t OFF_X = OFF_TB;
-    static constexpr uint32_t BYTES = OFF_TB + 8192;
+    static constexpr uint32_t OFF_TB = OFF_AT + C * LDT * 4;   // bf16 [j][j'], 128-byte swizzled rows
+    static constexpr uint32_t OFF_TG = OFF_TB + 8192;          // fp32 [j][j'], two 8 KB blocks of 32 columns
+    static constexpr uint32_t BYTES = OFF_TG + 16384;
 };
-static_assert(ReplayLayout::OFF_TB % 1024 == 0 && ReplayLayout::OFF_AT % 1024 == 0, "operands on 1 KB");
-static_assert(4 * 16 * 24 * 4 <= 8192, "inverse scratch fits the T operand's space");
-static_assert(2 * 8192 <= C * LDT * 4, "the fp32 T operand fits over T");
+static_assert(ReplayLayout::OFF_TB % 1024 == 0 && ReplayLayout::OFF_TG == ReplayLayout::OFF_TB + 8192,
+              "operands on 1 KB, TG right after TB");
 static_assert(2 * (ReplayLayout::BYTES + 1024 + 4096) <= 228 * 1024, "two replay CTAs per SM");
 
 // TMEM columns: the state S~^T (fp32, lane = value row), then two 64-column
@@ -67,68 +69,88 @@ constexpr uint32_t BAR_CHAIN = 2;   // named barrier of warps 4-7 (the state cha
 constexpr uint32_t BAR_A = 4;       // warps 6-7 -> warps 2-3: their part of A is written
 constexpr uint32_t BAR_KK = 5;      // warps 0-3 -> warp 4: K K^T in TM_Y is read, P may overwrite it
 
-// From T (fp32, in place in AT) write the two T operands of a chunk, with
-// 256 threads (thread -> row j = tid % 64, columns 16 part .. 16 part + 15):
-//   tb : E T diag(beta), bf16 [j][j'] in 128-byte swizzled rows (U' = that V);
-//   AT : -sigma E T diag(beta gamma), fp32 K-major [j][j'] in two 8 KB blocks of
-//        32 columns (128-byte swizzled), over T itself: every thread reads its
-//        values, the block meets at a barrier, then writes.
-// Consecutive threads take consecutive rows, so the row reads (stride LDT) and
-// the swizzled stores are free of bank conflicts.
-__device__ __forceinline__ void write_t_operands(float* AT, const Gates& G, float sigma, uint8_t* tb, int tid) {
-    const int j = tid & (C - 1), part = tid >> 6;
-    const float ej = G.e[j];
-    const float nsj = -sigma * ej;
-    float vb[16], vg[16];
+// The inverse's emitter (see invert_unit_lower_inplace): each final block of T
+// goes from registers into the two T operands of the chunk,
+//   tb[j][j'] = e_j T[j][j'] beta_j'               (bf16, 128-byte swizzled rows),
+//   tg[j][j'] = -sigma' e_j T[j][j'] beta_j' gamma_j' (fp32, K-major, two 8 KB blocks
+//                                                   of 32 columns, 128-byte swizzled),
+// with e_j = gamma_C / gamma_j and sigma' the state's scale after the chunk before.
+struct TOperandEmit {
+    const Gates* G;
+    float nsig;    // -sigma'
+    uint8_t* tb;   // tg follows at tb + 8192
+    __device__ __forceinline__ static uint32_t off_b(int j, int jj) {
+        return (uint32_t)(j * 128 + (((jj >> 3) ^ (j & 7)) << 4) + (jj & 7) * 2);
+    }
+    __device__ __forceinline__ static uint32_t off_g(int j, int jj) {
+        return (uint32_t)(8192 + (jj >> 5) * 8192 + j * 128 + ((((jj & 31) >> 2) ^ (j & 7)) << 4) + (jj & 3) * 4);
+    }
+    // thread q: row j = 16 (q / 16) + q % 16 of its diagonal block, 16 columns
+    __device__ __forceinline__ void diagonal(const float* AT, int q) const {
+        const int o = (q >> 4) * 16, j = o + (q & 15);
+        const float ej = G->e[j], ejg = nsig * ej;
+        float v[16];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const int col = part * 16 + 4 * q;
-        float4 tt = make_float4(0.f, 0.f, 0.f, 0.f);
-        if ((col >> 4) <= (j >> 4)) tt = *reinterpret_cast<const float4*>(AT + j * LDT + col);
-        const float4 b4 = *reinterpret_cast<const float4*>(G.beta + col);
-        const float4 g4 = *reinterpret_cast<const float4*>(G.gam + col);
-        const float tv[4] = {tt.x, tt.y, tt.z, tt.w};
-        const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
-        const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
+        for (int k = 0; k < 4; ++k) {
+            const float4 t4 = *reinterpret_cast<const float4*>(AT + j * LDT + o + 4 * k);
+            const float4 b4 = *reinterpret_cast<const float4*>(G->beta + o + 4 * k);
+            const float4 g4 = *reinterpret_cast<const float4*>(G->gam + o + 4 * k);
+            v[4 * k + 0] = t4.x * b4.x;
+            v[4 * k + 1] = t4.y * b4.y;
+            v[4 * k + 2] = t4.z * b4.z;
+            v[4 * k + 3] = t4.w * b4.w;
+            const float4 w4 = make_float4(v[4 * k] * g4.x * ejg, v[4 * k + 1] * g4.y * ejg,
+                                          v[4 * k + 2] * g4.z * ejg, v[4 * k + 3] * g4.w * ejg);
+            *reinterpret_cast<float4*>(tb + off_g(j, o + 4 * k)) = w4;
+        }
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float tbv = tv[e] * bv[e];
-            vb[4 * q + e] = tbv * ej;
-            vg[4 * q + e] = tbv * gv[e] * nsj;
+        for (int hh = 0; hh < 2; ++hh) {
+            uint4 x;
+            x.x = pack_bf16(v[8 * hh + 0] * ej, v[8 * hh + 1] * ej);
+            x.y = pack_bf16(v[8 * hh + 2] * ej, v[8 * hh + 3] * ej);
+            x.z = pack_bf16(v[8 * hh + 4] * ej, v[8 * hh + 5] * ej);
+            x.w = pack_bf16(v[8 * hh + 6] * ej, v[8 * hh + 7] * ej);
+            st_shared_v4(tb, off_b(j, o + 8 * hh), x);
         }
     }
-    __syncthreads();   // every read of T is done before the fp32 operand overwrites it
+    __device__ __forceinline__ void block(int r0, int c0, const float (&acc)[2][4], float scale, int g,
+                                          int t) const {
 #pragma unroll
-    for (int ch = 0; ch < 2; ++ch) {
-        uint4 x;
-        x.x = pack_bf16(vb[ch * 8 + 0], vb[ch * 8 + 1]);
-        x.y = pack_bf16(vb[ch * 8 + 2], vb[ch * 8 + 3]);
-        x.z = pack_bf16(vb[ch * 8 + 4], vb[ch * 8 + 5]);
-        x.w = pack_bf16(vb[ch * 8 + 6], vb[ch * 8 + 7]);
-        st_shared_v4(tb, (uint32_t)(j * 128 + (((2 * part + ch) ^ (j & 7)) << 4)), x);
+        for (int nt = 0; nt < 2; ++nt) {
+            const int jj = c0 + 8 * nt + 2 * t;
+            const float2 b2 = *reinterpret_cast<const float2*>(G->beta + jj);
+            const float2 g2 = *reinterpret_cast<const float2*>(G->gam + jj);
+            const float bg0 = nsig * b2.x * g2.x, bg1 = nsig * b2.y * g2.y;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int j = r0 + g + 8 * hh;
+                const float ej = scale * G->e[j];
+                const float v0 = acc[nt][2 * hh] * ej, v1 = acc[nt][2 * hh + 1] * ej;
+                *reinterpret_cast<uint32_t*>(tb + off_b(j, jj)) = pack_bf16(v0 * b2.x, v1 * b2.y);
+                *reinterpret_cast<float2*>(tb + off_g(j, jj)) = make_float2(v0 * bg0, v1 * bg1);
+            }
+        }
     }
-    uint8_t* blk = reinterpret_cast<uint8_t*>(AT) + (part >> 1) * 8192 + j * 128;
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<float4*>(blk + (((4 * (part & 1) + q) ^ (j & 7)) << 4)) =
-            make_float4(vg[4 * q], vg[4 * q + 1], vg[4 * q + 2], vg[4 * q + 3]);
-}
+};
 
 // ---------------------------------------------------------------------------
 // Tail replay, two chunks in flight inside the CTA.  Iteration c:
 //   phase X  warps 0-3: A of chunk c + 1 (columns 0-31; its K K^T was issued in the
-//                       last phase Y), then T = (I + A)^-1;
-//            warps 4-7: chunk c's chain: the U epilogue (U~ to bf16 in TMEM), the
-//                       state update, a bf16 copy of the new state in TMEM, then P
-//                       of chunk c + 1 from that copy and the chunk's bf16 keys, and
-//                       the TMA of chunk c + 2's keys (warp 4); warps 6-7 first
-//                       write the lower-right quarter of A.
-//   phase Y  all warps: the T operands of chunk c + 1; then warp 2 issues the P term
-//                       and U' of chunk c + 1 into one accumulator, and K K^T of
-//                       chunk c + 2 once the P term has read its region; warps 0-1
-//                       build the gates of chunk c + 2; then the TMA of chunk
-//                       c + 2's values.
-// 74 KB of shared memory, 256 TMEM columns and at most 128 registers per
+//                       last phase Y), then T = (I + A)^-1, writing the chunk's two
+//                       T operands as each block of T is final;
+//            warps 4-7: chunk c's chain: wait for E U of chunk c (and load the values
+//                       of chunk c + 1 into the slot its U' freed), the U epilogue
+//                       (U~ to bf16 in TMEM), the state update, a bf16 copy of the
+//                       new state in TMEM, then P of chunk c + 1 from that copy and
+//                       the chunk's bf16 keys, and the TMA of chunk c + 2's keys
+//                       (warp 4); warps 6-7 first write the lower-right quarter of A.
+//   phase Y  warp 2 issues the P term of chunk c + 1, then K K^T of chunk c + 2 as
+//                       soon as the P term has read TM_Y, then U' of chunk c + 1
+//                       (K K^T is on the front's path, U' only on the chain's);
+//                       warps 0-1 build the gates of chunk c + 2.  Nobody waits for
+//                       U' here: the chain waits before its U epilogue, the front
+//                       before its inverse writes over the T operands U' reads.
+// 90 KB of shared memory, 256 TMEM columns and at most 128 registers per
 // thread, so two CTAs share an SM.
 __global__ void __launch_bounds__(NT, 2)
 replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
@@ -202,8 +224,11 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     }
 
     float* AT = reinterpret_cast<float*>(sm + RL::OFF_AT);
-    float* Xs = reinterpret_cast<float*>(sm + RL::OFF_X);
-    const uint32_t s_at = smem_u32(sm + RL::OFF_AT), s_tb = smem_u32(sm + RL::OFF_TB);
+    const uint32_t s_tg = smem_u32(sm + RL::OFF_TG), s_tb = smem_u32(sm + RL::OFF_TB);
+    // the T operands' blocks above the diagonal stay zero (made visible to the tensor
+    // core by the proxy fence before the first MMA that reads them)
+    for (int e = tid; e < (8192 + 16384) / 16; e += NT)
+        st_shared_v4(sm + RL::OFF_TB, (uint32_t)(e * 16), make_uint4(0, 0, 0, 0));
     const uint32_t s_v = smem_u32(sm + RL::OFF_V);
     const size_t state_base = ((size_t)b * H + h) * D * D;
     {   // zero state: TMEM lane dv holds column dv of S / sigma (a row of S^T)
@@ -358,8 +383,20 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 // their columns 32-63 come from warps 6-7 (the later stages of the inverse
                 // start after a barrier of warps 0-3 that follows this one)
                 if (wq >= 2) named_sync(BAR_A, 128);
-                // ---- T = (I + A)^-1 in place ----
-                invert_unit_lower_inplace<GDN_INV_SCRATCH_SEPARATE>(AT, Xs, tid, BAR_INV);
+                if (c >= 0) {   // U' of chunk c is done with the T operands' space
+                    const bool tu = mbar_wait_bounded(&bar_u, c & 1, kWaitNs);
+                    if (!tu) report_timeout(a, 4);
+                    xok = xok && tu;
+                }
+                // ---- T = (I + A)^-1 in place, and the T operands of chunk cn, scaled with
+                //      the state's scale after chunk c ----
+                float sig = sigma;
+                if (c >= 0) {
+                    const float sn = sigma * s_gates[c & 1].gam[C - 1];
+                    sig = sn < kRenormBelow ? 1.0f : sn;
+                }
+                const TOperandEmit em{&s_gates[cn & 1], -sig, sm + RL::OFF_TB};
+                invert_unit_lower_inplace<GDN_INV_SCRATCH_IN_AT>(AT, AT + 32, tid, BAR_INV, em);
             }
         } else {
             if (has_next && warp >= 6) {
@@ -372,6 +409,16 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 //      first 32 columns of TM_X (half hf lands on columns 16 hf .. 16 hf + 15,
                 //      which this thread has read already); the decay is folded into the TMEM
                 //      state when sigma gets small ----
+                {
+                    const bool tu = mbar_wait_bounded(&bar_u, c & 1, kWaitNs);
+                    if (!tu) report_timeout(a, 4);
+                    xok = xok && tu;
+                }
+                tc_fence_after();
+                if (warp == 4 && xok && has_next) {   // U' of chunk c is done with the value slot
+                    if (elect_one()) issue_v(cn);
+                    __syncwarp();
+                }
                 Gates& G = s_gates[c & 1];
                 float snew = sigma * G.gam[C - 1];
                 if (snew < kRenormBelow) {   // uniform
@@ -464,9 +511,8 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         tc_fence_after();
 
         // =============================== phase Y ===============================
-        // ---- T operands of chunk cn: E T diag(beta) (bf16) and -sigma E T diag(beta gamma)
-        //      (fp32, over T); partial tiles get their rows past the window zeroed first ----
-        const Gates& Gn = s_gates[cn & 1];
+        // ---- partial tiles get their rows past the window zeroed; the T operands of chunk
+        //      cn are written (phase X) ----
         const int ncn = nrows_of(cn);
         const bool has_nn = cn + 1 < nchunks;
         const int nnn = has_nn ? nrows_of(cn + 1) : C;
@@ -483,7 +529,6 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             else report_timeout(a, 1);
             tok = tok && t;
         }
-        write_t_operands(AT, Gn, sigma, sm + RL::OFF_TB, tid);
         fence_proxy_async_smem();
         tc_fence_before();
         tok = __syncthreads_and(tok) != 0;
@@ -503,15 +548,28 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                     if (!t) report_timeout(a, 3);
                 }
                 tc_fence_after();
-                if (t) {
-                    if (cn > 0) {
-                        const uint64_t d2 = smem_desc_sw128(s_at, 16, 1024);
+                if (t && cn > 0) {
+                    const uint64_t d2 = smem_desc_sw128(s_tg, 16, 1024);
 #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)
-                            mma_tf32_ts(tbase + TM_X, tbase + TM_Y + kk * 8,
-                                        desc_advance(d2, (kk >> 2) * 8192 + (kk & 3) * 32), id_t, kk > 0);
-                        mma_commit(&bar_x);
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_tf32_ts(tbase + TM_X, tbase + TM_Y + kk * 8,
+                                    desc_advance(d2, (kk >> 2) * 8192 + (kk & 3) * 32), id_t, kk > 0);
+                }
+                mma_commit(&bar_x);
+                if (has_nn) {
+                    if (t && nnn == C) {
+                        t = mbar_wait_bounded(&bar_k[(cn + 1) & 1], ((cn + 1) >> 1) & 1, kWaitNs);
+                        if (!t) report_timeout(a, 1);
                     }
+                    if (t) {   // the P term is done reading TM_Y
+                        t = mbar_wait_bounded(&bar_x, cn & 1, kWaitNs);
+                        if (!t) report_timeout(a, 5);
+                    }
+                    tc_fence_after();
+                    if (t) issue_kk(cn + 1);
+                    mma_commit(&bar_kk);
+                }
+                if (t) {
                     const uint64_t dv = smem_desc_sw128(s_v, RL::BOX, 1024);
                     const uint64_t dt = smem_desc_sw128(s_tb, 16, 1024);
 #pragma unroll
@@ -520,35 +578,13 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                                     (cn > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(&bar_u);
-                if (has_nn) {
-                    if (t && nnn == C) {
-                        t = mbar_wait_bounded(&bar_k[(cn + 1) & 1], ((cn + 1) >> 1) & 1, kWaitNs);
-                        if (!t) report_timeout(a, 1);
-                    }
-                    if (t && cn > 0) {   // the P term is done reading TM_Y
-                        t = mbar_wait_bounded(&bar_x, (cn - 1) & 1, kWaitNs);
-                        if (!t) report_timeout(a, 5);
-                    }
-                    tc_fence_after();
-                    if (t) issue_kk(cn + 1);
-                    mma_commit(&bar_kk);
-                }
             }
             tok = __all_sync(0xffffffffu, t) && tok;
         } else if (tid < C && has_nn) {
             build_gates(s_gates[(cn + 1) & 1], al_nxt, be_nxt, tid, lane);
         }
         if (has_nn) load_gates(cn + 2, al_nxt, be_nxt);
-        {
-            const bool okw = mbar_wait_bounded(&bar_u, cn & 1, kWaitNs);
-            ok = __syncthreads_and(okw && tok) != 0;
-            if (!ok && tid == 0) report_timeout(a, 4);
-        }
-        // U' of chunk cn is done with the value slot: the values of chunk cn + 1 go there
-        if (ok && warp == 2 && has_nn) {
-            if (elect_one()) issue_v(cn + 1);
-            __syncwarp();
-        }
+        ok = __syncthreads_and(tok) != 0;
     }
 
     // ---- final state: S[dk][dv] = sigma * TMEM[lane dv][dk] ----

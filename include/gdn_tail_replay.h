@@ -73,11 +73,18 @@ typedef enum gdn_status {
 typedef enum gdn_dtype { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
 
 /* Kernel selection.  AUTO picks the tensor-core chunked kernel for bf16 with
- * d_k = d_v = 128 and the exact fp32 CUDA-core recurrent kernel otherwise. */
+ * d_k = d_v = 128 and the exact fp32 CUDA-core recurrent kernel otherwise.
+ * The chunked path runs the state-only replay on one of two kernels: with at
+ * most one (sequence, head) unit per SM a warp-specialised kernel (one CTA per
+ * SM), otherwise a kernel with two CTAs per SM.  The last two values pin that
+ * choice whatever the launch size (for tests and measurements); every other
+ * entry point treats them as GDN_KERNEL_CHUNKED_TC. */
 typedef enum gdn_kernel {
     GDN_KERNEL_AUTO = 0,
-    GDN_KERNEL_RECURRENT = 1,   /* token-recurrent, fp32 CUDA cores, any supported shape */
-    GDN_KERNEL_CHUNKED_TC = 2   /* chunked WY/UT form on tcgen05 tensor cores (bf16, d = 128) */
+    GDN_KERNEL_RECURRENT = 1,              /* token-recurrent, fp32 CUDA cores, any supported shape */
+    GDN_KERNEL_CHUNKED_TC = 2,             /* chunked WY/UT form on tcgen05 tensor cores (bf16, d = 128) */
+    GDN_KERNEL_CHUNKED_TC_TWO_CTA = 3,     /* as 2, the replay always on the two-CTA-per-SM kernel */
+    GDN_KERNEL_CHUNKED_TC_WARP_SPEC = 4    /* as 2, the replay always on the warp-specialised kernel */
 } gdn_kernel;
 
 /* Varlen batch descriptor.  Sequence b occupies rows [seq_offsets[b],

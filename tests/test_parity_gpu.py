@@ -12,13 +12,19 @@ from helpers import TOL, oracle_view, per_request_rows_err, per_request_state_er
 
 pytestmark = pytest.mark.gpu
 
-KERNELS = {"recurrent": gdn.GDN_KERNEL_RECURRENT, "chunked": gdn.GDN_KERNEL_CHUNKED_TC}
+# "two_cta" and "warp_spec" run the chunked path with the state-only replay pinned to
+# one of its two kernels (by default the launch size picks: the warp-specialised
+# kernel for at most one unit per SM, which the small cases here are)
+KERNELS = {"recurrent": gdn.GDN_KERNEL_RECURRENT, "chunked": gdn.GDN_KERNEL_CHUNKED_TC,
+           "two_cta": gdn.GDN_KERNEL_CHUNKED_TC_TWO_CTA, "warp_spec": gdn.GDN_KERNEL_CHUNKED_TC_WARP_SPEC}
+CHUNKED = ("chunked", "two_cta", "warp_spec")
+REPLAY_KERNELS = ["recurrent", "two_cta", "warp_spec"]
 
 
 def kernel_or_skip(name, dtype, dk, dv):
-    if name == "chunked" and not (dtype == "bf16" and dk == 128 and dv == 128):
+    if name in CHUNKED and not (dtype == "bf16" and dk == 128 and dv == 128):
         pytest.skip("chunked kernel serves bf16 with d = 128")
-    if name == "chunked":
+    if name in CHUNKED:
         try:
             gdn.ReplayPlan(1, 128, 128, "bf16", [0, 64], [64], [64], KERNELS[name]).close()
         except gdn.GdnError as e:
@@ -88,7 +94,7 @@ def test_tiny_f32_replay_then_suffix(kname):
     assert per_request_state_err(st2.cpu().numpy(), ref_st2) <= TOL["f32"]
 
 
-@pytest.mark.parametrize("kname", ["recurrent", "chunked"])
+@pytest.mark.parametrize("kname", REPLAY_KERNELS)
 @pytest.mark.parametrize("dtype,dk,dv", [("bf16", 128, 128), ("f32", 128, 128), ("bf16", 64, 128),
                                          ("f32", 128, 64)])
 def test_varlen_replay_edges(kname, dtype, dk, dv):
@@ -125,7 +131,7 @@ def test_varlen_prefill(kname, dtype, dk, dv, with_state):
     assert per_request_state_err(st.cpu().numpy(), ref_st) <= TOL[dtype]
 
 
-@pytest.mark.parametrize("kname", ["recurrent", "chunked"])
+@pytest.mark.parametrize("kname", REPLAY_KERNELS)
 def test_window_indexing_bit_exact(kname):
     """Orthonormal cycling keys, alpha = beta = 1, v_t carrying its row index:
     the state records exactly which rows were replayed (bf16 digits are exact)."""
@@ -187,7 +193,7 @@ def test_call_validation_on_device():
     plan.close()
 
 
-@pytest.mark.parametrize("kname", ["recurrent", "chunked"])
+@pytest.mark.parametrize("kname", REPLAY_KERNELS)
 def test_rerun_bit_identical(kname):
     kernel = kernel_or_skip(kname, "bf16", 128, 128)
     t = make_cache([700], 4, 128, 128, "bf16", seed=15)
@@ -196,7 +202,7 @@ def test_rerun_bit_identical(kname):
     assert torch.equal(a, b)
 
 
-@pytest.mark.parametrize("kname", ["recurrent", "chunked"])
+@pytest.mark.parametrize("kname", REPLAY_KERNELS)
 def test_replay_then_suffix_equals_one_prefill(kname):
     """Replay(R) then prefill(suffix) matches one prefill from zero over tail ++ suffix."""
     kernel = kernel_or_skip(kname, "bf16", 128, 128)
@@ -211,7 +217,7 @@ def test_replay_then_suffix_equals_one_prefill(kname):
     assert rel_err(o1.float().cpu().numpy(), o2[R:].float().cpu().numpy()) <= TOL["bf16"]
 
 
-@pytest.mark.parametrize("kname", ["recurrent", "chunked"])
+@pytest.mark.parametrize("kname", REPLAY_KERNELS)
 def test_full_window_replay_equals_prefill_state(kname):
     """R = L: the replay kernel reproduces the state of a prefill from zero over the same
     L tokens (the prefill kernel), and both match the oracle."""
@@ -246,7 +252,7 @@ def _gates(case, rows, H, seed, last_window_row):
     return torch.tensor(a, dtype=torch.float32), torch.tensor(b, dtype=torch.float32)
 
 
-@pytest.mark.parametrize("kname", ["recurrent", "chunked"])
+@pytest.mark.parametrize("kname", REPLAY_KERNELS)
 @pytest.mark.parametrize("case", ["strong_decay", "zero_gates", "no_write", "identity", "mixed_heads"])
 def test_gate_extremes(kname, case):
     """Degenerate and extreme gates: the replay of a 500-token window and the suffix prefill
@@ -254,7 +260,7 @@ def test_gate_extremes(kname, case):
     exponent path and folds the running scale into the state every chunk; alpha = 0 at the
     window's last token leaves beta k v^T; beta = 0 leaves a zero replay and a decayed
     state_in; alpha = 1, beta = 0 carries state_in through unchanged."""
-    dtype, dk, dv = ("bf16", 128, 128) if kname == "chunked" else ("f32", 64, 128)
+    dtype, dk, dv = ("bf16", 128, 128) if kname in CHUNKED else ("f32", 64, 128)
     kernel = kernel_or_skip(kname, dtype, dk, dv)
     L, R, N, H = 700, 500, 300, 2   # window of 7 chunks and a ragged tail; suffix of 4 and a tail
     t = make_cache([L + N], H, dk, dv, dtype, seed=31)
@@ -306,12 +312,12 @@ def test_bounded_wait_timeout_is_reported_and_context_survives():
     assert per_request_state_err(st.cpu().numpy(), ref) <= TOL["bf16"]
 
 
-@pytest.mark.parametrize("kname", ["recurrent", "chunked"])
+@pytest.mark.parametrize("kname", REPLAY_KERNELS)
 def test_random_varlen_batches(kname):
     """Seeded random batches: request count, heads, cached length, match, budget and suffix
     length drawn per batch (R = 0, R > L, L = 0 and partial chunks all occur); replay states,
     suffix outputs and final states against the oracle."""
-    dtype, dk, dv = ("bf16", 128, 128) if kname == "chunked" else ("f32", 64, 128)
+    dtype, dk, dv = ("bf16", 128, 128) if kname in CHUNKED else ("f32", 64, 128)
     kernel = kernel_or_skip(kname, dtype, dk, dv)
     rng = np.random.default_rng(2024)
     for trial in range(12):
@@ -355,7 +361,7 @@ def test_longest_windows_against_oracle():
     assert per_request_state_err(st2.cpu().numpy(), ref_st2) <= TOL["bf16"]
 
 
-@pytest.mark.parametrize("kname", ["recurrent", "chunked"])
+@pytest.mark.parametrize("kname", REPLAY_KERNELS)
 def test_chunk_boundary_window_lengths(kname):
     """Windows of 1, 63, 64, 65, 127, 128, 129, 191, 192 and 193 rows in one launch: one to
     four chunks, with and without a partial last chunk (whose key and value rows past the
