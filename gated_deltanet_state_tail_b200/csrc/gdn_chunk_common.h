@@ -109,13 +109,17 @@ __device__ __forceinline__ void store16x16(float* D, int ldd, const float acc[2]
 // thread's index among the 128 threads that run it; bar_id names the barrier
 // those threads share.
 //
-// emit sees each 16 x 16 block of T once it is final: emit.diagonal(AT, q)
-// runs on 64 threads (q = 0..63, warps 0-1, while warps 2-3 merge) once the four
-// diagonal blocks are in AT (zeros above their diagonals); emit.block(r0, c0,
-// acc, scale, g, t) gets block (r0 / 16, c0 / 16) below the diagonal from the
-// registers of the warp that computed it, as scale times an m16n8 fragment pair
-// (T[r0 + g + 8 h][c0 + 8 nt + 2 t + e] = scale * acc[nt][2 h + e]).
+// emit sees each 16 x 16 block of T once it is final: emit.prepare() runs on
+// all 128 threads after the diagonal solves, before any other emit call (a
+// caller whose output buffers are still being read waits there);
+// emit.diagonal(AT, q) runs on 64 threads (q = 0..63, warps 0-1, while warps
+// 2-3 merge) once the four diagonal blocks are in AT (zeros above their
+// diagonals); emit.block(r0, c0, acc, scale, g, t) gets block (r0 / 16, c0 / 16)
+// below the diagonal from the registers of the warp that computed it, as scale
+// times an m16n8 fragment pair (T[r0 + g + 8 h][c0 + 8 nt + 2 t + e] = scale *
+// acc[nt][2 h + e]).
 struct NoEmit {
+    __device__ __forceinline__ void prepare() const {}
     __device__ __forceinline__ void diagonal(const float*, int) const {}
     __device__ __forceinline__ void block(int, int, const float (&)[2][4], float, int, int) const {}
 };
@@ -156,6 +160,7 @@ __device__ __forceinline__ void invert_unit_lower_inplace(float* AT, float* Xs, 
         }
     }
     named_sync(bar_id, 128);
+    emit.prepare();
     const int g = lane >> 2, t = lane & 3;
     // Level A, warps 0-1: 32 x 32 merges, warp 0 -> block (1, 0), warp 1 -> block (3, 2),
     // T_ba = -D_b (A_ba D_a).  Warps 2-3 meanwhile start block row r = warp of the

@@ -19,8 +19,9 @@
 // P needs only the chunk's keys and the state, so it is formed on the tensor
 // core as soon as the previous chunk's state update is done, while the
 // chunk's T is still being built; once T is ready, E U is two MMAs into one
-// accumulator (E U' from V, then the P term).  The serial part of a chunk is
-// therefore: T operands -> U MMAs -> U epilogue -> state update -> P.
+// accumulator (the P term, then E U' from V).  The serial part of a chunk is
+// therefore: E U MMAs -> U epilogue -> state update -> P, with the next
+// chunk's K K^T and A behind P and the chunk's inverse beside it.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -34,18 +35,18 @@ using namespace sm100;
 using namespace chunk;
 
 // ---- shared memory (byte offsets from a 1 KB aligned base) ----
-// K of a chunk stays from its K K^T until its state update (two slots; P of
-// the chunk reads them too); V only until its U' MMA (one slot).  AT holds A,
-// then T in place, with the inverse's scratch in its unused upper-right
-// quarter.  The inverse writes the T operands as their blocks become final: TB
-// the bf16 E T diag(beta) (the B operand of U'), TG the fp32 -sigma' E T
-// diag(beta gamma) (the B operand of the P term); the blocks above the
-// diagonal are zeroed once and never written.
+// K of a chunk stays from its K K^T (one iteration before the chunk's own)
+// until its state update (one iteration after): three slots.  V stays only
+// until its U' MMA (one slot).  AT holds A, then T in place, with the
+// inverse's scratch in its unused upper-right quarter.  The inverse writes the
+// T operands as their blocks become final: TB the bf16 E T diag(beta) (the B
+// operand of U'), TG the fp32 -sigma' E T diag(beta gamma) (the B operand of
+// the P term); the blocks above the diagonal are zeroed once and never written.
 struct ReplayLayout {
     static constexpr uint32_t BOX = 8192;                   // 64 rows x 64 bf16 (128-byte swizzle)
     static constexpr uint32_t K_SLOT = 2 * BOX;             // [dk 0-63 | dk 64-127]
-    static constexpr uint32_t OFF_K = 0;                    // chunk c in slot c % 2
-    static constexpr uint32_t OFF_V = OFF_K + 2 * K_SLOT;   // [dv 0-63 | dv 64-127]
+    static constexpr uint32_t OFF_K = 0;                    // chunk c in slot c % 3
+    static constexpr uint32_t OFF_V = OFF_K + 3 * K_SLOT;   // [dv 0-63 | dv 64-127]
     static constexpr uint32_t OFF_AT = OFF_V + 2 * BOX;     // fp32 64 x LDT
     static constexpr uint32_t OFF_TB = OFF_AT + C * LDT * 4;   // bf16 [j][j'], 128-byte swizzled rows
     static constexpr uint32_t OFF_TG = OFF_TB + 8192;          // fp32 [j][j'], two 8 KB blocks of 32 columns
@@ -53,21 +54,20 @@ struct ReplayLayout {
 };
 static_assert(ReplayLayout::OFF_TB % 1024 == 0 && ReplayLayout::OFF_TG == ReplayLayout::OFF_TB + 8192,
               "operands on 1 KB, TG right after TB");
-static_assert(2 * (ReplayLayout::BYTES + 1024 + 4096) <= 228 * 1024, "two replay CTAs per SM");
+static_assert(2 * (ReplayLayout::BYTES + 1024 + 1024 + 5120) <= 228 * 1024,
+              "two replay CTAs per SM (dynamic + alignment + reserved + static)");
 
 // TMEM columns: the state S~^T (fp32, lane = value row), then two 64-column
-// regions with fixed roles.  TM_X holds E U of chunk c (M = 128, lane = value
-// row), then U~ = E U / sigma in bf16 over its first 32 columns, and after
-// chunk c's state update a bf16 copy of S~^T (two keys per column), the A
-// operand of P.  TM_Y holds K K^T of chunk c + 1 (M = 64), then, once its A
-// epilogue has read it, P^T of chunk c + 1 = S~^T K^T (fp32, lane = value row),
-// the A operand of the P term.
+// regions with fixed roles.  TM_X holds E U of chunk c - 1 (M = 128, lane =
+// value row), then U~ = E U / sigma in bf16 over its first 32 columns, then
+// after the state update a bf16 copy of S~^T (two keys per column, the A
+// operand of P), then K K^T of chunk c + 1 (M = 64) until its A epilogue, then
+// E U of chunk c.  TM_Y holds P^T of chunk c = S~^T K^T (fp32, lane = value
+// row), the A operand of the P term.
 constexpr uint32_t TM_X = 128;
 constexpr uint32_t TM_Y = 192;
 
 constexpr uint32_t BAR_CHAIN = 2;   // named barrier of warps 4-7 (the state chain)
-constexpr uint32_t BAR_A = 4;       // warps 6-7 -> warps 2-3: their part of A is written
-constexpr uint32_t BAR_KK = 5;      // warps 0-3 -> warp 4: K K^T in TM_Y is read, P may overwrite it
 
 // The inverse's emitter (see invert_unit_lower_inplace): each final block of T
 // goes from registers into the two T operands of the chunk,
@@ -79,6 +79,16 @@ struct TOperandEmit {
     const Gates* G;
     float nsig;    // -sigma'
     uint8_t* tb;   // tg follows at tb + 8192
+    uint64_t* bar_rd;    // null, or the mbarrier of the MMAs still reading tb and tg
+    uint32_t parity;
+    const CallArgs* a;
+    int* abort_flag;
+    __device__ __forceinline__ void prepare() const {
+        if (bar_rd != nullptr && !mbar_wait_bounded(bar_rd, parity, kWaitNs)) {
+            report_timeout(*a, 8);
+            *abort_flag = 1;
+        }
+    }
     __device__ __forceinline__ static uint32_t off_b(int j, int jj) {
         return (uint32_t)(j * 128 + (((jj >> 3) ^ (j & 7)) << 4) + (jj & 7) * 2);
     }
@@ -134,23 +144,23 @@ struct TOperandEmit {
 };
 
 // ---------------------------------------------------------------------------
-// Tail replay, two chunks in flight inside the CTA.  Iteration c:
-//   phase X  warps 0-3: A of chunk c + 1 (columns 0-31; its K K^T was issued in the
-//                       last phase Y), then T = (I + A)^-1, writing the chunk's two
-//                       T operands as each block of T is final;
-//            warps 4-7: chunk c's chain: wait for E U of chunk c (and load the values
-//                       of chunk c + 1 into the slot its U' freed), the U epilogue
-//                       (U~ to bf16 in TMEM), the state update, a bf16 copy of the
-//                       new state in TMEM, then P of chunk c + 1 from that copy and
-//                       the chunk's bf16 keys, and the TMA of chunk c + 2's keys
-//                       (warp 4); warps 6-7 first write the lower-right quarter of A.
-//   phase Y  warp 2 issues the P term of chunk c + 1, then K K^T of chunk c + 2 as
-//                       soon as the P term has read TM_Y, then U' of chunk c + 1
-//                       (K K^T is on the front's path, U' only on the chain's);
-//                       warps 0-1 build the gates of chunk c + 2.  Nobody waits for
-//                       U' here: the chain waits before its U epilogue, the front
-//                       before its inverse writes over the T operands U' reads.
-// 90 KB of shared memory, 256 TMEM columns and at most 128 registers per
+// Tail replay.  Iteration c = 0 .. nchunks (the last one only ends the chain):
+//   phase X  warps 0-3 (front): T = (I + A)^-1 of chunk c (its A was written in
+//                       the last phase X), writing the chunk's T operands as each
+//                       block of T is final, once E U of chunk c - 1 has read the
+//                       previous ones;
+//            warps 4-7 (chain): wait for E U of chunk c - 1 and load chunk c's
+//                       values into the slot its U' freed; the U epilogue (U~ to
+//                       bf16 in TM_X), the state update with chunk c - 1's keys,
+//                       the keys of chunk c + 2 into the slot they free, a bf16
+//                       copy of the new state in TM_X, P of chunk c into TM_Y, and
+//                       once P has read the copy, K K^T of chunk c + 1 into TM_X;
+//            then all warps: A of chunk c + 1 from TM_X into AT.
+//   phase Y  warp 2: the P term of chunk c, then U', into TM_X (E U of chunk c);
+//                       warps 0-1 build the gates of chunk c + 2.  No barrier
+//                       follows: the next phase X waits on the mbarriers of what
+//                       it reads.
+// 105 KB of shared memory, 256 TMEM columns and at most 128 registers per
 // thread, so two CTAs share an SM.
 __global__ void __launch_bounds__(NT, 2)
 replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
@@ -158,12 +168,12 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     using RL = ReplayLayout;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    // bar_k: keys of chunk c (slot c % 2); bar_v: values; bar_kk: K K^T; bar_s: the
-    // state update; bar_p: P; bar_x: the P term of E U; bar_u: E U (the P term and U').
-    // One issuer each.
-    __shared__ uint64_t bar_k[2], bar_v, bar_kk, bar_s, bar_p, bar_x, bar_u;
+    // bar_k: keys of chunk c (slot c % 3); bar_v: values; bar_kk: K K^T; bar_s: the
+    // state update; bar_p: P; bar_u: E U (the P term and U').  One issuer each.
+    __shared__ uint64_t bar_k[3], bar_v, bar_kk, bar_s, bar_p, bar_u;
     __shared__ uint32_t tmem_slot;
-    __shared__ Gates s_gates[2];    // chunk c uses s_gates[c & 1]
+    __shared__ Gates s_gates[3];    // chunk c uses s_gates[c % 3]
+    __shared__ int s_abort;         // a wait outside the block-wide barriers gave up
 
     const CallArgs& a = p.a;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -183,13 +193,12 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         return;
 
     if (tid == 0) {
-        mbar_init(&bar_k[0], 1);
-        mbar_init(&bar_k[1], 1);
+        s_abort = 0;
+        for (int i = 0; i < 3; ++i) mbar_init(&bar_k[i], 1);
         mbar_init(&bar_v, 1);
         mbar_init(&bar_kk, 1);
         mbar_init(&bar_s, 1);
         mbar_init(&bar_p, 1);
-        mbar_init(&bar_x, 1);
         mbar_init(&bar_u, 1);
         mbar_fence_init();
         tma_prefetch_desc(&map_k);
@@ -199,18 +208,26 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         tmem_alloc(&tmem_slot, 256);
         tmem_relinquish();
     }
+    float* AT = reinterpret_cast<float*>(sm + RL::OFF_AT);
+    // the T operands' blocks above the diagonal stay zero (made visible to the tensor
+    // core by the proxy fence before the first MMA that reads them)
+    for (int e = tid; e < (8192 + 16384) / 16; e += NT)
+        st_shared_v4(sm + RL::OFF_TB, (uint32_t)(e * 16), make_uint4(0, 0, 0, 0));
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = tmem_slot;
     const uint32_t tlane = tbase + ((uint32_t)(wq * 32) << 16);
-    auto kslot = [&](int cc) { return sm + RL::OFF_K + (cc & 1) * RL::K_SLOT; };
+    auto kslot = [&](int cc) { return sm + RL::OFF_K + (cc % 3) * RL::K_SLOT; };
+    auto kbar = [&](int cc) { return &bar_k[cc % 3]; };
+    auto kpar = [](int cc) { return (uint32_t)((cc / 3) & 1); };
     auto issue_k = [&](int cc) {
         uint8_t* dst = kslot(cc);
         const int r0 = (int)(w.row0 + (long long)cc * C);
-        mbar_arrive_expect_tx(&bar_k[cc & 1], RL::K_SLOT);
-        tma_load_3d(dst, &map_k, &bar_k[cc & 1], 0, h, r0);
-        tma_load_3d(dst + RL::BOX, &map_k, &bar_k[cc & 1], 64, h, r0);
+        mbar_arrive_expect_tx(kbar(cc), RL::K_SLOT);
+        tma_load_3d(dst, &map_k, kbar(cc), 0, h, r0);
+        tma_load_3d(dst + RL::BOX, &map_k, kbar(cc), 64, h, r0);
     };
     auto issue_v = [&](int cc) {
         const int r0 = (int)(w.row0 + (long long)cc * C);
@@ -219,16 +236,11 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         tma_load_3d(sm + RL::OFF_V + RL::BOX, &map_v, &bar_v, 64, h, r0);
     };
     if (tid == 0) {
-        for (int cc = 0; cc < 2 && cc < nchunks; ++cc) issue_k(cc);
+        for (int cc = 0; cc < 3 && cc < nchunks; ++cc) issue_k(cc);
         if (nchunks > 0) issue_v(0);
     }
 
-    float* AT = reinterpret_cast<float*>(sm + RL::OFF_AT);
     const uint32_t s_tg = smem_u32(sm + RL::OFF_TG), s_tb = smem_u32(sm + RL::OFF_TB);
-    // the T operands' blocks above the diagonal stay zero (made visible to the tensor
-    // core by the proxy fence before the first MMA that reads them)
-    for (int e = tid; e < (8192 + 16384) / 16; e += NT)
-        st_shared_v4(sm + RL::OFF_TB, (uint32_t)(e * 16), make_uint4(0, 0, 0, 0));
     const uint32_t s_v = smem_u32(sm + RL::OFF_V);
     const size_t state_base = ((size_t)b * H + h) * D * D;
     {   // zero state: TMEM lane dv holds column dv of S / sigma (a row of S^T)
@@ -239,7 +251,7 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         tmem_st32(tlane + TM_S + (2 * wh + 1) * 32, v);
         tmem_wait_st();
     }
-    float sigma = 1.0f;
+    float sigma = 1.0f;   // the scale of the state entering chunk c - 1 (1 up to chunk 0)
 
     const uint32_t id_kk = idesc_bf16(64, 64, false, false);   // K K^T; row r in lane 32 (r/16) + r%16
     const uint32_t id_w = idesc_bf16(128, 64, true, false);    // V^T (E T diag(beta))^T
@@ -261,7 +273,7 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     };
     auto nrows_of = [&](int cc) { return min(C, w.len - cc * C); };
 
-    // Epilogue 1 of chunk cc over the 32 columns [cb, cb + 32) of its K K^T:
+    // Epilogue 1 of chunk cc over the 32 columns [cb, cb + 32) of its K K^T (in TM_X):
     // A = strict_tril(beta_i (gamma_i / gamma_j) K K^T), fp32 into AT.  The M = 64
     // accumulator keeps rows 16 wq .. 16 wq + 15 in the quarter's first 16 lanes; this
     // thread takes rows i0 = 16 wq + lane / 4 and i0 + 8, columns cb + 8 k + 2 (lane % 4)
@@ -269,10 +281,10 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     // store through AT may alias them for the compiler, which would then serialise each
     // load behind the previous store), and while the TMEM load is in flight.
     auto epi1_half = [&](int cc, int cb) {
-        const Gates& Gn = s_gates[cc & 1];
+        const Gates& Gn = s_gates[cc % 3];
         const bool fast = Gn.g2[C - 1] >= kFastGateFloor;
         float v[16];
-        tmem_ld16x256b_x4(tlane + TM_Y + cb, v);
+        tmem_ld16x256b_x4(tlane + TM_X + cb, v);
         const int i0 = 16 * wq + (lane >> 2), jb = cb + 2 * (lane & 3);
         const float* colf = fast ? Gn.binv : Gn.g2;   // column factor: 2^-G_j, or G_j
         float2 cf[4];
@@ -307,19 +319,22 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             }
         }
     };
-    // wait for K K^T of chunk cc (every thread that reads it); false if the wait ran out
-    auto kk_ready = [&](int cc) -> bool {
+    // A of chunk cc from its K K^T: warps 0-3 take columns 0-31 of their quarter's rows,
+    // warps 6-7 columns 32-63 of rows 32-63 (rows 0-31 have no entries there); false if
+    // the wait for K K^T ran out
+    auto a_epilogue = [&](int cc) -> bool {
+        if (warp >= 4 && warp < 6) return true;
         const bool t = mbar_wait_bounded(&bar_kk, cc & 1, kWaitNs);
         if (!t) report_timeout(a, 2);
         tc_fence_after();
+        epi1_half(cc, warp < 4 ? 0 : 32);
         return t;
     };
-
-    // zero the rows past the window of a partial chunk's key (bx = 0) or value slot;
-    // every thread takes part, after the tile has arrived
-    auto zero_tail_rows = [&](uint8_t* slot, int nrows) {
+    // zero the rows past the window of a partial chunk's key (bx = 0) or value slot,
+    // with nth threads (index ct), after the tile has arrived
+    auto zero_tail_rows = [&](uint8_t* slot, int nrows, int ct, int nth) {
         const int nz = C - nrows;
-        for (int e = tid; e < 2 * nz * 8; e += NT) {
+        for (int e = ct; e < 2 * nz * 8; e += nth) {
             const int bx = e / (nz * 8), rr = nrows + (e / 8) % nz, ch = e % 8;
             st_shared_v4(slot + bx * RL::BOX, (uint32_t)(rr * 128 + ch * 16), make_uint4(0, 0, 0, 0));
         }
@@ -329,29 +344,31 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
             const uint64_t d = desc_advance(dk0, (kk >> 2) * RL::BOX + (kk & 3) * 32);
-            mma_bf16_ss(tbase + TM_Y, d, d, id_kk, kk > 0);
+            mma_bf16_ss(tbase + TM_X, d, d, id_kk, kk > 0);
         }
     };
 
-    // ---- prologue: gates of chunk 0 (built) and 1 (registers), K K^T of chunk 0 ----
+    // ---- prologue: gates of chunks 0 and 1, A of chunk 0 ----
     float al_nxt, be_nxt;
     load_gates(0, al_nxt, be_nxt);
     if (tid < C) build_gates(s_gates[0], al_nxt, be_nxt, tid, lane);
     load_gates(1, al_nxt, be_nxt);
+    if (tid < C) build_gates(s_gates[1], al_nxt, be_nxt, tid, lane);
+    load_gates(2, al_nxt, be_nxt);
     if (nchunks > 0) {
         bool t = true;
         if (nrows_of(0) < C) {
-            t = mbar_wait_bounded(&bar_k[0], 0, kWaitNs);
-            if (t) zero_tail_rows(kslot(0), nrows_of(0));
+            t = mbar_wait_bounded(kbar(0), 0, kWaitNs);
+            if (t) zero_tail_rows(kslot(0), nrows_of(0), tid, NT);
             else report_timeout(a, 1);
             fence_proxy_async_smem();
         }
         ok = __syncthreads_and(t) != 0;
         if (ok && warp == 0) {
-            bool tw = true;
             if (elect_one()) {
+                bool tw = true;
                 if (nrows_of(0) == C) {
-                    tw = mbar_wait_bounded(&bar_k[0], 0, kWaitNs);
+                    tw = mbar_wait_bounded(kbar(0), 0, kWaitNs);
                     if (!tw) report_timeout(a, 1);
                 }
                 tc_fence_after();
@@ -360,68 +377,51 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             }
             __syncwarp();
         }
+        if (ok) ok = a_epilogue(0);
     }
-    __syncthreads();
+    tc_fence_before();
+    ok = __syncthreads_and(ok) != 0;
+    tc_fence_after();
 
-    for (int c = -1; c < nchunks && ok; ++c) {
-        const int cn = c + 1;
-        const bool has_next = cn < nchunks;
+    for (int c = 0; c <= nchunks && ok; ++c) {
+        const bool has_cur = c < nchunks, has_prev = c >= 1, has_nx = c + 1 < nchunks;
+        // the scale of the state entering chunk c, after chunk c - 1's update (the same
+        // fp32 arithmetic in every thread); below 2^-40 it is folded into the state
+        float snew = 1.0f, sig_c = sigma;
+        bool fold = false;
+        if (has_prev) {
+            snew = sigma * s_gates[(c - 1) % 3].gam[C - 1];
+            fold = snew < kRenormBelow;
+            sig_c = fold ? 1.0f : snew;
+        }
         bool xok = true;
         // =============================== phase X ===============================
         if (warp < 4) {
-            if (has_next) {
-                // ---- epilogue 1 of chunk cn, columns 0-31 (warps 6-7 take rows 32-63 x
-                //      columns 32-63; rows 0-31 have no entries there) ----
-                xok = kk_ready(cn) && xok;
-                epi1_half(cn, 0);
-                __syncwarp();
-                if (c >= 0) {   // K K^T of chunk cn is read: P of chunk cn may take TM_Y
-                    tc_fence_before();
-                    named_arrive(BAR_KK, 160);
-                }
-                // the diagonal solve of block wq reads rows 16 wq .. 16 wq + 15; for wq >= 2
-                // their columns 32-63 come from warps 6-7 (the later stages of the inverse
-                // start after a barrier of warps 0-3 that follows this one)
-                if (wq >= 2) named_sync(BAR_A, 128);
-                if (c >= 0) {   // U' of chunk c is done with the T operands' space
-                    const bool tu = mbar_wait_bounded(&bar_u, c & 1, kWaitNs);
-                    if (!tu) report_timeout(a, 4);
-                    xok = xok && tu;
-                }
-                // ---- T = (I + A)^-1 in place, and the T operands of chunk cn, scaled with
-                //      the state's scale after chunk c ----
-                float sig = sigma;
-                if (c >= 0) {
-                    const float sn = sigma * s_gates[c & 1].gam[C - 1];
-                    sig = sn < kRenormBelow ? 1.0f : sn;
-                }
-                const TOperandEmit em{&s_gates[cn & 1], -sig, sm + RL::OFF_TB};
+            if (has_cur) {
+                // ---- T = (I + A)^-1 of chunk c in place, writing its T operands once the P
+                //      term and U' of chunk c - 1 have read the previous ones ----
+                const TOperandEmit em{&s_gates[c % 3], -sig_c, sm + RL::OFF_TB, has_prev ? &bar_u : nullptr,
+                                      (uint32_t)((c - 1) & 1), &a, &s_abort};
                 invert_unit_lower_inplace<GDN_INV_SCRATCH_IN_AT>(AT, AT + 32, tid, BAR_INV, em);
+                fence_proxy_async_smem();   // the T operands, for phase Y's MMAs
             }
         } else {
-            if (has_next && warp >= 6) {
-                xok = kk_ready(cn) && xok;
-                epi1_half(cn, 32);
-                named_arrive(BAR_A, 128);
-            }
-            if (c >= 0) {
-                // ---- epilogue U of chunk c: U~ = E U / sigma_new, bf16 back into TMEM over the
-                //      first 32 columns of TM_X (half hf lands on columns 16 hf .. 16 hf + 15,
-                //      which this thread has read already); the decay is folded into the TMEM
-                //      state when sigma gets small ----
-                {
-                    const bool tu = mbar_wait_bounded(&bar_u, c & 1, kWaitNs);
-                    if (!tu) report_timeout(a, 4);
-                    xok = xok && tu;
-                }
+            const int ct = tid - 128;
+            if (has_prev) {
+                // ---- E U of chunk c - 1 is done: its U' has read the value slot ----
+                bool t = mbar_wait_bounded(&bar_u, (c - 1) & 1, kWaitNs);
+                if (!t) report_timeout(a, 4);
+                xok = xok && t;
                 tc_fence_after();
-                if (warp == 4 && xok && has_next) {   // U' of chunk c is done with the value slot
-                    if (elect_one()) issue_v(cn);
+                if (warp == 4 && xok && has_cur) {
+                    if (elect_one()) issue_v(c);
                     __syncwarp();
                 }
-                Gates& G = s_gates[c & 1];
-                float snew = sigma * G.gam[C - 1];
-                if (snew < kRenormBelow) {   // uniform
+                // ---- epilogue U of chunk c - 1: U~ = E U / sigma_new, bf16 back into TMEM over
+                //      the first 32 columns of TM_X (half hf lands on columns 16 hf .. 16 hf + 15,
+                //      which this thread has read already); the decay is folded into the TMEM
+                //      state when sigma gets small ----
+                if (fold) {   // uniform
 #pragma unroll
                     for (int cb = 0; cb < 4; ++cb) {
                         float sv[32];
@@ -431,9 +431,8 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                         for (int q = 0; q < 32; ++q) sv[q] *= snew;
                         tmem_st32(tlane + TM_S + cb * 32, sv);
                     }
-                    snew = 1.0f;
                 }
-                const float inv = 1.0f / snew;
+                const float inv = fold ? 1.0f : 1.0f / snew;
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     float v[32];   // value dv = row, chunk rows [32 hf, 32 hf + 32)
@@ -447,12 +446,12 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 tmem_wait_st();
                 tc_fence_before();
                 xok = named_sync_and(BAR_CHAIN, 128, xok);
-                // ---- S~^T += U~^T K of chunk c ----
+                // ---- S~^T += U~^T K of chunk c - 1 ----
                 if (warp == 4) {
                     tc_fence_after();
                     if (elect_one()) {
                         if (xok) {
-                            const uint64_t db = smem_desc_sw128(smem_u32(kslot(c)), RL::BOX, 1024);
+                            const uint64_t db = smem_desc_sw128(smem_u32(kslot(c - 1)), RL::BOX, 1024);
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk)
                                 mma_bf16_ts(tbase + TM_S, tbase + TM_X + kk * 8, desc_advance(db, kk * 2048), id_s, 1u);
@@ -461,12 +460,17 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                     }
                     __syncwarp();
                 }
-                // ---- every chain thread waits for the update; then the bf16 copy of its
-                //      lane of S~^T into TM_X (U~ is read), two keys per column ----
-                bool t = xok && mbar_wait_bounded(&bar_s, c & 1, kWaitNs);
+                // ---- every chain thread waits for the update; the keys of chunk c + 2 go into
+                //      the slot chunk c - 1 frees; then the bf16 copy of this thread's lane of
+                //      S~^T into TM_X (U~ is read), two keys per column ----
+                t = xok && mbar_wait_bounded(&bar_s, (c - 1) & 1, kWaitNs);
                 if (xok && !t) report_timeout(a, 6);
                 tc_fence_after();
-                if (t && has_next) {
+                if (warp == 4 && t && c + 2 < nchunks) {
+                    if (elect_one()) issue_k(c + 2);
+                    __syncwarp();
+                }
+                if (t && has_cur) {
 #pragma unroll
                     for (int cb = 0; cb < 4; ++cb) {
                         float sv[32];
@@ -481,93 +485,92 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 }
                 tc_fence_before();
                 xok = named_sync_and(BAR_CHAIN, 128, t) && xok;
-                // ---- P^T of chunk cn = S~^T K_cn^T into TM_Y once warps 0-3 have read K K^T
-                //      there, and the keys of chunk c + 2 into the slot chunk c frees ----
-                if (warp == 4) {
-                    if (has_next) named_sync(BAR_KK, 160);
+                // ---- P^T of chunk c = S~^T K_c^T into TM_Y (the P term of chunk c - 1 has
+                //      read it) ----
+                if (warp == 4 && has_cur) {
                     tc_fence_after();
                     if (elect_one()) {
-                        if (xok && has_next) {
-                            const uint64_t dk = smem_desc_sw128(smem_u32(kslot(cn)), 16, 1024);
+                        if (xok) {
+                            const uint64_t dk = smem_desc_sw128(smem_u32(kslot(c)), 16, 1024);
 #pragma unroll
                             for (int kk = 0; kk < 8; ++kk)
                                 mma_bf16_ts(tbase + TM_Y, tbase + TM_X + kk * 8,
                                             desc_advance(dk, (kk >> 2) * RL::BOX + (kk & 3) * 32), id_p, kk > 0);
                         }
-                        if (has_next) mma_commit(&bar_p);
-                        if (xok && c + 2 < nchunks) issue_k(c + 2);
+                        mma_commit(&bar_p);
                     }
                     __syncwarp();
                 }
             }
+            if (has_nx) {
+                // ---- K K^T of chunk c + 1 into TM_X once P of chunk c has read the state copy
+                //      there; a partial tile first gets its rows past the window zeroed ----
+                if (nrows_of(c + 1) < C) {   // uniform
+                    const bool t = mbar_wait_bounded(kbar(c + 1), kpar(c + 1), kWaitNs);
+                    if (t) zero_tail_rows(kslot(c + 1), nrows_of(c + 1), ct, 128);
+                    else report_timeout(a, 1);
+                    fence_proxy_async_smem();
+                    xok = named_sync_and(BAR_CHAIN, 128, t && xok);
+                }
+                if (warp == 4) {
+                    tc_fence_after();
+                    if (elect_one()) {
+                        bool tw = xok;
+                        if (tw && nrows_of(c + 1) == C) {
+                            tw = mbar_wait_bounded(kbar(c + 1), kpar(c + 1), kWaitNs);
+                            if (!tw) report_timeout(a, 1);
+                        }
+                        if (tw && has_prev) {
+                            tw = mbar_wait_bounded(&bar_p, (c - 1) & 1, kWaitNs);
+                            if (!tw) report_timeout(a, 3);
+                        }
+                        tc_fence_after();
+                        if (tw) issue_kk(c + 1);
+                        mma_commit(&bar_kk);
+                        if (!tw) s_abort = 1;
+                    }
+                    __syncwarp();
+                }
+            }
+            if (has_cur && nrows_of(c) < C) {   // a partial chunk's values, before its U'
+                const bool t = mbar_wait_bounded(&bar_v, c & 1, kWaitNs);
+                if (t) zero_tail_rows(sm + RL::OFF_V, nrows_of(c), ct, 128);
+                else report_timeout(a, 1);
+                fence_proxy_async_smem();
+                xok = xok && t;
+            }
         }
-        if (c >= 0) {   // every thread keeps the same running scale
-            const float snew = sigma * s_gates[c & 1].gam[C - 1];
-            sigma = snew < kRenormBelow ? 1.0f : snew;
-        }
+        // ---- A of chunk c + 1 (the front is done with AT, and K K^T is issued) ----
         tc_fence_before();
-        ok = __syncthreads_and(xok) != 0;   // T of chunk cn is in AT; chunk c's state update is done
-        if (!ok || !has_next) break;
+        xok = __syncthreads_and(xok) != 0;
+        if (has_nx && xok) xok = a_epilogue(c + 1);
+        if (has_prev) sigma = sig_c;
+        tc_fence_before();
+        ok = __syncthreads_and(xok && s_abort == 0) != 0;
+        if (!ok || !has_cur) break;
         tc_fence_after();
 
         // =============================== phase Y ===============================
-        // ---- partial tiles get their rows past the window zeroed; the T operands of chunk
-        //      cn are written (phase X) ----
-        const int ncn = nrows_of(cn);
-        const bool has_nn = cn + 1 < nchunks;
-        const int nnn = has_nn ? nrows_of(cn + 1) : C;
-        bool tok = true;
-        if (ncn < C) {   // values of chunk cn
-            const bool t = mbar_wait_bounded(&bar_v, cn & 1, kWaitNs);
-            if (t) zero_tail_rows(sm + RL::OFF_V, ncn);
-            else report_timeout(a, 1);
-            tok = tok && t;
-        }
-        if (nnn < C) {   // keys of chunk cn + 1 (its K K^T is issued below)
-            const bool t = mbar_wait_bounded(&bar_k[(cn + 1) & 1], ((cn + 1) >> 1) & 1, kWaitNs);
-            if (t) zero_tail_rows(kslot(cn + 1), nnn);
-            else report_timeout(a, 1);
-            tok = tok && t;
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        tok = __syncthreads_and(tok) != 0;
         if (warp == 2) {
-            // ---- (E U)^T of chunk cn into TM_X: P^T (-sigma E T diag(beta gamma))^T, then
-            //      + V^T (E T diag(beta))^T; then K K^T of chunk cn + 1 into TM_Y once the P
-            //      term has read it ----
-            tc_fence_after();
-            bool t = tok;
+            // ---- (E U)^T of chunk c into TM_X: P^T (-sigma E T diag(beta gamma))^T, then
+            //      + V^T (E T diag(beta))^T ----
             if (elect_one()) {
-                if (t && ncn == C) {
-                    t = mbar_wait_bounded(&bar_v, cn & 1, kWaitNs);
+                bool t = true;
+                if (nrows_of(c) == C) {
+                    t = mbar_wait_bounded(&bar_v, c & 1, kWaitNs);
                     if (!t) report_timeout(a, 1);
                 }
-                if (t && cn > 0) {   // the state is zero before chunk 0
-                    t = mbar_wait_bounded(&bar_p, (cn - 1) & 1, kWaitNs);
+                if (t && has_prev && !has_nx) {   // with a next chunk its K K^T waited for P
+                    t = mbar_wait_bounded(&bar_p, (c - 1) & 1, kWaitNs);
                     if (!t) report_timeout(a, 3);
                 }
                 tc_fence_after();
-                if (t && cn > 0) {
+                if (t && has_prev) {   // the state is zero before chunk 0
                     const uint64_t d2 = smem_desc_sw128(s_tg, 16, 1024);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
                         mma_tf32_ts(tbase + TM_X, tbase + TM_Y + kk * 8,
                                     desc_advance(d2, (kk >> 2) * 8192 + (kk & 3) * 32), id_t, kk > 0);
-                }
-                mma_commit(&bar_x);
-                if (has_nn) {
-                    if (t && nnn == C) {
-                        t = mbar_wait_bounded(&bar_k[(cn + 1) & 1], ((cn + 1) >> 1) & 1, kWaitNs);
-                        if (!t) report_timeout(a, 1);
-                    }
-                    if (t) {   // the P term is done reading TM_Y
-                        t = mbar_wait_bounded(&bar_x, cn & 1, kWaitNs);
-                        if (!t) report_timeout(a, 5);
-                    }
-                    tc_fence_after();
-                    if (t) issue_kk(cn + 1);
-                    mma_commit(&bar_kk);
                 }
                 if (t) {
                     const uint64_t dv = smem_desc_sw128(s_v, RL::BOX, 1024);
@@ -575,16 +578,16 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_bf16_ss(tbase + TM_X, desc_advance(dv, kk * 2048), desc_advance(dt, kk * 32), id_w,
-                                    (cn > 0 || kk > 0) ? 1u : 0u);
+                                    (has_prev || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(&bar_u);
+                if (!t) s_abort = 1;
             }
-            tok = __all_sync(0xffffffffu, t) && tok;
-        } else if (tid < C && has_nn) {
-            build_gates(s_gates[(cn + 1) & 1], al_nxt, be_nxt, tid, lane);
+            __syncwarp();
+        } else if (tid < C && c + 2 < nchunks) {
+            build_gates(s_gates[(c + 2) % 3], al_nxt, be_nxt, tid, lane);
         }
-        if (has_nn) load_gates(cn + 2, al_nxt, be_nxt);
-        ok = __syncthreads_and(tok) != 0;
+        if (c + 2 < nchunks) load_gates(c + 3, al_nxt, be_nxt);
     }
 
     // ---- final state: S[dk][dv] = sigma * TMEM[lane dv][dk] ----
