@@ -60,13 +60,17 @@ __device__ __forceinline__ void report_timeout(const CallArgs& a, uint32_t where
     atomicCAS(&a.ws->timeout_where, 0u, where);
 }
 
-// acc[nt] += A (16 x 8 ksteps) * B (8 ksteps x 16), nt = two 8-column halves
-// of the 16-wide result; A and B row-major fp32 in shared memory (strides
-// lda, ldb), read as tf32 (the tensor core uses the top 19 bits).
+// acc[nt] += A (16 x 16) * B (16 x 16), nt = two 8-column halves of the result;
+// A and B row-major fp32 in shared memory (strides lda, ldb), read as tf32 (the
+// tensor core uses the top 19 bits).  With SPLIT_K the two 8-deep k-steps go to
+// separate accumulators, summed at the end, so neither product waits for the
+// other: a warp-level MMA shares the tensor pipe with the CTA's tcgen05 work and
+// its latency grows with it.  That pays where one CTA per SM waits on the
+// inverse; with two CTAs per SM the extra instructions cost more than it saves.
+template <bool SPLIT_K>
 __device__ __forceinline__ void mma16x16_tf32(float acc[2][4], const float* A, int lda, const float* B, int ldb,
-                                              int ksteps, int g, int t) {
-    for (int ks = 0; ks < ksteps; ++ks) {
-        uint32_t af[4], bf[2][2];
+                                              int g, int t) {
+    auto load_ks = [&](int ks, uint32_t af[4], uint32_t bf[2][2]) {
         af[0] = __float_as_uint(A[g * lda + 8 * ks + t]);
         af[1] = __float_as_uint(A[(g + 8) * lda + 8 * ks + t]);
         af[2] = __float_as_uint(A[g * lda + 8 * ks + t + 4]);
@@ -76,8 +80,28 @@ __device__ __forceinline__ void mma16x16_tf32(float acc[2][4], const float* A, i
             bf[nt][0] = __float_as_uint(B[(8 * ks + t) * ldb + 8 * nt + g]);
             bf[nt][1] = __float_as_uint(B[(8 * ks + t + 4) * ldb + 8 * nt + g]);
         }
+    };
+    if (SPLIT_K) {
+        float acc1[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        uint32_t af[2][4], bf[2][2][2];
+        load_ks(0, af[0], bf[0]);
+        load_ks(1, af[1], bf[1]);
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) mma_sync_tf32(acc[nt], af, bf[nt]);
+        for (int nt = 0; nt < 2; ++nt) {
+            mma_sync_tf32(acc[nt], af[0], bf[0][nt]);
+            mma_sync_tf32(acc1[nt], af[1], bf[1][nt]);
+        }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[nt][e] += acc1[nt][e];
+    } else {
+        for (int ks = 0; ks < 2; ++ks) {
+            uint32_t af[4], bf[2][2];
+            load_ks(ks, af, bf);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) mma_sync_tf32(acc[nt], af, bf[nt]);
+        }
     }
 }
 
@@ -124,7 +148,7 @@ struct NoEmit {
     __device__ __forceinline__ void block(int, int, const float (&)[2][4], float, int, int) const {}
 };
 
-template <int LDX, int XHI, int XLO, class Emit = NoEmit>
+template <int LDX, int XHI, int XLO, class Emit = NoEmit, bool SPLIT_K = false>
 __device__ __forceinline__ void invert_unit_lower_inplace(float* AT, float* Xs, int ltid, uint32_t bar_id,
                                                           const Emit& emit = Emit()) {
     const int warp = ltid >> 5, lane = ltid & 31;
@@ -172,23 +196,23 @@ __device__ __forceinline__ void invert_unit_lower_inplace(float* AT, float* Xs, 
         float* X = xslot(warp);
         const int bo = warp ? 48 : 16, ao = warp ? 32 : 0;   // row block b, column block a
         float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        mma16x16_tf32(acc, AT + bo * LDT + ao, LDT, AT + ao * LDT + ao, LDT, 2, g, t);     // A_ba D_a
+        mma16x16_tf32<SPLIT_K>(acc, AT + bo * LDT + ao, LDT, AT + ao * LDT + ao, LDT, g, t);     // A_ba D_a
         store16x16(X, LDX, acc, 1.0f, g, t);
         __syncwarp();
         float r[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        mma16x16_tf32(r, AT + bo * LDT + bo, LDT, X, LDX, 2, g, t);                      // D_b (A_ba D_a)
+        mma16x16_tf32<SPLIT_K>(r, AT + bo * LDT + bo, LDT, X, LDX, g, t);                      // D_b (A_ba D_a)
         store16x16(AT + bo * LDT + ao, LDT, r, -1.0f, g, t);
         emit.block(bo, ao, r, -1.0f, g, t);
     } else {
         const int r = warp;
-        mma16x16_tf32(pr0, AT + 16 * r * LDT, LDT, AT, LDT, 2, g, t);                    // A_r0 D_0
-        mma16x16_tf32(xr1, AT + 16 * r * LDT + 16, LDT, AT + 16 * LDT + 16, LDT, 2, g, t);  // A_r1 D_1
+        mma16x16_tf32<SPLIT_K>(pr0, AT + 16 * r * LDT, LDT, AT, LDT, g, t);                    // A_r0 D_0
+        mma16x16_tf32<SPLIT_K>(xr1, AT + 16 * r * LDT + 16, LDT, AT + 16 * LDT + 16, LDT, g, t);  // A_r1 D_1
     }
     named_sync(bar_id, 128);
     // Level B: X_r0 = P_r0 + A_r1 T_10 (warps 2-3), X blocks to the scratch, slot 2 (r - 2) + c
     if (warp >= 2) {
         const int r = warp;
-        mma16x16_tf32(pr0, AT + 16 * r * LDT + 16, LDT, AT + 16 * LDT, LDT, 2, g, t);      // + A_r1 T_10
+        mma16x16_tf32<SPLIT_K>(pr0, AT + 16 * r * LDT + 16, LDT, AT + 16 * LDT, LDT, g, t);      // + A_r1 T_10
         store16x16(xslot(2 * (r - 2)), LDX, pr0, 1.0f, g, t);
         store16x16(xslot(2 * (r - 2) + 1), LDX, xr1, 1.0f, g, t);
     } else {
@@ -201,11 +225,11 @@ __device__ __forceinline__ void invert_unit_lower_inplace(float* AT, float* Xs, 
         float rr[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         const float* X2c = xslot(c);
         if (r == 2) {
-            mma16x16_tf32(rr, AT + 32 * LDT + 32, LDT, X2c, LDX, 2, g, t);              // D_2 X_2c
+            mma16x16_tf32<SPLIT_K>(rr, AT + 32 * LDT + 32, LDT, X2c, LDX, g, t);              // D_2 X_2c
         } else {
             const float* X3c = xslot(2 + c);
-            mma16x16_tf32(rr, AT + 48 * LDT + 32, LDT, X2c, LDX, 2, g, t);              // T_32 X_2c
-            mma16x16_tf32(rr, AT + 48 * LDT + 48, LDT, X3c, LDX, 2, g, t);              // D_3 X_3c
+            mma16x16_tf32<SPLIT_K>(rr, AT + 48 * LDT + 32, LDT, X2c, LDX, g, t);              // T_32 X_2c
+            mma16x16_tf32<SPLIT_K>(rr, AT + 48 * LDT + 48, LDT, X3c, LDX, g, t);              // D_3 X_3c
         }
         store16x16(AT + 16 * r * LDT + 16 * c, LDT, rr, -1.0f, g, t);
         emit.block(16 * r, 16 * c, rr, -1.0f, g, t);

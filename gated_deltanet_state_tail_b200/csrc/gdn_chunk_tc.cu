@@ -308,7 +308,7 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                     }
                 }
                 named_sync(BAR_INV, 128);   // every row of A is in before the inverse reads it
-                invert_unit_lower_inplace<GDN_INV_SCRATCH_SEPARATE>(AT, Xs, tid, BAR_INV);
+                invert_unit_lower_inplace<GDN_INV_SCRATCH_SEPARATE, NoEmit, true>(AT, Xs, tid, BAR_INV);
             }
         } else if (c >= 0) {
             // ---- chain of chunk c: U~ (and U^T for the outputs), the state update and
