@@ -368,6 +368,84 @@ __device__ __forceinline__ void build_gates(Gates& G, float al, float be, int ti
     }
 }
 
+// An emitter for invert_unit_lower_inplace: each final block of T goes from
+// registers (or, for the diagonal blocks, from AT) into the chunk's two T
+// operands,
+//   tb[j][j'] = r_j T[j][j'] beta_j'                  (bf16, 128-byte swizzled rows),
+//   tg[j][j'] = -sigma' r_j T[j][j'] beta_j' gamma_j' (fp32, K-major, two 8 KB blocks
+//                                                      of 32 columns, 128-byte swizzled),
+// with r_j = gamma_C / gamma_j (ROW_E, the replay's chunk decay folded into the
+// rows) or 1 (the prefill, whose outputs need U itself), and sigma' the state's
+// scale entering the chunk.  tg follows tb at tb + 8192.
+template <bool ROW_E>
+struct TOperandEmit {
+    const Gates* G;
+    float nsig;    // -sigma'
+    uint8_t* tb;   // tg follows at tb + 8192
+    uint64_t* bar_rd;    // null, or the mbarrier of the MMAs still reading tb and tg
+    uint32_t parity;
+    const CallArgs* a;
+    int* abort_flag;
+    __device__ __forceinline__ void prepare() const {
+        if (bar_rd != nullptr && !mbar_wait_bounded(bar_rd, parity, kWaitNs)) {
+            report_timeout(*a, 8);
+            *abort_flag = 1;
+        }
+    }
+    __device__ __forceinline__ static uint32_t off_b(int j, int jj) {
+        return (uint32_t)(j * 128 + (((jj >> 3) ^ (j & 7)) << 4) + (jj & 7) * 2);
+    }
+    __device__ __forceinline__ static uint32_t off_g(int j, int jj) {
+        return (uint32_t)(8192 + (jj >> 5) * 8192 + j * 128 + ((((jj & 31) >> 2) ^ (j & 7)) << 4) + (jj & 3) * 4);
+    }
+    // thread q: row j = 16 (q / 16) + q % 16 of its diagonal block, 16 columns
+    __device__ __forceinline__ void diagonal(const float* AT, int q) const {
+        const int o = (q >> 4) * 16, j = o + (q & 15);
+        const float ej = ROW_E ? G->e[j] : 1.0f, ejg = nsig * ej;
+        float v[16];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float4 t4 = *reinterpret_cast<const float4*>(AT + j * LDT + o + 4 * k);
+            const float4 b4 = *reinterpret_cast<const float4*>(G->beta + o + 4 * k);
+            const float4 g4 = *reinterpret_cast<const float4*>(G->gam + o + 4 * k);
+            v[4 * k + 0] = t4.x * b4.x;
+            v[4 * k + 1] = t4.y * b4.y;
+            v[4 * k + 2] = t4.z * b4.z;
+            v[4 * k + 3] = t4.w * b4.w;
+            const float4 w4 = make_float4(v[4 * k] * g4.x * ejg, v[4 * k + 1] * g4.y * ejg,
+                                          v[4 * k + 2] * g4.z * ejg, v[4 * k + 3] * g4.w * ejg);
+            *reinterpret_cast<float4*>(tb + off_g(j, o + 4 * k)) = w4;
+        }
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            uint4 x;
+            x.x = pack_bf16(v[8 * hh + 0] * ej, v[8 * hh + 1] * ej);
+            x.y = pack_bf16(v[8 * hh + 2] * ej, v[8 * hh + 3] * ej);
+            x.z = pack_bf16(v[8 * hh + 4] * ej, v[8 * hh + 5] * ej);
+            x.w = pack_bf16(v[8 * hh + 6] * ej, v[8 * hh + 7] * ej);
+            st_shared_v4(tb, off_b(j, o + 8 * hh), x);
+        }
+    }
+    __device__ __forceinline__ void block(int r0, int c0, const float (&acc)[2][4], float scale, int g,
+                                          int t) const {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const int jj = c0 + 8 * nt + 2 * t;
+            const float2 b2 = *reinterpret_cast<const float2*>(G->beta + jj);
+            const float2 g2 = *reinterpret_cast<const float2*>(G->gam + jj);
+            const float bg0 = nsig * b2.x * g2.x, bg1 = nsig * b2.y * g2.y;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int j = r0 + g + 8 * hh;
+                const float ej = ROW_E ? scale * G->e[j] : scale;
+                const float v0 = acc[nt][2 * hh] * ej, v1 = acc[nt][2 * hh + 1] * ej;
+                *reinterpret_cast<uint32_t*>(tb + off_b(j, jj)) = pack_bf16(v0 * b2.x, v1 * b2.y);
+                *reinterpret_cast<float2*>(tb + off_g(j, jj)) = make_float2(v0 * bg0, v1 * bg1);
+            }
+        }
+    }
+};
+
 // Block-wide agreement after a bounded wait: every thread leaves together.
 __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, const CallArgs& a, uint32_t where) {
     bool ok = mbar_wait_bounded(bar, parity, kWaitNs);

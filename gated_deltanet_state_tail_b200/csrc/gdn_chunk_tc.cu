@@ -49,29 +49,40 @@ using namespace chunk;
 
 // ---------------------------------------------------------------------------
 // Prefill (and fused replay + suffix) with two chunks in flight per CTA.
-//
-// Warps 0-3 form A and M of chunk c + 1 and invert T while warps 4-7 finish
-// chunk c: the U epilogue, the state update and O += U M^T on the tensor core,
-// then chunk c's outputs and the TMA of chunk c + 2 into the slot that frees.
-// M is double-buffered so chunk c + 1's can be written while chunk c's output
-// product reads its own.  192 KB of shared memory, 512 TMEM columns, one CTA
-// per SM.
+// Iteration c (chunk cn = c + 1 is the next one):
+//   phase X  warps 0-3 (front): A and M of chunk cn from [K; Q] K^T (TM_P), then
+//                       T = (I + A)^-1, writing the chunk's T operands T diag(beta)
+//                       (bf16) and -sigma' T diag(beta gamma) (fp32) as each block of
+//                       T is final;
+//            warps 4-7 (chain): chunk c's U epilogue, its state update and
+//                       O += U M^T, the TMA of chunk c + 2, chunk c's outputs; then
+//                       a bf16 copy of the new state in TMEM, sigma' gamma Q of chunk
+//                       cn in bf16, and, once the front has read TM_P, P = K S~ of
+//                       chunk cn into TM_P and the outputs' state term sigma' diag(gamma)
+//                       Q S~ into TM_O, both from the bf16 state copy.
+//   phase Y  warp 2: U of chunk cn = P^T (-sigma' T diag(beta gamma))^T (tf32) + U'
+//                       into TM_U; warp 3: [K; Q] K^T of chunk cn + 1 into TM_P once
+//                       the P term has read it; warps 0-1: the gates of chunk cn + 1.
+// 185 KB of shared memory, 512 TMEM columns, one CTA per SM.
 constexpr uint32_t BAR_CHAIN = 2;   // named barrier of warps 4-7
+constexpr uint32_t BAR_KK = 5;      // warps 0-3 -> warp 4: [K; Q] K^T in TM_P is read, P may overwrite it
+constexpr uint32_t TM_SB = 384;     // 64 columns (prefill): bf16 S~^T, two keys per column
 struct PipeLayout {
     static constexpr uint32_t TILE = TileLayout::TILE;       // [K0 | Q0 | K1 | Q1 | V0 | V1]
     static constexpr uint32_t OFF_TILE = 0;
-    static constexpr uint32_t OFF_PREP = 2 * TILE;              // A / T, T diag(..), -sigma W
-    static constexpr uint32_t OFF_AT = OFF_PREP;
-    static constexpr uint32_t OFF_X = OFF_PREP + 17408;
-    static constexpr uint32_t OFF_TB = OFF_PREP;
-    static constexpr uint32_t OFF_TBG = OFF_PREP + 8192;
-    static constexpr uint32_t OFF_BU = OFF_PREP;
-    static constexpr uint32_t OFF_UB = OFF_PREP + 32768;        // the output stage, bf16 O [i][dv]
+    static constexpr uint32_t OFF_AT = 2 * TILE;                // fp32 A, then T (scratch in its upper right)
+    static constexpr uint32_t OFF_TB = OFF_AT + C * LDT * 4;    // bf16 T diag(beta)
+    static constexpr uint32_t OFF_TG = OFF_TB + 8192;           // fp32 -sigma T diag(beta gamma), K-major
+    static constexpr uint32_t OFF_UB = OFF_TG + 16384;          // the output stage, bf16 O [i][dv]
     static constexpr uint32_t OFF_MB = OFF_UB + 16384;          // two bf16 M [i][j], chunk c in c % 2
-    static constexpr uint32_t OFF_BQ = OFF_MB + 16384;          // fp32 sigma diag(gamma) Q, K-major
-    static constexpr uint32_t BYTES = OFF_BQ + 32768;
+    static constexpr uint32_t OFF_BQ = OFF_MB + 16384;          // bf16 sigma diag(gamma) Q, K-major
+    static constexpr uint32_t BYTES = OFF_BQ + 16384;
 };
+static_assert(PipeLayout::OFF_TB % 1024 == 0 && PipeLayout::OFF_TG == PipeLayout::OFF_TB + 8192 &&
+                  PipeLayout::OFF_BQ % 1024 == 0,
+              "operands on 1 KB, TG right after TB");
 static_assert(PipeLayout::BYTES + 1024 <= 227 * 1024, "fits one CTA per SM");
+static_assert(TM_SB + 64 <= 512, "TMEM map");
 
 __global__ void __launch_bounds__(NT, 1)
 prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
@@ -81,7 +92,10 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     using PL = PipeLayout;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t bar_tile[2], bar_w, bar_u, bar_s;
+    // bar_tile: the tiles of chunk c (slot c % 2); bar_kk: [K; Q] K^T; bar_s: the state
+    // update and O += U M^T; bar_p: P and the outputs' state term; bar_x: the P term;
+    // bar_u: U (the P term and U').  One issuer each.
+    __shared__ uint64_t bar_tile[2], bar_kk, bar_s, bar_p, bar_x, bar_u;
     __shared__ uint32_t tmem_slot;
     __shared__ Gates s_gates[2];    // chunk c uses s_gates[c & 1]
 
@@ -128,13 +142,19 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         else
             issue_tiles(tile_of(cc), &bar_tile[cc & 1], &map_k0, &map_v0, &map_q, h, (int)cs.r0, false);
     };
+    // the state entering chunk 0 is zero unless the call passes one (a fused call starts
+    // from zero): then chunk 0 has no P term and no state term in its outputs
+    const bool s0_zero = fused || a.state_in == nullptr;
+    auto has_state_terms = [&](int cc) { return cc > 0 || !s0_zero; };
 
     if (tid == 0) {
         mbar_init(&bar_tile[0], 1);
         mbar_init(&bar_tile[1], 1);
-        mbar_init(&bar_w, 2);
-        mbar_init(&bar_u, 2);
+        mbar_init(&bar_kk, 1);
         mbar_init(&bar_s, 1);
+        mbar_init(&bar_p, 1);
+        mbar_init(&bar_x, 1);
+        mbar_init(&bar_u, 1);
         mbar_fence_init();
         tma_prefetch_desc(&map_k);
         tma_prefetch_desc(&map_v);
@@ -148,6 +168,10 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         tmem_alloc(&tmem_slot, 512);
         tmem_relinquish();
     }
+    // the T operands' blocks above the diagonal stay zero
+    for (int e = tid; e < (8192 + 16384) / 16; e += NT)
+        st_shared_v4(sm + PL::OFF_TB, (uint32_t)(e * 16), make_uint4(0, 0, 0, 0));
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -158,9 +182,7 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     }
 
     float* AT = reinterpret_cast<float*>(sm + PL::OFF_AT);
-    float* Xs = reinterpret_cast<float*>(sm + PL::OFF_X);
-    const uint32_t s_bu = smem_u32(sm + PL::OFF_BU);
-    const uint32_t s_tb = smem_u32(sm + PL::OFF_TB), s_tbg = smem_u32(sm + PL::OFF_TBG);
+    const uint32_t s_tb = smem_u32(sm + PL::OFF_TB), s_tg = smem_u32(sm + PL::OFF_TG);
     const uint32_t s_bq = smem_u32(sm + PL::OFF_BQ);
     const size_t state_base = ((size_t)b * H + h) * D * D;
     {   // initial state: TMEM lane dv holds column dv of S (a row of S^T)
@@ -181,11 +203,12 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     float sigma = 1.0f;
 
     const uint32_t id_kk = idesc_bf16(128, 64, false, false);   // [K;Q] K^T
-    const uint32_t id_w = idesc_bf16(128, 64, true, false);
-    const uint32_t id_u = idesc_tf32(128, 64, false, false);
-    const uint32_t id_s = idesc_bf16(128, 128, false, true);
+    const uint32_t id_w = idesc_bf16(128, 64, true, false);     // V^T (T diag(beta))^T
+    const uint32_t id_t = idesc_tf32(128, 64, false, false);    // P^T (-sigma T diag(beta gamma))^T, A in TMEM
+    const uint32_t id_p = idesc_bf16(128, 64, false, false);    // S~^T K^T and S~^T (sigma gamma Q)^T, A in TMEM
+    const uint32_t id_s = idesc_bf16(128, 128, false, true);    // U~^T K, A in TMEM
     const uint32_t id_o2 = idesc_bf16(128, 64, false, false);   // U^T M^T, A (U^T) in TMEM
-    uint32_t ph_w = 0, ph_u = 0, ph_s = 0;
+    uint32_t ph_u = 0, ph_s = 0, ph_p = 0, ph_x = 0;
     bool ok = true;
 
     auto load_gates = [&](int cc, float& al, float& be) {
@@ -241,23 +264,21 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     load_gates(1, al_nxt, be_nxt);
     if (nchunks > 0) {
         ok = tiles_ready(0);
-        if (ok && (warp == 2 || warp == 3)) {
+        if (ok && warp == 3) {
             tc_fence_after();
             if (elect_one()) {
-                if (warp == 3) issue_kk(0);
-                mma_commit(&bar_u);
+                issue_kk(0);
+                mma_commit(&bar_kk);
             }
             __syncwarp();
-        }
-        if (ok) {
-            ok = wait_all(&bar_u, ph_u, a, 2);
-            ph_u ^= 1;
         }
     }
 
     for (int c = -1; c < nchunks && ok; ++c) {
         const int cn = c + 1;
         const bool has_next = cn < nchunks;
+        // P and the outputs' state term of chunk cn are formed in this phase X
+        const bool st_next = has_next && has_state_terms(cn);
         bool xok = true;
         tc_fence_after();
         if (warp < 4) {
@@ -265,6 +286,12 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 // ---- epilogue 1 of chunk cn: warps 0-1 hold K rows (lane = row), warps 2-3 the
                 //      Q rows; A = strict_tril(beta_i (gamma_i / gamma_j) K K^T) (fp32, in AT) and
                 //      M = tril((gamma_i / gamma_j) Q K^T) (bf16, MB[cn % 2]) ----
+                {
+                    const bool t = mbar_wait_bounded(&bar_kk, cn & 1, kWaitNs);
+                    if (!t) report_timeout(a, 2);
+                    xok = xok && t;
+                    tc_fence_after();
+                }
                 Gates& Gn = s_gates[cn & 1];
                 const bool outn = chunk_src(cn).out;
                 const bool krow = wq < 2;
@@ -307,115 +334,194 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                         }
                     }
                 }
+                if (st_next) {   // [K; Q] K^T is read: P of chunk cn may take TM_P
+                    tc_fence_before();
+                    named_arrive(BAR_KK, 160);
+                }
                 named_sync(BAR_INV, 128);   // every row of A is in before the inverse reads it
-                invert_unit_lower_inplace<GDN_INV_SCRATCH_SEPARATE, NoEmit, true>(AT, Xs, tid, BAR_INV);
+                // ---- T = (I + A)^-1 in place, writing the T operands of chunk cn scaled with the
+                //      state's scale entering it ----
+                float sig = sigma;
+                if (c >= 0) {
+                    const float sn = sigma * s_gates[c & 1].gam[C - 1];
+                    sig = sn < kRenormBelow ? 1.0f : sn;
+                }
+                const TOperandEmit<false> em{&Gn, -sig, sm + PL::OFF_TB, nullptr, 0u, &a, nullptr};
+                invert_unit_lower_inplace<GDN_INV_SCRATCH_IN_AT, TOperandEmit<false>, true>(AT, AT + 32, tid, BAR_INV,
+                                                                                            em);
+                fence_proxy_async_smem();   // the T operands, for phase Y's MMAs
             }
-        } else if (c >= 0) {
-            // ---- chain of chunk c: U~ (and U^T for the outputs), the state update and
-            //      O += U M^T, then chunk c's outputs ----
-            Gates& G = s_gates[c & 1];
-            const ChunkSrc src = chunk_src(c);
-            const bool outc = src.out;
-            uint8_t* tile = tile_of(c);
-            float snew = sigma * G.gam[C - 1];
-            if (snew < kRenormBelow) {   // uniform
+        } else {
+            const int ct = tid - 128;   // this thread among the chain's 128
+            if (c >= 0) {
+                // ---- chain of chunk c: U~ (and U^T for the outputs), the state update and
+                //      O += U M^T, then chunk c's outputs ----
+                Gates& G = s_gates[c & 1];
+                const ChunkSrc src = chunk_src(c);
+                const bool outc = src.out;
+                uint8_t* tile = tile_of(c);
+                float snew = sigma * G.gam[C - 1];
+                if (snew < kRenormBelow) {   // uniform
+#pragma unroll
+                    for (int cb = 0; cb < 4; ++cb) {
+                        float sv[32];
+                        tmem_ld32(tlane + TM_S + cb * 32, sv);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) sv[q] *= snew;
+                        tmem_st32(tlane + TM_S + cb * 32, sv);
+                    }
+                    tmem_wait_st();
+                    snew = 1.0f;
+                }
+                const float inv = 1.0f / snew;
+                // U^T (for the outputs) and U~^T = U^T diag(e) / sigma (for the state update) as
+                // bf16 in TMEM, two chunk rows per 32-bit column: the A operands of both MMAs
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    float v[32];
+                    tmem_ld32(tlane + TM_U + 32 * hf, v);
+                    tmem_wait_ld();
+                    uint32_t pk[16];
+                    if (outc) {
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) pk[q] = pack_bf16(v[2 * q], v[2 * q + 1]);
+                        tmem_st16(tlane + TM_UB + 16 * hf, pk);
+                    }
+                    const float4* ev = reinterpret_cast<const float4*>(G.e + 32 * hf);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 e4 = ev[q];
+                        pk[2 * q] = pack_bf16(v[4 * q] * (e4.x * inv), v[4 * q + 1] * (e4.y * inv));
+                        pk[2 * q + 1] = pack_bf16(v[4 * q + 2] * (e4.z * inv), v[4 * q + 3] * (e4.w * inv));
+                    }
+                    tmem_st16(tlane + TM_UT + 16 * hf, pk);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                named_sync(BAR_CHAIN, 128);
+                if (warp == 4) {
+                    tc_fence_after();
+                    if (elect_one()) {
+                        const uint32_t s_tile = smem_u32(tile);
+                        const uint32_t s_mb = smem_u32(sm + PL::OFF_MB + (c & 1) * 8192);
+                        const uint64_t db = smem_desc_sw128(s_tile, L::K_BLK, 1024);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_bf16_ts(tbase + TM_S, tbase + TM_UT + kk * 8, desc_advance(db, kk * 2048), id_s, 1u);
+                        if (outc) {   // O holds the state term unless the state entering chunk c is zero
+                            const uint64_t dmb = smem_desc_sw128(s_mb, 16, 1024);
+                            const bool acc = has_state_terms(c);
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk)
+                                mma_bf16_ts(tbase + TM_O, tbase + TM_UB + kk * 8, desc_advance(dmb, kk * 32), id_o2,
+                                            (acc || kk > 0) ? 1u : 0u);
+                        }
+                        mma_commit(&bar_s);
+                        if (mbar_wait_bounded(&bar_s, ph_s, kWaitNs)) {
+                            if (c + 2 < nchunks) issue_chunk(c + 2);
+                        } else {
+                            report_timeout(a, 6);
+                            xok = false;
+                        }
+                    }
+                    __syncwarp();
+                }
+                sigma = snew;
+                named_sync(BAR_CHAIN, 128);   // the state update (and O) of chunk c are complete
+                tc_fence_after();
+                if (outc) {
+                    // outputs: stage O as bf16 rows [i][dv] in the UB region, then 16-byte stores of
+                    // whole rows
+                    __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(sm + PL::OFF_UB);
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        float v[32];   // O^T: value dim = row, chunk rows [32 hf, 32 hf + 32)
+                        tmem_ld32(tlane + TM_O + 32 * hf, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int ii = 0; ii < 32; ++ii) stage[(32 * hf + ii) * D + row] = __float2bfloat16_rn(v[ii]);
+                    }
+                    named_sync(BAR_CHAIN, 128);
+                    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o_out);
+#pragma unroll
+                    for (int k = 0; k < (C * D / 8) / 128; ++k) {   // 16-byte pieces: 16 per row
+                        const int idx = ct + k * 128, i = idx >> 4, ch = idx & 15;
+                        if (i < src.nc && index_ok(a.ws, src.r0 + i < a.rows_total))
+                            *reinterpret_cast<uint4*>(o + ((src.r0 + i) * H + h) * (long long)D + ch * 8) =
+                                *reinterpret_cast<const uint4*>(stage + i * D + ch * 8);
+                    }
+                }
+                if (fused && c == nA - 1 && a.state_mid) {   // the state at L (chunk c is the window's last)
+#pragma unroll
+                    for (int cb = 0; cb < 4; ++cb) {
+                        float v[32];
+                        tmem_ld32(tlane + TM_S + cb * 32, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            a.state_mid[state_base + (size_t)(cb * 32 + i) * D + row] = sigma * v[i];
+                    }
+                }
+            }
+            if (st_next) {
+                // ---- chunk cn's state terms from a bf16 copy of S~^T (TM_SB): P^T = S~^T K^T into
+                //      TM_P once the front has read it, and, with outputs, the state term of O^T =
+                //      S~^T (sigma diag(gamma) Q)^T into TM_O (chunk c's outputs are read) ----
+                const bool outn = chunk_src(cn).out;
 #pragma unroll
                 for (int cb = 0; cb < 4; ++cb) {
                     float sv[32];
                     tmem_ld32(tlane + TM_S + cb * 32, sv);
                     tmem_wait_ld();
+                    uint32_t pk[16];
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) sv[q] *= snew;
-                    tmem_st32(tlane + TM_S + cb * 32, sv);
+                    for (int q = 0; q < 16; ++q) pk[q] = pack_bf16(sv[2 * q], sv[2 * q + 1]);
+                    tmem_st16(tlane + TM_SB + cb * 16, pk);
+                }
+                if (outn) {   // sigma gamma_i Q[i] in bf16, the Q tile's 128-byte swizzle kept
+                    const Gates& Gn = s_gates[cn & 1];
+                    const uint8_t* qt = tile_of(cn) + L::Q0;
+                    uint8_t* bq = sm + PL::OFF_BQ;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {   // 1024 16-byte pieces: 2 blocks x 64 rows x 8
+                        // consecutive threads take consecutive pieces of a row: a warp reads and
+                        // writes four whole 128-byte rows, free of bank conflicts
+                        const int idx = ct + k * 128, chn = idx & 7, i = (idx >> 3) & (C - 1), blk = idx >> 9;
+                        const uint32_t off = (uint32_t)(i * 128 + (chn << 4));
+                        const uint4 raw = *reinterpret_cast<const uint4*>(qt + blk * L::K_BLK + off);
+                        const float sg = sigma * Gn.gam[i];
+                        const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
+                        uint32_t pq[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            pq[e] = pack_bf16(sg * __uint_as_float(wd[e] << 16), sg * __uint_as_float(wd[e] & 0xffff0000u));
+                        *reinterpret_cast<uint4*>(bq + blk * 8192 + off) = make_uint4(pq[0], pq[1], pq[2], pq[3]);
+                    }
+                    fence_proxy_async_smem();
                 }
                 tmem_wait_st();
-                snew = 1.0f;
-            }
-            const float inv = 1.0f / snew;
-            // U^T (for the outputs) and U~^T = U^T diag(e) / sigma (for the state update) as
-            // bf16 in TMEM, two chunk rows per 32-bit column: the A operands of both MMAs
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                float v[32];
-                tmem_ld32(tlane + TM_U + 32 * hf, v);
-                tmem_wait_ld();
-                uint32_t pk[16];
-                if (outc) {
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) pk[q] = pack_bf16(v[2 * q], v[2 * q + 1]);
-                    tmem_st16(tlane + TM_UB + 16 * hf, pk);
-                }
-                const float4* ev = reinterpret_cast<const float4*>(G.e + 32 * hf);
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 e4 = ev[q];
-                    pk[2 * q] = pack_bf16(v[4 * q] * (e4.x * inv), v[4 * q + 1] * (e4.y * inv));
-                    pk[2 * q + 1] = pack_bf16(v[4 * q + 2] * (e4.z * inv), v[4 * q + 3] * (e4.w * inv));
-                }
-                tmem_st16(tlane + TM_UT + 16 * hf, pk);
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            named_sync(BAR_CHAIN, 128);
-            if (warp == 4) {
-                tc_fence_after();
-                if (elect_one()) {
-                    const uint32_t s_tile = smem_u32(tile);
-                    const uint32_t s_mb = smem_u32(sm + PL::OFF_MB + (c & 1) * 8192);
-                    const uint64_t db = smem_desc_sw128(s_tile, L::K_BLK, 1024);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ts(tbase + TM_S, tbase + TM_UT + kk * 8, desc_advance(db, kk * 2048), id_s, 1u);
-                    if (outc) {
-                        const uint64_t dmb = smem_desc_sw128(s_mb, 16, 1024);
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            mma_bf16_ts(tbase + TM_O, tbase + TM_UB + kk * 8, desc_advance(dmb, kk * 32), id_o2, 1u);
-                    }
-                    mma_commit(&bar_s);
-                    if (mbar_wait_bounded(&bar_s, ph_s, kWaitNs)) {
-                        if (c + 2 < nchunks) issue_chunk(c + 2);
-                    } else {
-                        report_timeout(a, 6);
-                        xok = false;
-                    }
-                }
-                __syncwarp();
-            }
-            sigma = snew;
-            named_sync(BAR_CHAIN, 128);   // the state update (and O) of chunk c are complete
-            tc_fence_after();
-            if (outc) {
-                // outputs: stage O as bf16 rows [i][dv] in the UB region, then 16-byte stores of
-                // whole rows
-                __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(sm + PL::OFF_UB);
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    float v[32];   // O^T: value dim = row, chunk rows [32 hf, 32 hf + 32)
-                    tmem_ld32(tlane + TM_O + 32 * hf, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int ii = 0; ii < 32; ++ii) stage[(32 * hf + ii) * D + row] = __float2bfloat16_rn(v[ii]);
-                }
+                tc_fence_before();
                 named_sync(BAR_CHAIN, 128);
-                __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o_out);
-                const int ct = tid - 128;   // this thread among the chain's 128
+                if (warp == 4) {
+                    named_sync(BAR_KK, 160);
+                    tc_fence_after();
+                    if (elect_one()) {
+                        const uint64_t dk = smem_desc_sw128(smem_u32(tile_of(cn)), 16, 1024);
 #pragma unroll
-                for (int k = 0; k < (C * D / 8) / 128; ++k) {   // 16-byte pieces: 16 per row
-                    const int idx = ct + k * 128, i = idx >> 4, ch = idx & 15;
-                    if (i < src.nc && index_ok(a.ws, src.r0 + i < a.rows_total))
-                        *reinterpret_cast<uint4*>(o + ((src.r0 + i) * H + h) * (long long)D + ch * 8) =
-                            *reinterpret_cast<const uint4*>(stage + i * D + ch * 8);
-                }
-            }
-            if (fused && c == nA - 1 && a.state_mid) {   // the state at L (chunk c is the window's last)
+                        for (int kk = 0; kk < 8; ++kk)
+                            mma_bf16_ts(tbase + TM_P, tbase + TM_SB + kk * 8,
+                                        desc_advance(dk, (kk >> 2) * L::K_BLK + (kk & 3) * 32), id_p, kk > 0);
+                        if (outn) {
+                            const uint64_t dq = smem_desc_sw128(s_bq, 16, 1024);
 #pragma unroll
-                for (int cb = 0; cb < 4; ++cb) {
-                    float v[32];
-                    tmem_ld32(tlane + TM_S + cb * 32, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) a.state_mid[state_base + (size_t)(cb * 32 + i) * D + row] = sigma * v[i];
+                            for (int kk = 0; kk < 8; ++kk)
+                                mma_bf16_ts(tbase + TM_O, tbase + TM_SB + kk * 8,
+                                            desc_advance(dq, (kk >> 2) * 8192 + (kk & 3) * 32), id_p, kk > 0);
+                        }
+                        mma_commit(&bar_p);
+                    }
+                    __syncwarp();
                 }
             }
         }
@@ -427,129 +533,71 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         ok = __syncthreads_and(xok) != 0;
         if (!ok || !has_next) break;
 
-        // ---- phase Y, chunk cn ----
-        Gates& Gn = s_gates[cn & 1];
-        const ChunkSrc srcn = chunk_src(cn);
-        uint8_t* tile_n = tile_of(cn);
-        const uint32_t s_tile_n = smem_u32(tile_n);
-        write_scaled_t<NT>(AT, Gn.beta, Gn.gam, sm + PL::OFF_TB, sm + PL::OFF_TBG, tid, 0);
-        fence_proxy_async_smem();
-        __syncthreads();
-        if (warp == 0) {
-            tc_fence_after();
-            if (elect_one()) {
-                const uint64_t da = smem_desc_sw128(s_tile_n, L::K_BLK, 1024);
-                const uint64_t db = smem_desc_sw128(s_tbg, 16, 1024);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ss(tbase + TM_P, desc_advance(da, kk * 2048), desc_advance(db, kk * 32), id_w, kk > 0);
-                mma_commit(&bar_w);
-            }
-            __syncwarp();
-        } else if (warp == 1) {
-            tc_fence_after();
-            if (elect_one()) {
-                const uint64_t da = smem_desc_sw128(s_tile_n + L::V0, L::V_LBO, 1024);
-                const uint64_t db = smem_desc_sw128(s_tb, 16, 1024);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ss(tbase + TM_U, desc_advance(da, kk * 2048), desc_advance(db, kk * 32), id_w, kk > 0);
-                mma_commit(&bar_w);
-            }
-            __syncwarp();
-        }
-        ok = wait_all(&bar_w, ph_w, a, 3);
-        ph_w ^= 1;
-        if (!ok) break;
-        tc_fence_after();
-        // ---- epilogue 2: BU = -sigma W (fp32, K-major); BQ = sigma diag(gamma) Q ----
-        {
-            float v[32];
-            tmem_ld32(tlane + TM_P + 32 * wh, v);
-            tmem_wait_ld();
-            uint8_t* bu = sm + PL::OFF_BU + wq * 8192;
-            const float ns = -sigma;
-#pragma unroll
-            for (int jj = 0; jj < 32; ++jj)
-                *reinterpret_cast<float*>(bu + sw128_offset_f32(32 * wh + jj, lane)) = ns * v[jj];
-            if (srcn.out) {
-                // row i, keys [32 qk, 32 qk + 32): consecutive threads take consecutive rows
-                const int i = tid & (C - 1), qk = tid >> 6;
-                const uint8_t* qb = tile_n + L::Q0 + (qk >> 1) * 16384;
-                uint8_t* blk = sm + PL::OFF_BQ + qk * 8192;
-                const float sg = sigma * Gn.gam[i];
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    const int cidx = (qk & 1) * 4 + ch;
-                    const uint4 raw = *reinterpret_cast<const uint4*>(qb + i * 128 + ((cidx ^ (i & 7)) << 4));
-                    const uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
-                    float f[8];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        f[2 * e] = sg * __uint_as_float(wds[e] << 16);
-                        f[2 * e + 1] = sg * __uint_as_float(wds[e] & 0xffff0000u);
-                    }
-                    *reinterpret_cast<float4*>(blk + sw128_offset_f32(i, 8 * ch)) = make_float4(f[0], f[1], f[2], f[3]);
-                    *reinterpret_cast<float4*>(blk + sw128_offset_f32(i, 8 * ch + 4)) =
-                        make_float4(f[4], f[5], f[6], f[7]);
-                }
-            }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        // ---- state product and O = sigma diag(gamma) Q S0 of chunk cn (warp 2) at once; [K; Q] K^T
-        //      of chunk cn + 1 (warp 3) once its tiles are in, while warps 0-1 build chunk cn + 1's
-        //      gate factors ----
-        if (warp == 2) {
-            tc_fence_after();
-            if (elect_one()) {
-                const uint64_t dbu = smem_desc_sw128(s_bu, 16, 1024);
-#pragma unroll
-                for (int kk = 0; kk < 16; ++kk)
-                    mma_tf32_ts(tbase + TM_U, tbase + TM_S + kk * 8, desc_advance(dbu, (kk >> 2) * 8192 + (kk & 3) * 32),
-                                id_u, 1u);
-                if (srcn.out) {
-                    const uint64_t dbq = smem_desc_sw128(s_bq, 16, 1024);
-#pragma unroll
-                    for (int kk = 0; kk < 16; ++kk)
-                        mma_tf32_ts(tbase + TM_O, tbase + TM_S + kk * 8,
-                                    desc_advance(dbq, (kk >> 2) * 8192 + (kk & 3) * 32), id_u, kk > 0);
-                }
-                mma_commit(&bar_u);
-            }
-            __syncwarp();
-        }
-        // A full next chunk: warp 3 alone waits for its tiles (the next block-wide barrier
-        // orders them for every later reader).  A partial one: the block zero-pads it first.
-        // A tile timeout still waits for the state product below before the block leaves.
+        // ---- phase Y, chunk cn: U = U' + P^T (-sigma T diag(beta gamma))^T (warp 2); [K; Q] K^T
+        //      of chunk cn + 1 once the P term has read TM_P (warp 3); the gates of chunk cn + 1
+        //      (warps 0-1).  A partial next chunk is zero-padded by the block first. ----
         const bool has_nn = cn + 1 < nchunks;
         const bool nn_partial = has_nn && chunk_src(cn + 1).nc < C;   // uniform
         bool tok = true;
         if (nn_partial) tok = tiles_ready(cn + 1);
-        if (warp == 3) {
-            // the thread that sees the tiles arrive is the one that issues the MMA reading them
-            bool t = true;
+        uint8_t* tile_n = tile_of(cn);
+        const uint32_t s_tile_n = smem_u32(tile_n);
+        if (warp == 2) {
+            tc_fence_after();
+            bool t = tok;
             if (elect_one()) {
-                if (has_nn && !nn_partial) {
+                if (t && st_next) {
+                    t = mbar_wait_bounded(&bar_p, ph_p, kWaitNs);
+                    if (!t) report_timeout(a, 3);
+                }
+                tc_fence_after();
+                if (t && st_next) {
+                    const uint64_t dg = smem_desc_sw128(s_tg, 16, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_tf32_ts(tbase + TM_U, tbase + TM_P + kk * 8, desc_advance(dg, (kk >> 2) * 8192 + (kk & 3) * 32),
+                                    id_t, kk > 0);
+                }
+                mma_commit(&bar_x);
+                if (t) {
+                    const uint64_t da = smem_desc_sw128(s_tile_n + L::V0, L::V_LBO, 1024);
+                    const uint64_t db = smem_desc_sw128(s_tb, 16, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ss(tbase + TM_U, desc_advance(da, kk * 2048), desc_advance(db, kk * 32), id_w,
+                                    (st_next || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(&bar_u);
+            }
+            tok = __all_sync(0xffffffffu, t) && tok;
+        } else if (warp == 3) {
+            bool t = tok;
+            if (elect_one()) {
+                if (t && has_nn && !nn_partial) {
                     t = mbar_wait_bounded(&bar_tile[(cn + 1) & 1], ((cn + 1) >> 1) & 1, kWaitNs);
                     if (!t) report_timeout(a, 1);
                 }
+                if (t && has_nn) {   // the P term is done reading TM_P
+                    t = mbar_wait_bounded(&bar_x, ph_x, kWaitNs);
+                    if (!t) report_timeout(a, 5);
+                }
                 tc_fence_after();
-                if (t && tok && has_nn) issue_kk(cn + 1);
-                mma_commit(&bar_u);
+                if (t && has_nn) issue_kk(cn + 1);
+                if (has_nn) mma_commit(&bar_kk);
             }
             tok = __all_sync(0xffffffffu, t) && tok;
         } else if (warp < 2 && tid < C && has_nn) {
             build_gates(s_gates[(cn + 1) & 1], al_nxt, be_nxt, tid, lane);
         }
         if (has_nn) load_gates(cn + 2, al_nxt, be_nxt);
-        {   // wait_all, with warp 3's tile flag in the same vote
+        {   // U of chunk cn is complete (its MMAs are done with the T operands and the tile)
             const bool okw = mbar_wait_bounded(&bar_u, ph_u, kWaitNs);
             ok = __syncthreads_and(okw && tok) != 0;
             if (!ok && tid == 0) report_timeout(a, 4);
         }
         ph_u ^= 1;
+        ph_x ^= 1;
+        if (st_next) ph_p ^= 1;
     }
 
     // ---- final state: S[dk][dv] = sigma * TMEM[lane dv][dk] ----

@@ -69,80 +69,6 @@ constexpr uint32_t TM_Y = 192;
 
 constexpr uint32_t BAR_CHAIN = 2;   // named barrier of warps 4-7 (the state chain)
 
-// The inverse's emitter (see invert_unit_lower_inplace): each final block of T
-// goes from registers into the two T operands of the chunk,
-//   tb[j][j'] = e_j T[j][j'] beta_j'               (bf16, 128-byte swizzled rows),
-//   tg[j][j'] = -sigma' e_j T[j][j'] beta_j' gamma_j' (fp32, K-major, two 8 KB blocks
-//                                                   of 32 columns, 128-byte swizzled),
-// with e_j = gamma_C / gamma_j and sigma' the state's scale after the chunk before.
-struct TOperandEmit {
-    const Gates* G;
-    float nsig;    // -sigma'
-    uint8_t* tb;   // tg follows at tb + 8192
-    uint64_t* bar_rd;    // null, or the mbarrier of the MMAs still reading tb and tg
-    uint32_t parity;
-    const CallArgs* a;
-    int* abort_flag;
-    __device__ __forceinline__ void prepare() const {
-        if (bar_rd != nullptr && !mbar_wait_bounded(bar_rd, parity, kWaitNs)) {
-            report_timeout(*a, 8);
-            *abort_flag = 1;
-        }
-    }
-    __device__ __forceinline__ static uint32_t off_b(int j, int jj) {
-        return (uint32_t)(j * 128 + (((jj >> 3) ^ (j & 7)) << 4) + (jj & 7) * 2);
-    }
-    __device__ __forceinline__ static uint32_t off_g(int j, int jj) {
-        return (uint32_t)(8192 + (jj >> 5) * 8192 + j * 128 + ((((jj & 31) >> 2) ^ (j & 7)) << 4) + (jj & 3) * 4);
-    }
-    // thread q: row j = 16 (q / 16) + q % 16 of its diagonal block, 16 columns
-    __device__ __forceinline__ void diagonal(const float* AT, int q) const {
-        const int o = (q >> 4) * 16, j = o + (q & 15);
-        const float ej = G->e[j], ejg = nsig * ej;
-        float v[16];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float4 t4 = *reinterpret_cast<const float4*>(AT + j * LDT + o + 4 * k);
-            const float4 b4 = *reinterpret_cast<const float4*>(G->beta + o + 4 * k);
-            const float4 g4 = *reinterpret_cast<const float4*>(G->gam + o + 4 * k);
-            v[4 * k + 0] = t4.x * b4.x;
-            v[4 * k + 1] = t4.y * b4.y;
-            v[4 * k + 2] = t4.z * b4.z;
-            v[4 * k + 3] = t4.w * b4.w;
-            const float4 w4 = make_float4(v[4 * k] * g4.x * ejg, v[4 * k + 1] * g4.y * ejg,
-                                          v[4 * k + 2] * g4.z * ejg, v[4 * k + 3] * g4.w * ejg);
-            *reinterpret_cast<float4*>(tb + off_g(j, o + 4 * k)) = w4;
-        }
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            uint4 x;
-            x.x = pack_bf16(v[8 * hh + 0] * ej, v[8 * hh + 1] * ej);
-            x.y = pack_bf16(v[8 * hh + 2] * ej, v[8 * hh + 3] * ej);
-            x.z = pack_bf16(v[8 * hh + 4] * ej, v[8 * hh + 5] * ej);
-            x.w = pack_bf16(v[8 * hh + 6] * ej, v[8 * hh + 7] * ej);
-            st_shared_v4(tb, off_b(j, o + 8 * hh), x);
-        }
-    }
-    __device__ __forceinline__ void block(int r0, int c0, const float (&acc)[2][4], float scale, int g,
-                                          int t) const {
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            const int jj = c0 + 8 * nt + 2 * t;
-            const float2 b2 = *reinterpret_cast<const float2*>(G->beta + jj);
-            const float2 g2 = *reinterpret_cast<const float2*>(G->gam + jj);
-            const float bg0 = nsig * b2.x * g2.x, bg1 = nsig * b2.y * g2.y;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int j = r0 + g + 8 * hh;
-                const float ej = scale * G->e[j];
-                const float v0 = acc[nt][2 * hh] * ej, v1 = acc[nt][2 * hh + 1] * ej;
-                *reinterpret_cast<uint32_t*>(tb + off_b(j, jj)) = pack_bf16(v0 * b2.x, v1 * b2.y);
-                *reinterpret_cast<float2*>(tb + off_g(j, jj)) = make_float2(v0 * bg0, v1 * bg1);
-            }
-        }
-    }
-};
-
 // ---------------------------------------------------------------------------
 // Tail replay.  Iteration c = 0 .. nchunks (the last one only ends the chain):
 //   phase X  warps 0-3 (front): T = (I + A)^-1 of chunk c (its A was written in
@@ -400,8 +326,8 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             if (has_cur) {
                 // ---- T = (I + A)^-1 of chunk c in place, writing its T operands once the P
                 //      term and U' of chunk c - 1 have read the previous ones ----
-                const TOperandEmit em{&s_gates[c % 3], -sig_c, sm + RL::OFF_TB, has_prev ? &bar_u : nullptr,
-                                      (uint32_t)((c - 1) & 1), &a, &s_abort};
+                const TOperandEmit<true> em{&s_gates[c % 3], -sig_c, sm + RL::OFF_TB, has_prev ? &bar_u : nullptr,
+                                            (uint32_t)((c - 1) & 1), &a, &s_abort};
                 invert_unit_lower_inplace<GDN_INV_SCRATCH_IN_AT>(AT, AT + 32, tid, BAR_INV, em);
                 fence_proxy_async_smem();   // the T operands, for phase Y's MMAs
             }
