@@ -28,8 +28,8 @@ GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT,
     GDN_ERR_ALLOC, GDN_ERR_MISMATCH, GDN_ERR_BOUNDS = range(8)
 GDN_F32, GDN_BF16 = 0, 1
 GDN_KERNEL_AUTO, GDN_KERNEL_RECURRENT, GDN_KERNEL_CHUNKED_TC = 0, 1, 2
-# the chunked kernel with the state-only replay pinned to its two-CTA-per-SM or its
-# warp-specialised kernel, whatever the launch size
+# the chunked kernel with the state-only replay pinned to its two-CTA-per-SM kernel (the
+# default) or to its warp-specialised one
 GDN_KERNEL_CHUNKED_TC_TWO_CTA, GDN_KERNEL_CHUNKED_TC_WARP_SPEC = 3, 4
 
 EXPORTED = (

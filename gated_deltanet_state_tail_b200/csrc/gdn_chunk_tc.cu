@@ -657,30 +657,16 @@ bool make_tile_map(CUtensorMap* m, const void* base, int H, long long rows, long
 
 bool chunk_tc_supported(int dtype, int dk, int dv) { return dtype == 1 && dk == 128 && dv == 128; }
 
-// SMs of the current device, looked up once per device (0 if the query fails).
-static int device_sm_count() {
-    static std::atomic<int> cache[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    int v = cache[dev].load(std::memory_order_relaxed);
-    if (v > 0) return v;
-    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    cache[dev].store(v, std::memory_order_relaxed);
-    return v;
-}
-
 cudaError_t launch_chunk_tc(const CallArgs& a, cudaStream_t stream) {
     if (a.units == 0) return cudaSuccess;
     if (!chunk_tc_supported(a.dtype, a.dk, a.dv)) return cudaErrorInvalidValue;
     // the state-only replay kernels unless outputs are asked for (a prefill, a fused replay
-    // + suffix, or a replay that also emits the window's outputs): with at most one unit
-    // per SM the warp-specialised kernel (one CTA per SM, the front of a unit's chunks
-    // decoupled from its state chain); otherwise the two-chunk kernel, two CTAs per SM
+    // + suffix, or a replay that also emits the window's outputs): the two-CTA-per-SM
+    // kernel, which is the faster one at every launch size measured (one to 296 units);
+    // the warp-specialised kernel (one CTA per SM, the front of a unit's chunks decoupled
+    // from its state chain) only when the descriptor pins it
     if (a.kind == kReplay && a.o_out == nullptr)
-        return (a.replay_variant == kReplayWarpSpec ||
-                (a.replay_variant == kReplayBySize && a.units <= (long long)device_sm_count()))
-                   ? launch_replay_ws(a, stream)
-                   : launch_replay_tc(a, stream);
+        return a.replay_variant == kReplayWarpSpec ? launch_replay_ws(a, stream) : launch_replay_tc(a, stream);
     TcParams p;
     p.a = a;
     // a call with no rows to read (every window empty) still runs, to write the states;

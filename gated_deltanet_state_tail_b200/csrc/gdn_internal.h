@@ -102,14 +102,14 @@ struct CallArgs {
     int replay_variant;     // ReplayVariant: which chunked kernel runs the state-only replay
 };
 
-// The chunked path's state-only replay kernel: chosen by launch size, or pinned by
-// the descriptor's kernel field (GDN_KERNEL_CHUNKED_TC_TWO_CTA / _WARP_SPEC).
-enum ReplayVariant { kReplayBySize = 0, kReplayTwoCta = 1, kReplayWarpSpec = 2 };
+// The chunked path's state-only replay kernel: the two-CTA-per-SM kernel unless the
+// descriptor's kernel field pins the warp-specialised one (GDN_KERNEL_CHUNKED_TC_WARP_SPEC).
+enum ReplayVariant { kReplayDefault = 0, kReplayTwoCta = 1, kReplayWarpSpec = 2 };
 
 inline int replay_variant_of(int kernel) {
     return kernel == GDN_KERNEL_CHUNKED_TC_TWO_CTA    ? kReplayTwoCta
            : kernel == GDN_KERNEL_CHUNKED_TC_WARP_SPEC ? kReplayWarpSpec
-                                                        : kReplayBySize;
+                                                        : kReplayDefault;
 }
 
 // The kernel family a descriptor's kernel field names (the pinned replay variants

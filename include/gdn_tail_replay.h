@@ -74,11 +74,10 @@ typedef enum gdn_dtype { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
 
 /* Kernel selection.  AUTO picks the tensor-core chunked kernel for bf16 with
  * d_k = d_v = 128 and the exact fp32 CUDA-core recurrent kernel otherwise.
- * The chunked path runs the state-only replay on one of two kernels: with at
- * most one (sequence, head) unit per SM a warp-specialised kernel (one CTA per
- * SM), otherwise a kernel with two CTAs per SM.  The last two values pin that
- * choice whatever the launch size (for tests and measurements); every other
- * entry point treats them as GDN_KERNEL_CHUNKED_TC. */
+ * The chunked path has two state-only replay kernels: one with two CTAs per SM
+ * (the one AUTO and GDN_KERNEL_CHUNKED_TC run) and a warp-specialised one with
+ * one CTA per SM.  The last two values pin one of them (for tests and
+ * measurements); every other entry point treats them as GDN_KERNEL_CHUNKED_TC. */
 typedef enum gdn_kernel {
     GDN_KERNEL_AUTO = 0,
     GDN_KERNEL_RECURRENT = 1,              /* token-recurrent, fp32 CUDA cores, any supported shape */

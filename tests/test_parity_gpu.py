@@ -13,8 +13,8 @@ from helpers import TOL, oracle_view, per_request_rows_err, per_request_state_er
 pytestmark = pytest.mark.gpu
 
 # "two_cta" and "warp_spec" run the chunked path with the state-only replay pinned to
-# one of its two kernels (by default the launch size picks: the warp-specialised
-# kernel for at most one unit per SM, which the small cases here are)
+# one of its two kernels (the default, "chunked", is the two-CTA kernel); every other
+# entry point runs the chunked prefill kernel under all three
 KERNELS = {"recurrent": gdn.GDN_KERNEL_RECURRENT, "chunked": gdn.GDN_KERNEL_CHUNKED_TC,
            "two_cta": gdn.GDN_KERNEL_CHUNKED_TC_TWO_CTA, "warp_spec": gdn.GDN_KERNEL_CHUNKED_TC_WARP_SPEC}
 CHUNKED = ("chunked", "two_cta", "warp_spec")

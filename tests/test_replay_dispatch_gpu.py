@@ -1,13 +1,14 @@
-"""The state-only replay's two tensor-core kernels, on each side of the launch
-size that picks between them.
+"""The state-only replay's two tensor-core kernels, each pinned through the
+descriptor, on launches on both sides of one unit per SM.
 
-A replay launch with at most one (request, head) unit per SM runs the
-warp-specialised kernel (one CTA per SM; the state-independent work of a unit's
-chunks runs ahead of its state chain); a larger launch runs the two-chunk kernel
-(two CTAs per SM).  Both launches here replay ragged windows (several 64-token
-chunks and a partial last chunk) and are checked element by element against the
-fp64 oracle on every unit; the units the two launches share must agree within
-the same bound.
+The chunked path runs the replay on a kernel with two CTAs per SM (the default)
+or, when the descriptor pins it, on a warp-specialised kernel with one CTA per
+SM (the front of a unit's chunks runs ahead of its state chain).  Each kernel
+replays the same ragged windows (several 64-token chunks and a partial last
+chunk) on a launch with at most one (request, head) unit per SM and on one with
+more; every unit is checked element by element against the fp64 oracle, the
+default must be the two-CTA kernel bit for bit, and the two kernels must agree
+within the same bound.
 """
 import numpy as np
 import pytest
@@ -23,8 +24,8 @@ pytestmark = pytest.mark.gpu
 H, D = 4, 128
 
 
-def _replay(t, off, ml, R):
-    plan = gdn.ReplayPlan(H, D, D, "bf16", off, ml, R)
+def _replay(t, off, ml, R, kernel):
+    plan = gdn.ReplayPlan(H, D, D, "bf16", off, ml, R, kernel)
     out = torch.full((len(ml), H, D, D), float("nan"), device="cuda")
     plan.run(t["k"], t["v"], t["alpha"], t["beta"], out)
     plan.check()
@@ -45,10 +46,13 @@ def test_both_replay_kernels_around_one_unit_per_sm():
     ref = oracle.replay_state(oracle_view(t["k"]), oracle_view(t["v"]), oracle_view(t["alpha"]),
                               oracle_view(t["beta"]), off, ml, R)
     assert H * b_small <= sms < H * b_large
-    small = _replay(t, off[:b_small + 1], ml[:b_small], R[:b_small])
-    large = _replay(t, off, ml, R)
-    for b in range(b_large):
-        assert rel_err(large[b], ref[b]) <= TOL["bf16"], f"request {b} (two-chunk kernel)"
-    for b in range(b_small):
-        assert rel_err(small[b], ref[b]) <= TOL["bf16"], f"request {b} (warp-specialised kernel)"
-        assert rel_err(small[b], large[b]) <= TOL["bf16"], f"request {b}: the kernels disagree"
+    for nb in (b_small, b_large):
+        o, m, r = off[:nb + 1], ml[:nb], R[:nb]
+        two = _replay(t, o, m, r, gdn.GDN_KERNEL_CHUNKED_TC_TWO_CTA)
+        ws = _replay(t, o, m, r, gdn.GDN_KERNEL_CHUNKED_TC_WARP_SPEC)
+        auto = _replay(t, o, m, r, gdn.GDN_KERNEL_AUTO)
+        assert np.array_equal(auto, two), f"{nb} requests: the default is not the two-CTA kernel"
+        for b in range(nb):
+            assert rel_err(two[b], ref[b]) <= TOL["bf16"], f"{nb} requests, request {b} (two-CTA kernel)"
+            assert rel_err(ws[b], ref[b]) <= TOL["bf16"], f"{nb} requests, request {b} (warp-specialised kernel)"
+            assert rel_err(ws[b], two[b]) <= TOL["bf16"], f"{nb} requests, request {b}: the kernels disagree"
