@@ -431,25 +431,42 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 named_sync(BAR_CHAIN, 128);   // the state update (and O) of chunk c are complete
                 tc_fence_after();
                 if (outc) {
-                    // outputs: stage O as bf16 rows [i][dv] in the UB region, then 16-byte stores of
-                    // whole rows
-                    __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(sm + PL::OFF_UB);
+                    // outputs: stage O as bf16 rows [i][dv] in the UB region (256-byte rows whose
+                    // 16-byte pieces are XOR-swizzled by i % 8), then 16-byte stores of whole rows.
+                    // O^T (lane = value dim dv, column = chunk row i) is read in the 16x256b shape,
+                    // whose registers are the fragments of 8 x 8 blocks [dv][i]; stmatrix .trans
+                    // writes each block as 8 rows i of 8 values dv.
+                    const uint32_t s_stage = smem_u32(sm + PL::OFF_UB);
 #pragma unroll
-                    for (int hf = 0; hf < 2; ++hf) {
-                        float v[32];   // O^T: value dim = row, chunk rows [32 hf, 32 hf + 32)
-                        tmem_ld32(tlane + TM_O + 32 * hf, v);
+                    for (int lh = 0; lh < 2; ++lh) {   // lanes 16 lh .. 16 lh + 15 of the quarter
+                        float v[32];   // register 4k + e: dv = 16 lh + lane/4 + 8 (e/2), i = 8k + 2 (lane%4) + e%2
+                        tmem_ld16x256b_x8(tlane + ((uint32_t)(16 * lh) << 16) + TM_O, v);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int ii = 0; ii < 32; ++ii) stage[(32 * hf + ii) * D + row] = __float2bfloat16_rn(v[ii]);
+                        for (int hf = 0; hf < 2; ++hf) {
+                            const int v0 = 32 * wq + 16 * lh + 8 * hf;   // the blocks' first dv
+#pragma unroll
+                            for (int kg = 0; kg < 2; ++kg) {   // blocks i = 8k.., k = 4 kg + m
+                                uint32_t r[4];
+#pragma unroll
+                                for (int m = 0; m < 4; ++m) {
+                                    const int k = 4 * kg + m;
+                                    r[m] = pack_bf16(v[4 * k + 2 * hf], v[4 * k + 2 * hf + 1]);
+                                }
+                                const int i = 32 * kg + 8 * (lane >> 3) + (lane & 7);   // this lane's row
+                                stmatrix_x4_trans(s_stage + (uint32_t)(i * 256 + (((v0 >> 3) ^ (i & 7)) << 4)), r);
+                            }
+                        }
                     }
                     named_sync(BAR_CHAIN, 128);
+                    const uint8_t* stage = sm + PL::OFF_UB;
                     __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o_out);
 #pragma unroll
                     for (int k = 0; k < (C * D / 8) / 128; ++k) {   // 16-byte pieces: 16 per row
                         const int idx = ct + k * 128, i = idx >> 4, ch = idx & 15;
                         if (i < src.nc && index_ok(a.ws, src.r0 + i < a.rows_total))
                             *reinterpret_cast<uint4*>(o + ((src.r0 + i) * H + h) * (long long)D + ch * 8) =
-                                *reinterpret_cast<const uint4*>(stage + i * D + ch * 8);
+                                *reinterpret_cast<const uint4*>(stage + i * 256 + ((ch ^ (i & 7)) << 4));
                     }
                 }
                 if (fused && c == nA - 1 && a.state_mid) {   // the state at L (chunk c is the window's last)

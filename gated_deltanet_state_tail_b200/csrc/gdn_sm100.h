@@ -339,6 +339,16 @@ __device__ __forceinline__ uint32_t sw128_offset_f32(int row, int col) {
     return (uint32_t)(row * 128 + ((((col >> 2) ^ (row & 7))) << 4) + ((col & 3) << 2));
 }
 
+// Store four 8 x 8 matrices of 16-bit elements to shared memory, transposed
+// (stmatrix .trans): thread t holds in r[m] the elements (row t/4, columns 2 (t%4)
+// and 2 (t%4) + 1) of matrix m; lanes 8m .. 8m + 7 give the 16-byte-aligned
+// addresses of rows 0..7 of matrix m's transpose, i.e. of its columns.
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t saddr, const uint32_t r[4]) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(r[0]),
+                 "r"(r[1]), "r"(r[2]), "r"(r[3])
+                 : "memory");
+}
+
 // Warp-level m16n8k8 tf32 MMA with fp32 accumulate (registers hold tf32
 // bit patterns).  Fragment layout, g = lane / 4, t = lane % 4:
 //   a0 = A[g][t], a1 = A[g+8][t], a2 = A[g][t+4], a3 = A[g+8][t+4]
