@@ -105,14 +105,26 @@ __device__ __forceinline__ void mma16x16_tf32(float acc[2][4], const float* A, i
     }
 }
 
-// Store a 16 x 16 fragment pair (times `scale`) row-major at D (stride ldd).
+// Store a 16 x 16 fragment pair (times `scale`) row-major at D (stride ldd).  WIDE:
+// one 8-byte store per pair of values (ldd even, D 8-byte aligned), which a warp
+// issues as 256 bytes in the minimum two wavefronts, where two 4-byte stores each
+// conflict two ways; it keeps both values live, which a kernel at its register cap
+// pays for in spills.
+template <bool WIDE>
 __device__ __forceinline__ void store16x16(float* D, int ldd, const float acc[2][4], float scale, int g, int t) {
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
-        D[g * ldd + 8 * nt + 2 * t] = scale * acc[nt][0];
-        D[g * ldd + 8 * nt + 2 * t + 1] = scale * acc[nt][1];
-        D[(g + 8) * ldd + 8 * nt + 2 * t] = scale * acc[nt][2];
-        D[(g + 8) * ldd + 8 * nt + 2 * t + 1] = scale * acc[nt][3];
+        if (WIDE) {
+            *reinterpret_cast<float2*>(D + g * ldd + 8 * nt + 2 * t) =
+                make_float2(scale * acc[nt][0], scale * acc[nt][1]);
+            *reinterpret_cast<float2*>(D + (g + 8) * ldd + 8 * nt + 2 * t) =
+                make_float2(scale * acc[nt][2], scale * acc[nt][3]);
+        } else {
+            D[g * ldd + 8 * nt + 2 * t] = scale * acc[nt][0];
+            D[g * ldd + 8 * nt + 2 * t + 1] = scale * acc[nt][1];
+            D[(g + 8) * ldd + 8 * nt + 2 * t] = scale * acc[nt][2];
+            D[(g + 8) * ldd + 8 * nt + 2 * t + 1] = scale * acc[nt][3];
+        }
     }
 }
 
@@ -148,6 +160,8 @@ struct NoEmit {
     __device__ __forceinline__ void block(int, int, const float (&)[2][4], float, int, int) const {}
 };
 
+// SPLIT_K selects the variant for a kernel with registers to spare (one CTA per
+// SM): the products' k-steps in separate accumulators and 8-byte fragment stores.
 template <int LDX, int XHI, int XLO, class Emit = NoEmit, bool SPLIT_K = false>
 __device__ __forceinline__ void invert_unit_lower_inplace(float* AT, float* Xs, int ltid, uint32_t bar_id,
                                                           const Emit& emit = Emit()) {
@@ -197,11 +211,11 @@ __device__ __forceinline__ void invert_unit_lower_inplace(float* AT, float* Xs, 
         const int bo = warp ? 48 : 16, ao = warp ? 32 : 0;   // row block b, column block a
         float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         mma16x16_tf32<SPLIT_K>(acc, AT + bo * LDT + ao, LDT, AT + ao * LDT + ao, LDT, g, t);     // A_ba D_a
-        store16x16(X, LDX, acc, 1.0f, g, t);
+        store16x16<SPLIT_K>(X, LDX, acc, 1.0f, g, t);
         __syncwarp();
         float r[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         mma16x16_tf32<SPLIT_K>(r, AT + bo * LDT + bo, LDT, X, LDX, g, t);                      // D_b (A_ba D_a)
-        store16x16(AT + bo * LDT + ao, LDT, r, -1.0f, g, t);
+        store16x16<SPLIT_K>(AT + bo * LDT + ao, LDT, r, -1.0f, g, t);
         emit.block(bo, ao, r, -1.0f, g, t);
     } else {
         const int r = warp;
@@ -213,8 +227,8 @@ __device__ __forceinline__ void invert_unit_lower_inplace(float* AT, float* Xs, 
     if (warp >= 2) {
         const int r = warp;
         mma16x16_tf32<SPLIT_K>(pr0, AT + 16 * r * LDT + 16, LDT, AT + 16 * LDT, LDT, g, t);      // + A_r1 T_10
-        store16x16(xslot(2 * (r - 2)), LDX, pr0, 1.0f, g, t);
-        store16x16(xslot(2 * (r - 2) + 1), LDX, xr1, 1.0f, g, t);
+        store16x16<SPLIT_K>(xslot(2 * (r - 2)), LDX, pr0, 1.0f, g, t);
+        store16x16<SPLIT_K>(xslot(2 * (r - 2) + 1), LDX, xr1, 1.0f, g, t);
     } else {
         emit.diagonal(AT, ltid);
     }
@@ -231,7 +245,7 @@ __device__ __forceinline__ void invert_unit_lower_inplace(float* AT, float* Xs, 
             mma16x16_tf32<SPLIT_K>(rr, AT + 48 * LDT + 32, LDT, X2c, LDX, g, t);              // T_32 X_2c
             mma16x16_tf32<SPLIT_K>(rr, AT + 48 * LDT + 48, LDT, X3c, LDX, g, t);              // D_3 X_3c
         }
-        store16x16(AT + 16 * r * LDT + 16 * c, LDT, rr, -1.0f, g, t);
+        store16x16<SPLIT_K>(AT + 16 * r * LDT + 16 * c, LDT, rr, -1.0f, g, t);
         emit.block(16 * r, 16 * c, rr, -1.0f, g, t);
     }
     named_sync(bar_id, 128);
