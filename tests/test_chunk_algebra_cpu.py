@@ -273,10 +273,13 @@ def test_renormalisation_is_exercised():
     assert np.sum(np.log2(a)) >= FAST_FLOOR
 
 
-def chunk_algebra_prefill(q, k, v, alpha, beta, S0=None):
-    """The prefill's variant: U stays unscaled (the outputs use it); E and 1/sigma_new
-    are applied to U only for the state update.  Per chunk the outputs are
-    O = sigma diag(gamma) Q (S / sigma) + M U with M_ij = (q_i . k_j) 2^(G_i - G_j), j <= i."""
+def chunk_algebra_prefill(q, k, v, alpha, beta, S0=None, unscaled_output_state_term=False):
+    """The prefill's grouping (the P-form): P = K (S / sigma) from the state entering
+    the chunk, U = T diag(beta) V + (-sigma T diag(beta gamma)) P, unscaled (the
+    outputs use it); E and 1/sigma_new are applied to U only for the state update.
+    Per chunk the outputs are O = (sigma diag(gamma) Q) (S / sigma) + M U with
+    M_ij = (q_i . k_j) 2^(G_i - G_j), j <= i.  A zero entering state skips chunk 0's
+    state terms (P and the outputs' state term), as the kernel does."""
     n, dk = k.shape
     dv = v.shape[1]
     St = np.zeros((dk, dv)) if S0 is None else np.array(S0, dtype=np.float64)
@@ -302,8 +305,14 @@ def chunk_algebra_prefill(q, k, v, alpha, beta, S0=None):
         A = np.tril(bc[:, None] * ratio * (kc @ kc.T), -1)
         Mq = np.tril(ratio * (qc @ kc.T))
         T = np.linalg.inv(np.eye(C) + A)
-        U = (T * bc[None, :]) @ vc - sigma * ((T * (bc * gam)[None, :]) @ kc) @ St
-        O = sigma * (gam[:, None] * qc) @ St + Mq @ U
+        U = (T * bc[None, :]) @ vc
+        O = Mq @ U
+        if c0 > 0 or S0 is not None:
+            P = kc @ St
+            Tg = -sigma * (T * (bc * gam)[None, :])
+            U = U + Tg @ P
+            qs = gam if unscaled_output_state_term else sigma * gam
+            O = (qs[:, None] * qc) @ St + Mq @ U
         o[c0:c0 + m] = O[:m]
         snew = sigma * gam[-1]
         if snew < RENORM_BELOW:
@@ -323,10 +332,27 @@ def test_prefill_chunk_algebra_matches_recurrence(case, n):
     q = g.standard_normal((n, dk))
     q /= np.linalg.norm(q, axis=1, keepdims=True)
     S0 = g.standard_normal((dk, dv))
-    S_ref, o_ref = oracle.recurrence(k, v, a, b, q=q, S0=S0)
-    S, o = chunk_algebra_prefill(q, k, v, a, b, S0=S0)
-    assert np.abs(S - S_ref).max() / np.abs(S_ref).max() <= 1e-10
-    assert np.abs(o - o_ref).max() / np.abs(o_ref).max() <= 1e-10
+    for s0 in (S0, None):
+        S_ref, o_ref = oracle.recurrence(k, v, a, b, q=q, S0=s0)
+        S, o = chunk_algebra_prefill(q, k, v, a, b, S0=s0)
+        assert np.abs(S - S_ref).max() / np.abs(S_ref).max() <= 1e-10
+        assert np.abs(o - o_ref).max() / np.abs(o_ref).max() <= 1e-10
+
+
+def test_prefill_output_state_term_needs_sigma():
+    """Planted mistake: the outputs' state term built from gamma Q instead of sigma gamma Q
+    (the bf16 copy holds S / sigma, so sigma must come with Q)."""
+    dk, dv, n = 16, 8, 150
+    k, v, a, b = _inputs(n, dk, dv, "normal", seed=9)
+    g = np.random.default_rng(10)
+    q = g.standard_normal((n, dk))
+    S0 = g.standard_normal((dk, dv))
+    _, o_ref = oracle.recurrence(k, v, a, b, q=q, S0=S0)
+    _, good = chunk_algebra_prefill(q, k, v, a, b, S0=S0)
+    _, bad = chunk_algebra_prefill(q, k, v, a, b, S0=S0, unscaled_output_state_term=True)
+    scale = np.abs(o_ref).max()
+    assert np.abs(good - o_ref).max() / scale <= 1e-10
+    assert np.abs(bad - o_ref).max() / scale > 1e-3
 
 
 def blocked_unit_lower_inverse(A):
