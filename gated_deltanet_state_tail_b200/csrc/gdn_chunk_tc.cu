@@ -17,22 +17,26 @@
 //   U    = U' - W S0
 //   S_C  = gamma_C S0 + K^T diag(gamma_C / gamma) U
 //   O    = diag(gamma) Q S0 + (tril(Q K^T) * exp(G_i - G_j)) U
-// Every chunk contraction is a tcgen05.mma with M = 128 (the key or value
-// dimension, or the 64 chunk rows of K stacked on 64 rows of Q/V) and
-// accumulators in TMEM.  The state lives in TMEM transposed (lane = value
-// row) as S / sigma with a running scalar sigma, so the state-dependent
-// product U' - W S reads it straight from TMEM as a tf32 operand and the
-// decay costs no pass over the state (sigma is folded back only when it gets
-// small).  T is built from 16 x 16 diagonal inverses on CUDA cores and
-// warp-level tf32 tensor-core products for the blocks below the diagonal.
+// This kernel groups the state term through P = K (S0 / sigma):
+//   U = U' - sigma (T diag(beta gamma)) P,   O = (sigma diag(gamma) Q) (S0 / sigma) + M U
+// Every chunk contraction is a tcgen05.mma with M = 128 (the value dimension,
+// or the 64 chunk rows of K stacked on 64 rows of Q) and accumulators in TMEM.
+// The state lives in TMEM transposed (lane = value row) as S / sigma with a
+// running scalar sigma, so the decay costs no pass over the state (sigma is
+// folded back only when it gets small).  After each state update a bf16 copy
+// of S / sigma goes into TMEM, the A operand of P and of the outputs' state
+// term; the P term reads P from TMEM as a tf32 operand.  T is built from
+// 16 x 16 diagonal inverses on CUDA cores and warp-level tf32 tensor-core
+// products for the blocks below the diagonal, and the inverse writes the T
+// operands as its blocks become final.
 //
 // Work: one CTA of 8 warps per (sequence, head) unit, chunks in order, two in
 // flight: warps 0-3 build A and M of chunk c + 1 and invert T while warps 4-7
-// finish chunk c (its state update, outputs and the next tile prefetch).
-// Warps w and w + 4 share TMEM lane quarter w (the only lanes a warp may
-// read).  prefill_pipe_kernel runs the prefill with outputs and the fused
-// replay + suffix (the replay window's chunks first, without outputs):
-// 192 KB of shared memory, 512 TMEM columns, one CTA per SM.
+// finish chunk c (its state update, outputs and the next tile prefetch) and
+// form P of chunk c + 1.  Warps w and w + 4 share TMEM lane quarter w (the only
+// lanes a warp may read).  prefill_pipe_kernel runs the prefill with outputs
+// and the fused replay + suffix (the replay window's chunks first, without
+// outputs): 185 KB of shared memory, 448 of 512 TMEM columns, one CTA per SM.
 #include <atomic>
 
 #include <cuda.h>

@@ -1,6 +1,8 @@
 // gdn_replay_ws.cu -- the state-only tail replay on tcgen05 tensor cores with
 // warp-specialised roles (bf16 k/v, d_k = d_v = 128, fp32 state in tensor
-// memory), one CTA per SM.
+// memory), one CTA per SM.  Plans run it only when the descriptor pins it
+// (GDN_KERNEL_CHUNKED_TC_WARP_SPEC); by default every replay runs the
+// two-CTA-per-SM kernel of gdn_replay.cu, which is faster at every launch size.
 //
 // Tail-Replay ("Tail-Replay: Escaping the Curse of Linear Attention in
 // Prefix Caching for Hybrid LLMs", section "Mecanismos Principais", item
