@@ -134,7 +134,7 @@ __device__ __forceinline__ void store16x16(float* D, int ldd, const float acc[2]
 // triangles of the diagonal blocks are written as zeros; the blocks above
 // them are left untouched and must be read as zero).  Xs holds the merges'
 // four 16 x 16 scratch blocks: block s at Xs + (s / 2) XHI + (s % 2) XLO, row
-// stride LDX (see the placements below).
+// stride LDX (see GDN_INV_SCRATCH_IN_AT below).
 //
 // Diagonal blocks: forward substitution on CUDA cores, warp w solves block w
 // with one lane per column.  Then recursive doubling with
@@ -251,64 +251,9 @@ __device__ __forceinline__ void invert_unit_lower_inplace(float* AT, float* Xs, 
     named_sync(bar_id, 128);
 }
 
-// The scratch placements of the inverse: a separate buffer of four 16 x 24
-// blocks, or the upper-right 32 x 32 quarter of AT itself (rows 0-31, columns
-// 32-63), which neither A nor T uses.
-#define GDN_INV_SCRATCH_SEPARATE 24, 2 * 16 * 24, 16 * 24
+// The inverse's scratch placement: the upper-right 32 x 32 quarter of AT itself
+// (rows 0-31, columns 32-63), which neither A nor T uses; pass AT + 32 as Xs.
 #define GDN_INV_SCRATCH_IN_AT LDT, 16 * LDT, 16
-
-// From the inverse T (in place in AT, see above) write the bf16 operands
-// T diag(beta) -> tb and T diag(beta gamma) -> tbg, [j][j'] in 128-byte
-// swizzled rows, with NTH threads (ltid < NTH) sharing barrier bar_id (the
-// prefill's W and U' operands).  beta and gam are 16-byte aligned.  tb / tbg
-// overlap AT, so every thread reads its values before a barrier and writes
-// after it.
-template <int NTH>
-__device__ __forceinline__ void write_scaled_t(const float* AT, const float* beta, const float* gam,
-                                               uint8_t* tb, uint8_t* tbg, int ltid, uint32_t bar_id) {
-    constexpr int PER = C * C / NTH;   // values of one row per thread
-    constexpr int TPR = C / PER;       // threads per row
-    static_assert(PER % 8 == 0 && TPR * PER == C, "whole 16-byte chunks per thread");
-    // thread -> (row j, column part): consecutive threads take consecutive rows, so
-    // the fp32 row loads (stride LDT) and the swizzled bf16 row stores are both
-    // free of bank conflicts, and a warp reads one set of gate factors
-    const int j = ltid % C, part = ltid / C;
-    float vb[PER], vbg[PER];
-#pragma unroll
-    for (int q = 0; q < PER; q += 4) {
-        const int col = part * PER + q;
-        float4 tt = make_float4(0.f, 0.f, 0.f, 0.f);
-        if ((col >> 4) <= (j >> 4)) tt = *reinterpret_cast<const float4*>(AT + j * LDT + col);
-        const float4 b4 = *reinterpret_cast<const float4*>(beta + col);
-        const float4 g4 = *reinterpret_cast<const float4*>(gam + col);
-        const float tv[4] = {tt.x, tt.y, tt.z, tt.w};
-        const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
-        const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float x = tv[e] * bv[e];
-            vb[q + e] = x;
-            vbg[q + e] = x * gv[e];
-        }
-    }
-    named_sync(bar_id, NTH);
-#pragma unroll
-    for (int ch = 0; ch < PER / 8; ++ch) {
-        const int chunk = part * (PER / 8) + ch;
-        uint4 x, y;
-        x.x = pack_bf16(vb[ch * 8 + 0], vb[ch * 8 + 1]);
-        x.y = pack_bf16(vb[ch * 8 + 2], vb[ch * 8 + 3]);
-        x.z = pack_bf16(vb[ch * 8 + 4], vb[ch * 8 + 5]);
-        x.w = pack_bf16(vb[ch * 8 + 6], vb[ch * 8 + 7]);
-        y.x = pack_bf16(vbg[ch * 8 + 0], vbg[ch * 8 + 1]);
-        y.y = pack_bf16(vbg[ch * 8 + 2], vbg[ch * 8 + 3]);
-        y.z = pack_bf16(vbg[ch * 8 + 4], vbg[ch * 8 + 5]);
-        y.w = pack_bf16(vbg[ch * 8 + 6], vbg[ch * 8 + 7]);
-        const uint32_t off = (uint32_t)(j * 128 + ((chunk ^ (j & 7)) << 4));
-        st_shared_v4(tb, off, x);
-        st_shared_v4(tbg, off, y);
-    }
-}
 
 // ---------------------------------------------------------------- kernel building blocks
 // Shared by the replay and prefill kernels of the chunked tensor-core path.
