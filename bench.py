@@ -1056,43 +1056,49 @@ def bench_overlap(args):
 
 
 def bench_fused(args):
-    """The 24-layer cache hit as 3 fused launches (replay window then suffix, 8 layers each)
-    against the 3 replay + 3 prefill launches of the bench line."""
+    """Fused replay + suffix calls against separate replay and prefill launches, on the
+    24-layer cache hit (3 calls of 8 layers; 256 units and 3277-token windows, so each fused
+    call runs as a replay launch then a prefill launch) and on the one-layer 8K prefix at 5%
+    (16 units, 410-token windows: one launch)."""
     import gated_deltanet_state_tail_b200 as gdn
-    wl = inputs.stack_workload(24)
-    data = StackData(wl, "cuda", compact=True)
-    rp, pp, state, o, st_out, _ = build_stack_runner(data, gdn.GDN_KERNEL_AUTO)
-    fp = []
-    for slots in data.launches:
-        off, ml, R = data.replay_desc(slots)
-        fp.append(gdn.FusedPlan(wl.H, wl.dk, wl.dv, wl.dtype, off, ml, R, data.suffix_cu(slots)))
-    per = data.per_launch
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
-    mid = torch.empty_like(state)
+    lines = []
+    for wl in (inputs.stack_workload(24), inputs.single_layer_workload()):
+        data = StackData(wl, "cuda", compact=True)
+        rp, pp, state, o, st_out, _ = build_stack_runner(data, gdn.GDN_KERNEL_AUTO)
+        fp = []
+        for slots in data.launches:
+            off, ml, R = data.replay_desc(slots)
+            fp.append(gdn.FusedPlan(wl.H, wl.dk, wl.dv, wl.dtype, off, ml, R, data.suffix_cu(slots)))
+        per = data.per_launch
+        flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+        mid = torch.empty_like(state)
 
-    def separate():
-        run_step(data, rp, pp, state, o, st_out)
+        def separate():
+            run_step(data, rp, pp, state, o, st_out)
 
-    def fused():
-        for j, plan in enumerate(fp):
-            sl = slice(j * per, (j + 1) * per)
-            plan.run(data.k, data.v, data.alpha, data.beta, data.sq, data.sk, data.sv, data.sa, data.sb, o,
-                     st_out[sl], state_mid=mid[sl])
+        def fused():
+            for j, plan in enumerate(fp):
+                sl = slice(j * per, (j + 1) * per)
+                plan.run(data.k, data.v, data.alpha, data.beta, data.sq, data.sk, data.sv, data.sa, data.sb, o,
+                         st_out[sl], state_mid=mid[sl])
 
-    for _ in range(args.warmup):
-        separate()
-        fused()
-    sep_ms = _time_ms(separate, 10, flush)
-    ref = st_out.clone()
-    fused_ms = _time_ms(fused, 10, flush)
-    rel = float(((st_out - ref).norm() / ref.norm()).item())
-    for p in rp + pp + fp:
-        p.check()
-        p.close()
-    return [{"metric": "fused replay + suffix prefill", "workload": wl.name, "layers": wl.layers,
-             "separate_ms": sep_ms, "fused_ms": fused_ms, "launches_separate": 2 * len(data.launches),
-             "launches_fused": len(data.launches), "final_state_rel_diff_fused_vs_separate": rel,
-             "dtype": "bf16", "data": "synthetic"}]
+        for _ in range(args.warmup):
+            separate()
+            fused()
+        sep_ms = _time_ms(separate, 10, flush)
+        ref = st_out.clone()
+        fused_ms = _time_ms(fused, 10, flush)
+        rel = float(((st_out - ref).norm() / ref.norm()).item())
+        launches_fused = sum(p.launches for p in fp)
+        for p in rp + pp + fp:
+            p.check()
+            p.close()
+        lines.append({"metric": "fused replay + suffix prefill", "workload": wl.name, "layers": wl.layers,
+                      "separate_ms": sep_ms, "fused_ms": fused_ms, "launches_separate": 2 * len(data.launches),
+                      "launches_fused": launches_fused, "final_state_rel_diff_fused_vs_separate": rel,
+                      "dtype": "bf16", "data": "synthetic"})
+        del data, state, o, st_out, mid, flush
+    return lines
 
 
 # --------------------------------------------------------------------------

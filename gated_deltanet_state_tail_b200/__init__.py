@@ -35,7 +35,7 @@ GDN_KERNEL_CHUNKED_TC_TWO_CTA, GDN_KERNEL_CHUNKED_TC_WARP_SPEC = 3, 4
 EXPORTED = (
     "gdn_plan_create_replay", "gdn_plan_create_prefill", "gdn_plan_destroy", "gdn_replay_windows",
     "gdn_plan_window",
-    "gdn_plan_info", "gdn_workspace_bytes", "gdn_tail_replay_state", "gdn_chunk_prefill",
+    "gdn_plan_info", "gdn_plan_launches", "gdn_workspace_bytes", "gdn_tail_replay_state", "gdn_chunk_prefill",
     "gdn_workspace_status", "gdn_status_string", "gdn_version", "gdn_tail_replay_state_noalloc",
     "gdn_tail_replay_outputs", "gdn_decode_step", "gdn_plan_create_fused", "gdn_tail_replay_prefill",
     "gdn_selftest_bounded_wait", "gdn_debug_fail_plan_allocations", "gdn_selftest_index_check",
@@ -77,6 +77,7 @@ def _load():
         "gdn_replay_windows": (I32, [I32, P, P, P, P, P]),
         "gdn_plan_window": (I32, [P, I32, ctypes.POINTER(I64), ctypes.POINTER(I32)]),
         "gdn_plan_info": (I32, [P, ctypes.POINTER(I64), ctypes.POINTER(I64), ctypes.POINTER(I32)]),
+        "gdn_plan_launches": (I32, [P, ctypes.POINTER(I32)]),
         "gdn_workspace_bytes": (ctypes.c_size_t, [P]),
         "gdn_tail_replay_state": (I32, [P, P, P, P, P, P, P, P, P, P, P, P]),
         "gdn_chunk_prefill": (I32, [P, P, P, P, P, P, P, P, P, P, P, P]),
@@ -248,6 +249,12 @@ def gdn_plan_info(handle):
     return {"units": u.value, "total_tokens": t.value, "kernel": k.value}
 
 
+def gdn_plan_launches(handle) -> int:
+    n = ctypes.c_int32()
+    _check(_lib.gdn_plan_launches(handle, ctypes.byref(n)), "gdn_plan_launches")
+    return n.value
+
+
 def gdn_workspace_bytes(handle) -> int:
     return int(_lib.gdn_workspace_bytes(handle))
 
@@ -349,6 +356,7 @@ class _Plan:
         import torch
         self.handle, self.H, self.dk, self.dv, self.dtype, self.batch = handle, H, dk, dv, dtype, batch
         self.info = gdn_plan_info(handle)
+        self.launches = gdn_plan_launches(handle)   # kernel launches per call
         self.workspace = torch.zeros(gdn_workspace_bytes(handle), dtype=torch.uint8, device="cuda")
 
     def window(self, b):

@@ -26,6 +26,7 @@ struct gdn_plan {
     int kind;
     int batch, num_heads, dk, dv, dtype, kernel;
     int replay_variant;       // gdn::ReplayVariant (chunked kernel, state-only replay)
+    bool fused_one_launch;    // fused plan, chunked kernel: the windows and the suffix in one launch
     long long rs_qk, rs_v;    // row strides (elements) of q/k and of v
     int device;
     std::vector<Window> windows;   // replay: the tail windows; prefill and fused: the (suffix) sequences
@@ -96,6 +97,33 @@ int resolve_kernel(const gdn_varlen_desc* d) {
                                                               : GDN_KERNEL_RECURRENT;
 }
 
+// Longest replay window (tokens) that a fused call on the chunked kernel still runs as one
+// launch.  One launch keeps the state on chip between the window and the suffix and saves a
+// launch, but its window chunks run on the one-CTA-per-SM prefill kernel, slower per chunk
+// than the two-CTA state-only replay kernel.  Measured on B200 (bf16, d = 128, 512-token
+// suffix): with at most one unit per SM, one launch is 2-12 us faster up to 13 chunks, within
+// 2 us either way at 20 and up to 28 us slower at 52; with more units than SMs, two launches
+// win from 7 chunks on.
+constexpr int kFusedOneLaunchMaxTokens = 16 * 64;
+
+// A fused plan on the chunked kernel runs as one launch when every (sequence, head) unit has
+// an SM of its own and no window is longer than kFusedOneLaunchMaxTokens; otherwise as the
+// state-only replay launch followed by the prefill launch.  A descriptor that pins a replay
+// kernel always takes the two launches.
+gdn_status choose_fused_schedule(gdn_plan* p) {
+    p->fused_one_launch = false;
+    if (p->kernel != GDN_KERNEL_CHUNKED_TC || p->replay_variant != gdn::kReplayDefault) return GDN_OK;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, p->device) != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_CUDA;
+    }
+    int longest = 0;
+    for (const Window& w : p->windows0) longest = std::max(longest, (int)w.len);
+    p->fused_one_launch = (long long)p->batch * p->num_heads <= sms && longest <= kFusedOneLaunchMaxTokens;
+    return GDN_OK;
+}
+
 gdn_status finish_plan(gdn_plan* p, gdn_plan_t* out) {
     // Work units: every (sequence, head); longest window first so the long
     // units start early and the short ones fill the tail of the grid.
@@ -122,6 +150,10 @@ gdn_status finish_plan(gdn_plan* p, gdn_plan_t* out) {
     // an injected failure stands where the device allocation would fail
     if (take_injected_alloc_failure()) return GDN_ERR_ALLOC;
     if (cudaGetDevice(&p->device) != cudaSuccess) return GDN_ERR_CUDA;
+    if (p->kind == gdn::kFused) {
+        const gdn_status s = choose_fused_schedule(p);
+        if (s != GDN_OK) return s;
+    }
     const size_t wbytes = sizeof(Window) * p->windows.size();
     const size_t w0bytes = sizeof(Window) * p->windows0.size();
     const size_t ubytes = sizeof(Unit) * p->units.size();
@@ -169,6 +201,7 @@ gdn_plan* new_plan(const gdn_varlen_desc* d, int kind) {
     p->replay_variant = gdn::replay_variant_of(d->kernel);
     p->rs_qk = gdn::row_stride_qk(d);
     p->rs_v = gdn::row_stride_v(d);
+    p->fused_one_launch = false;
     p->dev_block = nullptr;
     p->d_windows0 = nullptr;
     return p;
@@ -360,6 +393,12 @@ gdn_status gdn_plan_info(gdn_plan_t plan, int64_t* units, int64_t* total_tokens,
     return GDN_OK;
 }
 
+gdn_status gdn_plan_launches(gdn_plan_t plan, int32_t* launches) {
+    if (!plan || !launches) return GDN_ERR_INVALID_ARG;
+    *launches = plan->kind == gdn::kFused && !plan->fused_one_launch ? 2 : 1;
+    return GDN_OK;
+}
+
 size_t gdn_workspace_bytes(gdn_plan_t plan) {
     (void)plan;
     return sizeof(WorkspaceHeader);
@@ -519,7 +558,7 @@ gdn_status gdn_tail_replay_prefill(gdn_plan_t plan, const void* k, const void* v
     CallArgs a;
     std::memset(&a, 0, sizeof a);
     fill_common(plan, a, workspace);
-    if (plan->kernel == GDN_KERNEL_CHUNKED_TC) {
+    if (plan->fused_one_launch) {
         // one launch: window chunks, then suffix chunks, the state kept on chip
         a.kind = gdn::kFused;
         a.q = sq;
@@ -538,7 +577,9 @@ gdn_status gdn_tail_replay_prefill(gdn_plan_t plan, const void* k, const void* v
         a.state_mid = state_mid;
         return launch(plan, a, st);
     }
-    // the exact fp32 recurrent kernel: the same results as a replay launch then a prefill launch
+    // two launches, one status reset for both: the state-only replay of the windows into
+    // state_mid (or state_out), then the prefill of the suffix from that state
+    auto run = plan->kernel == GDN_KERNEL_CHUNKED_TC ? gdn::launch_chunk_tc : gdn::launch_recurrent;
     if (cudaMemsetAsync(a.ws, 0, sizeof(WorkspaceHeader), st) != cudaSuccess) {
         cudaGetLastError();
         return GDN_ERR_CUDA;
@@ -552,7 +593,7 @@ gdn_status gdn_tail_replay_prefill(gdn_plan_t plan, const void* k, const void* v
     a.alpha = alpha;
     a.beta = beta;
     a.state_out = mid;
-    if (gdn::launch_recurrent(a, st) != cudaSuccess) {
+    if (run(a, st) != cudaSuccess) {
         cudaGetLastError();
         return GDN_ERR_CUDA;
     }
@@ -566,7 +607,7 @@ gdn_status gdn_tail_replay_prefill(gdn_plan_t plan, const void* k, const void* v
     a.state_in = mid;
     a.o_out = o_out;
     a.state_out = state_out;
-    if (gdn::launch_recurrent(a, st) != cudaSuccess) {
+    if (run(a, st) != cudaSuccess) {
         cudaGetLastError();
         return GDN_ERR_CUDA;
     }

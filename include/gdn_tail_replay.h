@@ -169,6 +169,12 @@ GDN_API gdn_status gdn_plan_window(gdn_plan_t plan, int32_t b, int64_t* row0, in
 GDN_API gdn_status gdn_plan_info(gdn_plan_t plan, int64_t* units, int64_t* total_tokens,
                          int32_t* kernel);
 
+/* Kernel launches that one call on this plan makes: 1 for a replay or a
+ * prefill plan; 1 or 2 for a fused plan (see gdn_tail_replay_prefill).  The
+ * workspace status reset each call does first is a memset, not counted.
+ * INVALID_ARG for a NULL plan or pointer. */
+GDN_API gdn_status gdn_plan_launches(gdn_plan_t plan, int32_t* launches);
+
 /* Bytes of device workspace a call on this plan needs (>= 256, multiple of
  * 256).  The caller allocates it (16-byte aligned) and passes it to each
  * call; calls running concurrently need separate workspaces. */
@@ -264,9 +270,14 @@ GDN_API gdn_status gdn_chunk_prefill(gdn_plan_t plan, const void* q, const void*
 /*
  * Fused rebuild + suffix prefill on a fused plan: equal (up to rounding
  * order) to gdn_tail_replay_state followed by gdn_chunk_prefill from the
- * rebuilt states.  With the tensor-core kernel it is one launch and the
- * state never leaves the chip between the two phases; the fp32 recurrent
- * kernel runs it as those two launches.
+ * rebuilt states.  The plan fixes how it runs.  On the tensor-core kernel,
+ * when the plan has no more (sequence, head) units than the GPU has SMs and
+ * no replay window is longer than 1024 tokens, it is one launch and the
+ * state stays on chip between the two phases.  Otherwise, on that kernel
+ * with a replay kernel pinned, and on the fp32 recurrent kernel, it is a
+ * state-only replay launch writing state_mid (or state_out) and a prefill
+ * launch reading it back: longer windows replay faster on the replay
+ * kernel than inside the one-launch kernel.  gdn_plan_launches tells which.
  *   k, v, alpha, beta        the cache rows (as for the replay).
  *   sq, sk, sv, salpha, sbeta
  *                            the suffix rows (as for the prefill).

@@ -32,6 +32,14 @@ def test_every_declared_symbol_is_exported():
     assert set(gdn.EXPORTED) <= names
 
 
+def test_plan_launches_rejects_null():
+    lib = gdn.library()
+    n = ctypes.c_int32(-1)
+    assert lib.gdn_plan_launches(None, ctypes.byref(n)) == gdn.GDN_ERR_INVALID_ARG
+    assert n.value == -1
+    assert lib.gdn_plan_launches(ctypes.c_void_p(1), None) == gdn.GDN_ERR_INVALID_ARG
+
+
 def test_version_and_status_strings():
     assert gdn.gdn_version() >= 100
     for s in range(8):
