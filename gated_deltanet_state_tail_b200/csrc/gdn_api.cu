@@ -49,6 +49,13 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 namespace gdn {
 
+unsigned int next_call_number() {
+    static std::atomic<unsigned int> counter{0};
+    unsigned int n = counter.fetch_add(1, std::memory_order_relaxed) + 1;
+    while (n == 0) n = counter.fetch_add(1, std::memory_order_relaxed) + 1;   // 0 is never a call number
+    return n;
+}
+
 gdn_status check_varlen_desc(const gdn_varlen_desc* d) {
     if (!d || !d->seq_offsets_host) return GDN_ERR_INVALID_ARG;
     if (d->batch < 1 || d->num_heads < 1) return GDN_ERR_INVALID_ARG;
@@ -247,10 +254,6 @@ gdn_status check_call_common(gdn_plan_t plan, void* workspace) {
 }
 
 gdn_status launch(gdn_plan_t plan, CallArgs& a, cudaStream_t stream) {
-    if (cudaMemsetAsync(a.ws, 0, sizeof(WorkspaceHeader), stream) != cudaSuccess) {
-        cudaGetLastError();
-        return GDN_ERR_CUDA;
-    }
     cudaError_t e = plan->kernel == GDN_KERNEL_CHUNKED_TC ? gdn::launch_chunk_tc(a, stream)
                                                           : gdn::launch_recurrent(a, stream);
     if (e != cudaSuccess) {
@@ -274,6 +277,7 @@ void fill_common(gdn_plan_t plan, CallArgs& a, void* workspace) {
     a.windows = plan->d_windows;
     a.unit_list = plan->d_units;
     a.ws = static_cast<WorkspaceHeader*>(workspace);
+    a.epoch = gdn::next_call_number();
     a.replay_variant = plan->replay_variant;
 }
 
@@ -577,13 +581,9 @@ gdn_status gdn_tail_replay_prefill(gdn_plan_t plan, const void* k, const void* v
         a.state_mid = state_mid;
         return launch(plan, a, st);
     }
-    // two launches, one status reset for both: the state-only replay of the windows into
+    // two launches under one call number: the state-only replay of the windows into
     // state_mid (or state_out), then the prefill of the suffix from that state
     auto run = plan->kernel == GDN_KERNEL_CHUNKED_TC ? gdn::launch_chunk_tc : gdn::launch_recurrent;
-    if (cudaMemsetAsync(a.ws, 0, sizeof(WorkspaceHeader), st) != cudaSuccess) {
-        cudaGetLastError();
-        return GDN_ERR_CUDA;
-    }
     float* mid = state_mid ? state_mid : state_out;
     a.kind = gdn::kReplay;
     a.windows = plan->d_windows0;
@@ -597,7 +597,9 @@ gdn_status gdn_tail_replay_prefill(gdn_plan_t plan, const void* k, const void* v
         cudaGetLastError();
         return GDN_ERR_CUDA;
     }
+    const unsigned int call = a.epoch;
     fill_common(plan, a, workspace);
+    a.epoch = call;
     a.kind = gdn::kPrefill;
     a.q = sq;
     a.k = sk;
@@ -621,11 +623,12 @@ gdn_status gdn_workspace_status(const void* workspace, void* stream) {
         cudaGetLastError();
         return GDN_ERR_CUDA;
     }
-    unsigned int status = 0;
-    if (cudaMemcpy(&status, workspace, sizeof status, cudaMemcpyDeviceToHost) != cudaSuccess) {
+    WorkspaceHeader h;
+    if (cudaMemcpy(&h, workspace, sizeof h, cudaMemcpyDeviceToHost) != cudaSuccess) {
         cudaGetLastError();
         return GDN_ERR_CUDA;
     }
+    const unsigned int status = gdn::header_status(h);
     if (status & gdn::kStatusTimeout) return GDN_ERR_TIMEOUT;
     if (status & gdn::kStatusBounds) return GDN_ERR_BOUNDS;
     if (status & gdn::kStatusMismatch) return GDN_ERR_MISMATCH;

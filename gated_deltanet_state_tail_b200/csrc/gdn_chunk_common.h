@@ -56,8 +56,8 @@ __device__ __forceinline__ void write_row32_bf16(uint8_t* tile, int row, int c0,
 }
 
 __device__ __forceinline__ void report_timeout(const CallArgs& a, uint32_t where) {
-    atomicOr(&a.ws->status, kStatusTimeout);
-    atomicCAS(&a.ws->timeout_where, 0u, where);
+    report_status(a, kStatusTimeout);
+    tag_merge(&a.ws->where, a.epoch, where, true);
 }
 
 // acc[nt] += A (16 x 16) * B (16 x 16), nt = two 8-column halves of the result;

@@ -104,13 +104,14 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     __shared__ Gates s_gates[2];    // chunk c uses s_gates[c & 1]
 
     const CallArgs& a = p.a;
+    record_call(a);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wq = warp & 3, wh = warp >> 2;
     const int row = wq * 32 + lane;
     const Unit u = a.unit_list[blockIdx.x];
     const int b = u.seq, h = u.head, H = a.num_heads;
     if (!window_agrees(a, b)) {
-        if (tid == 0) atomicOr(&a.ws->status, kStatusMismatch);
+        if (tid == 0) report_status(a, kStatusMismatch);
         return;
     }
     // Chunk stream of this unit: the fused call's replay window first (cache rows, no
@@ -124,7 +125,7 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     const int nA = (w0.len + C - 1) / C;
     const int nchunks = nA + (w.len + C - 1) / C;
     // debug build: the unit and its row ranges lie inside the plan's extents (uniform)
-    if (!index_ok(a.ws, b >= 0 && b < a.batch && h >= 0 && h < H && w.row0 >= 0 && w.len >= 0 &&
+    if (!index_ok(a, b >= 0 && b < a.batch && h >= 0 && h < H && w.row0 >= 0 && w.len >= 0 &&
                             w.row0 + w.len <= a.rows_total && w0.row0 >= 0 && w0.len >= 0 &&
                             w0.row0 + w0.len <= (fused ? a.rows_total0 : 0)))
         return;
@@ -224,7 +225,7 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 const float* pa = cc < nA ? a.alpha0 : a.alpha;
                 const float* pb = cc < nA ? a.beta0 : a.beta;
                 const long long r = cs.r0 + tid;
-                if (index_ok(a.ws, r < (cc < nA ? a.rows_total0 : a.rows_total))) {
+                if (index_ok(a, r < (cc < nA ? a.rows_total0 : a.rows_total))) {
                     al = pa[r * H + h];
                     be = pb[r * H + h];
                 }
@@ -468,7 +469,7 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
 #pragma unroll
                     for (int k = 0; k < (C * D / 8) / 128; ++k) {   // 16-byte pieces: 16 per row
                         const int idx = ct + k * 128, i = idx >> 4, ch = idx & 15;
-                        if (i < src.nc && index_ok(a.ws, src.r0 + i < a.rows_total))
+                        if (i < src.nc && index_ok(a, src.r0 + i < a.rows_total))
                             *reinterpret_cast<uint4*>(o + ((src.r0 + i) * H + h) * (long long)D + ch * 8) =
                                 *reinterpret_cast<const uint4*>(stage + i * 256 + ((ch ^ (i & 7)) << 4));
                     }

@@ -33,17 +33,54 @@ struct Unit {
     int head;
 };
 
-// Per-call device scratch at the start of the caller's workspace.
+// Per-call device status at the start of the caller's workspace.  Nothing clears
+// it between calls.  Each call carries a nonzero call number (CallArgs::epoch);
+// every report tags a word with that number, dropping whatever an earlier number
+// left in it, and the first thread of each launch records the number in `epoch`.
+// A reader counts only the words whose tag equals that record (header_status), so
+// no reset has to run on the stream ahead of the kernel.
 struct WorkspaceHeader {
-    unsigned int status;        // bit set of kStatus*
-    unsigned int timeout_where; // first wait that gave up (kernel-defined code)
-    unsigned int pad[62];
+    unsigned long long status;  // (call number << 32) | kStatus* bits reported under it
+    unsigned long long where;   // (call number << 32) | first wait that gave up (kernel-defined code)
+    unsigned int epoch;         // call number of the last launch on this workspace
+    unsigned int pad[59];
 };
 static_assert(sizeof(WorkspaceHeader) == 256, "header is 256 bytes");
 
 constexpr unsigned int kStatusMismatch = 1u;
 constexpr unsigned int kStatusTimeout = 2u;
 constexpr unsigned int kStatusBounds = 4u;   // a checked index fell outside the plan (debug build)
+
+// The kStatus* bits, and the first wait site that gave up, of the last call, from a
+// header read back once the call is done.
+__host__ __device__ inline unsigned int header_status(const WorkspaceHeader& h) {
+    return (unsigned int)(h.status >> 32) == h.epoch ? (unsigned int)h.status : 0u;
+}
+__host__ __device__ inline unsigned int header_where(const WorkspaceHeader& h) {
+    return (unsigned int)(h.where >> 32) == h.epoch ? (unsigned int)h.where : 0u;
+}
+
+// Next call number (never 0), for the host side of every entry point.
+unsigned int next_call_number();
+
+// Tags `word` with call number `epoch` and merges `val` into its low half: OR-ed in,
+// or (first_only) stored only while the low half is still zero.  A retry follows
+// another thread's change, and a word changes at most a few times per call (one
+// retag, then once per status bit), so the loop ends; the cap only bounds it.  Out
+// of line: inlined at every wait site, the loop slowed the prefill kernel by 3%.
+static __device__ __noinline__ void tag_merge(unsigned long long* word, unsigned int epoch, unsigned int val,
+                                          bool first_only) {
+    unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(word);
+    for (int i = 0; i < 64; ++i) {
+        const unsigned int low = (unsigned int)(old >> 32) == epoch ? (unsigned int)old : 0u;
+        const unsigned int nlow = first_only ? (low ? low : val) : (low | val);
+        const unsigned long long want = ((unsigned long long)epoch << 32) | nlow;
+        if (want == old) return;
+        const unsigned long long seen = atomicCAS(word, old, want);
+        if (seen == old) return;
+        old = seen;
+    }
+}
 
 // Index checks of the debug build (compiled with -DGDN_DEBUG_BOUNDS).  Each
 // computed global row, head, column and state index is compared with the
@@ -52,13 +89,13 @@ constexpr unsigned int kStatusBounds = 4u;   // a checked index fell outside the
 // build every check is the constant `true` and compiles away.
 #ifdef GDN_DEBUG_BOUNDS
 constexpr bool kDebugBounds = true;
-__device__ __forceinline__ bool index_ok(WorkspaceHeader* ws, bool cond) {
-    if (!cond) atomicOr(&ws->status, kStatusBounds);
+__device__ __forceinline__ bool index_ok(WorkspaceHeader* ws, unsigned int epoch, bool cond) {
+    if (!cond) tag_merge(&ws->status, epoch, kStatusBounds, false);
     return cond;
 }
 #else
 constexpr bool kDebugBounds = false;
-__device__ __forceinline__ bool index_ok(WorkspaceHeader*, bool) { return true; }
+__device__ __forceinline__ bool index_ok(WorkspaceHeader*, unsigned int, bool) { return true; }
 #endif
 
 // kFused: the replay window of each sequence, then its suffix with outputs, in one launch
@@ -90,6 +127,7 @@ struct CallArgs {
     void* o_out;            // null = no outputs (the state-only replay)
     float* state_out;       // may be null for prefill
     WorkspaceHeader* ws;
+    unsigned int epoch;     // this call's number (see WorkspaceHeader)
     // fused replay + suffix (chunked kernel): a first segment of rows per sequence,
     // replayed from the zero state without outputs before the rows of `windows`
     const Window* windows0; // [batch] or null
@@ -101,6 +139,17 @@ struct CallArgs {
     float* state_mid;       // null, or [batch, H, dk, dv]: the state after the first segment
     int replay_variant;     // ReplayVariant: which chunked kernel runs the state-only replay
 };
+
+// A status report of this call (see WorkspaceHeader).
+__device__ __forceinline__ void report_status(const CallArgs& a, unsigned int bits) {
+    tag_merge(&a.ws->status, a.epoch, bits, false);
+}
+__device__ __forceinline__ bool index_ok(const CallArgs& a, bool cond) { return index_ok(a.ws, a.epoch, cond); }
+// The first thread of a launch records the call number; every kernel that takes a
+// CallArgs does this before anything else.
+__device__ __forceinline__ void record_call(const CallArgs& a) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) a.ws->epoch = a.epoch;
+}
 
 // The chunked path's state-only replay kernel: the two-CTA-per-SM kernel unless the
 // descriptor's kernel field pins the warp-specialised one (GDN_KERNEL_CHUNKED_TC_WARP_SPEC).

@@ -127,7 +127,7 @@ extern "C" gdn_status gdn_tail_replay_state_noalloc(const gdn_varlen_desc* cache
         unsigned char* scratch = static_cast<unsigned char*>(scratch_address());
         if (!scratch) return GDN_ERR_CUDA;
         cudaStream_t st = static_cast<cudaStream_t>(stream);
-        std::memset(host, 0, sizeof(WorkspaceHeader));   // status word and wait site start at zero
+        std::memset(host, 0, sizeof(WorkspaceHeader));   // no status reported under any call number
         if (cudaMemcpyAsync(scratch, host, need, cudaMemcpyHostToDevice, st) != cudaSuccess) {
             cudaGetLastError();
             return GDN_ERR_CUDA;
@@ -152,6 +152,7 @@ extern "C" gdn_status gdn_tail_replay_state_noalloc(const gdn_varlen_desc* cache
         a.beta = beta;
         a.state_out = state_out;
         a.ws = reinterpret_cast<WorkspaceHeader*>(scratch);
+        a.epoch = gdn::next_call_number();
         a.replay_variant = gdn::replay_variant_of(cache->kernel);
         cudaError_t e = kernel == GDN_KERNEL_CHUNKED_TC ? gdn::launch_chunk_tc(a, st) : gdn::launch_recurrent(a, st);
         if (e != cudaSuccess) {
@@ -159,13 +160,13 @@ extern "C" gdn_status gdn_tail_replay_state_noalloc(const gdn_varlen_desc* cache
             return GDN_ERR_CUDA;
         }
         if (status_out) {
-            uint32_t status = 0;
-            if (cudaMemcpyAsync(&status, scratch, sizeof status, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+            WorkspaceHeader hdr;
+            if (cudaMemcpyAsync(&hdr, scratch, sizeof hdr, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
                 cudaStreamSynchronize(st) != cudaSuccess) {
                 cudaGetLastError();
                 return GDN_ERR_CUDA;
             }
-            *status_out = status;
+            *status_out = gdn::header_status(hdr);
         }
     }
     return GDN_OK;

@@ -60,19 +60,19 @@ __device__ __forceinline__ void stage_rows(const CallArgs& a, long long row0, in
     const T* q = static_cast<const T*>(a.q);
     for (int e = threadIdx.x * 4; e < n * DK; e += blockDim.x * 4) {
         int j = e / DK, i = e % DK;
-        if (!index_ok(a.ws, row0 + t0 + j < a.rows_total)) continue;
+        if (!index_ok(a, row0 + t0 + j < a.rows_total)) continue;
         long long g = (row0 + t0 + j) * a.rs_qk + (long long)h * DK + i;
         load4<T>(k + g, sk + e);
         if (OUT) load4<T>(q + g, sq + e);
     }
     for (int e = threadIdx.x * 4; e < n * DV; e += blockDim.x * 4) {
         int j = e / DV, i = e % DV;
-        if (!index_ok(a.ws, row0 + t0 + j < a.rows_total)) continue;
+        if (!index_ok(a, row0 + t0 + j < a.rows_total)) continue;
         long long g = (row0 + t0 + j) * a.rs_v + (long long)h * DV + i;
         load4<T>(v + g, sv + e);
     }
     for (int j = threadIdx.x; j < n; j += blockDim.x) {
-        if (!index_ok(a.ws, row0 + t0 + j < a.rows_total)) continue;
+        if (!index_ok(a, row0 + t0 + j < a.rows_total)) continue;
         long long g = (row0 + t0 + j) * H + h;
         sa[j] = a.alpha[g];
         sb[j] = a.beta[g];
@@ -92,17 +92,18 @@ __global__ void __launch_bounds__(64 * (DK / 64), 3) recurrent_kernel(const Call
     __shared__ __align__(16) float sv[kStageTokens * DV];
     __shared__ float sa[kStageTokens], sb[kStageTokens];
 
+    record_call(a);
     const Unit u = a.unit_list[blockIdx.x];
     const int b = u.seq, h = u.head;
     const int c = blockIdx.y * COLS + threadIdx.x / KS, part = threadIdx.x % KS, r0 = part * KR;
     if (!window_agrees(a, b)) {
-        if (threadIdx.x == 0) atomicOr(&a.ws->status, kStatusMismatch);
+        if (threadIdx.x == 0) report_status(a, kStatusMismatch);
         return;
     }
     const Window w = a.windows[b];
     const size_t state_base = ((size_t)b * a.num_heads + h) * DK * DV;
     // debug build: the unit, its column block and its window lie inside the plan (uniform)
-    if (!index_ok(a.ws, b >= 0 && b < a.batch && h >= 0 && h < a.num_heads && blockIdx.y * COLS + COLS <= DV &&
+    if (!index_ok(a, b >= 0 && b < a.batch && h >= 0 && h < a.num_heads && blockIdx.y * COLS + COLS <= DV &&
                             w.row0 >= 0 && w.len >= 0 && w.row0 + w.len <= a.rows_total))
         return;
 
@@ -178,7 +179,7 @@ __global__ void __launch_bounds__(64 * (DK / 64), 3) recurrent_kernel(const Call
                 }
                 float ov = ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
                 if (KS == 2) ov += __shfl_xor_sync(0xffffffffu, ov, 1);
-                if (part == 0 && index_ok(a.ws, w.row0 + t0 + j < a.rows_total))
+                if (part == 0 && index_ok(a, w.row0 + t0 + j < a.rows_total))
                     store1(o + ((w.row0 + t0 + j) * a.num_heads + h) * (long long)DV + c, sigma * ov);
             }
         }

@@ -102,19 +102,20 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     __shared__ int s_abort;         // a wait outside the block-wide barriers gave up
 
     const CallArgs& a = p.a;
+    record_call(a);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wq = warp & 3, wh = warp >> 2;   // TMEM lane quarter; which half of the warps
     const int row = wq * 32 + lane;            // this thread's TMEM lane
     const Unit u = a.unit_list[blockIdx.x];
     const int b = u.seq, h = u.head, H = a.num_heads;
     if (!window_agrees(a, b)) {
-        if (tid == 0) atomicOr(&a.ws->status, kStatusMismatch);
+        if (tid == 0) report_status(a, kStatusMismatch);
         return;
     }
     const Window w = a.windows[b];
     const int nchunks = (w.len + C - 1) / C;
     // debug build: the unit and its window lie inside the plan's extents (uniform)
-    if (!index_ok(a.ws, b >= 0 && b < a.batch && h >= 0 && h < H && w.row0 >= 0 && w.len >= 0 &&
+    if (!index_ok(a, b >= 0 && b < a.batch && h >= 0 && h < H && w.row0 >= 0 && w.len >= 0 &&
                             w.row0 + w.len <= a.rows_total))
         return;
 
@@ -191,7 +192,7 @@ replay_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
         be = 0.0f;
         if (tid < C && cc * C + tid < w.len) {
             const long long r = w.row0 + (long long)cc * C + tid;
-            if (index_ok(a.ws, r < a.rows_total)) {
+            if (index_ok(a, r < a.rows_total)) {
                 al = a.alpha[r * H + h];
                 be = a.beta[r * H + h];
             }

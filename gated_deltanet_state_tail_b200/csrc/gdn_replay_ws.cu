@@ -302,17 +302,18 @@ replay_ws_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
     __shared__ float s_msg_scale;
 
     const CallArgs& a = p.a;
+    record_call(a);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wq = warp & 3;   // TMEM lane quarter
     const Unit u = a.unit_list[blockIdx.x];
     const int b = u.seq, h = u.head, H = a.num_heads;
     if (!window_agrees(a, b)) {
-        if (tid == 0) atomicOr(&a.ws->status, kStatusMismatch);
+        if (tid == 0) report_status(a, kStatusMismatch);
         return;
     }
     const Window w = a.windows[b];
     const int nchunks = (w.len + C - 1) / C;
-    if (!index_ok(a.ws, b >= 0 && b < a.batch && h >= 0 && h < H && w.row0 >= 0 && w.len >= 0 &&
+    if (!index_ok(a, b >= 0 && b < a.batch && h >= 0 && h < H && w.row0 >= 0 && w.len >= 0 &&
                             w.row0 + w.len <= a.rows_total))
         return;
 
@@ -371,7 +372,7 @@ replay_ws_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                 be[q] = 0.0f;
                 if (n < nchunks && n * C + jj < w.len) {
                     const long long r = w.row0 + (long long)n * C + jj;
-                    if (index_ok(a.ws, r < a.rows_total)) {
+                    if (index_ok(a, r < a.rows_total)) {
                         al[q] = a.alpha[r * H + h];
                         be[q] = a.beta[r * H + h];
                     }

@@ -16,13 +16,14 @@ namespace {
 constexpr unsigned int kSelftestWhere = 99u;   // wait-site code reported by the self-test
 
 // One thread waits, bounded by limit_ns, on an mbarrier that nothing arrives on.
-__global__ void bounded_wait_selftest_kernel(WorkspaceHeader* ws, unsigned long long limit_ns) {
+__global__ void bounded_wait_selftest_kernel(WorkspaceHeader* ws, unsigned int epoch, unsigned long long limit_ns) {
     __shared__ uint64_t bar;
+    ws->epoch = epoch;
     sm100::mbar_init(&bar, 1);
     sm100::mbar_fence_init();
     if (!sm100::mbar_wait_bounded(&bar, 0u, limit_ns)) {
-        atomicOr(&ws->status, kStatusTimeout);
-        atomicCAS(&ws->timeout_where, 0u, kSelftestWhere);
+        tag_merge(&ws->status, epoch, kStatusTimeout, false);
+        tag_merge(&ws->where, epoch, kSelftestWhere, true);
     }
 }
 
@@ -30,9 +31,10 @@ __global__ void bounded_wait_selftest_kernel(WorkspaceHeader* ws, unsigned long 
 // the check records kStatusBounds and skips the store it guards.  (The index
 // is still inside the header's pad array, so even an unchecked store would
 // stay in the caller's workspace.)
-__global__ void index_check_selftest_kernel(WorkspaceHeader* ws) {
+__global__ void index_check_selftest_kernel(WorkspaceHeader* ws, unsigned int epoch) {
     const long long extent = 4, idx = extent;   // one past the end
-    if (index_ok(ws, idx < extent)) ws->pad[idx] = 1u;
+    ws->epoch = epoch;
+    if (index_ok(ws, epoch, idx < extent)) ws->pad[idx] = 1u;
 }
 
 }  // namespace
@@ -43,11 +45,7 @@ extern "C" gdn_status gdn_selftest_bounded_wait(uint64_t limit_ns, void* workspa
     if (limit_ns == 0 || limit_ns > 1000000000ull) return GDN_ERR_INVALID_ARG;   // at most 1 s
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     auto* ws = static_cast<gdn::WorkspaceHeader*>(workspace);
-    if (cudaMemsetAsync(ws, 0, sizeof(gdn::WorkspaceHeader), st) != cudaSuccess) {
-        cudaGetLastError();
-        return GDN_ERR_CUDA;
-    }
-    gdn::bounded_wait_selftest_kernel<<<1, 1, 0, st>>>(ws, (unsigned long long)limit_ns);
+    gdn::bounded_wait_selftest_kernel<<<1, 1, 0, st>>>(ws, gdn::next_call_number(), (unsigned long long)limit_ns);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     return GDN_OK;
 }
@@ -57,11 +55,7 @@ extern "C" gdn_status gdn_selftest_index_check(void* workspace, void* stream) {
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 15u) != 0) return GDN_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     auto* ws = static_cast<gdn::WorkspaceHeader*>(workspace);
-    if (cudaMemsetAsync(ws, 0, sizeof(gdn::WorkspaceHeader), st) != cudaSuccess) {
-        cudaGetLastError();
-        return GDN_ERR_CUDA;
-    }
-    gdn::index_check_selftest_kernel<<<1, 1, 0, st>>>(ws);
+    gdn::index_check_selftest_kernel<<<1, 1, 0, st>>>(ws, gdn::next_call_number());
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     return GDN_OK;
 }

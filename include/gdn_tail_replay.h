@@ -170,14 +170,18 @@ GDN_API gdn_status gdn_plan_info(gdn_plan_t plan, int64_t* units, int64_t* total
                          int32_t* kernel);
 
 /* Kernel launches that one call on this plan makes: 1 for a replay or a
- * prefill plan; 1 or 2 for a fused plan (see gdn_tail_replay_prefill).  The
- * workspace status reset each call does first is a memset, not counted.
- * INVALID_ARG for a NULL plan or pointer. */
+ * prefill plan; 1 or 2 for a fused plan (see gdn_tail_replay_prefill).  A
+ * call puts nothing else on its stream.  INVALID_ARG for a NULL plan or
+ * pointer. */
 GDN_API gdn_status gdn_plan_launches(gdn_plan_t plan, int32_t* launches);
 
 /* Bytes of device workspace a call on this plan needs (>= 256, multiple of
  * 256).  The caller allocates it (16-byte aligned) and passes it to each
- * call; calls running concurrently need separate workspaces. */
+ * call; calls running concurrently need separate workspaces.  Its contents
+ * need no initialisation and no reset between calls: each call tags the
+ * status it reports with a call number of its own, and the call's first
+ * thread records that number, so gdn_workspace_status reads only what the
+ * last call reported. */
 GDN_API size_t gdn_workspace_bytes(gdn_plan_t plan);
 
 /*

@@ -177,6 +177,33 @@ def test_descriptor_mismatch_is_reported():
     plan.close()
 
 
+def test_status_belongs_to_the_last_call_without_a_reset():
+    """No call clears the workspace: each tags its reports with its own call number.  A
+    workspace of arbitrary bytes reads GDN_OK after a good call, and neither a timeout nor
+    a mismatch outlives the call that reported it."""
+    t = make_cache([100, 100], 2, 128, 128, "bf16", seed=16)
+    off, ml, R = [0, 100, 200], [90, 100], [30, 40]
+    plan = gdn.ReplayPlan(2, 128, 128, "bf16", off, ml, R)
+    out = torch.zeros((2, 2, 128, 128), device="cuda")
+    ref = oracle_replay(t, np.array(off, np.int32), ml, R)
+    ws = torch.full((256,), 0xFF, dtype=torch.uint8, device="cuda")
+    ws[:8].fill_(0x07)                                       # every status bit set, under a stale tag
+    plan.run(t["k"], t["v"], t["alpha"], t["beta"], out, workspace=ws)
+    assert gdn.gdn_workspace_status(ws) == gdn.GDN_OK
+    assert per_request_state_err(out.cpu().numpy(), ref) <= TOL["bf16"]
+    gdn.gdn_selftest_bounded_wait(1_000_000, ws)
+    assert gdn.gdn_workspace_status(ws) == gdn.GDN_ERR_TIMEOUT
+    plan.run(t["k"], t["v"], t["alpha"], t["beta"], out, workspace=ws)
+    assert gdn.gdn_workspace_status(ws) == gdn.GDN_OK
+    bad = torch.tensor([90, 99], dtype=torch.int32, device="cuda")
+    plan.run(t["k"], t["v"], t["alpha"], t["beta"], out, match_len=bad, workspace=ws)
+    assert gdn.gdn_workspace_status(ws) == gdn.GDN_ERR_MISMATCH
+    plan.run(t["k"], t["v"], t["alpha"], t["beta"], out, workspace=ws)
+    assert gdn.gdn_workspace_status(ws) == gdn.GDN_OK
+    assert per_request_state_err(out.cpu().numpy(), ref) <= TOL["bf16"]
+    plan.close()
+
+
 def test_call_validation_on_device():
     t = make_cache([64], 1, 64, 64, "f32", seed=14)
     plan = gdn.ReplayPlan(1, 64, 64, "f32", [0, 64], [64], [10])
@@ -303,8 +330,10 @@ def test_bounded_wait_timeout_is_reported_and_context_survives():
     ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
     gdn.gdn_selftest_bounded_wait(1_000_000, ws)
     assert gdn.gdn_workspace_status(ws) == gdn.GDN_ERR_TIMEOUT
+    # header words: status (bits, call number), wait site (code, call number), recorded call number
     header = ws.view(torch.int32).cpu().numpy()
-    assert header[1] == 99                                   # the wait site the self-test reports
+    assert header[2] == 99                                   # the wait site the self-test reports
+    assert header[1] == header[3] == header[4] != 0          # both tagged with the recorded call
     # the context is still usable: a small replay runs and matches the oracle
     t = make_cache([200], 2, 128, 128, "bf16", seed=3)
     st = run_replay(t, np.array([0, 200], np.int32), [200], [150], gdn.GDN_KERNEL_AUTO, "bf16")
