@@ -29,8 +29,8 @@ GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT,
 GDN_F32, GDN_BF16 = 0, 1
 GDN_KERNEL_AUTO, GDN_KERNEL_RECURRENT, GDN_KERNEL_CHUNKED_TC = 0, 1, 2
 # the chunked kernel with the state-only replay pinned to its two-CTA-per-SM kernel (the
-# default) or to its warp-specialised one
-GDN_KERNEL_CHUNKED_TC_TWO_CTA, GDN_KERNEL_CHUNKED_TC_WARP_SPEC = 3, 4
+# default), its warp-specialised one or its cluster-pair one
+GDN_KERNEL_CHUNKED_TC_TWO_CTA, GDN_KERNEL_CHUNKED_TC_WARP_SPEC, GDN_KERNEL_CHUNKED_TC_PAIR = 3, 4, 5
 
 EXPORTED = (
     "gdn_plan_create_replay", "gdn_plan_create_prefill", "gdn_plan_destroy", "gdn_replay_windows",

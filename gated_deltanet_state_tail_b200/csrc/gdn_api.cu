@@ -61,7 +61,7 @@ gdn_status check_varlen_desc(const gdn_varlen_desc* d) {
     if (d->batch < 1 || d->num_heads < 1) return GDN_ERR_INVALID_ARG;
     if (d->dtype != GDN_F32 && d->dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
     if ((d->d_k != 64 && d->d_k != 128) || (d->d_v != 64 && d->d_v != 128)) return GDN_ERR_UNSUPPORTED;
-    if (d->kernel < GDN_KERNEL_AUTO || d->kernel > GDN_KERNEL_CHUNKED_TC_WARP_SPEC) return GDN_ERR_INVALID_ARG;
+    if (d->kernel < GDN_KERNEL_AUTO || d->kernel > GDN_KERNEL_CHUNKED_TC_PAIR) return GDN_ERR_INVALID_ARG;
     // row stride: 0 = packed; otherwise every head of a row fits and rows start on 16 bytes
     if (d->row_stride_elems != 0) {
         const long long elem = d->dtype == GDN_BF16 ? 2 : 4;

@@ -684,11 +684,16 @@ cudaError_t launch_chunk_tc(const CallArgs& a, cudaStream_t stream) {
     if (!chunk_tc_supported(a.dtype, a.dk, a.dv)) return cudaErrorInvalidValue;
     // the state-only replay kernels unless outputs are asked for (a prefill, a fused replay
     // + suffix, or a replay that also emits the window's outputs): the two-CTA-per-SM
-    // kernel, which is the faster one at every launch size measured (one to 296 units);
-    // the warp-specialised kernel (one CTA per SM, the front of a unit's chunks decoupled
-    // from its state chain) only when the descriptor pins it
-    if (a.kind == kReplay && a.o_out == nullptr)
-        return a.replay_variant == kReplayWarpSpec ? launch_replay_ws(a, stream) : launch_replay_tc(a, stream);
+    // kernel, the fastest or as fast at every launch size measured (one to 296 units); the
+    // warp-specialised kernel (one CTA per SM) and the cluster-pair kernel (two SMs per
+    // unit) only when the descriptor pins them
+    if (a.kind == kReplay && a.o_out == nullptr) {
+        switch (a.replay_variant) {
+            case kReplayWarpSpec: return launch_replay_ws(a, stream);
+            case kReplayPair: return launch_replay_pair(a, stream);
+            default: return launch_replay_tc(a, stream);
+        }
+    }
     TcParams p;
     p.a = a;
     // a call with no rows to read (every window empty) still runs, to write the states;

@@ -152,19 +152,21 @@ __device__ __forceinline__ void record_call(const CallArgs& a) {
 }
 
 // The chunked path's state-only replay kernel: the two-CTA-per-SM kernel unless the
-// descriptor's kernel field pins the warp-specialised one (GDN_KERNEL_CHUNKED_TC_WARP_SPEC).
-enum ReplayVariant { kReplayDefault = 0, kReplayTwoCta = 1, kReplayWarpSpec = 2 };
+// descriptor's kernel field pins the warp-specialised or the cluster-pair one.
+enum ReplayVariant { kReplayDefault = 0, kReplayTwoCta = 1, kReplayWarpSpec = 2, kReplayPair = 3 };
 
 inline int replay_variant_of(int kernel) {
     return kernel == GDN_KERNEL_CHUNKED_TC_TWO_CTA    ? kReplayTwoCta
            : kernel == GDN_KERNEL_CHUNKED_TC_WARP_SPEC ? kReplayWarpSpec
+           : kernel == GDN_KERNEL_CHUNKED_TC_PAIR      ? kReplayPair
                                                         : kReplayDefault;
 }
 
 // The kernel family a descriptor's kernel field names (the pinned replay variants
 // are the chunked kernel).
 inline int kernel_family_of(int kernel) {
-    return (kernel == GDN_KERNEL_CHUNKED_TC_TWO_CTA || kernel == GDN_KERNEL_CHUNKED_TC_WARP_SPEC)
+    return (kernel == GDN_KERNEL_CHUNKED_TC_TWO_CTA || kernel == GDN_KERNEL_CHUNKED_TC_WARP_SPEC ||
+            kernel == GDN_KERNEL_CHUNKED_TC_PAIR)
                ? GDN_KERNEL_CHUNKED_TC
                : kernel;
 }
@@ -230,6 +232,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_chunk_tc(const CallArgs& a, cudaStream_t stream);   // dispatches the replay below
 cudaError_t launch_replay_tc(const CallArgs& a, cudaStream_t stream);
 cudaError_t launch_replay_ws(const CallArgs& a, cudaStream_t stream);
+cudaError_t launch_replay_pair(const CallArgs& a, cudaStream_t stream);
 bool chunk_tc_supported(int dtype, int dk, int dv);
 
 }  // namespace gdn

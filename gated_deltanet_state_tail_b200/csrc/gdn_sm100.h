@@ -62,6 +62,77 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     return true;
 }
 
+// ---------------------------------------------------------------- clusters
+// Thread-block clusters of two CTAs on two SMs, talking through distributed
+// shared memory.  No multicast anywhere: each copy has one destination.
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// The shared::cluster address of the location at `saddr` (a shared::cta
+// address) in the shared memory of cluster CTA `rank`.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+
+// Every thread of both CTAs (each warp executes it whole): release this
+// thread's prior accesses, then wait for the rest of the cluster.
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Copy `bytes` (a multiple of 16, both addresses 16-byte aligned) from this
+// CTA's shared memory at `src` to a peer CTA's at `peer_dst` (a shared::cluster
+// address), completing `bytes` of transaction count on the peer's mbarrier at
+// `peer_bar` (a shared::cluster address).
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t peer_dst, uint32_t src, uint32_t bytes,
+                                                  uint32_t peer_bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            peer_dst),
+        "r"(src), "r"(bytes), "r"(peer_bar)
+        : "memory");
+}
+
+// Arrive (count 1) on a peer CTA's mbarrier (a shared::cluster address),
+// releasing this thread's prior accesses at cluster scope.
+__device__ __forceinline__ void mbar_arrive_peer(uint32_t peer_bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(peer_bar) : "memory");
+}
+
+// A 32-bit load from a peer CTA's shared memory (a shared::cluster address).
+__device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+// mbar_wait_bounded for a phase that a peer CTA completes: acquire at cluster
+// scope, so what the peer released before its arrive is visible here.
+__device__ __forceinline__ bool mbar_wait_bounded_cluster(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+    auto try_wait = [&]() {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+        return done != 0;
+    };
+    if (try_wait()) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (!try_wait()) {
+        if (global_timer_ns() - t0 > limit_ns) return false;
+    }
+    return true;
+}
+
 // ---------------------------------------------------------------- barriers
 // Arrive (count 1) on an mbarrier from this thread.
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {

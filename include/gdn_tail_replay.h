@@ -74,16 +74,20 @@ typedef enum gdn_dtype { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
 
 /* Kernel selection.  AUTO picks the tensor-core chunked kernel for bf16 with
  * d_k = d_v = 128 and the exact fp32 CUDA-core recurrent kernel otherwise.
- * The chunked path has two state-only replay kernels: one with two CTAs per SM
- * (the one AUTO and GDN_KERNEL_CHUNKED_TC run) and a warp-specialised one with
- * one CTA per SM.  The last two values pin one of them (for tests and
- * measurements); every other entry point treats them as GDN_KERNEL_CHUNKED_TC. */
+ * The chunked path has three state-only replay kernels: one with two CTAs per
+ * SM (the one AUTO and GDN_KERNEL_CHUNKED_TC run), a warp-specialised one with
+ * one CTA per SM, and a cluster-pair one that runs each (sequence, head) unit
+ * on two CTAs on two SMs (one builds the chunks' T operands, the other runs
+ * the state chain).  The values 3 to 5 pin one of them (for tests and
+ * measurements); every other entry point treats them as
+ * GDN_KERNEL_CHUNKED_TC. */
 typedef enum gdn_kernel {
     GDN_KERNEL_AUTO = 0,
     GDN_KERNEL_RECURRENT = 1,              /* token-recurrent, fp32 CUDA cores, any supported shape */
     GDN_KERNEL_CHUNKED_TC = 2,             /* chunked WY/UT form on tcgen05 tensor cores (bf16, d = 128) */
     GDN_KERNEL_CHUNKED_TC_TWO_CTA = 3,     /* as 2, the replay always on the two-CTA-per-SM kernel */
-    GDN_KERNEL_CHUNKED_TC_WARP_SPEC = 4    /* as 2, the replay always on the warp-specialised kernel */
+    GDN_KERNEL_CHUNKED_TC_WARP_SPEC = 4,   /* as 2, the replay always on the warp-specialised kernel */
+    GDN_KERNEL_CHUNKED_TC_PAIR = 5         /* as 2, the replay always on the cluster-pair kernel */
 } gdn_kernel;
 
 /* Varlen batch descriptor.  Sequence b occupies rows [seq_offsets[b],

@@ -118,14 +118,15 @@ def test_chunked_kernel_needs_bf16_d128():
 
 
 def test_pinned_replay_kernels_validate_as_chunked():
-    """The two values that pin the state-only replay to one of the chunked path's
+    """The three values that pin the state-only replay to one of the chunked path's
     kernels validate like the chunked kernel; the value after them is rejected."""
-    for k in (gdn.GDN_KERNEL_CHUNKED_TC_TWO_CTA, gdn.GDN_KERNEL_CHUNKED_TC_WARP_SPEC):
+    for k in (gdn.GDN_KERNEL_CHUNKED_TC_TWO_CTA, gdn.GDN_KERNEL_CHUNKED_TC_WARP_SPEC,
+              gdn.GDN_KERNEL_CHUNKED_TC_PAIR):
         d, off = _desc(dtype=gdn.GDN_F32, kernel=k)
         assert _create_replay(d, [50], [10]) == gdn.GDN_ERR_UNSUPPORTED
         d, off = _desc(dk=64, dv=64, kernel=k)
         assert _create_replay(d, [50], [10]) == gdn.GDN_ERR_UNSUPPORTED
-    d, off = _desc(kernel=gdn.GDN_KERNEL_CHUNKED_TC_WARP_SPEC + 1)
+    d, off = _desc(kernel=gdn.GDN_KERNEL_CHUNKED_TC_PAIR + 1)
     assert _create_replay(d, [50], [10]) == gdn.GDN_ERR_INVALID_ARG
 
 

@@ -12,13 +12,14 @@ from helpers import TOL, oracle_view, per_request_rows_err, per_request_state_er
 
 pytestmark = pytest.mark.gpu
 
-# "two_cta" and "warp_spec" run the chunked path with the state-only replay pinned to
-# one of its two kernels (the default, "chunked", is the two-CTA kernel); every other
-# entry point runs the chunked prefill kernel under all three
+# "two_cta", "warp_spec" and "pair" run the chunked path with the state-only replay
+# pinned to one of its three kernels (the default, "chunked", is the two-CTA kernel);
+# every other entry point runs the chunked prefill kernel under all four
 KERNELS = {"recurrent": gdn.GDN_KERNEL_RECURRENT, "chunked": gdn.GDN_KERNEL_CHUNKED_TC,
-           "two_cta": gdn.GDN_KERNEL_CHUNKED_TC_TWO_CTA, "warp_spec": gdn.GDN_KERNEL_CHUNKED_TC_WARP_SPEC}
-CHUNKED = ("chunked", "two_cta", "warp_spec")
-REPLAY_KERNELS = ["recurrent", "two_cta", "warp_spec"]
+           "two_cta": gdn.GDN_KERNEL_CHUNKED_TC_TWO_CTA, "warp_spec": gdn.GDN_KERNEL_CHUNKED_TC_WARP_SPEC,
+           "pair": gdn.GDN_KERNEL_CHUNKED_TC_PAIR}
+CHUNKED = ("chunked", "two_cta", "warp_spec", "pair")
+REPLAY_KERNELS = ["recurrent", "two_cta", "warp_spec", "pair"]
 
 
 def kernel_or_skip(name, dtype, dk, dv):

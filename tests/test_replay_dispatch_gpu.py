@@ -1,14 +1,15 @@
-"""The state-only replay's two tensor-core kernels, each pinned through the
-descriptor, on launches on both sides of one unit per SM.
+"""The state-only replay's three tensor-core kernels, each pinned through the
+descriptor, on launches of three sizes.
 
-The chunked path runs the replay on a kernel with two CTAs per SM (the default)
-or, when the descriptor pins it, on a warp-specialised kernel with one CTA per
-SM (the front of a unit's chunks runs ahead of its state chain).  Each kernel
-replays the same ragged windows (several 64-token chunks and a partial last
-chunk) on a launch with at most one (request, head) unit per SM and on one with
-more; every unit is checked element by element against the fp64 oracle, the
-default must be the two-CTA kernel bit for bit, and the two kernels must agree
-within the same bound.
+The chunked path runs the replay on a kernel with two CTAs per SM by default, on a
+warp-specialised kernel with one CTA per SM or on a cluster-pair kernel (each unit
+on two CTAs on two SMs) when the descriptor pins one.  Each kernel replays the same
+ragged windows (several 64-token chunks and a partial last chunk) on a launch with
+at most one (request, head) unit per two SMs, one with at most one per SM and one
+with more; every unit is checked element by element against the fp64 oracle, the
+default must equal the two-CTA kernel bit for bit, and so must the pair kernel (the
+same operations in the same order); the warp-specialised kernel must agree within
+the oracle's bound.
 """
 import numpy as np
 import pytest
@@ -33,9 +34,10 @@ def _replay(t, off, ml, R, kernel):
     return out.cpu().numpy()
 
 
-def test_both_replay_kernels_around_one_unit_per_sm():
+def test_replay_kernels_across_launch_sizes():
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    b_small = sms // H                  # units = H * b_small <= SMs
+    b_pair = sms // (2 * H)             # units = H * b_pair <= SMs / 2
+    b_small = sms // H                  # units <= SMs
     b_large = b_small + 2               # units > SMs
     rng = np.random.default_rng(5)
     ml = rng.integers(70, 330, size=b_large).astype(np.int32)
@@ -45,14 +47,16 @@ def test_both_replay_kernels_around_one_unit_per_sm():
     t = inputs.draw_tensors(int(off[-1]), H, D, D, "bf16", 0.9, 0.999, 21, device="cuda", with_q=False)
     ref = oracle.replay_state(oracle_view(t["k"]), oracle_view(t["v"]), oracle_view(t["alpha"]),
                               oracle_view(t["beta"]), off, ml, R)
-    assert H * b_small <= sms < H * b_large
-    for nb in (b_small, b_large):
+    assert 2 * H * b_pair <= sms < 2 * H * (b_pair + 1) and H * b_small <= sms < H * b_large
+    names = {"two_cta": gdn.GDN_KERNEL_CHUNKED_TC_TWO_CTA, "warp_spec": gdn.GDN_KERNEL_CHUNKED_TC_WARP_SPEC,
+             "pair": gdn.GDN_KERNEL_CHUNKED_TC_PAIR}
+    for nb in (b_pair, b_small, b_large):
         o, m, r = off[:nb + 1], ml[:nb], R[:nb]
-        two = _replay(t, o, m, r, gdn.GDN_KERNEL_CHUNKED_TC_TWO_CTA)
-        ws = _replay(t, o, m, r, gdn.GDN_KERNEL_CHUNKED_TC_WARP_SPEC)
+        got = {k: _replay(t, o, m, r, v) for k, v in names.items()}
         auto = _replay(t, o, m, r, gdn.GDN_KERNEL_AUTO)
-        assert np.array_equal(auto, two), f"{nb} requests: the default is not the two-CTA kernel"
+        assert np.array_equal(auto, got["two_cta"]), f"{nb} requests: the default is not the two-CTA kernel"
+        assert np.array_equal(got["pair"], got["two_cta"]), f"{nb} requests: the pair kernel's bits differ"
         for b in range(nb):
-            assert rel_err(two[b], ref[b]) <= TOL["bf16"], f"{nb} requests, request {b} (two-CTA kernel)"
-            assert rel_err(ws[b], ref[b]) <= TOL["bf16"], f"{nb} requests, request {b} (warp-specialised kernel)"
-            assert rel_err(ws[b], two[b]) <= TOL["bf16"], f"{nb} requests, request {b}: the kernels disagree"
+            for k, g in got.items():
+                assert rel_err(g[b], ref[b]) <= TOL["bf16"], f"{nb} requests, request {b} ({k} kernel)"
+                assert rel_err(g[b], got["two_cta"][b]) <= TOL["bf16"], f"{nb} requests, request {b}: {k} vs two_cta"
