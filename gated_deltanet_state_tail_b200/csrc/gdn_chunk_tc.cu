@@ -77,21 +77,22 @@ struct PipeLayout {
     static constexpr uint32_t OFF_AT = 2 * TILE;                // fp32 A, then T (scratch in its upper right)
     static constexpr uint32_t OFF_TB = OFF_AT + C * LDT * 4;    // bf16 T diag(beta)
     static constexpr uint32_t OFF_TG = OFF_TB + 8192;           // fp32 -sigma T diag(beta gamma), K-major
-    static constexpr uint32_t OFF_UB = OFF_TG + 16384;          // the output stage, bf16 O [i][dv]
+    static constexpr uint32_t OFF_UB = OFF_TG + 16384;          // the output stage: bf16 O, two [i][dv] tiles
     static constexpr uint32_t OFF_MB = OFF_UB + 16384;          // two bf16 M [i][j], chunk c in c % 2
     static constexpr uint32_t OFF_BQ = OFF_MB + 16384;          // bf16 sigma diag(gamma) Q, K-major
     static constexpr uint32_t BYTES = OFF_BQ + 16384;
 };
 static_assert(PipeLayout::OFF_TB % 1024 == 0 && PipeLayout::OFF_TG == PipeLayout::OFF_TB + 8192 &&
-                  PipeLayout::OFF_BQ % 1024 == 0,
-              "operands on 1 KB, TG right after TB");
+                  PipeLayout::OFF_BQ % 1024 == 0 && PipeLayout::OFF_UB % 1024 == 0,
+              "operands and the output stage (a TMA source) on 1 KB, TG right after TB");
 static_assert(PipeLayout::BYTES + 1024 <= 227 * 1024, "fits one CTA per SM");
 static_assert(TM_SB + 64 <= 512, "TMEM map");
 
 __global__ void __launch_bounds__(NT, 1)
 prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_q,
-                    const __grid_constant__ CUtensorMap map_k0, const __grid_constant__ CUtensorMap map_v0) {
+                    const __grid_constant__ CUtensorMap map_k0, const __grid_constant__ CUtensorMap map_v0,
+                    const __grid_constant__ CUtensorMap map_o) {
     using L = TileLayout;
     using PL = PipeLayout;
     extern __shared__ uint8_t smem_raw[];
@@ -433,14 +434,17 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                     __syncwarp();
                 }
                 sigma = snew;
+                if (ct == 0 && outc) bulk_wait_group_read0();   // the last chunk's output store has read the stage
                 named_sync(BAR_CHAIN, 128);   // the state update (and O) of chunk c are complete
                 tc_fence_after();
                 if (outc) {
-                    // outputs: stage O as bf16 rows [i][dv] in the UB region (256-byte rows whose
-                    // 16-byte pieces are XOR-swizzled by i % 8), then 16-byte stores of whole rows.
-                    // O^T (lane = value dim dv, column = chunk row i) is read in the 16x256b shape,
-                    // whose registers are the fragments of 8 x 8 blocks [dv][i]; stmatrix .trans
-                    // writes each block as 8 rows i of 8 values dv.
+                    // outputs: stage O as bf16 in the UB region, two 8 KB tiles of 64 rows i by
+                    // 64 values dv (128-byte rows, 16-byte pieces XOR-swizzled by i % 8: the TMA
+                    // layout), then one TMA store per tile for a full chunk, or 16-byte stores of
+                    // the chunk's rows for a partial one.  O^T (lane = value dim dv, column =
+                    // chunk row i) is read in the 16x256b shape, whose registers are the
+                    // fragments of 8 x 8 blocks [dv][i]; stmatrix .trans writes each block as 8
+                    // rows i of 8 values dv.
                     const uint32_t s_stage = smem_u32(sm + PL::OFF_UB);
 #pragma unroll
                     for (int lh = 0; lh < 2; ++lh) {   // lanes 16 lh .. 16 lh + 15 of the quarter
@@ -459,19 +463,32 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                                     r[m] = pack_bf16(v[4 * k + 2 * hf], v[4 * k + 2 * hf + 1]);
                                 }
                                 const int i = 32 * kg + 8 * (lane >> 3) + (lane & 7);   // this lane's row
-                                stmatrix_x4_trans(s_stage + (uint32_t)(i * 256 + (((v0 >> 3) ^ (i & 7)) << 4)), r);
+                                stmatrix_x4_trans(s_stage + (uint32_t)((v0 >> 6) * 8192 + i * 128 +
+                                                                       ((((v0 & 63) >> 3) ^ (i & 7)) << 4)),
+                                                  r);
                             }
                         }
                     }
+                    const bool tma_out = src.nc == C && index_ok(a, src.r0 + C <= a.rows_total);   // uniform
+                    if (tma_out) fence_proxy_async_smem();   // the stage, for the TMA store
                     named_sync(BAR_CHAIN, 128);
-                    const uint8_t* stage = sm + PL::OFF_UB;
-                    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o_out);
+                    if (tma_out) {
+                        if (ct == 0) {
+                            tma_store_3d(&map_o, s_stage, 0, h, (int)src.r0);
+                            tma_store_3d(&map_o, s_stage + 8192, 64, h, (int)src.r0);
+                            bulk_commit_group();
+                        }
+                    } else {
+                        const uint8_t* stage = sm + PL::OFF_UB;
+                        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o_out);
 #pragma unroll
-                    for (int k = 0; k < (C * D / 8) / 128; ++k) {   // 16-byte pieces: 16 per row
-                        const int idx = ct + k * 128, i = idx >> 4, ch = idx & 15;
-                        if (i < src.nc && index_ok(a, src.r0 + i < a.rows_total))
-                            *reinterpret_cast<uint4*>(o + ((src.r0 + i) * H + h) * (long long)D + ch * 8) =
-                                *reinterpret_cast<const uint4*>(stage + i * 256 + ((ch ^ (i & 7)) << 4));
+                        for (int k = 0; k < (C * D / 8) / 128; ++k) {   // 16-byte pieces: 16 per row
+                            const int idx = ct + k * 128, i = idx >> 4, ch = idx & 15;
+                            if (i < src.nc && index_ok(a, src.r0 + i < a.rows_total))
+                                *reinterpret_cast<uint4*>(o + ((src.r0 + i) * H + h) * (long long)D + ch * 8) =
+                                    *reinterpret_cast<const uint4*>(stage + (ch >> 3) * 8192 + i * 128 +
+                                                                    (((ch & 7) ^ (i & 7)) << 4));
+                        }
                     }
                 }
                 if (fused && c == nA - 1 && a.state_mid) {   // the state at L (chunk c is the window's last)
@@ -634,6 +651,7 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             for (int i = 0; i < 32; ++i) a.state_out[state_base + (size_t)(cb * 32 + i) * D + row] = sigma * v[i];
         }
     }
+    if (tid == 128) bulk_wait_group0();   // the outputs' TMA stores are done before the CTA leaves
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -719,7 +737,11 @@ cudaError_t launch_chunk_tc(const CallArgs& a, cudaStream_t stream) {
     const uint32_t smem = PipeLayout::BYTES + 1024;
     const cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(prefill_pipe_kernel), (int)smem, smem_set);
     if (e != cudaSuccess) return e;
-    prefill_pipe_kernel<<<(unsigned)a.units, NT, smem, stream>>>(p, mk, mv, mq, mk0, mv0);
+    // the outputs' map ([rows, H, 128] bf16, packed), stored into by whole full chunks
+    CUtensorMap mo = mk;
+    if (a.o_out && !make_tile_map(&mo, a.o_out, a.num_heads, a.rows_total, (long long)a.num_heads * D))
+        return cudaErrorInvalidValue;
+    prefill_pipe_kernel<<<(unsigned)a.units, NT, smem, stream>>>(p, mk, mv, mq, mk0, mv0, mo);
     return cudaGetLastError();
 }
 
