@@ -18,7 +18,7 @@
 //   S_C  = gamma_C S0 + K^T diag(gamma_C / gamma) U
 //   O    = diag(gamma) Q S0 + (tril(Q K^T) * exp(G_i - G_j)) U
 // This kernel groups the state term through P = K (S0 / sigma):
-//   U = U' - sigma (T diag(beta gamma)) P,   O = (sigma diag(gamma) Q) (S0 / sigma) + M U
+//   U = U' - sigma (T diag(beta gamma)) P,   O = M U + diag(sigma gamma) (Q (S0 / sigma))
 // Every chunk contraction is a tcgen05.mma with M = 128 (the value dimension,
 // or the 64 chunk rows of K stacked on 64 rows of Q) and accumulators in TMEM.
 // The state lives in TMEM transposed (lane = value row) as S / sigma with a
@@ -36,7 +36,7 @@
 // form P of chunk c + 1.  Warps w and w + 4 share TMEM lane quarter w (the only
 // lanes a warp may read).  prefill_pipe_kernel runs the prefill with outputs
 // and the fused replay + suffix (the replay window's chunks first, without
-// outputs): 185 KB of shared memory, 448 of 512 TMEM columns, one CTA per SM.
+// outputs): 169 KB of shared memory, 512 TMEM columns, one CTA per SM.
 #include <atomic>
 
 #include <cuda.h>
@@ -59,18 +59,20 @@ using namespace chunk;
 //                       (bf16) and -sigma' T diag(beta gamma) (fp32) as each block of
 //                       T is final;
 //            warps 4-7 (chain): chunk c's U epilogue, its state update and
-//                       O += U M^T, the TMA of chunk c + 2, chunk c's outputs; then
-//                       a bf16 copy of the new state in TMEM, sigma' gamma Q of chunk
-//                       cn in bf16, and, once the front has read TM_P, P = K S~ of
-//                       chunk cn into TM_P and the outputs' state term sigma' diag(gamma)
-//                       Q S~ into TM_O, both from the bf16 state copy.
+//                       O = U M^T, the TMA of chunk c + 2, chunk c's outputs
+//                       O + diag(sigma gamma) (Q S~) (the state term scaled per row
+//                       in fp32); then a bf16 copy of the new state in TMEM, and,
+//                       once the front has read TM_P, P = K S~ of chunk cn into TM_P
+//                       and the outputs' state term Q S~ of chunk cn into TM_OS, both
+//                       from the bf16 state copy and the chunk's own K and Q tiles.
 //   phase Y  warp 2: U of chunk cn = P^T (-sigma' T diag(beta gamma))^T (tf32) + U'
 //                       into TM_U; warp 3: [K; Q] K^T of chunk cn + 1 into TM_P once
 //                       the P term has read it; warps 0-1: the gates of chunk cn + 1.
-// 185 KB of shared memory, 512 TMEM columns, one CTA per SM.
+// 169 KB of shared memory, 512 TMEM columns, one CTA per SM.
 constexpr uint32_t BAR_CHAIN = 2;   // named barrier of warps 4-7
 constexpr uint32_t BAR_KK = 5;      // warps 0-3 -> warp 4: [K; Q] K^T in TM_P is read, P may overwrite it
 constexpr uint32_t TM_SB = 384;     // 64 columns (prefill): bf16 S~^T, two keys per column
+constexpr uint32_t TM_OS = 448;     // 64 columns (prefill): the outputs' state term (Q S~)^T
 struct PipeLayout {
     static constexpr uint32_t TILE = TileLayout::TILE;       // [K0 | Q0 | K1 | Q1 | V0 | V1]
     static constexpr uint32_t OFF_TILE = 0;
@@ -79,14 +81,13 @@ struct PipeLayout {
     static constexpr uint32_t OFF_TG = OFF_TB + 8192;           // fp32 -sigma T diag(beta gamma), K-major
     static constexpr uint32_t OFF_UB = OFF_TG + 16384;          // the output stage: bf16 O, two [i][dv] tiles
     static constexpr uint32_t OFF_MB = OFF_UB + 16384;          // two bf16 M [i][j], chunk c in c % 2
-    static constexpr uint32_t OFF_BQ = OFF_MB + 16384;          // bf16 sigma diag(gamma) Q, K-major
-    static constexpr uint32_t BYTES = OFF_BQ + 16384;
+    static constexpr uint32_t BYTES = OFF_MB + 16384;
 };
 static_assert(PipeLayout::OFF_TB % 1024 == 0 && PipeLayout::OFF_TG == PipeLayout::OFF_TB + 8192 &&
-                  PipeLayout::OFF_BQ % 1024 == 0 && PipeLayout::OFF_UB % 1024 == 0,
+                  PipeLayout::OFF_MB % 1024 == 0 && PipeLayout::OFF_UB % 1024 == 0,
               "operands and the output stage (a TMA source) on 1 KB, TG right after TB");
 static_assert(PipeLayout::BYTES + 1024 <= 227 * 1024, "fits one CTA per SM");
-static_assert(TM_SB + 64 <= 512, "TMEM map");
+static_assert(TM_OS + 64 <= 512, "TMEM map");
 
 __global__ void __launch_bounds__(NT, 1)
 prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
@@ -189,7 +190,6 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
 
     float* AT = reinterpret_cast<float*>(sm + PL::OFF_AT);
     const uint32_t s_tb = smem_u32(sm + PL::OFF_TB), s_tg = smem_u32(sm + PL::OFF_TG);
-    const uint32_t s_bq = smem_u32(sm + PL::OFF_BQ);
     const size_t state_base = ((size_t)b * H + h) * D * D;
     {   // initial state: TMEM lane dv holds column dv of S (a row of S^T)
         float v[32];
@@ -415,13 +415,12 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
                             mma_bf16_ts(tbase + TM_S, tbase + TM_UT + kk * 8, desc_advance(db, kk * 2048), id_s, 1u);
-                        if (outc) {   // O holds the state term unless the state entering chunk c is zero
+                        if (outc) {   // O = U M^T; the state term is added in the epilogue
                             const uint64_t dmb = smem_desc_sw128(s_mb, 16, 1024);
-                            const bool acc = has_state_terms(c);
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk)
                                 mma_bf16_ts(tbase + TM_O, tbase + TM_UB + kk * 8, desc_advance(dmb, kk * 32), id_o2,
-                                            (acc || kk > 0) ? 1u : 0u);
+                                            kk > 0 ? 1u : 0u);
                         }
                         mma_commit(&bar_s);
                         if (mbar_wait_bounded(&bar_s, ph_s, kWaitNs)) {
@@ -433,6 +432,7 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                     }
                     __syncwarp();
                 }
+                const float sig_c = sigma;   // the scale of the state entering chunk c
                 sigma = snew;
                 if (ct == 0 && outc) bulk_wait_group_read0();   // the last chunk's output store has read the stage
                 named_sync(BAR_CHAIN, 128);   // the state update (and O) of chunk c are complete
@@ -446,11 +446,37 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                     // fragments of 8 x 8 blocks [dv][i]; stmatrix .trans writes each block as 8
                     // rows i of 8 values dv.
                     const uint32_t s_stage = smem_u32(sm + PL::OFF_UB);
+                    // the state term's row factors sigma gamma_i for this thread's rows
+                    // i = 8 k + 2 (lane % 4) + {0, 1}
+                    const bool st_c = has_state_terms(c);   // uniform
+                    float2 sg[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const float2 g = *reinterpret_cast<const float2*>(s_gates[c & 1].gam + 8 * k + 2 * (lane & 3));
+                        sg[k] = make_float2(sig_c * g.x, sig_c * g.y);
+                    }
 #pragma unroll
                     for (int lh = 0; lh < 2; ++lh) {   // lanes 16 lh .. 16 lh + 15 of the quarter
                         float v[32];   // register 4k + e: dv = 16 lh + lane/4 + 8 (e/2), i = 8k + 2 (lane%4) + e%2
-                        tmem_ld16x256b_x8(tlane + ((uint32_t)(16 * lh) << 16) + TM_O, v);
+                        const uint32_t tq = tlane + ((uint32_t)(16 * lh) << 16);
+                        tmem_ld16x256b_x8(tq + TM_O, v);
                         tmem_wait_ld();
+                        if (st_c) {   // O = U M^T + diag(sigma gamma) Q S~, in two halves of the rows
+#pragma unroll
+                            for (int half = 0; half < 2; ++half) {
+                                float w[16];
+                                tmem_ld16x256b_x4(tq + TM_OS + 32 * half, w);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int kh = 0; kh < 4; ++kh) {
+                                    const int k = 4 * half + kh;
+                                    v[4 * k + 0] += sg[k].x * w[4 * kh + 0];
+                                    v[4 * k + 1] += sg[k].y * w[4 * kh + 1];
+                                    v[4 * k + 2] += sg[k].x * w[4 * kh + 2];
+                                    v[4 * k + 3] += sg[k].y * w[4 * kh + 3];
+                                }
+                            }
+                        }
 #pragma unroll
                         for (int hf = 0; hf < 2; ++hf) {
                             const int v0 = 32 * wq + 16 * lh + 8 * hf;   // the blocks' first dv
@@ -505,8 +531,9 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
             }
             if (st_next) {
                 // ---- chunk cn's state terms from a bf16 copy of S~^T (TM_SB): P^T = S~^T K^T into
-                //      TM_P once the front has read it, and, with outputs, the state term of O^T =
-                //      S~^T (sigma diag(gamma) Q)^T into TM_O (chunk c's outputs are read) ----
+                //      TM_P once the front has read it, and, with outputs, (Q S~)^T = S~^T Q^T into
+                //      TM_OS (chunk c's outputs have read it); the row factors sigma' gamma_i are
+                //      applied in chunk cn's output epilogue ----
                 const bool outn = chunk_src(cn).out;
 #pragma unroll
                 for (int cb = 0; cb < 4; ++cb) {
@@ -517,27 +544,6 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
 #pragma unroll
                     for (int q = 0; q < 16; ++q) pk[q] = pack_bf16(sv[2 * q], sv[2 * q + 1]);
                     tmem_st16(tlane + TM_SB + cb * 16, pk);
-                }
-                if (outn) {   // sigma gamma_i Q[i] in bf16, the Q tile's 128-byte swizzle kept
-                    const Gates& Gn = s_gates[cn & 1];
-                    const uint8_t* qt = tile_of(cn) + L::Q0;
-                    uint8_t* bq = sm + PL::OFF_BQ;
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {   // 1024 16-byte pieces: 2 blocks x 64 rows x 8
-                        // consecutive threads take consecutive pieces of a row: a warp reads and
-                        // writes four whole 128-byte rows, free of bank conflicts
-                        const int idx = ct + k * 128, chn = idx & 7, i = (idx >> 3) & (C - 1), blk = idx >> 9;
-                        const uint32_t off = (uint32_t)(i * 128 + (chn << 4));
-                        const uint4 raw = *reinterpret_cast<const uint4*>(qt + blk * L::K_BLK + off);
-                        const float sg = sigma * Gn.gam[i];
-                        const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
-                        uint32_t pq[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            pq[e] = pack_bf16(sg * __uint_as_float(wd[e] << 16), sg * __uint_as_float(wd[e] & 0xffff0000u));
-                        *reinterpret_cast<uint4*>(bq + blk * 8192 + off) = make_uint4(pq[0], pq[1], pq[2], pq[3]);
-                    }
-                    fence_proxy_async_smem();
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -551,12 +557,12 @@ prefill_pipe_kernel(const TcParams p, const __grid_constant__ CUtensorMap map_k,
                         for (int kk = 0; kk < 8; ++kk)
                             mma_bf16_ts(tbase + TM_P, tbase + TM_SB + kk * 8,
                                         desc_advance(dk, (kk >> 2) * L::K_BLK + (kk & 3) * 32), id_p, kk > 0);
-                        if (outn) {
-                            const uint64_t dq = smem_desc_sw128(s_bq, 16, 1024);
+                        if (outn) {   // (Q S~)^T of chunk cn from its Q tile
+                            const uint64_t dq = smem_desc_sw128(smem_u32(tile_of(cn) + L::Q0), 16, 1024);
 #pragma unroll
                             for (int kk = 0; kk < 8; ++kk)
-                                mma_bf16_ts(tbase + TM_O, tbase + TM_SB + kk * 8,
-                                            desc_advance(dq, (kk >> 2) * 8192 + (kk & 3) * 32), id_p, kk > 0);
+                                mma_bf16_ts(tbase + TM_OS, tbase + TM_SB + kk * 8,
+                                            desc_advance(dq, (kk >> 2) * L::K_BLK + (kk & 3) * 32), id_p, kk > 0);
                         }
                         mma_commit(&bar_p);
                     }

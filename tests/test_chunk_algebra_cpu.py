@@ -11,8 +11,9 @@ chunk they
   * keep the state as S / sigma with a running scalar sigma, multiply the state
     product by -sigma, and fold sigma back into the state when sigma * gamma_C
     falls below 2^-40.
-The prefill keeps U unscaled for its outputs, O = sigma diag(gamma) Q (S / sigma)
-+ M U, and applies E and 1 / sigma_new to U for the state update only.
+The prefill keeps U unscaled for its outputs, O = M U + diag(sigma gamma)
+(Q (S / sigma)) (the state term formed from Q itself and scaled per row after),
+and applies E and 1 / sigma_new to U for the state update only.
 This test restates those steps (not the kernels' code) and shows that they
 reproduce the recurrence (states and outputs) to fp64 rounding, including under
 strong and zero gates, so the kernels' parity rests on an exact reformulation."""
@@ -277,9 +278,10 @@ def chunk_algebra_prefill(q, k, v, alpha, beta, S0=None, unscaled_output_state_t
     """The prefill's grouping (the P-form): P = K (S / sigma) from the state entering
     the chunk, U = T diag(beta) V + (-sigma T diag(beta gamma)) P, unscaled (the
     outputs use it); E and 1/sigma_new are applied to U only for the state update.
-    Per chunk the outputs are O = (sigma diag(gamma) Q) (S / sigma) + M U with
-    M_ij = (q_i . k_j) 2^(G_i - G_j), j <= i.  A zero entering state skips chunk 0's
-    state terms (P and the outputs' state term), as the kernel does."""
+    Per chunk the outputs are O = M U + diag(sigma gamma) (Q (S / sigma)) with
+    M_ij = (q_i . k_j) 2^(G_i - G_j), j <= i: the state term is formed from Q itself
+    and its rows are scaled afterwards.  A zero entering state skips chunk 0's state
+    terms (P and the outputs' state term), as the kernel does."""
     n, dk = k.shape
     dv = v.shape[1]
     St = np.zeros((dk, dv)) if S0 is None else np.array(S0, dtype=np.float64)
@@ -312,7 +314,7 @@ def chunk_algebra_prefill(q, k, v, alpha, beta, S0=None, unscaled_output_state_t
             Tg = -sigma * (T * (bc * gam)[None, :])
             U = U + Tg @ P
             qs = gam if unscaled_output_state_term else sigma * gam
-            O = (qs[:, None] * qc) @ St + Mq @ U
+            O = Mq @ U + qs[:, None] * (qc @ St)
         o[c0:c0 + m] = O[:m]
         snew = sigma * gam[-1]
         if snew < RENORM_BELOW:
