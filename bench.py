@@ -613,8 +613,10 @@ def cpu_suffix_sample(wl):
 def e2e_host_buffers(data, kernel, args, world):
     """Same metric through the C ABI with host buffers: every step copies the
     tail windows and the suffix inputs from pinned host memory, runs the
-    replay and the suffix prefill, and reads states and outputs back; the
-    copies of one launch group overlap the kernels of the previous one."""
+    replay and the suffix prefill, and reads states and outputs back.  The
+    copies of one launch group overlap the kernels of another, and a step's
+    read-back overlaps the next step's input copies (PCIe carries both
+    directions at once)."""
     import gated_deltanet_state_tail_b200 as gdn
     wl = data.wl
     H, dk, dv = wl.H, wl.dk, wl.dv
@@ -644,27 +646,31 @@ def e2e_host_buffers(data, kernel, args, world):
 
     # The three launch groups are independent, so group j + 1's inputs cross PCIe while
     # group j replays and prefills (copy-in stream, compute stream), and group j's states
-    # and outputs are read back on a third stream.
+    # and outputs are read back on a third stream.  Across steps, group j's inputs are
+    # overwritten once the last step's kernels of group j have read them (ev_done), and
+    # its states and outputs once the last step has read them back (ev_out).
     cur = torch.cuda.current_stream()
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     n_groups = len(rp)
     ev_in = [torch.cuda.Event() for _ in range(n_groups)]
     ev_done = [torch.cuda.Event() for _ in range(n_groups)]
+    ev_out = [torch.cuda.Event() for _ in range(n_groups)]
 
     def rows_of(name, j):
         per_rows = per * (R if name.startswith("t") else N)
         return slice(j * per_rows, (j + 1) * per_rows)
 
     def step():
-        s_in.wait_stream(cur)                  # the previous step no longer reads the inputs
-        with torch.cuda.stream(s_in):
-            for j in range(n_groups):
+        for j in range(n_groups):
+            s_in.wait_event(ev_done[j])        # the last step's kernels of group j are done
+            with torch.cuda.stream(s_in):
                 for k in dev:
                     sl = rows_of(k, j)
                     dev[k][sl].copy_(host[k][sl], non_blocking=True)
-                ev_in[j].record(s_in)
+            ev_in[j].record(s_in)
         for j in range(n_groups):
             cur.wait_event(ev_in[j])
+            cur.wait_event(ev_out[j])          # the last step has read group j's results back
             gs, rs = slice(j * per, (j + 1) * per), slice(j * per * N, (j + 1) * per * N)
             rp[j].run(dev["tk"], dev["tv"], dev["talpha"], dev["tbeta"], state[gs])
             pp[j].run(dev["sq"], dev["sk"], dev["sv"], dev["salpha"], dev["sbeta"], o,
@@ -674,17 +680,20 @@ def e2e_host_buffers(data, kernel, args, world):
             with torch.cuda.stream(s_out):
                 h_state[gs].copy_(st_out[gs], non_blocking=True)
                 h_o[rs].copy_(o[rs], non_blocking=True)
-        cur.wait_stream(s_out)                 # the step ends with its results on the host
+            ev_out[j].record(s_out)
 
     steps = max(3, min(args.steps, 10))
     for _ in range(2):
         step()
+    cur.wait_stream(s_out)
     torch.cuda.synchronize()
     barrier(world)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
+    s_in.wait_stream(cur)                      # no timed copy starts before the start event
     for _ in range(steps):
         step()
+    cur.wait_stream(s_out)                     # the last step's results are on the host
     b.record()
     torch.cuda.synchronize()
     t = max_over_ranks(a.elapsed_time(b) / 1e3, world)
