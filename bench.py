@@ -953,9 +953,10 @@ def cpu_varlen_sample(wl, off, cu, cache, suf, nreq=4):
 def bench_decode(args):
     """One decode step (the token after the prefill) of the 24-layer stack for 64 requests:
     32 heads, d = 128, bf16 q/k/v/o, fp32 states updated in place.  The layers are folded into
-    the batch (24 x 64 = 1536 state slots, 6.4 GB of state, larger than L2), one launch."""
+    the batch (24 x 64 = 1536 state slots, 6.4 GB of state, larger than L2), one launch.
+    --layers sets fewer layers for a profiling capture."""
     import gated_deltanet_state_tail_b200 as gdn
-    layers, B, H, d = 24, 64, 32, 128
+    layers, B, H, d = args.layers, 64, 32, 128
     nb = layers * B
     t = inputs.draw_tensors(nb, H, d, d, "bf16", 0.9, 0.999, 7, device="cuda")
     g = torch.Generator(device="cuda").manual_seed(8)
@@ -971,13 +972,14 @@ def bench_decode(args):
     nbytes = nb * H * (2 * d * d * 4 + 4 * d * 2 + 8)   # state read + write, q k v o, alpha beta
     peaks = measured_peaks()
     gbs = nbytes / (ms / 1e3) / 1e9
-    return [{"metric": "GDN decode step (24 layers x 64 requests)", "value": ms, "unit": "ms",
-             "higher_is_better": False, "workload": "decode24-B64-H32-d128-bf16", "layers": layers,
+    return [{"metric": f"GDN decode step ({layers} layers x {B} requests)", "value": ms, "unit": "ms",
+             "higher_is_better": False, "workload": f"decode{layers}-B{B}-H{H}-d{d}-bf16", "layers": layers,
              "requests": B, "heads": H, "tokens_per_s": B / (ms / 1e3),
              "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                           "frac": gbs / peaks["hbm_gbs"], "traffic": None, "peak_source": peaks["source"],
                           "bytes_per_launch": nbytes},
-             "l2": "6.4 GB of state per launch, larger than L2", "dtype": "bf16", "data": "synthetic"}]
+             "l2": f"{nb * H * d * d * 4 / 1e9:.2f} GB of state per launch (L2 is 126 MB)", "dtype": "bf16",
+             "data": "synthetic"}]
 
 
 def bench_outputs(args):
