@@ -104,19 +104,21 @@ int resolve_kernel(const gdn_varlen_desc* d) {
                                                               : GDN_KERNEL_RECURRENT;
 }
 
-// Longest replay window (tokens) that a fused call on the chunked kernel still runs as one
+// Longest replay windows (tokens) that a fused call on the chunked kernel still runs as one
 // launch.  One launch keeps the state on chip between the window and the suffix and saves a
 // launch, but its window chunks run on the one-CTA-per-SM prefill kernel, slower per chunk
 // than the two-CTA state-only replay kernel.  Measured on B200 (bf16, d = 128, 512-token
 // suffix): with at most one unit per SM, one launch is 2-12 us faster up to 13 chunks, within
-// 2 us either way at 20 and up to 28 us slower at 52; with more units than SMs, two launches
-// win from 7 chunks on.
-constexpr int kFusedOneLaunchMaxTokens = 16 * 64;
+// 2 us either way at 20 and up to 28 us slower at 52; with 192 to 444 units, 2-18 us faster
+// up to 5 chunks and 3.5-5 us slower at 7.
+constexpr int kFusedOneLaunchMaxTokens = 16 * 64;         // at most one unit per SM
+constexpr int kFusedOneLaunchMaxTokensAnyUnits = 5 * 64;  // any number of units
 
-// A fused plan on the chunked kernel runs as one launch when every (sequence, head) unit has
-// an SM of its own and no window is longer than kFusedOneLaunchMaxTokens; otherwise as the
-// state-only replay launch followed by the prefill launch.  A descriptor that pins a replay
-// kernel always takes the two launches.
+// A fused plan on the chunked kernel runs as one launch when no window is longer than
+// kFusedOneLaunchMaxTokensAnyUnits, or when every (sequence, head) unit has an SM of its own
+// and no window is longer than kFusedOneLaunchMaxTokens; otherwise as the state-only replay
+// launch followed by the prefill launch.  A descriptor that pins a replay kernel always takes
+// the two launches.
 gdn_status choose_fused_schedule(gdn_plan* p) {
     p->fused_one_launch = false;
     if (p->kernel != GDN_KERNEL_CHUNKED_TC || p->replay_variant != gdn::kReplayDefault) return GDN_OK;
@@ -127,7 +129,8 @@ gdn_status choose_fused_schedule(gdn_plan* p) {
     }
     int longest = 0;
     for (const Window& w : p->windows0) longest = std::max(longest, (int)w.len);
-    p->fused_one_launch = (long long)p->batch * p->num_heads <= sms && longest <= kFusedOneLaunchMaxTokens;
+    p->fused_one_launch = longest <= kFusedOneLaunchMaxTokensAnyUnits ||
+                          ((long long)p->batch * p->num_heads <= sms && longest <= kFusedOneLaunchMaxTokens);
     return GDN_OK;
 }
 

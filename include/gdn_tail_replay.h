@@ -279,9 +279,10 @@ GDN_API gdn_status gdn_chunk_prefill(gdn_plan_t plan, const void* q, const void*
  * Fused rebuild + suffix prefill on a fused plan: equal (up to rounding
  * order) to gdn_tail_replay_state followed by gdn_chunk_prefill from the
  * rebuilt states.  The plan fixes how it runs.  On the tensor-core kernel,
- * when the plan has no more (sequence, head) units than the GPU has SMs and
- * no replay window is longer than 1024 tokens, it is one launch and the
- * state stays on chip between the two phases.  Otherwise, on that kernel
+ * when no replay window is longer than 320 tokens, or when the plan has no
+ * more (sequence, head) units than the GPU has SMs and no window is longer
+ * than 1024 tokens, it is one launch and the state stays on chip between
+ * the two phases.  Otherwise, on that kernel
  * with a replay kernel pinned, and on the fp32 recurrent kernel, it is a
  * state-only replay launch writing state_mid (or state_out) and a prefill
  * launch reading it back: longer windows replay faster on the replay

@@ -3,11 +3,12 @@ replay followed by its prefill, on ragged batches that include an empty window,
 an empty suffix, R = 0 and R > L.  Tolerance: max|err|/max|ref| per request and
 tensor.
 
-The tensor-core kernel runs a fused call as one launch when the plan has at
-most one (sequence, head) unit per SM and no replay window is longer than 1024
-tokens, and otherwise (or with a replay kernel pinned) as the state-only replay
-launch followed by the prefill launch; both schedules are covered, and the
-two-launch one must equal separate replay and prefill plans bit for bit."""
+The tensor-core kernel runs a fused call as one launch when no replay window is
+longer than 320 tokens, or when the plan has at most one (sequence, head) unit per
+SM and no window is longer than 1024 tokens, and otherwise (or with a replay kernel
+pinned) as the state-only replay launch followed by the prefill launch; both
+schedules are covered, and the two-launch one must equal separate replay and
+prefill plans bit for bit."""
 import numpy as np
 import pytest
 import torch
@@ -128,18 +129,36 @@ def test_fused_long_window_runs_as_replay_then_prefill():
 
 
 def test_fused_more_units_than_sms_runs_as_replay_then_prefill():
+    # more units than SMs and one window over 320 tokens: two launches
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     H = 4
-    B = sms // H + 2                  # H * B > SMs, short windows
+    B = sms // H + 2                  # H * B > SMs
     rng = np.random.default_rng(9)
     cached = rng.integers(40, 200, size=B)
     ml = np.minimum(cached, rng.integers(30, 200, size=B)).astype(np.int32)
     R = rng.integers(0, 160, size=B).astype(np.int32)
+    cached[0] = ml[0] = R[0] = 330
     slen = rng.integers(0, 90, size=B)
     launches, got, sep = _fused_vs_separate(H, cached, ml, R, slen, 71)
     assert launches == 2
     for g, e in zip(got, sep):
         assert np.array_equal(g, e)
+
+
+def test_fused_more_units_than_sms_short_windows_run_as_one_launch():
+    # more units than SMs, every window <= 320 tokens (one of exactly 320): one launch,
+    # checked against the oracle
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    H = 4
+    B = sms // H + 2
+    rng = np.random.default_rng(12)
+    cached = rng.integers(40, 400, size=B)
+    ml = np.minimum(cached, rng.integers(30, 400, size=B)).astype(np.int32)
+    R = np.minimum(rng.integers(0, 321, size=B), 320).astype(np.int32)
+    cached[0] = ml[0] = R[0] = 320
+    slen = rng.integers(0, 90, size=B)
+    launches, _, _ = _fused_vs_separate(H, cached, ml, R, slen, 91)
+    assert launches == 1
 
 
 def test_fused_short_windows_run_as_one_launch():
